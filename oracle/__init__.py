@@ -1,0 +1,190 @@
+"""CPU oracle for the quantized linear layer -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its binding) never imports, links or executes anything here, and this package
+imports nothing from the product.
+
+The arithmetic lives in ``qlin_oracle.c`` (plain C, one separately rounded
+binary32 operation per step, exact integer sums); this module only marshals
+numpy arrays to it.  bf16 tensors travel as their uint16 bit patterns.
+
+Format codes: 0 = INT8 (W8A8), 1 = FP8 e4m3 per-token/per-channel,
+2 = Block-FP8 (1x128 activation groups, 128x128 weight blocks), the three
+formats named on the page "Helion in vLLM: A Unified Route to Tunable Linear
+Kernels", section "What the integration changes".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+FMT_INT8 = 0
+FMT_FP8 = 1
+FMT_FP8_BLOCK = 2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "qlin_oracle.c")
+_LIB = os.path.join(_HERE, "libqlin_oracle.so")
+
+# Flags that keep every binary32 operation rounded exactly as written.
+CFLAGS = ["-O2", "-std=c99", "-fno-fast-math", "-ffp-contract=off", "-fexcess-precision=standard",
+          "-fPIC", "-shared"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library with gcc (idempotent)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        f32p = ctypes.POINTER(ctypes.c_float)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        i64 = ctypes.c_int64
+        lib.qo_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.qo_bf16_to_f32.restype = ctypes.c_float
+        lib.qo_f32_to_bf16.argtypes = [ctypes.c_float]
+        lib.qo_f32_to_bf16.restype = ctypes.c_uint16
+        lib.qo_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.qo_e4m3_decode.restype = ctypes.c_float
+        lib.qo_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.qo_e4m3_encode.restype = ctypes.c_uint8
+        lib.qo_e4m3_units.argtypes = [ctypes.c_uint8]
+        lib.qo_e4m3_units.restype = ctypes.c_int64
+        lib.qo_quantize_per_token.argtypes = [ctypes.c_int, u16p, i64, i64, i64, u8p, f32p]
+        lib.qo_quantize_per_token.restype = None
+        lib.qo_quantize_block.argtypes = [u16p, i64, i64, i64, i64, i64, u8p, f32p]
+        lib.qo_quantize_block.restype = None
+        lib.qo_scaled_mm.argtypes = [ctypes.c_int, i64, i64, i64, u8p, f32p, u8p, f32p, u16p,
+                                     i64p, i64, i64p, i64, u16p, i32p]
+        lib.qo_scaled_mm.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray | None, ctype):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 input as a contiguous uint16 array (accepts torch bf16 or uint16 numpy)."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch  # plumbing only: reinterpret bf16 storage as raw bits
+
+    assert x.dtype == torch.bfloat16 and x.device.type == "cpu"
+    return np.ascontiguousarray(x.contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+# ------------------------------------------------------------------ scalars --
+def bf16_to_f32(b: int) -> float:
+    return _load().qo_bf16_to_f32(b)
+
+
+def f32_to_bf16(f: float) -> int:
+    return _load().qo_f32_to_bf16(f)
+
+
+def e4m3_decode(code: int) -> float:
+    return _load().qo_e4m3_decode(code)
+
+
+def e4m3_encode(v: float) -> int:
+    return _load().qo_e4m3_encode(v)
+
+
+def e4m3_units(code: int) -> int:
+    return _load().qo_e4m3_units(code)
+
+
+# --------------------------------------------------------------- quantisers --
+def quantize_per_token(fmt: int, x) -> tuple[np.ndarray, np.ndarray]:
+    """Per-token dynamic quantisation of a bf16 [rows, cols] matrix.
+
+    Returns (q uint8 [rows, cols] -- int8 bits for INT8, e4m3 codes for FP8 --,
+    s float32 [rows]).
+    """
+    assert fmt in (FMT_INT8, FMT_FP8)
+    xb = _bits(x)
+    rows, cols = xb.shape
+    q = np.empty((rows, cols), np.uint8)
+    s = np.empty((rows,), np.float32)
+    _load().qo_quantize_per_token(fmt, _ptr(xb, ctypes.c_uint16), rows, cols, cols,
+                                  _ptr(q, ctypes.c_uint8), _ptr(s, ctypes.c_float))
+    return q, s
+
+
+def quantize_block(x, block_rows: int, block_cols: int = 128) -> tuple[np.ndarray, np.ndarray]:
+    """Block-FP8 quantisation; scales [ceil(rows/block_rows), cols/block_cols]."""
+    xb = _bits(x)
+    rows, cols = xb.shape
+    assert cols % block_cols == 0
+    q = np.empty((rows, cols), np.uint8)
+    s = np.empty(((rows + block_rows - 1) // block_rows, cols // block_cols), np.float32)
+    _load().qo_quantize_block(_ptr(xb, ctypes.c_uint16), rows, cols, cols, block_rows, block_cols,
+                              _ptr(q, ctypes.c_uint8), _ptr(s, ctypes.c_float))
+    return q, s
+
+
+# -------------------------------------------------------------- scaled GEMM --
+def scaled_mm(fmt: int, a_q: np.ndarray, s_a: np.ndarray, w_q: np.ndarray, s_w: np.ndarray,
+              bias=None, m_idx=None, n_idx=None, want_acc: bool = False):
+    """C = (A_q W_q^T) * s_a * s_w + bias as bf16 bits, optionally on a row/column sample.
+
+    Returns uint16 C [len(m_idx), len(n_idx)] (or [M, N]); with want_acc (INT8)
+    also the int32 accumulators.
+    """
+    a_q = np.ascontiguousarray(a_q, dtype=np.uint8)
+    w_q = np.ascontiguousarray(w_q, dtype=np.uint8)
+    s_a = np.ascontiguousarray(s_a, dtype=np.float32)
+    s_w = np.ascontiguousarray(s_w, dtype=np.float32)
+    M, K = a_q.shape
+    N, K2 = w_q.shape
+    assert K == K2 and K % 128 == 0
+    if fmt == FMT_FP8_BLOCK:
+        assert bias is None
+        assert s_a.shape == (M, K // 128) and s_w.shape == ((N + 127) // 128, K // 128)
+    else:
+        assert s_a.shape == (M,) and s_w.shape == (N,)
+    bb = None if bias is None else _bits(bias).reshape(-1)
+    mi = None if m_idx is None else np.ascontiguousarray(m_idx, dtype=np.int64)
+    ni = None if n_idx is None else np.ascontiguousarray(n_idx, dtype=np.int64)
+    mc = M if mi is None else len(mi)
+    nc = N if ni is None else len(ni)
+    c = np.empty((mc, nc), np.uint16)
+    acc = np.empty((mc, nc), np.int32) if want_acc else None
+    rc = _load().qo_scaled_mm(fmt, M, N, K, _ptr(a_q, ctypes.c_uint8), _ptr(s_a, ctypes.c_float),
+                              _ptr(w_q, ctypes.c_uint8), _ptr(s_w, ctypes.c_float),
+                              _ptr(bb, ctypes.c_uint16), _ptr(mi, ctypes.c_int64), mc,
+                              _ptr(ni, ctypes.c_int64), nc, _ptr(c, ctypes.c_uint16),
+                              _ptr(acc, ctypes.c_int32))
+    if rc == -1:
+        raise OverflowError("INT8 accumulator left the int32 range")
+    if rc != 0:
+        raise MemoryError("oracle allocation failed")
+    return (c, acc) if want_acc else c
+
+
+def bf16_bits_to_f32(c: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns to float32 values (exact)."""
+    return (c.astype(np.uint32) << 16).view(np.float32)

@@ -1,0 +1,276 @@
+/*
+ * qlin_oracle.c -- plain, slow, obviously-correct CPU oracle for the quantized
+ * linear layer (dynamic activation quantisation followed by a scaled GEMM).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package smoke check and
+ * the CPU-baseline leg of the benchmark may load this library.  It shares no
+ * code, header, table or constant generator with the CUDA library; neither
+ * side includes or links the other.
+ *
+ * What it follows.  The page "Helion in vLLM: A Unified Route to Tunable Linear
+ * Kernels", section "What the integration changes", names the three formats
+ * (FP8 dynamic quantisation, W8A8 INT8, Block-FP8) and the three GEMM
+ * strategies (plain, Split-K, Swap-AB).  The page prints no formula, so each
+ * function below states the arithmetic it implements, in the plainest reading:
+ *
+ *   per-token (INT8 / FP8):   s[m] = amax_k |x[m,k]| / Qmax, Qmax = 127 / 448
+ *                             q[m,k] = Q(x[m,k] / s[m])
+ *   Block-FP8:                one scale per 1x128 (activations) or 128x128
+ *                             (weights) block, s = amax_block / 448
+ *   scaled GEMM:              C[m,n] = bf16( (acc[m,n] * s_a[m]) * s_w[n] + bias[n] )
+ *   Block-FP8 GEMM:           C[m,n] = bf16( sum_kb P_kb[m,n] * s_a[m,kb] * s_w[n/128,kb] )
+ *
+ * Every fp32 operation is a separately rounded IEEE binary32 operation
+ * (compile with -O2 -fno-fast-math -ffp-contract=off; x86-64 SSE arithmetic),
+ * round-to-nearest-even.  Sums of products are formed EXACTLY in 64-bit
+ * integers and rounded once, so the oracle is at least as accurate as any
+ * fp32 accumulation order.
+ *
+ * Readings taken where the pages are silent:
+ *   - amax == 0: the scale is 0 and every quantised value is +0.
+ *   - x / s is a true IEEE division, not a multiply by 1/s.
+ *   - INT8 rounds half-to-even and clamps to [-127, 127] (-128 never occurs).
+ *   - FP8 clamps x/s to [-448, 448] ("saturation"), then rounds to the nearest
+ *     OCP E4M3 (e4m3fn) code, ties to the even code, keeping the sign of zero.
+ *
+ * Parity pins for every function here live in tests/test_oracle_*.py.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <stdlib.h>
+
+#define QO_FMT_INT8 0
+#define QO_FMT_FP8 1
+#define QO_FMT_FP8_BLOCK 2
+
+/* ---------------------------------------------------------------- bf16 ---- */
+
+/* bfloat16 is the upper half of a binary32: widening is a 16-bit shift. */
+float qo_bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* binary32 -> bfloat16, round to nearest, ties to even (on the dropped 16 bits). */
+uint16_t qo_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if (isnan(f)) return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t upper = u >> 16;
+    uint32_t lower = u & 0xFFFFu;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;
+    return (uint16_t)upper;
+}
+
+/* ---------------------------------------------------------------- e4m3 ---- */
+/*
+ * OCP FP8 E4M3 ("e4m3fn"): 1 sign bit, 4 exponent bits (bias 7), 3 mantissa
+ * bits, no infinities; S.1111.111 is NaN, so the largest finite magnitude is
+ * S.1111.110 = 1.75 * 2^8 = 448.  Exponent field 0 holds subnormals m * 2^-9.
+ */
+
+/* Value of a code as an integer count of 2^-9 (exact for every finite code). */
+int64_t qo_e4m3_units(uint8_t code) {
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    int64_t mag;
+    if (e == 0)
+        mag = m;                              /* m * 2^-9                   */
+    else
+        mag = (int64_t)(8 + m) << (e - 1);    /* (1 + m/8) * 2^(e-7) / 2^-9 */
+    return (code & 0x80) ? -mag : mag;
+}
+
+float qo_e4m3_decode(uint8_t code) {
+    if ((code & 0x7F) == 0x7F) return NAN;
+    double v = (double)qo_e4m3_units(code) * ldexp(1.0, -9);
+    if (v == 0.0 && (code & 0x80)) return -0.0f;
+    return (float)v;
+}
+
+/* floor(v + 1/2) with exact ties going to the even integer; v >= 0. */
+static double round_half_even_nonneg(double v) {
+    double f = floor(v);
+    double frac = v - f;                      /* exact: v has few bits here */
+    if (frac > 0.5) return f + 1.0;
+    if (frac < 0.5) return f;
+    return (fmod(f, 2.0) == 0.0) ? f : f + 1.0;
+}
+
+/* Nearest e4m3fn code to v (ties to even code), saturating at +-448. */
+uint8_t qo_e4m3_encode(float v) {
+    if (isnan(v)) return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal range: grid step 2^-9; rounding up to 8 steps lands on
+         * 2^-6, which is code 0x08, the smallest normal -- the same integer. */
+        double r = round_half_even_nonneg(a * 512.0);
+        return (uint8_t)(sign | (uint8_t)r);
+    }
+    int e = (int)floor(log2(a));              /* unbiased exponent, -6..8 */
+    /* guard log2 rounding at exact powers of two */
+    if (ldexp(1.0, e) > a) e -= 1;
+    if (ldexp(1.0, e + 1) <= a) e += 1;
+    double steps = a / ldexp(1.0, e - 3);     /* in [8, 16), exact */
+    double r = round_half_even_nonneg(steps); /* 8..16; 16 carries into e+1 */
+    int code = ((e + 7) << 3) + ((int)r - 8);
+    if (code > 0x7E) code = 0x7E;             /* cannot happen below 448 */
+    return (uint8_t)(sign | (uint8_t)code);
+}
+
+/* ----------------------------------------------------------- quantisers ---- */
+
+/* Round half to even to an integer, then clamp to [-127, 127]. */
+static int8_t int8_rne_clamp(float v) {
+    double a = round_half_even_nonneg(fabs((double)v));
+    double r = signbit(v) ? -a : a;
+    if (r > 127.0) r = 127.0;
+    if (r < -127.0) r = -127.0;
+    return (int8_t)r;
+}
+
+static uint8_t quantize_one(int fmt, float x, float s) {
+    if (s == 0.0f) return 0;                  /* amax == 0 reading: q = +0 */
+    float v = x / s;                          /* IEEE binary32 division */
+    if (fmt == QO_FMT_INT8) return (uint8_t)int8_rne_clamp(v);
+    if (v > 448.0f) v = 448.0f;               /* saturation */
+    if (v < -448.0f) v = -448.0f;
+    return qo_e4m3_encode(v);
+}
+
+/*
+ * Per-token dynamic quantisation (INT8 or FP8): one scale per row.
+ * x: bf16 bits [rows][ld], q: [rows][cols] row-major, s: [rows].
+ */
+void qo_quantize_per_token(int fmt, const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                           uint8_t* q, float* s) {
+    const float qmax = (fmt == QO_FMT_INT8) ? 127.0f : 448.0f;
+    for (int64_t r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int64_t c = 0; c < cols; ++c) {
+            float a = fabsf(qo_bf16_to_f32(x[r * ld + c]));
+            if (a > amax) amax = a;
+        }
+        float sr = amax / qmax;               /* IEEE binary32 division */
+        s[r] = sr;
+        for (int64_t c = 0; c < cols; ++c)
+            q[r * cols + c] = quantize_one(fmt, qo_bf16_to_f32(x[r * ld + c]), sr);
+    }
+}
+
+/*
+ * Block-FP8 quantisation: one e4m3 scale per block of block_rows x block_cols
+ * elements (1 x 128 for activations, 128 x 128 for weights).  A block at the
+ * bottom edge holds the rows that exist.  cols must be a multiple of
+ * block_cols.  s: [ceil(rows/block_rows)][cols/block_cols] row-major.
+ */
+void qo_quantize_block(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                       int64_t block_rows, int64_t block_cols, uint8_t* q, float* s) {
+    int64_t nbr = (rows + block_rows - 1) / block_rows;
+    int64_t nbc = cols / block_cols;
+    for (int64_t br = 0; br < nbr; ++br) {
+        int64_t r0 = br * block_rows;
+        int64_t r1 = r0 + block_rows < rows ? r0 + block_rows : rows;
+        for (int64_t bc = 0; bc < nbc; ++bc) {
+            int64_t c0 = bc * block_cols, c1 = c0 + block_cols;
+            float amax = 0.0f;
+            for (int64_t r = r0; r < r1; ++r)
+                for (int64_t c = c0; c < c1; ++c) {
+                    float a = fabsf(qo_bf16_to_f32(x[r * ld + c]));
+                    if (a > amax) amax = a;
+                }
+            float sb = amax / 448.0f;
+            s[br * nbc + bc] = sb;
+            for (int64_t r = r0; r < r1; ++r)
+                for (int64_t c = c0; c < c1; ++c)
+                    q[r * cols + c] = quantize_one(QO_FMT_FP8, qo_bf16_to_f32(x[r * ld + c]), sb);
+        }
+    }
+}
+
+/* ---------------------------------------------------------- scaled GEMM ---- */
+
+/* Exact integer value of a quantised element: int8 as is, e4m3 in 2^-9 units. */
+static int64_t element_units(int fmt, uint8_t code) {
+    if (fmt == QO_FMT_INT8) return (int64_t)(int8_t)code;
+    return qo_e4m3_units(code);
+}
+
+/*
+ * Scaled GEMM, C = A_q * W_q^T with scales, both operands K-major:
+ *   a_q [M][K], w_q [N][K], c [M][N] bf16 bits.
+ * Per-token formats: s_a [M], s_w [N]; bias bf16 [N] or NULL.
+ *   INT8: acc = sum_k a*w exactly (int32 range), y = fp32(acc)
+ *   FP8 : acc = sum_k a*w exactly in 2^-18 units, y = fp32(acc) (one rounding)
+ *   y = y * s_a[m]; y = y * s_w[n]; y = y + bias[n]; C = bf16(y)
+ * Block-FP8: s_a [M][K/128], s_w [ceil(N/128)][K/128]; bias must be NULL.
+ *   P_kb exact per 128-wide K block, acc = sum_kb P_kb*2^-18*s_a*s_w in fp64,
+ *   C = bf16(fp32(acc)).
+ * Only the rows m_idx[0..m_cnt) and columns n_idx[0..n_cnt) are computed
+ * (NULL index = all); outputs are dense [m_cnt][n_cnt].
+ * acc_out (INT8 only, may be NULL): the int32 accumulators, [m_cnt][n_cnt].
+ * Returns 0, or -1 if an INT8 accumulator leaves the int32 range.
+ */
+int qo_scaled_mm(int fmt, int64_t M, int64_t N, int64_t K,
+                 const uint8_t* a_q, const float* s_a, const uint8_t* w_q, const float* s_w,
+                 const uint16_t* bias, const int64_t* m_idx, int64_t m_cnt,
+                 const int64_t* n_idx, int64_t n_cnt, uint16_t* c, int32_t* acc_out) {
+    if (!m_idx) m_cnt = M;
+    if (!n_idx) n_cnt = N;
+    const int64_t kblocks = K / 128;
+    /* decode the selected rows once into exact integers */
+    int64_t* ua = (int64_t*)malloc(sizeof(int64_t) * (size_t)(m_cnt * K));
+    int64_t* uw = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_cnt * K));
+    if (!ua || !uw) { free(ua); free(uw); return -2; }
+    for (int64_t i = 0; i < m_cnt; ++i) {
+        int64_t m = m_idx ? m_idx[i] : i;
+        for (int64_t k = 0; k < K; ++k) ua[i * K + k] = element_units(fmt, a_q[m * K + k]);
+    }
+    for (int64_t j = 0; j < n_cnt; ++j) {
+        int64_t n = n_idx ? n_idx[j] : j;
+        for (int64_t k = 0; k < K; ++k) uw[j * K + k] = element_units(fmt, w_q[n * K + k]);
+    }
+    int rc = 0;
+    for (int64_t i = 0; i < m_cnt; ++i) {
+        int64_t m = m_idx ? m_idx[i] : i;
+        const int64_t* ra = ua + i * K;
+        for (int64_t j = 0; j < n_cnt; ++j) {
+            int64_t n = n_idx ? n_idx[j] : j;
+            const int64_t* rw = uw + j * K;
+            float y;
+            if (fmt == QO_FMT_FP8_BLOCK) {
+                double acc = 0.0;
+                for (int64_t kb = 0; kb < kblocks; ++kb) {
+                    int64_t p = 0;
+                    for (int64_t k = kb * 128; k < kb * 128 + 128; ++k) p += ra[k] * rw[k];
+                    acc += (double)p * ldexp(1.0, -18) * (double)s_a[m * kblocks + kb]
+                           * (double)s_w[(n / 128) * kblocks + kb];
+                }
+                y = (float)acc;
+            } else {
+                int64_t p = 0;
+                for (int64_t k = 0; k < K; ++k) p += ra[k] * rw[k];
+                if (fmt == QO_FMT_INT8) {
+                    if (p > INT32_MAX || p < INT32_MIN) rc = -1;
+                    if (acc_out) acc_out[i * n_cnt + j] = (int32_t)p;
+                    y = (float)(int32_t)p;            /* int32 -> fp32, RNE */
+                } else {
+                    y = (float)p;                     /* exact sum, one rounding */
+                    y = y * 0x1p-18f;                 /* exact power-of-two scaling */
+                }
+                y = y * s_a[m];
+                y = y * s_w[n];
+                if (bias) y = y + qo_bf16_to_f32(bias[n]);
+            }
+            c[i * n_cnt + j] = qo_f32_to_bf16(y);
+        }
+    }
+    free(ua);
+    free(uw);
+    return rc;
+}
