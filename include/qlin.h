@@ -1,0 +1,237 @@
+/*
+ * qlin.h -- C ABI of the B200 (sm_100a) quantized linear layer library.
+ *
+ * The hot path of a quantized linear layer in LLM serving: dynamic activation
+ * quantisation followed by a scaled GEMM whose epilogue applies the scales and
+ * the bias and stores bf16,
+ *
+ *     C[m,n] = bf16( (sum_k A_q[m,k] * W_q[n,k]) * s_a[m] * s_w[n] + bias[n] )
+ *
+ * in the three formats named on the page "Helion in vLLM: A Unified Route to
+ * Tunable Linear Kernels" (section "What the integration changes": FP8 dynamic
+ * quantisation, W8A8 INT8 and Block-FP8), with the three GEMM strategies the
+ * same section lists (ordinary GEMM, Split-K, Swap-AB) chosen per shape from a
+ * dispatch table ("Algorithm choice becomes part of tuning", same section).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named *_q, x, scale_*, bias, c_out and workspace are DEVICE
+ *     pointers owned by the caller; the library allocates no device memory and
+ *     keeps no pointer after a call returns.
+ *   - All device work is enqueued on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and is asynchronous: outputs are valid once the
+ *     stream has reached that point.  Apart from the table loader, no entry
+ *     point synchronises, allocates or compiles, so calls may be captured in a
+ *     CUDA graph.
+ *   - Arguments are validated on the host before anything is launched; a bad
+ *     argument returns an error status and launches nothing.  No entry point
+ *     aborts the process.
+ *   - Matrices are dense and row-major: A [M,K], W [N,K] (nn.Linear layout,
+ *     so both GEMM operands are K-major), C [M,N].
+ *   - bf16 data is IEEE bfloat16; e4m3 is the OCP FP8 E4M3 ("e4m3fn")
+ *     encoding; int8 is two's complement.
+ *   - Device kernels never wait unboundedly: a wait that exceeds its limit
+ *     records QLIN_ERR_DEVICE_TIMEOUT, which qlin_sync_status() reports.
+ */
+#ifndef QLIN_H
+#define QLIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QLIN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define QLIN_API __attribute__((visibility("default")))
+#else
+#define QLIN_API
+#endif
+
+typedef void* qlin_stream_t; /* cudaStream_t */
+
+typedef enum {
+    QLIN_OK = 0,
+    QLIN_ERR_INVALID_ARG = 1,   /* null pointer, bad enum, non-positive size, ... */
+    QLIN_ERR_UNSUPPORTED = 2,   /* shape/format/variant combination not provided */
+    QLIN_ERR_ALIGNMENT = 3,     /* pointer or stride not 16-byte aligned */
+    QLIN_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+    QLIN_ERR_TABLE_IO = 5,      /* dispatch table file unreadable */
+    QLIN_ERR_TABLE_FORMAT = 6,  /* dispatch table malformed or inconsistent */
+    QLIN_ERR_TABLE_DEVICE = 7,  /* dispatch table made for another device */
+    QLIN_ERR_CUDA = 8,          /* a CUDA runtime/driver call failed */
+    QLIN_ERR_DEVICE_TIMEOUT = 9,/* a device-side wait gave up (see qlin_sync_status) */
+    QLIN_ERR_NO_DEVICE = 10     /* no sm_100 device is current */
+} qlin_status;
+
+typedef enum {
+    QLIN_FMT_INT8 = 0,       /* W8A8 INT8, per-token / per-channel scales, int32 accumulate */
+    QLIN_FMT_FP8 = 1,        /* e4m3, per-token / per-channel scales, fp32 accumulate */
+    QLIN_FMT_FP8_BLOCK = 2   /* e4m3, 1x128 activation groups, 128x128 weight blocks */
+} qlin_format;
+
+typedef enum {
+    QLIN_VAR_AUTO = 0,          /* dispatch table entry, else the built-in rule */
+    QLIN_VAR_PLAIN = 1,         /* one CTA per output tile, all K segments in it */
+    QLIN_VAR_SPLITK = 2,        /* K segments of a tile spread over CTAs, fixed-order reduce */
+    QLIN_VAR_SWAPAB = 3,        /* C^T = W A^T: N fills the 128-row MMA side, M the narrow side */
+    QLIN_VAR_SWAPAB_SPLITK = 4  /* Swap-AB with the K segments spread over CTAs */
+} qlin_variant;
+
+/* flags for qlin_scaled_mm */
+#define QLIN_OUT_I32ACC 1u /* INT8 only: write the raw int32 accumulators instead of bf16 C */
+
+/* A resolved GEMM configuration (what qlin_dispatch_query returns). */
+typedef struct {
+    int32_t variant;    /* qlin_variant, never AUTO */
+    int32_t tile_n;     /* rows of the narrow MMA operand per tile: 16, 32, 64 (Swap-AB) or 128, 256 */
+    int32_t k_segments; /* S: K is cut into S equal segments; fixed per (format, N, K) */
+    int32_t stages;     /* shared-memory pipeline depth the kernel uses for tile_n */
+    int64_t m_max;      /* upper bound of the table bucket (0 for the built-in rule) */
+    int32_t from_table; /* 1 if the loaded table supplied the entry */
+} qlin_config;
+
+/*
+ * qlin_quantize_per_token -- dynamic per-token activation quantisation
+ * ("FP8 dynamic quantization" and "W8A8 INT8", page "Helion in vLLM: A Unified
+ * Route to Tunable Linear Kernels", section "What the integration changes").
+ *
+ * For each row r: amax = max_c |x[r,c]|; scale_out[r] = amax / Qmax (IEEE
+ * binary32 division; Qmax = 127 for INT8, 448 for FP8); q_out[r,c] =
+ * round(x[r,c] / scale_out[r]) -- INT8: half-to-even, clamped to [-127,127];
+ * FP8: clamped to [-448,448] then nearest e4m3, ties to even.  A row whose
+ * amax is 0 gets scale 0 and all-zero codes.  Also quantises weights
+ * per output channel (rows of W).
+ *
+ *   fmt        QLIN_FMT_INT8 or QLIN_FMT_FP8
+ *   x          bf16 [rows, ld_x] (device); only the first `cols` of each row are read
+ *   rows, cols rows >= 0 (0 is a no-op), cols >= 1, cols % 8 == 0
+ *   ld_x       row stride of x in elements, >= cols, ld_x % 8 == 0
+ *   q_out      int8 / e4m3 [rows, cols] dense (device)
+ *   scale_out  fp32 [rows] (device)
+ * Alignment: x, q_out 16-byte aligned; scale_out 4-byte aligned.
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA (launch failure).
+ */
+QLIN_API qlin_status qlin_quantize_per_token(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                                    void* q_out, float* scale_out, qlin_stream_t stream);
+
+/*
+ * qlin_quantize_block -- Block-FP8 quantisation ("Block-FP8", page "Helion in
+ * vLLM: A Unified Route to Tunable Linear Kernels", section "What the
+ * integration changes"): one scale per block of block_rows x block_cols
+ * elements, scale = block amax / 448, codes as in qlin_quantize_per_token's
+ * FP8 path.  block_rows = 1 gives the 1x128 activation groups (the dynamic,
+ * per-call path); block_rows = 128 gives the 128x128 weight blocks (done once
+ * per weight, offline).  A block on the bottom edge covers the rows that exist.
+ *
+ *   x           bf16 [rows, ld_x] (device)
+ *   block_rows  1 or 128;  block_cols  128;  cols % 128 == 0
+ *   q_out       e4m3 [rows, cols] dense (device)
+ *   scale_out   fp32 [ceil(rows/block_rows), cols/128] row-major (device)
+ * Alignment as qlin_quantize_per_token.
+ * Errors: INVALID_ARG, UNSUPPORTED (other block shapes), ALIGNMENT, CUDA.
+ */
+QLIN_API qlin_status qlin_quantize_block(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int block_rows,
+                                int block_cols, void* q_out, float* scale_out, qlin_stream_t stream);
+
+/*
+ * qlin_scaled_mm -- the scaled GEMM with a fused scale / bias / bf16 epilogue,
+ * strategies "ordinary GEMM", "Split-K" and "Swap-AB" (page "Helion in vLLM: A
+ * Unified Route to Tunable Linear Kernels", section "What the integration
+ * changes").  Runs as one persistent tcgen05 kernel (TMA-fed shared-memory
+ * stages, accumulators in tensor memory).
+ *
+ *   INT8, FP8:  C[m,n] = bf16( ((float)acc[m,n] * s_a[m]) * s_w[n] + bias[n] )
+ *               s_a fp32 [M], s_w fp32 [N]; acc exact int32 (INT8) or fp32 (FP8)
+ *   FP8_BLOCK:  C[m,n] = bf16( sum_kb P_kb[m,n] * (s_a[m,kb] * s_w[n/128,kb]) )
+ *               s_a fp32 [M, K/128], s_w fp32 [ceil(N/128), K/128]; bias must be NULL
+ *
+ * Determinism and batch invariance: K is cut into k_segments equal segments,
+ * a fixed number per (format, N, K) in the dispatch table; every variant sums
+ * the per-segment results in the same fixed order s = 0..S-1, so a row of C
+ * depends only on that row of A and never on M, on the variant or on the
+ * order in which CTAs finish.
+ *
+ *   fmt, variant        qlin_format, qlin_variant (AUTO = table / built-in rule)
+ *   tile_n, k_segments  0 = take from the table / rule; otherwise forced
+ *                       (a forced k_segments gives up invariance with calls that
+ *                       use another value)
+ *   M, N, K             M >= 0 (0 is a no-op), N >= 16, N % 16 == 0
+ *                       (FP8_BLOCK: N % 128 == 0), K % 128 == 0, k_segments | K/128
+ *   a_q, w_q            int8 / e4m3 [M,K] and [N,K] (device)
+ *   bias                bf16 [N] (device) or NULL
+ *   c_out               bf16 [M,N] (device); int32 [M,N] with QLIN_OUT_I32ACC
+ *   flags               0 or QLIN_OUT_I32ACC (INT8 only)
+ *   workspace           device buffer of at least qlin_scaled_mm_workspace_size()
+ *                       bytes (may be NULL when that size is 0).  It must be
+ *                       zero-filled once when first allocated; every call leaves
+ *                       its ticket words at zero again.  Calls that overlap in time
+ *                       must not share a workspace.
+ * Alignment: a_q, w_q, c_out, workspace 16-byte aligned; scales and bias 4 / 2.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
+                           const void* a_q, const float* s_a, const void* w_q, const float* s_w,
+                           const void* bias, void* c_out, uint32_t flags, void* workspace,
+                           size_t workspace_bytes, qlin_stream_t stream);
+
+/*
+ * qlin_scaled_mm_workspace_size -- bytes of workspace qlin_scaled_mm needs for
+ * the same (fmt, variant, tile_n, k_segments, M, N, K): the Split-K partial
+ * tiles plus one ticket word per output tile (0 for the other variants).
+ * Host-only; resolves AUTO through the table exactly as qlin_scaled_mm does.
+ * Errors: INVALID_ARG, UNSUPPORTED.
+ */
+QLIN_API qlin_status qlin_scaled_mm_workspace_size(int fmt, int variant, int tile_n, int k_segments, int64_t M,
+                                          int64_t N, int64_t K, size_t* bytes_out);
+
+/*
+ * qlin_dispatch_table_load -- load a per-shape dispatch table written by the
+ * offline sweep (format: see the sweep's source).  Per-shape configurations
+ * are looked up at launch, as the page "[Kernel][Perf] Add Hopper (SM90) tuned
+ * config for batch-invariant persistent matmul" describes (section "Summary":
+ * the config lookup runs at kernel launch and at initialisation).  The table
+ * header names the device it was measured on; a table from another device
+ * (name, compute capability or SM count) is refused, the lesson of that page's
+ * review thread about a table applied to the wrong Hopper parts.  Entries
+ * whose shared-memory need exceeds the device's opt-in limit, or whose
+ * k_segments differ between M buckets of one (format, N, K), are refused.
+ * Replaces any previously loaded table; a failed load leaves the previous
+ * table in place.  Blocking, host-only; call it before any graph capture.
+ * Errors: INVALID_ARG, TABLE_IO, TABLE_FORMAT, TABLE_DEVICE, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_dispatch_table_load(const char* path);
+
+/* Drop the loaded table (AUTO then uses the built-in rule).  Host-only. */
+QLIN_API qlin_status qlin_dispatch_table_clear(void);
+
+/*
+ * qlin_dispatch_query -- the configuration AUTO resolves to for a shape: the
+ * table entry for (fmt, N, K) with the smallest m_max >= M (the largest if M
+ * exceeds them all), else the built-in rule (Swap-AB for M <= 64, Split-K when
+ * the output tiles cannot fill the SMs, plain otherwise).  Host-only, no
+ * allocation.
+ * Errors: INVALID_ARG, UNSUPPORTED.
+ */
+QLIN_API qlin_status qlin_dispatch_query(int fmt, int64_t M, int64_t N, int64_t K, qlin_config* out);
+
+/* Human-readable text for a status code (static storage; never NULL). */
+QLIN_API const char* qlin_status_string(qlin_status status);
+
+/*
+ * qlin_sync_status -- synchronise `stream`, then report and clear the device
+ * status word that kernels set when a bounded wait gives up.  Returns QLIN_OK,
+ * QLIN_ERR_DEVICE_TIMEOUT or QLIN_ERR_CUDA.  Blocking.
+ */
+QLIN_API qlin_status qlin_sync_status(qlin_stream_t stream);
+
+/* ABI version of the loaded library (QLIN_ABI_VERSION at build time). */
+QLIN_API int qlin_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLIN_H */

@@ -1,0 +1,452 @@
+// api.cu -- the extern "C" entry points of include/qlin.h: host-side argument
+// validation, GEMM planning, the per-shape dispatch table and status codes.
+//
+// Dispatch follows the page "[Kernel][Perf] Add Hopper (SM90) tuned config for
+// batch-invariant persistent matmul" (section "Summary": a per-shape config is
+// looked up at kernel launch; the table is keyed by architecture family and
+// split into M buckets) and "Helion in vLLM: A Unified Route to Tunable Linear
+// Kernels" ("Algorithm choice becomes part of tuning": the variant is part of
+// each per-shape entry).  The table is plain text written by the offline
+// sweep:
+//
+//   qlin-dispatch 1
+//   device <sm_count> <cc_major> <cc_minor> <device name ...>
+//   # fmt N K m_max variant tile_n k_segments
+//   entry fp8 4096 2048 16 swapab_splitk 16 4
+//   ...
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <fstream>
+#include <mutex>
+#include <sstream>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+
+namespace qlin {
+
+namespace {
+
+struct TableEntry {
+    int fmt;
+    int64_t N, K, m_max;
+    int variant, tile_n, k_segments;
+};
+
+std::mutex g_table_mu;
+std::vector<TableEntry> g_table;  // sorted by (fmt, N, K, m_max)
+
+bool g_log = [] {
+    const char* e = std::getenv("QLIN_LOG");
+    return e && e[0] == '1';
+}();
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+const char* fmt_name(int f) {
+    switch (f) {
+        case QLIN_FMT_INT8: return "int8";
+        case QLIN_FMT_FP8: return "fp8";
+        case QLIN_FMT_FP8_BLOCK: return "fp8_block";
+    }
+    return "?";
+}
+
+int parse_fmt(const std::string& s) {
+    if (s == "int8") return QLIN_FMT_INT8;
+    if (s == "fp8") return QLIN_FMT_FP8;
+    if (s == "fp8_block") return QLIN_FMT_FP8_BLOCK;
+    return -1;
+}
+
+const char* variant_name(int v) {
+    switch (v) {
+        case QLIN_VAR_PLAIN: return "plain";
+        case QLIN_VAR_SPLITK: return "splitk";
+        case QLIN_VAR_SWAPAB: return "swapab";
+        case QLIN_VAR_SWAPAB_SPLITK: return "swapab_splitk";
+    }
+    return "auto";
+}
+
+int parse_variant(const std::string& s) {
+    if (s == "plain") return QLIN_VAR_PLAIN;
+    if (s == "splitk") return QLIN_VAR_SPLITK;
+    if (s == "swapab") return QLIN_VAR_SWAPAB;
+    if (s == "swapab_splitk") return QLIN_VAR_SWAPAB_SPLITK;
+    return -1;
+}
+
+bool is_swap(int v) { return v == QLIN_VAR_SWAPAB || v == QLIN_VAR_SWAPAB_SPLITK; }
+bool is_spread(int v) { return v == QLIN_VAR_SPLITK || v == QLIN_VAR_SWAPAB_SPLITK; }
+
+bool tile_supported(int fmt, bool swap, int tile_n) {
+    if (swap) return tile_n == 16 || tile_n == 32 || tile_n == 64;
+    if (fmt == QLIN_FMT_FP8_BLOCK) return tile_n == 128;
+    return tile_n == 128 || tile_n == 256;
+}
+
+// K segmentation of the built-in rule: the largest S <= 8 dividing K/128 such
+// that the Swap-AB tiles of the shape (ceil(N/128)) times S still fit in one
+// wave of CTAs.  Fixed per (format, N, K), independent of M.
+int default_segments(int fmt, int64_t N, int64_t K, int num_sms) {
+    (void)fmt;
+    const int64_t kblocks = K / 128;
+    const int64_t tiles = (N + 127) / 128;
+    int best = 1;
+    for (int s = 2; s <= 8; ++s)
+        if (kblocks % s == 0 && tiles * s <= num_sms) best = s;
+    return best;
+}
+
+qlin_config default_config(int fmt, int64_t M, int64_t N, int64_t K, int num_sms) {
+    qlin_config c{};
+    c.k_segments = default_segments(fmt, N, K, num_sms);
+    c.from_table = 0;
+    c.m_max = 0;
+    if (M <= 64) {
+        c.tile_n = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+        c.variant = c.k_segments > 1 ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB;
+    } else {
+        const bool multi = fmt == QLIN_FMT_FP8_BLOCK || (fmt == QLIN_FMT_FP8 && c.k_segments > 1);
+        c.tile_n = multi ? 128 : 256;
+        const int64_t tiles = ((M + 127) / 128) * ((N + c.tile_n - 1) / c.tile_n);
+        c.variant = (c.k_segments > 1 && tiles * 2 <= num_sms) ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN;
+    }
+    c.stages = gemm_stages_for(c.tile_n);
+    return c;
+}
+
+bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, qlin_config* out) {
+    std::lock_guard<std::mutex> lk(g_table_mu);
+    const TableEntry* best = nullptr;
+    const TableEntry* largest = nullptr;
+    for (const auto& e : g_table) {
+        if (e.fmt != fmt || e.N != N || e.K != K) continue;
+        if (!largest || e.m_max > largest->m_max) largest = &e;
+        if (e.m_max >= M && (!best || e.m_max < best->m_max)) best = &e;
+    }
+    if (!best) best = largest;
+    if (!best) return false;
+    out->variant = best->variant;
+    out->tile_n = best->tile_n;
+    out->k_segments = best->k_segments;
+    out->stages = gemm_stages_for(best->tile_n);
+    out->m_max = best->m_max;
+    out->from_table = 1;
+    return true;
+}
+
+qlin_status check_fmt_shape(int fmt, int64_t M, int64_t N, int64_t K) {
+    if (fmt < QLIN_FMT_INT8 || fmt > QLIN_FMT_FP8_BLOCK) return QLIN_ERR_INVALID_ARG;
+    if (M < 0 || N < 16 || K < 128) return QLIN_ERR_INVALID_ARG;
+    if (N % 16 != 0 || K % 128 != 0) return QLIN_ERR_UNSUPPORTED;
+    if (fmt == QLIN_FMT_FP8_BLOCK && N % 128 != 0) return QLIN_ERR_UNSUPPORTED;
+    if (M > (int64_t)1 << 30 || N > (int64_t)1 << 30 || K > (int64_t)1 << 24) return QLIN_ERR_UNSUPPORTED;
+    return QLIN_OK;
+}
+
+qlin_status resolve_config(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
+                           int num_sms, qlin_config* cfg) {
+    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_SWAPAB_SPLITK) return QLIN_ERR_INVALID_ARG;
+    if (tile_n < 0 || k_segments < 0) return QLIN_ERR_INVALID_ARG;
+    qlin_config base{};
+    if (!lookup_table(fmt, M, N, K, &base)) base = default_config(fmt, M, N, K, num_sms);
+    if (variant != QLIN_VAR_AUTO) {
+        // a forced variant keeps the shape's segmentation; its tile defaults
+        // to the rule's choice for that orientation
+        const qlin_config d = default_config(fmt, is_swap(variant) ? 1 : 65, N, K, num_sms);
+        const bool same_orientation = is_swap(variant) == is_swap(base.variant);
+        base.tile_n = same_orientation ? base.tile_n : d.tile_n;
+        if (is_swap(variant) && !same_orientation)
+            base.tile_n = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+        base.variant = variant;
+    }
+    if (tile_n) base.tile_n = tile_n;
+    if (k_segments) base.k_segments = k_segments;
+    base.stages = gemm_stages_for(base.tile_n);
+    *cfg = base;
+    return QLIN_OK;
+}
+
+}  // namespace
+
+int current_device_sms() {
+    static int cached_dev = -1, cached_sms = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (dev != cached_dev) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cached_sms = sms;
+        cached_dev = dev;
+    }
+    return cached_sms;
+}
+
+qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
+                           int num_sms, GemmPlan* plan) {
+    qlin_status st = check_fmt_shape(fmt, M, N, K);
+    if (st != QLIN_OK) return st;
+    if (num_sms <= 0) num_sms = kNumSMsB200;
+    qlin_config cfg{};
+    st = resolve_config(fmt, variant, tile_n, k_segments, M, N, K, num_sms, &cfg);
+    if (st != QLIN_OK) return st;
+    GemmPlan p;
+    p.fmt = fmt;
+    p.swap = is_swap(cfg.variant);
+    p.spread = is_spread(cfg.variant);
+    p.tile_n = cfg.tile_n;
+    p.k_segments = cfg.k_segments;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.kblocks = (int)(K / 128);
+    if (!tile_supported(fmt, p.swap, p.tile_n)) return QLIN_ERR_UNSUPPORTED;
+    if (p.k_segments < 1 || p.kblocks % p.k_segments != 0) return QLIN_ERR_UNSUPPORTED;
+    if (p.k_segments == 1) p.spread = false;
+    p.kb_per_seg = p.kblocks / p.k_segments;
+    // units with more than one accumulator chunk keep tile_n fp32 values per
+    // thread and a TMEM running total: only tiles up to 128 columns do that
+    const bool multi_chunk = (fmt == QLIN_FMT_FP8_BLOCK && (p.spread ? p.kb_per_seg : p.kblocks) > 1) ||
+                             (fmt == QLIN_FMT_FP8 && !p.spread && p.k_segments > 1);
+    if (multi_chunk && p.tile_n > 128) return QLIN_ERR_UNSUPPORTED;
+    p.stages = gemm_stages_for(p.tile_n);
+    p.smem_bytes = gemm_smem_bytes_for(p.tile_n);
+    p.p_rows = p.swap ? N : M;
+    p.q_rows = p.swap ? M : N;
+    p.p_tiles = (p.p_rows + 127) / 128;
+    p.q_tiles = (p.q_rows + p.tile_n - 1) / p.tile_n;
+    p.num_tiles = p.p_tiles * p.q_tiles;
+    p.units = p.num_tiles * (p.spread ? p.k_segments : 1);
+    if (p.units > (int64_t)INT32_MAX / 2) return QLIN_ERR_UNSUPPORTED;
+    p.grid = (int)std::min<int64_t>(p.units, num_sms);
+    if (p.grid < 1) p.grid = 1;
+    if (p.spread) {
+        p.ticket_bytes = ((size_t)p.num_tiles * 4 + 255) & ~size_t(255);
+        p.workspace_bytes = p.ticket_bytes + (size_t)p.k_segments * p.num_tiles * 128 * p.tile_n * 4;
+    } else {
+        p.ticket_bytes = 0;
+        p.workspace_bytes = 0;
+    }
+    *plan = p;
+    return QLIN_OK;
+}
+
+}  // namespace qlin
+
+using namespace qlin;
+
+extern "C" {
+
+int qlin_abi_version(void) { return QLIN_ABI_VERSION; }
+
+const char* qlin_status_string(qlin_status s) {
+    switch (s) {
+        case QLIN_OK: return "ok";
+        case QLIN_ERR_INVALID_ARG: return "invalid argument";
+        case QLIN_ERR_UNSUPPORTED: return "unsupported shape, format or variant";
+        case QLIN_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+        case QLIN_ERR_WORKSPACE: return "workspace missing or too small";
+        case QLIN_ERR_TABLE_IO: return "dispatch table file unreadable";
+        case QLIN_ERR_TABLE_FORMAT: return "dispatch table malformed";
+        case QLIN_ERR_TABLE_DEVICE: return "dispatch table made for another device";
+        case QLIN_ERR_CUDA: return "CUDA call failed";
+        case QLIN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case QLIN_ERR_NO_DEVICE: return "no sm_100 device";
+    }
+    return "unknown status";
+}
+
+qlin_status qlin_quantize_per_token(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld_x, void* q_out,
+                                    float* scale_out, qlin_stream_t stream) {
+    if (fmt != QLIN_FMT_INT8 && fmt != QLIN_FMT_FP8) return QLIN_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 1 || ld_x < cols) return QLIN_ERR_INVALID_ARG;
+    if (rows == 0) return QLIN_OK;
+    if (!x || !q_out || !scale_out) return QLIN_ERR_INVALID_ARG;
+    if (cols % 8 != 0 || ld_x % 8 != 0) return QLIN_ERR_ALIGNMENT;
+    if (!aligned16(x) || !aligned16(q_out) || (reinterpret_cast<uintptr_t>(scale_out) & 3u))
+        return QLIN_ERR_ALIGNMENT;
+    if (rows > (int64_t)1 << 34) return QLIN_ERR_UNSUPPORTED;
+    cudaError_t e = launch_quantize_per_token(fmt, x, rows, cols, ld_x, q_out, scale_out,
+                                              static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
+}
+
+qlin_status qlin_quantize_block(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int block_rows,
+                                int block_cols, void* q_out, float* scale_out, qlin_stream_t stream) {
+    if (rows < 0 || cols < 1 || ld_x < cols) return QLIN_ERR_INVALID_ARG;
+    if (block_cols != 128 || (block_rows != 1 && block_rows != 128)) return QLIN_ERR_UNSUPPORTED;
+    if (cols % 128 != 0) return QLIN_ERR_UNSUPPORTED;
+    if (rows == 0) return QLIN_OK;
+    if (!x || !q_out || !scale_out) return QLIN_ERR_INVALID_ARG;
+    if (ld_x % 8 != 0) return QLIN_ERR_ALIGNMENT;
+    if (!aligned16(x) || !aligned16(q_out) || (reinterpret_cast<uintptr_t>(scale_out) & 3u))
+        return QLIN_ERR_ALIGNMENT;
+    if (block_rows == 128 && (rows + 127) / 128 > 65535) return QLIN_ERR_UNSUPPORTED;
+    cudaError_t e =
+        launch_quantize_block(x, rows, cols, ld_x, block_rows, q_out, scale_out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
+}
+
+qlin_status qlin_scaled_mm_workspace_size(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N,
+                                          int64_t K, size_t* bytes_out) {
+    if (!bytes_out) return QLIN_ERR_INVALID_ARG;
+    *bytes_out = 0;
+    if (M == 0) {
+        qlin_status s = check_fmt_shape(fmt, 1, N, K);
+        return s;
+    }
+    GemmPlan p;
+    qlin_status st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, current_device_sms(), &p);
+    if (st != QLIN_OK) return st;
+    *bytes_out = p.workspace_bytes;
+    return QLIN_OK;
+}
+
+qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
+                           const void* a_q, const float* s_a, const void* w_q, const float* s_w, const void* bias,
+                           void* c_out, uint32_t flags, void* workspace, size_t workspace_bytes,
+                           qlin_stream_t stream) {
+    qlin_status st = check_fmt_shape(fmt, M, N, K);
+    if (st != QLIN_OK) return st;
+    if (flags & ~QLIN_OUT_I32ACC) return QLIN_ERR_INVALID_ARG;
+    const bool out_i32 = (flags & QLIN_OUT_I32ACC) != 0;
+    if (out_i32 && fmt != QLIN_FMT_INT8) return QLIN_ERR_INVALID_ARG;
+    if (fmt == QLIN_FMT_FP8_BLOCK && bias) return QLIN_ERR_INVALID_ARG;
+    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_SWAPAB_SPLITK || tile_n < 0 || k_segments < 0)
+        return QLIN_ERR_INVALID_ARG;
+    if (M == 0) return QLIN_OK;
+    if (!a_q || !s_a || !w_q || !s_w || !c_out) return QLIN_ERR_INVALID_ARG;
+    if (!aligned16(a_q) || !aligned16(w_q) || !aligned16(c_out)) return QLIN_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(s_a) & 3u) || (reinterpret_cast<uintptr_t>(s_w) & 3u) ||
+        (reinterpret_cast<uintptr_t>(bias) & 1u))
+        return QLIN_ERR_ALIGNMENT;
+    const int sms = current_device_sms();
+    if (sms <= 0) return QLIN_ERR_NO_DEVICE;
+    GemmPlan p;
+    st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, sms, &p);
+    if (st != QLIN_OK) return st;
+    if (p.workspace_bytes) {
+        if (!workspace || workspace_bytes < p.workspace_bytes) return QLIN_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return QLIN_ERR_ALIGNMENT;
+    }
+    if (g_log)
+        std::fprintf(stderr, "[qlin] scaled_mm %s M=%lld N=%lld K=%lld -> %s tile_n=%d S=%d grid=%d\n",
+                     fmt_name(fmt), (long long)M, (long long)N, (long long)K,
+                     variant_name(p.swap ? (p.spread ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB)
+                                         : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
+                     p.tile_n, p.k_segments, p.grid);
+    GemmOperands ops{a_q, s_a, w_q, s_w, bias, c_out, out_i32, workspace};
+    return launch_gemm(p, ops, static_cast<cudaStream_t>(stream));
+}
+
+qlin_status qlin_dispatch_query(int fmt, int64_t M, int64_t N, int64_t K, qlin_config* out) {
+    if (!out) return QLIN_ERR_INVALID_ARG;
+    qlin_status st = check_fmt_shape(fmt, M < 1 ? 1 : M, N, K);
+    if (st != QLIN_OK) return st;
+    int sms = current_device_sms();
+    if (sms <= 0) sms = kNumSMsB200;
+    return resolve_config(fmt, QLIN_VAR_AUTO, 0, 0, M < 1 ? 1 : M, N, K, sms, out);
+}
+
+qlin_status qlin_dispatch_table_clear(void) {
+    std::lock_guard<std::mutex> lk(g_table_mu);
+    g_table.clear();
+    return QLIN_OK;
+}
+
+qlin_status qlin_dispatch_table_load(const char* path) {
+    if (!path) return QLIN_ERR_INVALID_ARG;
+    std::ifstream f(path);
+    if (!f) return QLIN_ERR_TABLE_IO;
+    std::string line;
+    bool have_magic = false, have_device = false;
+    int t_sms = 0, t_major = 0, t_minor = 0;
+    std::string t_name;
+    std::vector<TableEntry> entries;
+    while (std::getline(f, line)) {
+        if (line.empty() || line[0] == '#') continue;
+        std::istringstream ss(line);
+        std::string key;
+        ss >> key;
+        if (key == "qlin-dispatch") {
+            int ver = 0;
+            if (!(ss >> ver) || ver != 1) return QLIN_ERR_TABLE_FORMAT;
+            have_magic = true;
+        } else if (key == "device") {
+            if (!(ss >> t_sms >> t_major >> t_minor)) return QLIN_ERR_TABLE_FORMAT;
+            std::getline(ss, t_name);
+            const size_t b = t_name.find_first_not_of(" \t");
+            t_name = b == std::string::npos ? "" : t_name.substr(b);
+            have_device = true;
+        } else if (key == "entry") {
+            std::string fs, vs;
+            TableEntry e{};
+            if (!(ss >> fs >> e.N >> e.K >> e.m_max >> vs >> e.tile_n >> e.k_segments)) return QLIN_ERR_TABLE_FORMAT;
+            e.fmt = parse_fmt(fs);
+            e.variant = parse_variant(vs);
+            if (e.fmt < 0 || e.variant < 0 || e.m_max < 1) return QLIN_ERR_TABLE_FORMAT;
+            if (check_fmt_shape(e.fmt, 1, e.N, e.K) != QLIN_OK) return QLIN_ERR_TABLE_FORMAT;
+            if (!tile_supported(e.fmt, is_swap(e.variant), e.tile_n)) return QLIN_ERR_TABLE_FORMAT;
+            if (e.k_segments < 1 || (e.K / 128) % e.k_segments != 0) return QLIN_ERR_TABLE_FORMAT;
+            entries.push_back(e);
+        } else {
+            return QLIN_ERR_TABLE_FORMAT;
+        }
+    }
+    if (!have_magic || !have_device) return QLIN_ERR_TABLE_FORMAT;
+    // every M bucket of one (format, N, K) must share the segmentation, or
+    // results would change with the batch size
+    for (size_t i = 0; i < entries.size(); ++i)
+        for (size_t j = i + 1; j < entries.size(); ++j) {
+            const auto &a = entries[i], &b = entries[j];
+            if (a.fmt == b.fmt && a.N == b.N && a.K == b.K) {
+                if (a.m_max == b.m_max) return QLIN_ERR_TABLE_FORMAT;
+                if (a.fmt != QLIN_FMT_INT8 && a.k_segments != b.k_segments) return QLIN_ERR_TABLE_FORMAT;
+            }
+        }
+    // every entry must be launchable (validates tile / segmentation / chunking)
+    for (const auto& e : entries) {
+        GemmPlan p;
+        if (make_gemm_plan(e.fmt, e.variant, e.tile_n, e.k_segments, e.m_max, e.N, e.K, t_sms > 0 ? t_sms : 148, &p) !=
+            QLIN_OK)
+            return QLIN_ERR_TABLE_FORMAT;
+    }
+    // device guard: the table must have been measured on this kind of device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return QLIN_ERR_NO_DEVICE;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return QLIN_ERR_CUDA;
+    if (prop.multiProcessorCount != t_sms || prop.major != t_major || prop.minor != t_minor ||
+        t_name != std::string(prop.name))
+        return QLIN_ERR_TABLE_DEVICE;
+    for (const auto& e : entries)
+        if (gemm_smem_bytes_for(e.tile_n) > prop.sharedMemPerBlockOptin) return QLIN_ERR_TABLE_FORMAT;
+    std::sort(entries.begin(), entries.end(), [](const TableEntry& a, const TableEntry& b) {
+        if (a.fmt != b.fmt) return a.fmt < b.fmt;
+        if (a.N != b.N) return a.N < b.N;
+        if (a.K != b.K) return a.K < b.K;
+        return a.m_max < b.m_max;
+    });
+    {
+        std::lock_guard<std::mutex> lk(g_table_mu);
+        g_table.swap(entries);
+    }
+    if (g_log) std::fprintf(stderr, "[qlin] loaded %zu dispatch entries from %s\n", g_table.size(), path);
+    return QLIN_OK;
+}
+
+qlin_status qlin_sync_status(qlin_stream_t stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QLIN_ERR_CUDA;
+    int v = 0;
+    if (device_status_read_clear(&v) != cudaSuccess) return QLIN_ERR_CUDA;
+    return v != 0 ? (qlin_status)v : QLIN_OK;
+}
+
+}  // extern "C"

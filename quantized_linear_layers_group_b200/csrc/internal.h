@@ -1,0 +1,71 @@
+// internal.h -- declarations shared by the library's translation units (not
+// part of the public ABI; see include/qlin.h for that).
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "qlin.h"
+
+namespace qlin {
+
+constexpr int kNumSMsB200 = 148;
+
+// ---------------------------------------------------------------- quantise
+cudaError_t launch_quantize_per_token(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld, void* q,
+                                      float* s, cudaStream_t st);
+cudaError_t launch_quantize_block(const void* x, int64_t rows, int64_t cols, int64_t ld, int block_rows, void* q,
+                                  float* s, cudaStream_t st);
+
+// ------------------------------------------------------------------- GEMM
+// A fully resolved GEMM launch: which operand feeds the 128-row MMA side
+// ("P") and which the narrow side ("Q", tile_n rows), how K is segmented and
+// whether the segments of one tile run in separate CTAs.
+struct GemmPlan {
+    int fmt = 0;
+    bool swap = false;    // P = W (rows of N), Q = A (rows of M)
+    bool spread = false;  // Split-K: one work unit per (tile, segment)
+    int tile_n = 0;       // Q rows per tile (MMA N)
+    int k_segments = 1;   // S
+    int stages = 0;
+    int64_t M = 0, N = 0, K = 0;
+    int64_t p_rows = 0, q_rows = 0;
+    int64_t p_tiles = 0, q_tiles = 0, num_tiles = 0, units = 0;
+    int kblocks = 0;       // K / 128
+    int kb_per_seg = 0;    // kblocks / S
+    int grid = 0;          // persistent CTAs
+    size_t smem_bytes = 0;
+    size_t ticket_bytes = 0;   // workspace prefix holding the per-tile tickets
+    size_t workspace_bytes = 0;
+};
+
+// Validates the (fmt, tile_n, S, variant) combination and fills the plan.
+// Returns QLIN_OK or an error status; touches no device state.
+qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
+                           int num_sms, GemmPlan* plan);
+
+// Shared-memory pipeline depth and dynamic smem size for a tile_n.
+int gemm_stages_for(int tile_n);
+size_t gemm_smem_bytes_for(int tile_n);
+
+struct GemmOperands {
+    const void* a_q;
+    const float* s_a;
+    const void* w_q;
+    const float* s_w;
+    const void* bias;
+    void* c;
+    bool out_i32;
+    void* workspace;
+};
+
+qlin_status launch_gemm(const GemmPlan& plan, const GemmOperands& ops, cudaStream_t st);
+
+// Reads and clears the device status word that bounded waits set on timeout.
+cudaError_t device_status_read_clear(int* value);
+
+// Number of SMs of the current device (cached per device); 0 if none.
+int current_device_sms();
+
+}  // namespace qlin

@@ -1,0 +1,292 @@
+// quantize.cu -- dynamic activation (and offline weight) quantisation kernels.
+//
+// Per-token INT8 / FP8 and Block-FP8 (1x128 groups, 128x128 blocks), the
+// formats named on the page "Helion in vLLM: A Unified Route to Tunable Linear
+// Kernels", section "What the integration changes".  Each kernel makes ONE
+// pass over HBM: a row (or block) is loaded with 16-byte vector loads into
+// registers, its absolute maximum is reduced with warp shuffles, and the codes
+// are produced from the registers.
+//
+// Arithmetic (bit-exact by construction, no fast-math anywhere):
+//   scale = amax / Qmax          IEEE binary32 division (__fdiv_rn)
+//   v     = x / scale            IEEE binary32 division (__fdiv_rn)
+//   INT8: q = clamp(rint_half_even(v), -127, 127)
+//   FP8 : q = e4m3_rn_satfinite(clamp(v, -448, 448))
+//   amax == 0 -> scale = 0, q = 0.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+
+namespace qlin {
+
+namespace {
+
+constexpr int kQuantWarps = 8;  // rows per CTA for the warp-per-row kernels
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+
+// 8 bf16 in a uint4 -> 8 floats (exact widening)
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
+        f[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+    }
+}
+
+__device__ __forceinline__ float absmax8(const uint4& v) {
+    float f[8];
+    unpack8(v, f);
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+    return m;
+}
+
+__device__ __forceinline__ uint32_t quant_int8_x4(const float* f, float s) {
+    uint32_t out = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int r = 0;
+        if (s != 0.f) {
+            r = __float2int_rn(__fdiv_rn(f[i], s));
+            r = max(-127, min(127, r));
+        }
+        out |= (uint32_t)(r & 0xFF) << (8 * i);
+    }
+    return out;
+}
+
+__device__ __forceinline__ uint32_t quant_e4m3_x4(const float* f, float s) {
+    if (s == 0.f) return 0u;
+    float v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = fminf(fmaxf(__fdiv_rn(f[i], s), -448.f), 448.f);
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v[0], v[1]), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(v[2], v[3]), __NV_SATFINITE, __NV_E4M3);
+    return (uint32_t)lo | ((uint32_t)hi << 16);
+}
+
+template <int FMT>
+__device__ __forceinline__ uint2 quant8(const uint4& v, float s) {
+    float f[8];
+    unpack8(v, f);
+    uint2 r;
+    if constexpr (FMT == QLIN_FMT_INT8) {
+        r.x = quant_int8_x4(f, s);
+        r.y = quant_int8_x4(f + 4, s);
+    } else {
+        r.x = quant_e4m3_x4(f, s);
+        r.y = quant_e4m3_x4(f + 4, s);
+    }
+    return r;
+}
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// ----------------------------------------------------------------------------
+// Per-token: one warp per row; lane l owns vectors l, l+32, l+64, ... of the
+// row (16 bytes = 8 bf16 each), all held in registers (VPL vectors per lane).
+template <int FMT, int VPL>
+__global__ void __launch_bounds__(kQuantWarps * 32)
+    quantize_per_token_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                              uint8_t* __restrict__ q, float* __restrict__ s) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
+    const int nvec = (int)(cols >> 3);
+    constexpr float QMAX = (FMT == QLIN_FMT_INT8) ? 127.f : 448.f;
+
+    uint4 v[VPL];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int idx = i * 32 + lane;
+        if (idx < nvec) {
+            v[i] = ld_stream(xr + idx);
+            amax = fmaxf(amax, absmax8(v[i]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sc = __fdiv_rn(amax, QMAX);
+    if (lane == 0) s[row] = sc;
+    uint2* qr = reinterpret_cast<uint2*>(q + row * cols);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+        const int idx = i * 32 + lane;
+        if (idx < nvec) qr[idx] = quant8<FMT>(v[i], sc);
+    }
+}
+
+// Per-token, rows too long to hold in registers: two passes over the row
+// (the second one hits L2).
+template <int FMT>
+__global__ void __launch_bounds__(kQuantWarps * 32)
+    quantize_per_token_long_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                                   uint8_t* __restrict__ q, float* __restrict__ s) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
+    const int64_t nvec = cols >> 3;
+    constexpr float QMAX = (FMT == QLIN_FMT_INT8) ? 127.f : 448.f;
+    float amax = 0.f;
+    for (int64_t idx = lane; idx < nvec; idx += 32) amax = fmaxf(amax, absmax8(xr[idx]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float sc = __fdiv_rn(amax, QMAX);
+    if (lane == 0) s[row] = sc;
+    uint2* qr = reinterpret_cast<uint2*>(q + row * cols);
+    for (int64_t idx = lane; idx < nvec; idx += 32) qr[idx] = quant8<FMT>(xr[idx], sc);
+}
+
+// ----------------------------------------------------------------------------
+// Block-FP8 activations, 1x128 groups: one warp per row.  In step i, lanes
+// 0-15 hold group 2i and lanes 16-31 group 2i+1 (16 vectors x 8 = 128), so the
+// group maximum is a 16-lane shuffle reduction.
+template <int VPL>
+__global__ void __launch_bounds__(kQuantWarps * 32)
+    quantize_group128_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                             uint8_t* __restrict__ q, float* __restrict__ s) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
+    const int nvec = (int)(cols >> 3);  // multiple of 16
+    const int ngroups = (int)(cols >> 7);
+    uint2* qr = reinterpret_cast<uint2*>(q + row * cols);
+    float* sr = s + row * ngroups;
+    for (int base = 0; base < nvec; base += VPL * 32) {
+        uint4 v[VPL];
+        float gmax[VPL];
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int idx = base + i * 32 + lane;
+            gmax[i] = 0.f;
+            if (idx < nvec) {
+                v[i] = ld_stream(xr + idx);
+                gmax[i] = absmax8(v[i]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) gmax[i] = fmaxf(gmax[i], __shfl_xor_sync(0xffffffffu, gmax[i], o));
+        }
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) {
+            const int idx = base + i * 32 + lane;
+            if (idx < nvec) {
+                const float sc = __fdiv_rn(gmax[i], 448.f);
+                if ((lane & 15) == 0) sr[idx >> 4] = sc;
+                qr[idx] = quant8<QLIN_FMT_FP8>(v[i], sc);
+            }
+        }
+    }
+    (void)ngroups;
+}
+
+// Block-FP8 weights, 128x128 blocks: one CTA (256 threads) per block.  Thread
+// t owns column vector t%16 of rows t/16 + 16*i, i = 0..7.
+__global__ void __launch_bounds__(256)
+    quantize_block128_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                             uint8_t* __restrict__ q, float* __restrict__ s) {
+    __shared__ float warp_max[8];
+    const int t = threadIdx.x;
+    const int64_t br = blockIdx.y, bc = blockIdx.x;
+    const int64_t nbc = cols >> 7;
+    const int cv = t & 15;
+    uint4 v[8];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t r = br * 128 + (t >> 4) + 16 * i;
+        if (r < rows) {
+            v[i] = ld_stream(reinterpret_cast<const uint4*>(x + r * ld + bc * 128) + cv);
+            amax = fmaxf(amax, absmax8(v[i]));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if ((t & 31) == 0) warp_max[t >> 5] = amax;
+    __syncthreads();
+    amax = warp_max[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
+    const float sc = __fdiv_rn(amax, 448.f);
+    if (t == 0) s[br * nbc + bc] = sc;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t r = br * 128 + (t >> 4) + 16 * i;
+        if (r < rows) reinterpret_cast<uint2*>(q + r * cols + bc * 128)[cv] = quant8<QLIN_FMT_FP8>(v[i], sc);
+    }
+}
+
+template <int FMT>
+cudaError_t launch_per_token_fmt(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* q, float* s,
+                                 cudaStream_t st) {
+    const int64_t nvec = cols >> 3;
+    const dim3 grid((unsigned)((rows + kQuantWarps - 1) / kQuantWarps)), block(kQuantWarps * 32);
+    if (nvec <= 32)
+        quantize_per_token_kernel<FMT, 1><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
+    else if (nvec <= 64)
+        quantize_per_token_kernel<FMT, 2><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
+    else if (nvec <= 128)
+        quantize_per_token_kernel<FMT, 4><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
+    else if (nvec <= 256)
+        quantize_per_token_kernel<FMT, 8><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
+    else if (nvec <= 512)
+        quantize_per_token_kernel<FMT, 16><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
+    else if (nvec <= 768)
+        quantize_per_token_kernel<FMT, 24><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
+    else if (nvec <= 1024)
+        quantize_per_token_kernel<FMT, 32><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
+    else
+        quantize_per_token_long_kernel<FMT><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_per_token(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld, void* q,
+                                      float* s, cudaStream_t st) {
+    const auto* xb = static_cast<const uint16_t*>(x);
+    auto* qb = static_cast<uint8_t*>(q);
+    if (fmt == QLIN_FMT_INT8) return launch_per_token_fmt<QLIN_FMT_INT8>(xb, rows, cols, ld, qb, s, st);
+    return launch_per_token_fmt<QLIN_FMT_FP8>(xb, rows, cols, ld, qb, s, st);
+}
+
+cudaError_t launch_quantize_block(const void* x, int64_t rows, int64_t cols, int64_t ld, int block_rows, void* q,
+                                  float* s, cudaStream_t st) {
+    const auto* xb = static_cast<const uint16_t*>(x);
+    auto* qb = static_cast<uint8_t*>(q);
+    if (block_rows == 1) {
+        const dim3 grid((unsigned)((rows + kQuantWarps - 1) / kQuantWarps)), block(kQuantWarps * 32);
+        const int64_t nvec = cols >> 3;
+        if (nvec <= 64)
+            quantize_group128_kernel<2><<<grid, block, 0, st>>>(xb, rows, cols, ld, qb, s);
+        else if (nvec <= 256)
+            quantize_group128_kernel<8><<<grid, block, 0, st>>>(xb, rows, cols, ld, qb, s);
+        else
+            quantize_group128_kernel<24><<<grid, block, 0, st>>>(xb, rows, cols, ld, qb, s);
+    } else {
+        const dim3 grid((unsigned)(cols >> 7), (unsigned)((rows + 127) / 128));
+        quantize_block128_kernel<<<grid, 256, 0, st>>>(xb, rows, cols, ld, qb, s);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace qlin

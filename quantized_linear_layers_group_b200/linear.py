@@ -1,0 +1,85 @@
+"""The quantized linear layer a user calls, composed from the C ABI.
+
+``QuantizedLinear(fmt, weight, bias)`` quantises the bf16 weight once
+(per output channel for INT8 / FP8, 128x128 blocks for Block-FP8) with the
+library's own kernels, and its ``forward(x)`` runs the hot path: dynamic
+activation quantisation (per token, or per 1x128 group) followed by the
+scaled GEMM with the fused scale / bias / bf16 epilogue.  Both steps run in
+libqlin.so; this module only allocates tensors (through PyTorch's caching
+allocator) and passes pointers.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import qlin
+
+
+class Workspace:
+    """A zero-initialised device buffer for Split-K partials and tickets.
+
+    The GEMM leaves the ticket words zeroed after every call, so the buffer is
+    zero-filled only when it is (re)allocated.  Calls that may overlap in time
+    (different streams) need separate workspaces.
+    """
+
+    def __init__(self, nbytes: int = 0, device="cuda"):
+        self.device = torch.device(device)
+        self.buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=self.device)
+
+    def ensure(self, nbytes: int) -> torch.Tensor:
+        if nbytes > self.buf.numel():
+            self.buf = torch.zeros(int(nbytes), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+def quantize_weight(fmt: int, weight: torch.Tensor, stream=None):
+    """Quantise a bf16 weight [N, K] on the device; returns (w_q uint8 [N, K], s_w fp32)."""
+    assert weight.dtype == torch.bfloat16 and weight.is_cuda and weight.dim() == 2
+    N, K = weight.shape
+    w_q = torch.empty(N, K, dtype=torch.uint8, device=weight.device)
+    if fmt == qlin.QLIN_FMT_FP8_BLOCK:
+        s_w = torch.empty((N + 127) // 128, K // 128, dtype=torch.float32, device=weight.device)
+        qlin.qlin_quantize_block(weight, 128, w_q, s_w, stream)
+    else:
+        s_w = torch.empty(N, dtype=torch.float32, device=weight.device)
+        qlin.qlin_quantize_per_token(fmt, weight, w_q, s_w, stream)
+    return w_q, s_w
+
+
+def quantize_activation(fmt: int, x: torch.Tensor, stream=None):
+    """Dynamic activation quantisation; returns (a_q uint8 [M, K], s_a fp32)."""
+    M, K = x.shape
+    a_q = torch.empty(M, K, dtype=torch.uint8, device=x.device)
+    if fmt == qlin.QLIN_FMT_FP8_BLOCK:
+        s_a = torch.empty(M, K // 128, dtype=torch.float32, device=x.device)
+        qlin.qlin_quantize_block(x, 1, a_q, s_a, stream)
+    else:
+        s_a = torch.empty(M, dtype=torch.float32, device=x.device)
+        qlin.qlin_quantize_per_token(fmt, x, a_q, s_a, stream)
+    return a_q, s_a
+
+
+class QuantizedLinear:
+    """y = x W^T + b with W8A8 INT8, FP8 per-token/per-channel or Block-FP8 arithmetic."""
+
+    def __init__(self, fmt: int, weight: torch.Tensor, bias: torch.Tensor | None = None, workspace=None):
+        self.fmt = fmt
+        self.N, self.K = weight.shape
+        self.w_q, self.s_w = quantize_weight(fmt, weight)
+        self.bias = bias
+        self.workspace = workspace if workspace is not None else Workspace(device=weight.device)
+
+    def forward(self, x: torch.Tensor, stream=None, variant: int = qlin.QLIN_VAR_AUTO, tile_n: int = 0,
+                k_segments: int = 0, out: torch.Tensor | None = None) -> torch.Tensor:
+        assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.shape[1] == self.K
+        M = x.shape[0]
+        a_q, s_a = quantize_activation(self.fmt, x, stream)
+        c = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
+        nbytes = qlin.qlin_scaled_mm_workspace_size(self.fmt, M, self.N, self.K, variant, tile_n, k_segments)
+        ws = self.workspace.ensure(nbytes) if nbytes else None
+        qlin.qlin_scaled_mm(self.fmt, a_q, s_a, self.w_q, self.s_w, self.bias, c, ws, stream, variant=variant,
+                            tile_n=tile_n, k_segments=k_segments)
+        return c
+
+    __call__ = forward

@@ -1,0 +1,183 @@
+"""Thin ctypes binding of the C ABI in include/qlin.h (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: torch tensors are turned into device pointers, the
+current CUDA stream into a ``cudaStream_t`` and a non-OK status into a
+``QlinError``.  PyTorch is used for device memory and streams only.
+
+The library ``libqlin.so`` is built in-tree by ``build.py``; if it is missing
+this module raises ImportError -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.environ.get("QLIN_LIB", os.path.join(_HERE, "libqlin.so"))
+
+# ------------------------------------------------------------ enums (qlin.h)
+QLIN_OK = 0
+QLIN_ERR_INVALID_ARG = 1
+QLIN_ERR_UNSUPPORTED = 2
+QLIN_ERR_ALIGNMENT = 3
+QLIN_ERR_WORKSPACE = 4
+QLIN_ERR_TABLE_IO = 5
+QLIN_ERR_TABLE_FORMAT = 6
+QLIN_ERR_TABLE_DEVICE = 7
+QLIN_ERR_CUDA = 8
+QLIN_ERR_DEVICE_TIMEOUT = 9
+QLIN_ERR_NO_DEVICE = 10
+
+QLIN_FMT_INT8 = 0
+QLIN_FMT_FP8 = 1
+QLIN_FMT_FP8_BLOCK = 2
+
+QLIN_VAR_AUTO = 0
+QLIN_VAR_PLAIN = 1
+QLIN_VAR_SPLITK = 2
+QLIN_VAR_SWAPAB = 3
+QLIN_VAR_SWAPAB_SPLITK = 4
+
+QLIN_OUT_I32ACC = 1
+
+VARIANT_NAMES = {QLIN_VAR_AUTO: "auto", QLIN_VAR_PLAIN: "plain", QLIN_VAR_SPLITK: "splitk",
+                 QLIN_VAR_SWAPAB: "swapab", QLIN_VAR_SWAPAB_SPLITK: "swapab_splitk"}
+
+# every symbol include/qlin.h declares
+EXPORTS = ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_scaled_mm_workspace_size",
+           "qlin_dispatch_table_load", "qlin_dispatch_table_clear", "qlin_dispatch_query", "qlin_status_string",
+           "qlin_sync_status", "qlin_abi_version")
+
+
+class qlin_config(ctypes.Structure):
+    _fields_ = [("variant", ctypes.c_int32), ("tile_n", ctypes.c_int32), ("k_segments", ctypes.c_int32),
+                ("stages", ctypes.c_int32), ("m_max", ctypes.c_int64), ("from_table", ctypes.c_int32)]
+
+    def as_dict(self):
+        return {f: getattr(self, f) for f, _ in self._fields_}
+
+
+class QlinError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libqlin.so not found at {LIB_PATH}; build it with "
+                      "`python quantized_linear_layers_group_b200/build.py`")
+
+lib = ctypes.CDLL(LIB_PATH)
+_vp, _i64, _i32, _u32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint32, ctypes.c_size_t
+lib.qlin_quantize_per_token.argtypes = [_i32, _vp, _i64, _i64, _i64, _vp, _vp, _vp]
+lib.qlin_quantize_block.argtypes = [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp]
+lib.qlin_scaled_mm.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _u32, _vp,
+                               _sz, _vp]
+lib.qlin_scaled_mm_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, ctypes.POINTER(_sz)]
+lib.qlin_dispatch_table_load.argtypes = [ctypes.c_char_p]
+lib.qlin_dispatch_table_clear.argtypes = []
+lib.qlin_dispatch_query.argtypes = [_i32, _i64, _i64, _i64, ctypes.POINTER(qlin_config)]
+lib.qlin_status_string.argtypes = [_i32]
+lib.qlin_status_string.restype = ctypes.c_char_p
+lib.qlin_sync_status.argtypes = [_vp]
+lib.qlin_abi_version.argtypes = []
+for _name in EXPORTS:
+    if _name != "qlin_status_string":
+        getattr(lib, _name).restype = _i32
+
+
+def status_string(status: int) -> str:
+    return lib.qlin_status_string(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != QLIN_OK:
+        raise QlinError(status, where)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ------------------------------------------------------------- entry points
+def qlin_quantize_per_token(fmt: int, x, q_out, scale_out, stream=None, *, rows=None, cols=None, ld_x=None):
+    """Per-token INT8/FP8 quantisation of bf16 x [rows, cols] into q_out / scale_out."""
+    rows = x.shape[0] if rows is None else rows
+    cols = x.shape[1] if cols is None else cols
+    ld_x = (x.stride(0) if x.dim() == 2 else cols) if ld_x is None else ld_x
+    _check(lib.qlin_quantize_per_token(fmt, _ptr(x), rows, cols, ld_x, _ptr(q_out), _ptr(scale_out),
+                                       _stream(stream)), "qlin_quantize_per_token")
+
+
+def qlin_quantize_block(x, block_rows: int, q_out, scale_out, stream=None, *, block_cols: int = 128, rows=None,
+                        cols=None, ld_x=None):
+    """Block-FP8 quantisation (1x128 activation groups or 128x128 weight blocks)."""
+    rows = x.shape[0] if rows is None else rows
+    cols = x.shape[1] if cols is None else cols
+    ld_x = (x.stride(0) if x.dim() == 2 else cols) if ld_x is None else ld_x
+    _check(lib.qlin_quantize_block(_ptr(x), rows, cols, ld_x, block_rows, block_cols, _ptr(q_out), _ptr(scale_out),
+                                   _stream(stream)), "qlin_quantize_block")
+
+
+def qlin_scaled_mm_workspace_size(fmt: int, M: int, N: int, K: int, variant: int = QLIN_VAR_AUTO, tile_n: int = 0,
+                                  k_segments: int = 0) -> int:
+    out = _sz(0)
+    _check(lib.qlin_scaled_mm_workspace_size(fmt, variant, tile_n, k_segments, M, N, K, ctypes.byref(out)),
+           "qlin_scaled_mm_workspace_size")
+    return out.value
+
+
+def qlin_scaled_mm(fmt: int, a_q, s_a, w_q, s_w, bias, c_out, workspace=None, stream=None, *,
+                   variant: int = QLIN_VAR_AUTO, tile_n: int = 0, k_segments: int = 0, flags: int = 0,
+                   M=None, N=None, K=None, workspace_bytes=None):
+    """C = (A_q W_q^T) * s_a * s_w + bias (bf16), or raw INT8 accumulators with QLIN_OUT_I32ACC."""
+    M = a_q.shape[0] if M is None else M
+    N = w_q.shape[0] if N is None else N
+    K = a_q.shape[1] if K is None else K
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.qlin_scaled_mm(fmt, variant, tile_n, k_segments, M, N, K, _ptr(a_q), _ptr(s_a), _ptr(w_q), _ptr(s_w),
+                              _ptr(bias), _ptr(c_out), flags, _ptr(workspace), workspace_bytes, _stream(stream)),
+           "qlin_scaled_mm")
+
+
+def qlin_dispatch_table_load(path: str):
+    _check(lib.qlin_dispatch_table_load(os.fsencode(path)), "qlin_dispatch_table_load")
+
+
+def qlin_dispatch_table_clear():
+    _check(lib.qlin_dispatch_table_clear(), "qlin_dispatch_table_clear")
+
+
+def qlin_dispatch_query(fmt: int, M: int, N: int, K: int) -> dict:
+    cfg = qlin_config()
+    _check(lib.qlin_dispatch_query(fmt, M, N, K, ctypes.byref(cfg)), "qlin_dispatch_query")
+    return cfg.as_dict()
+
+
+def qlin_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def qlin_sync_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return lib.qlin_sync_status(_stream(stream))
+
+
+def qlin_abi_version() -> int:
+    return lib.qlin_abi_version()

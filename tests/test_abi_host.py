@@ -1,0 +1,165 @@
+"""Host-only checks of the C ABI (no GPU): the library loads, exports every
+symbol include/qlin.h declares, validates arguments before launching
+anything, and plans / dispatches shapes as documented."""
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def q():
+    from quantized_linear_layers_group_b200 import build
+
+    build.build()
+    from quantized_linear_layers_group_b200 import qlin
+
+    return qlin
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "qlin.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^QLIN_API\s+[\w\s\*]+?\b(qlin_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    syms = _declared_symbols()
+    for name in ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_dispatch_table_load"):
+        assert name in syms
+    assert len(syms) == 10
+
+
+def test_library_exports_every_declared_symbol(q):
+    import ctypes
+
+    lib = ctypes.CDLL(q.LIB_PATH)
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(_declared_symbols()) == set(q.EXPORTS)
+    assert q.qlin_abi_version() == 1
+
+
+def test_status_strings(q):
+    for s in range(0, 11):
+        assert q.qlin_status_string(s) and q.qlin_status_string(s) != "unknown status"
+    assert q.qlin_status_string(99) == "unknown status"
+
+
+def _mm(q, **kw):
+    args = dict(fmt=1, variant=0, tile_n=0, k_segments=0, M=16, N=256, K=256, a=16, sa=16, w=16, sw=16,
+                bias=None, c=16, flags=0, ws=None, wsb=0)
+    args.update(kw)
+    return q.lib.qlin_scaled_mm(args["fmt"], args["variant"], args["tile_n"], args["k_segments"], args["M"],
+                                args["N"], args["K"], args["a"], args["sa"], args["w"], args["sw"], args["bias"],
+                                args["c"], args["flags"], args["ws"], args["wsb"], None)
+
+
+def test_scaled_mm_rejects_bad_arguments_before_launch(q):
+    assert _mm(q, fmt=7) == q.QLIN_ERR_INVALID_ARG
+    assert _mm(q, N=8) == q.QLIN_ERR_INVALID_ARG
+    assert _mm(q, N=250) == q.QLIN_ERR_UNSUPPORTED
+    assert _mm(q, K=200) == q.QLIN_ERR_UNSUPPORTED
+    assert _mm(q, fmt=2, N=320) == q.QLIN_ERR_UNSUPPORTED
+    assert _mm(q, M=-1) == q.QLIN_ERR_INVALID_ARG
+    assert _mm(q, variant=9) == q.QLIN_ERR_INVALID_ARG
+    assert _mm(q, flags=2) == q.QLIN_ERR_INVALID_ARG
+    assert _mm(q, flags=1) == q.QLIN_ERR_INVALID_ARG          # I32 accumulators are INT8 only
+    assert _mm(q, fmt=2, bias=16) == q.QLIN_ERR_INVALID_ARG   # Block-FP8 takes no bias
+    assert _mm(q, a=None) == q.QLIN_ERR_INVALID_ARG
+    assert _mm(q, a=24) == q.QLIN_ERR_ALIGNMENT
+    assert _mm(q, c=8) == q.QLIN_ERR_ALIGNMENT
+    assert _mm(q, sa=18) == q.QLIN_ERR_ALIGNMENT
+    assert _mm(q, M=0) == q.QLIN_OK                            # empty batch: no-op
+
+
+def test_quantize_rejects_bad_arguments(q):
+    L = q.lib
+    assert L.qlin_quantize_per_token(2, 16, 4, 64, 64, 16, 16, None) == q.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_per_token(1, 16, 4, 60, 64, 16, 16, None) == q.QLIN_ERR_ALIGNMENT
+    assert L.qlin_quantize_per_token(1, 16, 4, 64, 32, 16, 16, None) == q.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_per_token(1, 8, 4, 64, 64, 16, 16, None) == q.QLIN_ERR_ALIGNMENT
+    assert L.qlin_quantize_per_token(1, None, 4, 64, 64, 16, 16, None) == q.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_per_token(1, None, 0, 64, 64, None, None, None) == q.QLIN_OK
+    assert L.qlin_quantize_block(16, 4, 256, 256, 2, 128, 16, 16, None) == q.QLIN_ERR_UNSUPPORTED
+    assert L.qlin_quantize_block(16, 4, 256, 256, 1, 64, 16, 16, None) == q.QLIN_ERR_UNSUPPORTED
+    assert L.qlin_quantize_block(16, 4, 200, 200, 1, 128, 16, 16, None) == q.QLIN_ERR_UNSUPPORTED
+    assert L.qlin_quantize_block(16, 4, 256, 256, 1, 128, 16, 17, None) == q.QLIN_ERR_ALIGNMENT
+
+
+def test_workspace_sizes(q):
+    # Swap-AB + Split-K, FP8 N=4096 K=2048 M=16: S=4 segments of 32 tiles of 128x16
+    assert q.qlin_scaled_mm_workspace_size(1, 16, 4096, 2048) == 256 + 4 * 32 * 128 * 16 * 4
+    # plain variants need none
+    assert q.qlin_scaled_mm_workspace_size(1, 2048, 151936, 2048) == 0
+    assert q.qlin_scaled_mm_workspace_size(1, 16, 256, 256, variant=q.QLIN_VAR_PLAIN, tile_n=128,
+                                           k_segments=1) == 0
+    with pytest.raises(q.QlinError):
+        q.qlin_scaled_mm_workspace_size(1, 16, 256, 384, k_segments=2)          # 3 K blocks, 2 segments
+    with pytest.raises(q.QlinError):
+        q.qlin_scaled_mm_workspace_size(1, 200, 4096, 2048, variant=q.QLIN_VAR_PLAIN, tile_n=256,
+                                        k_segments=4)                            # multi-chunk on a 256 tile
+    with pytest.raises(q.QlinError):
+        q.qlin_scaled_mm_workspace_size(1, 16, 256, 256, variant=q.QLIN_VAR_SWAPAB, tile_n=128)
+
+
+def test_builtin_dispatch_rule(q):
+    q.qlin_dispatch_table_clear()
+    c = q.qlin_dispatch_query(q.QLIN_FMT_FP8, 1, 4096, 2048)
+    assert (c["variant"], c["tile_n"], c["k_segments"], c["from_table"]) == (q.QLIN_VAR_SWAPAB_SPLITK, 16, 4, 0)
+    c = q.qlin_dispatch_query(q.QLIN_FMT_FP8, 64, 4096, 2048)
+    assert (c["variant"], c["tile_n"]) == (q.QLIN_VAR_SWAPAB_SPLITK, 64)
+    c = q.qlin_dispatch_query(q.QLIN_FMT_FP8, 2048, 4096, 2048)
+    assert (c["variant"], c["tile_n"], c["k_segments"]) == (q.QLIN_VAR_PLAIN, 128, 4)
+    c = q.qlin_dispatch_query(q.QLIN_FMT_FP8, 2048, 151936, 2048)
+    assert (c["variant"], c["tile_n"], c["k_segments"]) == (q.QLIN_VAR_PLAIN, 256, 1)
+    c = q.qlin_dispatch_query(q.QLIN_FMT_FP8_BLOCK, 1, 2048, 6144)
+    assert (c["variant"], c["k_segments"]) == (q.QLIN_VAR_SWAPAB_SPLITK, 8)
+    # segmentation is a property of the shape, never of M
+    for fmt, N, K in ((1, 4096, 2048), (2, 2048, 6144), (1, 12288, 2048), (0, 2048, 2048)):
+        segs = {q.qlin_dispatch_query(fmt, M, N, K)["k_segments"] for M in (1, 8, 64, 65, 256, 2048)}
+        assert len(segs) == 1
+
+
+def _write(tmp_path, text):
+    p = tmp_path / "t.qlt"
+    p.write_text(text)
+    return str(p)
+
+
+def test_table_loader_rejects_bad_files(q, tmp_path):
+    with pytest.raises(q.QlinError) as e:
+        q.qlin_dispatch_table_load(str(tmp_path / "missing.qlt"))
+    assert e.value.status == q.QLIN_ERR_TABLE_IO
+    head = "qlin-dispatch 1\ndevice 148 10 0 NVIDIA B200\n"
+    bad = [
+        "nonsense\n",
+        "qlin-dispatch 2\ndevice 148 10 0 NVIDIA B200\n",
+        "qlin-dispatch 1\n",                                                    # no device line
+        head + "entry fp9 4096 2048 16 swapab 16 4\n",                         # bad format
+        head + "entry fp8 4096 2048 16 swapab 128 4\n",                        # tile not allowed for swap
+        head + "entry fp8 4096 2048 16 swapab 16 3\n",                         # 16 K blocks, 3 segments
+        head + "entry fp8 4096 2048 16 swapab 16 4\nentry fp8 4096 2048 256 plain 128 2\n",  # S differs by M
+        head + "entry fp8 4096 2048 16 swapab 16 4\nentry fp8 4096 2048 16 plain 128 4\n",  # duplicate bucket
+        head + "entry fp8 4096 2048 256 plain 256 4\n",                        # multi-chunk 256 tile
+        head + "entry fp8 4096 2048 16 swapab 16\n",                           # truncated
+    ]
+    for text in bad:
+        with pytest.raises(q.QlinError) as e:
+            q.qlin_dispatch_table_load(_write(tmp_path, text))
+        assert e.value.status == q.QLIN_ERR_TABLE_FORMAT, text
+
+
+def test_shipped_table_parses(q, tmp_path):
+    # the committed table passes every format check (the device check needs a GPU)
+    path = os.path.join(ROOT, "quantized_linear_layers_group_b200", "tables", "b200.qlt")
+    if not os.path.exists(path):
+        pytest.skip("no table shipped yet")
+    try:
+        q.qlin_dispatch_table_load(path)
+    except q.QlinError as e:
+        assert e.status in (q.QLIN_ERR_NO_DEVICE, q.QLIN_ERR_TABLE_DEVICE, q.QLIN_ERR_CUDA), e
+    finally:
+        q.qlin_dispatch_table_clear()

@@ -1,0 +1,131 @@
+"""GPU parity of the quantisation kernels against the oracle: bit-exact codes and
+scales (INT8 / FP8 per-token, Block-FP8 1x128 groups and 128x128 blocks)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import bits_u8, check_status
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from quantized_linear_layers_group_b200 import qlin
+    return qlin
+
+
+def _gpu_per_token(lib, fmt, x):
+    xd = x.cuda()
+    rows, cols = x.shape
+    q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    s = torch.empty(rows, dtype=torch.float32, device="cuda")
+    lib.qlin_quantize_per_token(fmt, xd, q, s)
+    torch.cuda.synchronize()
+    return bits_u8(q), s.cpu().numpy()
+
+
+def _gpu_block(lib, x, block_rows):
+    xd = x.cuda()
+    rows, cols = x.shape
+    q = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    s = torch.empty((rows + block_rows - 1) // block_rows, cols // 128, dtype=torch.float32, device="cuda")
+    lib.qlin_quantize_block(xd, block_rows, q, s)
+    torch.cuda.synchronize()
+    return bits_u8(q), s.cpu().numpy()
+
+
+def _assert_same(q_gpu, s_gpu, q_ref, s_ref, what):
+    assert np.array_equal(s_gpu.view(np.uint32), s_ref.view(np.uint32)), f"{what}: scales differ"
+    if not np.array_equal(q_gpu, q_ref):
+        bad = np.argwhere(q_gpu != q_ref)
+        raise AssertionError(f"{what}: {len(bad)} codes differ, first {bad[:5].tolist()} "
+                             f"gpu={q_gpu[tuple(bad[:5].T)]} ref={q_ref[tuple(bad[:5].T)]}")
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_INT8, oracle.FMT_FP8])
+@pytest.mark.parametrize("wname,M", [("int8_smoke", 16), ("fp8_attn", 1), ("fp8_attn", 333),
+                                     ("fp8_block_down", 64), ("fp8_attn", 2048)])
+def test_per_token_workload_rows(lib, fmt, wname, M):
+    x = synth.activations(synth.WORKLOADS[wname], M, seed=0)
+    qg, sg = _gpu_per_token(lib, fmt, x)
+    qr, sr = oracle.quantize_per_token(fmt, x)
+    _assert_same(qg, sg, qr, sr, f"{wname} M={M}")
+    check_status()
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_INT8, oracle.FMT_FP8])
+def test_per_token_exhaustive_bf16(lib, fmt):
+    # every finite bf16 value paired with the format's Qmax so the scale is 1
+    bits = np.arange(0, 1 << 16, dtype=np.uint32)
+    f = (bits << 16).view(np.float32)
+    qmax = 127.0 if fmt == oracle.FMT_INT8 else 448.0
+    vb = bits[np.isfinite(f) & (np.abs(f) <= qmax)].astype(np.uint16)
+    head = np.uint16(0x42FE if fmt == oracle.FMT_INT8 else 0x43E0)
+    x_bits = np.stack([np.full_like(vb, head)] + [vb] * 7, axis=1)  # 8 columns (16-byte rows)
+    x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16)
+    qg, sg = _gpu_per_token(lib, fmt, x)
+    qr, sr = oracle.quantize_per_token(fmt, x)
+    assert np.all(sg == 1.0)
+    _assert_same(qg, sg, qr, sr, "exhaustive")
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_INT8, oracle.FMT_FP8])
+def test_per_token_random_magnitudes_and_edges(lib, fmt):
+    g = torch.Generator().manual_seed(17)
+    x = torch.randn(67, 2056, generator=g) * torch.exp(torch.randn(67, 1, generator=g) * 4)
+    x[3] = 0.0                      # amax = 0
+    x[4] = -0.0
+    x[5, :] = -7.0                  # all -amax
+    x[6] = 0.0
+    x[6, 1000] = 3e-5               # single non-zero
+    x[7, ::2] = 1e-30               # subnormal-range quotients
+    x = x.to(torch.bfloat16)
+    qg, sg = _gpu_per_token(lib, fmt, x)
+    qr, sr = oracle.quantize_per_token(fmt, x)
+    _assert_same(qg, sg, qr, sr, "random")
+    assert sg[3] == 0 and np.all(qg[3] == 0) and np.all(qg[4] == 0)
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_INT8, oracle.FMT_FP8])
+@pytest.mark.parametrize("cols", [8, 136, 8192, 8200, 12288])
+def test_per_token_column_counts(lib, fmt, cols):
+    # register-resident paths up to 8192 columns, two-pass path above
+    x = synth.normal((9, cols), 1.0, cols)
+    qg, sg = _gpu_per_token(lib, fmt, x)
+    qr, sr = oracle.quantize_per_token(fmt, x)
+    _assert_same(qg, sg, qr, sr, f"cols={cols}")
+
+
+def test_per_token_strided_input(lib):
+    x = synth.normal((20, 512), 1.0, 3)
+    xd = x.cuda()
+    sub = xd[:, 128:384]                       # ld_x = 512, cols = 256
+    q = torch.empty(20, 256, dtype=torch.uint8, device="cuda")
+    s = torch.empty(20, dtype=torch.float32, device="cuda")
+    lib.qlin_quantize_per_token(oracle.FMT_FP8, sub, q, s)
+    torch.cuda.synchronize()
+    qr, sr = oracle.quantize_per_token(oracle.FMT_FP8, x[:, 128:384].contiguous())
+    _assert_same(bits_u8(q), s.cpu().numpy(), qr, sr, "strided")
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (37, 6144), (2048, 6144), (5, 16384)])
+def test_group128_activations(lib, rows, cols):
+    w = synth.WORKLOADS["fp8_block_down"]
+    x = synth.activations(w, rows, seed=1) if cols == 6144 else synth.normal((rows, cols), 3.0, 5)
+    qg, sg = _gpu_block(lib, x, 1)
+    qr, sr = oracle.quantize_block(x, 1, 128)
+    _assert_same(qg, sg, qr, sr, f"group128 {rows}x{cols}")
+
+
+@pytest.mark.parametrize("rows,cols", [(128, 128), (300, 384), (2048, 6144)])
+def test_block128_weights(lib, rows, cols):
+    x = synth.normal((rows, cols), 0.02, rows + cols)
+    if cols > 128:
+        x[:, 128:256] = 0  # an all-zero block column
+    qg, sg = _gpu_block(lib, x, 128)
+    qr, sr = oracle.quantize_block(x, 128, 128)
+    _assert_same(qg, sg, qr, sr, f"block128 {rows}x{cols}")
+    check_status()
