@@ -1,0 +1,506 @@
+"""Benchmark of the quantized linear layer hot path on B200.
+
+One step = one pass of the whole hot path over one batch per M of the
+workload's M sweep: dynamic activation quantisation (per token, or per 1x128
+group for Block-FP8) followed by the scaled GEMM with the variant the dispatch
+table (or the built-in rule) picks for that (M, N, K, format).  Each GEMM of a
+step reads a different copy of the quantised weight, rotating through enough
+copies that the weights read between two uses of one copy exceed 2x the L2
+(126 MB), so every GEMM streams its weight from HBM.
+
+Prints one JSON line (rank 0):
+  value       whole-job GEMM TFLOP/s over the device-timed steps (inputs resident)
+  e2e         the same steps through the same C ABI calls with the bf16
+              activations copied in from pinned host memory and C copied back
+  roofline    the dominant kernel (largest share of device time) against the
+              measured HBM / tensor peak
+  per_m       per (M, N, K, format): GEMM time, TFLOP/s, HBM GB/s, roofline fraction
+  cpu_baseline  the CPU oracle on a bounded sample (rank 0, N = 1 only)
+
+  --impl reference  times the CPU oracle as the reference arm instead.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs the same
+independent step on its own GPU (no data-path collective; weak scaling); the
+time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "scaled_mm TFLOPS & HBM GB/s vs roofline, per (M,N,K,format), 1×B200"
+L2_BYTES = 126 * 1024 * 1024
+FMT_NAME = {0: "int8", 1: "fp8", 2: "fp8_block"}
+DTYPE = {0: "int8 (int32 accumulate)", 1: "fp8_e4m3 (fp32 accumulate)", 2: "fp8_e4m3 block-scaled (fp32 accumulate)"}
+
+
+# ------------------------------------------------------------------ peaks
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def tensor_peak(peaks, fmt, sustained=True):
+    """8-bit dense tensor peak = measured bf16 cuBLAS peak x 2 (nominal 4.5 vs 2.25 PF)."""
+    base = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    return 2.0 * base
+
+
+def gemm_flops(M, N, K):
+    return 2.0 * M * N * K
+
+
+def gemm_bytes(M, N, K, fmt):
+    """Algorithmic bytes per GEMM launch: the 8-bit operands A and W (as the
+    roofline is defined on), plus scales, bias and the bf16 output separately."""
+    ab = M * K + N * K
+    scales = (M * (K // 128) + (N // 128) * (K // 128)) * 4 if fmt == 2 else (M + N) * 4
+    extra = scales + 2 * M * N
+    return ab, extra
+
+
+def quant_bytes(M, K, fmt):
+    return 2 * M * K + M * K + (M * (K // 128) if fmt == 2 else M) * 4
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# --------------------------------------------------------------- the step
+class HotPath:
+    """Device buffers and the per-step launch sequence for one workload."""
+
+    def __init__(self, workload: synth.Workload, m_values, device, seed=0):
+        from quantized_linear_layers_group_b200 import linear, qlin
+
+        self.qlin, self.linear = qlin, linear
+        self.w = workload
+        self.fmt = workload.fmt
+        self.ms = list(m_values)
+        self.device = device
+        N, K = workload.N, workload.K
+        w_cpu = synth.weights(workload, seed)
+        b_cpu = synth.bias(workload, seed)
+        w_dev = w_cpu.to(device)
+        w_q, s_w = linear.quantize_weight(self.fmt, w_dev)
+        del w_dev
+        self.bias = None if b_cpu is None else b_cpu.to(device)
+        wbytes = N * K
+        # enough weight copies that the bytes read between two uses of a copy exceed 2x L2
+        self.n_copies = max(2, math.ceil(2 * L2_BYTES / wbytes) + 1)
+        self.w_copies = [(w_q if i == 0 else w_q.clone(), s_w if i == 0 else s_w.clone())
+                         for i in range(self.n_copies)]
+        self.a = {M: synth.activations(workload, M, seed=seed).to(device) for M in self.ms}
+        self.a_host = {M: self.a[M].cpu().pin_memory() for M in self.ms}
+        self.a_q, self.s_a, self.c, self.c_host = {}, {}, {}, {}
+        ws = 0
+        for M in self.ms:
+            self.a_q[M] = torch.empty(M, K, dtype=torch.uint8, device=device)
+            self.s_a[M] = torch.empty(*((M, K // 128) if self.fmt == 2 else (M,)), dtype=torch.float32,
+                                      device=device)
+            self.c[M] = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+            self.c_host[M] = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+            ws = max(ws, qlin.qlin_scaled_mm_workspace_size(self.fmt, M, N, K))
+        self.workspace = torch.zeros(max(ws, 256), dtype=torch.uint8, device=device)
+        self.calls = 0
+        self.configs = {M: qlin.qlin_dispatch_query(self.fmt, M, N, K) for M in self.ms}
+        # weights are final: launches may overlap the previous kernel's tail
+        torch.cuda.synchronize(device)
+        self.flags = qlin.QLIN_PDL
+
+    def launch_quant(self, M, stream):
+        q = self.qlin
+        if self.fmt == 2:
+            q.qlin_quantize_block(self.a[M], 1, self.a_q[M], self.s_a[M], stream, flags=self.flags)
+        else:
+            q.qlin_quantize_per_token(self.fmt, self.a[M], self.a_q[M], self.s_a[M], stream, flags=self.flags)
+
+    def launch_gemm(self, M, stream):
+        w_q, s_w = self.w_copies[self.calls % self.n_copies]
+        self.calls += 1
+        self.qlin.qlin_scaled_mm(self.fmt, self.a_q[M], self.s_a[M], w_q, s_w, self.bias, self.c[M],
+                                 self.workspace, stream, flags=self.flags)
+
+    def step(self, stream, events=None):
+        for M in self.ms:
+            if events is not None:
+                events[M][0].record(stream)
+            self.launch_quant(M, stream)
+            if events is not None:
+                events[M][1].record(stream)
+            self.launch_gemm(M, stream)
+            if events is not None:
+                events[M][2].record(stream)
+
+    def step_e2e(self, stream):
+        """Same step with the activations copied in from pinned host memory and
+        C copied back; returns (h2d bytes, d2h bytes)."""
+        hb = db = 0
+        for M in self.ms:
+            self.a[M].copy_(self.a_host[M], non_blocking=True)
+            hb += self.a_host[M].numel() * 2
+            self.launch_quant(M, stream)
+            self.launch_gemm(M, stream)
+            self.c_host[M].copy_(self.c[M], non_blocking=True)
+            db += self.c[M].numel() * 2
+        return hb, db
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+# ----------------------------------------------------------- distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def aggregate(per_rank_units: float, max_seconds: float, world: int) -> float:
+    """Whole-job throughput: every rank processed per_rank_units; time is the max over ranks."""
+    return per_rank_units * world / max_seconds
+
+
+# -------------------------------------------------------------- CPU arm
+_ORACLE_WEIGHTS = {}
+
+
+def cpu_oracle_sample(workload: synth.Workload, M: int, seed=0):
+    """The CPU oracle (as it stands) on a bounded sample: quantise M activation
+    rows and compute their full C rows against the whole (offline-quantised)
+    weight.  Returns (seconds, GEMM flops, description)."""
+    import oracle
+
+    N, K = workload.N, workload.K
+    key = (workload.name, seed)
+    if key not in _ORACLE_WEIGHTS:
+        w = synth.weights(workload, seed)
+        if workload.fmt == 2:
+            _ORACLE_WEIGHTS[key] = oracle.quantize_block(w, 128, 128)
+        else:
+            _ORACLE_WEIGHTS[key] = oracle.quantize_per_token(workload.fmt, w)
+    wq, sw = _ORACLE_WEIGHTS[key]
+    a = synth.activations(workload, M, seed=seed)
+    b = synth.bias(workload, seed)
+    t0 = time.perf_counter()
+    if workload.fmt == 2:
+        aq, sa = oracle.quantize_block(a, 1, 128)
+    else:
+        aq, sa = oracle.quantize_per_token(workload.fmt, a)
+    oracle.scaled_mm(workload.fmt, aq, sa, wq, sw, b)
+    dt = time.perf_counter() - t0
+    return dt, gemm_flops(M, N, K), f"{workload.name}: quantise + scaled_mm of M={M} rows x N={N} x K={K}, 1 thread"
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    M = args.ref_rows
+    times, flops = [], 0.0
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, M)
+    desc = ""
+    for _ in range(args.steps):
+        dt, fl, desc = cpu_oracle_sample(w, M)
+        times.append(dt)
+        flops = fl
+    total = sum(times)
+    value = flops * len(times) / total / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE[w.fmt],
+            "data": "synthetic", "config": {"workload": w.name, "format": FMT_NAME[w.fmt], "N": w.N, "K": w.K,
+                                            "m_values": [M], "parallelism": "single process"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="fp8_attn", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--m", type=str, default=None, help="comma-separated M values (default: the workload's sweep)")
+    ap.add_argument("--table", default=os.path.join(ROOT, "quantized_linear_layers_group_b200", "tables",
+                                                    "b200.qlt"))
+    ap.add_argument("--no-table", action="store_true")
+    ap.add_argument("--graph", dest="graph", action="store_true", default=True,
+                    help="replay each device-timed step as a CUDA graph (default)")
+    ap.add_argument("--no-graph", dest="graph", action="store_false")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=256, help="rows per reference-arm step")
+    ap.add_argument("--baseline-rows", type=int, default=1024, help="rows of the cpu_baseline sample")
+    args = ap.parse_args(argv)
+    assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
+
+    rank, world, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        barrier(world)
+        return
+
+    from quantized_linear_layers_group_b200 import qlin
+
+    if not args.no_table and os.path.exists(args.table):
+        qlin.qlin_dispatch_table_load(args.table)
+    workload = synth.WORKLOADS[args.workload]
+    ms = [int(x) for x in args.m.split(",")] if args.m else list(workload.m_values)
+    device = torch.device("cuda", local)
+    hp = HotPath(workload, ms, device)
+    stream = torch.cuda.Stream(device)
+    peaks = load_peaks()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            hp.step(stream)
+        torch.cuda.synchronize()
+        st = qlin.qlin_sync_status(stream)
+        if st != 0:
+            raise RuntimeError(f"device status after warm-up: {qlin.qlin_status_string(st)}")
+
+        # ---------------------------------------------- device-timed steps
+        # Each step is one CUDA graph (the launch sequence of the hot path,
+        # as a serving engine replays it); G graphs use different weight
+        # copies so the rotation defeats L2.  Timing events are graph nodes.
+        n_graphs = max(1, math.ceil(hp.n_copies / len(ms))) if args.graph else 1
+        ev_sets, graphs = [], []
+        for _ in range(n_graphs):
+            ev = {M: [torch.cuda.Event(enable_timing=True, external=args.graph) for _ in range(3)] for M in ms}
+            ev_sets.append(ev)
+            if args.graph:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    hp.step(stream, ev)
+                graphs.append(g)
+        torch.cuda.synchronize()
+        for i in range(args.warmup):
+            if args.graph:
+                graphs[i % n_graphs].replay()
+            else:
+                hp.step(stream, ev_sets[0])
+        torch.cuda.synchronize()
+        per_m_q = {M: [] for M in ms}
+        per_m_g = {M: [] for M in ms}
+        clocks = ClockSampler(local)
+        clocks.start()
+        time.sleep(0.3)
+        barrier(world)
+        torch.cuda.synchronize()
+        step_ms = []
+        for i in range(args.steps):
+            ev = ev_sets[i % n_graphs]
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            if args.graph:
+                graphs[i % n_graphs].replay()
+            else:
+                hp.step(stream, ev)
+            s1.record(stream)
+            s1.synchronize()
+            step_ms.append(s0.elapsed_time(s1))
+            for M in ms:
+                per_m_q[M].append(ev[M][0].elapsed_time(ev[M][1]))
+                per_m_g[M].append(ev[M][1].elapsed_time(ev[M][2]))
+        torch.cuda.synchronize()
+        barrier(world)
+        clk = clocks.stop()
+        elapsed_s = max_over_ranks(sum(step_ms) / 1e3, world)
+        del graphs
+
+        # ------------------------------------------------- end-to-end steps
+        for _ in range(2):
+            hp.step_e2e(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        hb = db = 0
+        for _ in range(args.steps):
+            hb, db = hp.step_e2e(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+        st = qlin.qlin_sync_status(stream)
+        if st != 0:
+            raise RuntimeError(f"device status: {qlin.qlin_status_string(st)}")
+
+    N, K, fmt = workload.N, workload.K, workload.fmt
+    flops_step = sum(gemm_flops(M, N, K) for M in ms)
+    value = aggregate(flops_step * args.steps, elapsed_s, world) / 1e12
+    e2e_value = aggregate(flops_step * args.steps, e2e_s, world) / 1e12
+
+    tc_peak = tensor_peak(peaks, fmt, sustained=True)
+    hbm = peaks["hbm_gbs"]
+    per_m = []
+    dominant = None
+    total_dev = sum(statistics.mean(per_m_g[M]) + statistics.mean(per_m_q[M]) for M in ms)
+    for M in ms:
+        tg = statistics.mean(per_m_g[M]) / 1e3
+        tq = statistics.mean(per_m_q[M]) / 1e3
+        ab, extra = gemm_bytes(M, N, K, fmt)
+        fl = gemm_flops(M, N, K)
+        t_roof = max(ab / (hbm * 1e9), fl / (tc_peak * 1e12))
+        cfg = hp.configs[M]
+        per_m.append({"M": M, "N": N, "K": K, "format": FMT_NAME[fmt],
+                      "variant": qlin.VARIANT_NAMES[cfg["variant"]], "tile_n": cfg["tile_n"],
+                      "k_segments": cfg["k_segments"], "gemm_us": tg * 1e6, "quant_us": tq * 1e6,
+                      "tflops": fl / tg / 1e12, "hbm_gbs": ab / tg / 1e9,
+                      "hbm_gbs_all_bytes": (ab + extra) / tg / 1e9,
+                      "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / tg,
+                      "bound": "hbm" if ab / (hbm * 1e9) >= fl / (tc_peak * 1e12) else "tensor",
+                      "quant_gbs": quant_bytes(M, K, fmt) / tq / 1e9})
+        share = tg / (total_dev / 1e3)
+        if dominant is None or share > dominant[0]:
+            dominant = (share, M, tg, ab, fl)
+    _, Md, tgd, abd, fld = dominant
+    bound = "hbm" if abd / (hbm * 1e9) >= fld / (tc_peak * 1e12) else "tensor"
+    if bound == "tensor":
+        roof = {"bound": "tensor", "achieved": fld / tgd / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": fld / tgd / 1e12 / tc_peak}
+    else:
+        roof = {"bound": "hbm", "achieved": abd / tgd / 1e9, "peak": hbm, "unit": "GB/s",
+                "frac": abd / tgd / 1e9 / hbm}
+    roof.update({"traffic": None, "kernel": f"qlin_gemm_kernel M={Md} N={N} K={K} {FMT_NAME[fmt]}",
+                 "peak_source": f"{peaks['source']}: " + ("2 x bf16_tflops_sustained (8-bit = 2x bf16 nominal)"
+                                                          if bound == "tensor" else "hbm_gbs copy")})
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * elapsed_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": DTYPE[fmt], "data": "synthetic",
+            "config": {"workload": workload.name, "format": FMT_NAME[fmt], "N": N, "K": K, "m_values": ms,
+                       "bias": workload.bias,
+                       "l2": f"{hp.n_copies} rotating weight copies ({hp.n_copies * N * K / 1e6:.0f} MB) > 2x L2",
+                       "parallelism": "replicas" if world > 1 else "single GPU", "cuda_graph": args.graph,
+                       "pdl": True,
+                       "table": (not args.no_table and os.path.exists(args.table))},
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db},
+            "gpu_launches": 2 * len(ms) * args.steps,
+            "clocks": clk,
+            "per_m": per_m}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl, desc = cpu_oracle_sample(workload, args.baseline_rows)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                                "sample": desc, "seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

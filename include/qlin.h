@@ -80,8 +80,16 @@ typedef enum {
     QLIN_VAR_SWAPAB_SPLITK = 4  /* Swap-AB with the K segments spread over CTAs */
 } qlin_variant;
 
-/* flags for qlin_scaled_mm */
-#define QLIN_OUT_I32ACC 1u /* INT8 only: write the raw int32 accumulators instead of bf16 C */
+/* flags */
+#define QLIN_OUT_I32ACC 1u /* qlin_scaled_mm, INT8 only: write the raw int32 accumulators instead of bf16 C */
+/* Launch as a programmatic dependent of the previous kernel in the stream:
+ * the kernel may start before that kernel has finished, waits for it before
+ * reading activations or scales or writing outputs, and lets the next kernel
+ * start early in turn.  qlin_scaled_mm streams weight tiles (w_q) before the
+ * wait, so with this flag w_q must not be written by the kernel that
+ * immediately precedes the call in the stream.  Accepted by every launching
+ * entry point. */
+#define QLIN_PDL 2u
 
 /* A resolved GEMM configuration (what qlin_dispatch_query returns). */
 typedef struct {
@@ -111,11 +119,12 @@ typedef struct {
  *   ld_x       row stride of x in elements, >= cols, ld_x % 8 == 0
  *   q_out      int8 / e4m3 [rows, cols] dense (device)
  *   scale_out  fp32 [rows] (device)
+ *   flags      0 or QLIN_PDL
  * Alignment: x, q_out 16-byte aligned; scale_out 4-byte aligned.
  * Errors: INVALID_ARG, ALIGNMENT, CUDA (launch failure).
  */
 QLIN_API qlin_status qlin_quantize_per_token(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld_x,
-                                    void* q_out, float* scale_out, qlin_stream_t stream);
+                                             void* q_out, float* scale_out, uint32_t flags, qlin_stream_t stream);
 
 /*
  * qlin_quantize_block -- Block-FP8 quantisation ("Block-FP8", page "Helion in
@@ -130,11 +139,13 @@ QLIN_API qlin_status qlin_quantize_per_token(int fmt, const void* x, int64_t row
  *   block_rows  1 or 128;  block_cols  128;  cols % 128 == 0
  *   q_out       e4m3 [rows, cols] dense (device)
  *   scale_out   fp32 [ceil(rows/block_rows), cols/128] row-major (device)
+ *   flags       0 or QLIN_PDL
  * Alignment as qlin_quantize_per_token.
  * Errors: INVALID_ARG, UNSUPPORTED (other block shapes), ALIGNMENT, CUDA.
  */
 QLIN_API qlin_status qlin_quantize_block(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int block_rows,
-                                int block_cols, void* q_out, float* scale_out, qlin_stream_t stream);
+                                         int block_cols, void* q_out, float* scale_out, uint32_t flags,
+                                         qlin_stream_t stream);
 
 /*
  * qlin_scaled_mm -- the scaled GEMM with a fused scale / bias / bf16 epilogue,
@@ -163,12 +174,14 @@ QLIN_API qlin_status qlin_quantize_block(const void* x, int64_t rows, int64_t co
  *   a_q, w_q            int8 / e4m3 [M,K] and [N,K] (device)
  *   bias                bf16 [N] (device) or NULL
  *   c_out               bf16 [M,N] (device); int32 [M,N] with QLIN_OUT_I32ACC
- *   flags               0 or QLIN_OUT_I32ACC (INT8 only)
+ *   flags               QLIN_OUT_I32ACC (INT8 only) and / or QLIN_PDL
  *   workspace           device buffer of at least qlin_scaled_mm_workspace_size()
- *                       bytes (may be NULL when that size is 0).  It must be
- *                       zero-filled once when first allocated; every call leaves
- *                       its ticket words at zero again.  Calls that overlap in time
- *                       must not share a workspace.
+ *                       bytes (may be NULL when that size is 0).  Its first
+ *                       64 KiB hold the Split-K ticket words: they must be
+ *                       zero-filled once when the buffer is allocated, and every
+ *                       call leaves them at zero again; the rest holds partial
+ *                       tiles.  Calls that overlap in time must not share a
+ *                       workspace.
  * Alignment: a_q, w_q, c_out, workspace 16-byte aligned; scales and bias 4 / 2.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, NO_DEVICE.
  */

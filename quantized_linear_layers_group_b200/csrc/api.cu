@@ -227,8 +227,9 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     if (p.units > (int64_t)INT32_MAX / 2) return QLIN_ERR_UNSUPPORTED;
     p.grid = (int)std::min<int64_t>(p.units, num_sms);
     if (p.grid < 1) p.grid = 1;
+    if (p.spread && p.num_tiles > kMaxSplitTiles) return QLIN_ERR_UNSUPPORTED;
     if (p.spread) {
-        p.ticket_bytes = ((size_t)p.num_tiles * 4 + 255) & ~size_t(255);
+        p.ticket_bytes = kTicketBytes;
         p.workspace_bytes = p.ticket_bytes + (size_t)p.k_segments * p.num_tiles * 128 * p.tile_n * 4;
     } else {
         p.ticket_bytes = 0;
@@ -264,8 +265,9 @@ const char* qlin_status_string(qlin_status s) {
 }
 
 qlin_status qlin_quantize_per_token(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld_x, void* q_out,
-                                    float* scale_out, qlin_stream_t stream) {
+                                    float* scale_out, uint32_t flags, qlin_stream_t stream) {
     if (fmt != QLIN_FMT_INT8 && fmt != QLIN_FMT_FP8) return QLIN_ERR_INVALID_ARG;
+    if (flags & ~QLIN_PDL) return QLIN_ERR_INVALID_ARG;
     if (rows < 0 || cols < 1 || ld_x < cols) return QLIN_ERR_INVALID_ARG;
     if (rows == 0) return QLIN_OK;
     if (!x || !q_out || !scale_out) return QLIN_ERR_INVALID_ARG;
@@ -273,14 +275,15 @@ qlin_status qlin_quantize_per_token(int fmt, const void* x, int64_t rows, int64_
     if (!aligned16(x) || !aligned16(q_out) || (reinterpret_cast<uintptr_t>(scale_out) & 3u))
         return QLIN_ERR_ALIGNMENT;
     if (rows > (int64_t)1 << 34) return QLIN_ERR_UNSUPPORTED;
-    cudaError_t e = launch_quantize_per_token(fmt, x, rows, cols, ld_x, q_out, scale_out,
+    cudaError_t e = launch_quantize_per_token(fmt, x, rows, cols, ld_x, q_out, scale_out, (flags & QLIN_PDL) != 0,
                                               static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
 }
 
 qlin_status qlin_quantize_block(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int block_rows,
-                                int block_cols, void* q_out, float* scale_out, qlin_stream_t stream) {
+                                int block_cols, void* q_out, float* scale_out, uint32_t flags, qlin_stream_t stream) {
     if (rows < 0 || cols < 1 || ld_x < cols) return QLIN_ERR_INVALID_ARG;
+    if (flags & ~QLIN_PDL) return QLIN_ERR_INVALID_ARG;
     if (block_cols != 128 || (block_rows != 1 && block_rows != 128)) return QLIN_ERR_UNSUPPORTED;
     if (cols % 128 != 0) return QLIN_ERR_UNSUPPORTED;
     if (rows == 0) return QLIN_OK;
@@ -289,8 +292,8 @@ qlin_status qlin_quantize_block(const void* x, int64_t rows, int64_t cols, int64
     if (!aligned16(x) || !aligned16(q_out) || (reinterpret_cast<uintptr_t>(scale_out) & 3u))
         return QLIN_ERR_ALIGNMENT;
     if (block_rows == 128 && (rows + 127) / 128 > 65535) return QLIN_ERR_UNSUPPORTED;
-    cudaError_t e =
-        launch_quantize_block(x, rows, cols, ld_x, block_rows, q_out, scale_out, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_quantize_block(x, rows, cols, ld_x, block_rows, q_out, scale_out, (flags & QLIN_PDL) != 0,
+                                          static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
 }
 
@@ -315,7 +318,7 @@ qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int
                            qlin_stream_t stream) {
     qlin_status st = check_fmt_shape(fmt, M, N, K);
     if (st != QLIN_OK) return st;
-    if (flags & ~QLIN_OUT_I32ACC) return QLIN_ERR_INVALID_ARG;
+    if (flags & ~(QLIN_OUT_I32ACC | QLIN_PDL)) return QLIN_ERR_INVALID_ARG;
     const bool out_i32 = (flags & QLIN_OUT_I32ACC) != 0;
     if (out_i32 && fmt != QLIN_FMT_INT8) return QLIN_ERR_INVALID_ARG;
     if (fmt == QLIN_FMT_FP8_BLOCK && bias) return QLIN_ERR_INVALID_ARG;
@@ -342,7 +345,7 @@ qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int
                      variant_name(p.swap ? (p.spread ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB)
                                          : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
                      p.tile_n, p.k_segments, p.grid);
-    GemmOperands ops{a_q, s_a, w_q, s_w, bias, c_out, out_i32, workspace};
+    GemmOperands ops{a_q, s_a, w_q, s_w, bias, c_out, out_i32, workspace, (flags & QLIN_PDL) != 0};
     return launch_gemm(p, ops, static_cast<cudaStream_t>(stream));
 }
 

@@ -9,13 +9,15 @@
 // transposes": C^T = W A^T, so a small M becomes the narrow MMA side).
 //
 // One CTA per SM runs a static round-robin over work units.  Warp roles:
-//   warp 4  TMA producer: 128-byte-swizzled K-major tiles of both operands
+//   warp 8  TMA producer: 128-byte-swizzled K-major tiles of both operands
 //           into a STAGES-deep shared-memory ring (mbarrier full/empty pairs)
-//   warp 5  TMEM allocator + MMA issuer: one thread issues tcgen05.mma
+//   warp 9  TMEM allocator + MMA issuer: one thread issues tcgen05.mma
 //           (M = 128, N = tile_n, K = 32 per instruction) into one of two
 //           TMEM accumulator buffers and commits to mbarriers
-//   warps 0-3  epilogue: tcgen05.ld of the accumulator (warp w owns TMEM
-//           lanes 32w..32w+31), scales, bias, bf16 convert, global store.
+//   warps 0-7  epilogue: warp w reads TMEM lanes 32(w%4)..32(w%4)+31 (the
+//           hardware's lane quadrant for that warp) and the 32-column slices
+//           j with j % 2 == w / 4, so two warps share each quadrant; scales
+//           and bias are staged once per tile in shared memory.
 //
 // Fixed reduction order (batch invariance).  K is cut into S segments fixed
 // per (format, N, K).  Each segment is accumulated on its own in TMEM
@@ -27,6 +29,11 @@
 // them in the same order; so every variant gives bitwise the same C, and a
 // row of C never depends on the other rows.  INT8 sums are exact, so the
 // plain INT8 variant simply accumulates all of K in one TMEM buffer.
+//
+// Programmatic dependent launch: with QLIN_PDL the kernel starts while the
+// previous kernel of the stream (normally the activation quantiser) is still
+// running; the producer streams the first weight tiles before pdl_wait(), and
+// everything that reads activations, scales or writes C waits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -52,7 +59,7 @@ struct GemmArgs {
     const float* s_a;
     const float* s_w;
     const uint16_t* bias;
-    void* c;
+    void* c;  // bf16 C, or int32 C when out_i32
     int32_t* tickets;
     uint32_t* partials;
     int M, N;
@@ -61,8 +68,14 @@ struct GemmArgs {
     int spread, out_i32;
 };
 
-constexpr int kThreads = 192;  // 4 epilogue warps + producer warp + MMA warp
-constexpr int kSmemBudget = 232448 - 1024 - 256;
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kProducerWarp = kEpiWarps;
+constexpr int kMmaWarp = kEpiWarps + 1;
+constexpr int kThreads = (kEpiWarps + 2) * 32;
+constexpr int kStagingBytes = kEpiWarps * 2048;  // per epilogue warp: one 32x32 bf16 box
+constexpr int kScaleBytes = 2 * 256 * 4;         // column scale + column bias of one tile
+constexpr int kStageBudget = 232448 - 1024 - 256 - kStagingBytes - kScaleBytes;
 
 __host__ __device__ constexpr int pow2_at_least(int v) {
     int p = 32;
@@ -79,18 +92,23 @@ struct Cfg {
     static constexpr int P_BYTES = BM * BK;
     static constexpr int Q_BYTES = BN * BK;
     static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES;
-    static constexpr int STAGES_FIT = kSmemBudget / STAGE_BYTES;
+    static constexpr int STAGES_FIT = kStageBudget / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
-    static constexpr int SW = BN < 32 ? BN : 32;   // columns per TMEM load
+    static constexpr int SW = BN < 32 ? BN : 32;   // columns per TMEM load / per store box
     static constexpr int NSLICE = BN / SW;
+    static constexpr int MY_SLICES = (NSLICE + 1) / 2;  // slices per epilogue warp (at most)
     static constexpr int ACC_COLS = BN < 32 ? 32 : BN;
     static constexpr bool MULTI = BN <= 128;       // may run multi-chunk units
     static constexpr int TOTAL_COL = 2 * ACC_COLS; // running-total region
     static constexpr int TMEM_COLS = pow2_at_least(2 * ACC_COLS + (MULTI ? ACC_COLS : 0));
     static constexpr uint32_t IDESC = make_idesc(INT8, 128, BN);
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+    static constexpr size_t STAGING_OFF = (size_t)STAGES * STAGE_BYTES;
+    static constexpr size_t SCALE_OFF = STAGING_OFF + kStagingBytes;
+    static constexpr size_t BAR_OFF = SCALE_OFF + kScaleBytes;
+    static constexpr size_t SMEM = 1024 + BAR_OFF + 256;
     static_assert(TMEM_COLS <= 512, "TMEM overflow");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+    static_assert(SMEM <= 232448, "shared memory");
 };
 
 struct Unit {
@@ -123,99 +141,133 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    const __nv_bfloat16 l = __float2bfloat16_rn(lo);
-    const __nv_bfloat16 h = __float2bfloat16_rn(hi);
-    return (uint32_t)__bfloat16_as_ushort(l) | ((uint32_t)__bfloat16_as_ushort(h) << 16);
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half), .y = hi
+    return *reinterpret_cast<const uint32_t*>(&p);
 }
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts_u4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+// Per-thread epilogue context.
+struct EpiCtx {
+    int quad, half, lane, row_lane;  // TMEM lane quadrant, slice parity, lane, TMEM lane (row of P)
+    float row_scale;                 // s_a[m] (plain) or s_w[n] (Swap-AB)
+    float row_bias;                  // bias[n] (Swap-AB only)
+    uint32_t s_col;                  // shared address of the tile's column scales
+    uint32_t b_col;                  // shared address of the tile's column bias
+    uint32_t staging;                // shared address of this warp's 2 KB transpose buffer
+    bool has_bias;
+};
 
 // Final epilogue of one slice of SW accumulator columns.  `v` holds fp32 bits
 // (FP8 formats: the summed value) or int32 (INT8: the exact accumulator).
+//   y = ((float)acc * s_a[m]) * s_w[n] + bias[n]   (Block-FP8: y = acc)
 template <int FMT, bool SWAP, int BN>
-__device__ __forceinline__ void store_slice(const GemmArgs& a, const Unit& un, int j, int row_lane,
-                                            const uint32_t* v) {
+__device__ __forceinline__ void finish_slice(const GemmArgs& a, const Unit& un, int j, EpiCtx& e,
+                                             const uint32_t* v) {
     using C = Cfg<FMT, SWAP, BN>;
     constexpr int SW = C::SW;
-    if constexpr (!SWAP) {
-        const int m = un.pt * 128 + row_lane;
-        if (m >= a.M) return;
-        const int n0 = un.qt * BN + j * SW;
-        if (a.out_i32) {
-            int32_t* out = static_cast<int32_t*>(a.c) + (size_t)m * a.N + n0;
+    if (a.out_i32) {  // raw INT8 accumulators (test path): direct stores
+        int32_t* out = static_cast<int32_t*>(a.c);
+        if constexpr (!SWAP) {
+            const int m = un.pt * 128 + e.row_lane;
+            const int n0 = un.qt * BN + j * SW;
+            if (m < a.M) {
 #pragma unroll
-            for (int h = 0; h < SW / 16; ++h) {
-                if (n0 + h * 16 + 16 <= a.N) {
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        reinterpret_cast<uint4*>(out + h * 16)[q4] =
-                            make_uint4(v[h * 16 + q4 * 4], v[h * 16 + q4 * 4 + 1], v[h * 16 + q4 * 4 + 2],
-                                       v[h * 16 + q4 * 4 + 3]);
-                }
+                for (int c = 0; c < SW; ++c)
+                    if (n0 + c < a.N) out[(size_t)m * a.N + n0 + c] = (int32_t)v[c];
             }
-            return;
-        }
-        float sa = 0.f;
-        if constexpr (!C::BLOCK) sa = __ldg(a.s_a + m);
-        uint16_t* out = reinterpret_cast<uint16_t*>(a.c) + (size_t)m * a.N + n0;
+        } else {
+            const int n = un.pt * 128 + e.row_lane;
+            const int m0 = un.qt * BN + j * SW;
+            if (n < a.N) {
 #pragma unroll
-        for (int h = 0; h < SW / 16; ++h) {
-            if (n0 + h * 16 + 16 > a.N) continue;
-            uint32_t packed[8];
-#pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-                float y[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int c = h * 16 + i + e;
-                    const int n = n0 + c;
-                    float t;
-                    if constexpr (C::INT8)
-                        t = __int2float_rn((int)v[c]);
-                    else
-                        t = __uint_as_float(v[c]);
-                    if constexpr (!C::BLOCK) {
-                        t = __fmul_rn(t, sa);
-                        t = __fmul_rn(t, __ldg(a.s_w + n));
-                        if (a.bias) t = __fadd_rn(t, __uint_as_float((uint32_t)__ldg(a.bias + n) << 16));
-                    }
-                    y[e] = t;
-                }
-                packed[i / 2] = pack_bf16x2(y[0], y[1]);
+                for (int c = 0; c < SW; ++c)
+                    if (m0 + c < a.M) out[(size_t)(m0 + c) * a.N + n] = (int32_t)v[c];
             }
-            reinterpret_cast<uint4*>(out + h * 16)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            reinterpret_cast<uint4*>(out + h * 16)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         }
-    } else {
-        const int n = un.pt * 128 + row_lane;
-        if (n >= a.N) return;
-        const int m0 = un.qt * BN + j * SW;
-        if (a.out_i32) {
-            int32_t* out = static_cast<int32_t*>(a.c);
+        return;
+    }
+    float y[SW];
 #pragma unroll
-            for (int c = 0; c < SW; ++c)
-                if (m0 + c < a.M) out[(size_t)(m0 + c) * a.N + n] = (int32_t)v[c];
-            return;
-        }
-        float swv = 0.f, bv = 0.f;
+    for (int c4 = 0; c4 < SW; c4 += 4) {
+        float4 sc = make_float4(0.f, 0.f, 0.f, 0.f), bc = make_float4(0.f, 0.f, 0.f, 0.f);
         if constexpr (!C::BLOCK) {
-            swv = __ldg(a.s_w + n);
-            if (a.bias) bv = __uint_as_float((uint32_t)__ldg(a.bias + n) << 16);
+            sc = lds_f4(e.s_col + (uint32_t)(j * SW + c4) * 4u);
+            if (!SWAP && e.has_bias) bc = lds_f4(e.b_col + (uint32_t)(j * SW + c4) * 4u);
         }
-        uint16_t* out = reinterpret_cast<uint16_t*>(a.c);
+        const float scv[4] = {sc.x, sc.y, sc.z, sc.w};
+        const float bcv[4] = {bc.x, bc.y, bc.z, bc.w};
 #pragma unroll
-        for (int c = 0; c < SW; ++c) {
-            const int m = m0 + c;
-            if (m >= a.M) break;
+        for (int i = 0; i < 4; ++i) {
+            const int c = c4 + i;
             float t;
             if constexpr (C::INT8)
                 t = __int2float_rn((int)v[c]);
             else
                 t = __uint_as_float(v[c]);
             if constexpr (!C::BLOCK) {
-                t = __fmul_rn(t, __ldg(a.s_a + m));
-                t = __fmul_rn(t, swv);
-                if (a.bias) t = __fadd_rn(t, bv);
+                if constexpr (!SWAP) {
+                    t = __fmul_rn(t, e.row_scale);  // * s_a[m]
+                    t = __fmul_rn(t, scv[i]);       // * s_w[n]
+                    if (e.has_bias) t = __fadd_rn(t, bcv[i]);
+                } else {
+                    t = __fmul_rn(t, scv[i]);       // * s_a[m]
+                    t = __fmul_rn(t, e.row_scale);  // * s_w[n]
+                    if (e.has_bias) t = __fadd_rn(t, e.row_bias);
+                }
             }
-            out[(size_t)m * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(t));
+            y[c] = t;
+        }
+    }
+    uint16_t* cb = static_cast<uint16_t*>(a.c);
+    if constexpr (SWAP) {
+        // lane = column n of C; each store instruction writes 64 contiguous bytes of row m
+        const int n = un.pt * 128 + e.row_lane;
+        const int m0 = un.qt * BN + j * SW;
+        if (n < a.N) {
+#pragma unroll
+            for (int c = 0; c < SW; ++c)
+                if (m0 + c < a.M) cb[(size_t)(m0 + c) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y[c]));
+        }
+    } else {
+        // The warp's 32 x 32 box of C is transposed through shared memory so that
+        // every store instruction writes whole 64-byte row segments (4 lanes per
+        // row).  Chunk q of row r sits at q ^ ((r >> 1) & 3): conflict-free both ways.
+        const int bx = un.qt * BN + j * SW;
+        const int by = un.pt * 128 + e.quad * 32;
+        if (bx >= a.N || by >= a.M) return;  // warp-uniform: the whole box is outside C
+        uint32_t packed[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) packed[c / 2] = pack_bf16x2(y[c], y[c + 1]);
+        __syncwarp();  // every lane has read the previous box back
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            sts_u4(e.staging + e.lane * 64 + ((q ^ ((e.lane >> 1) & 3)) * 16),
+                   make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]));
+        __syncwarp();
+        const int q = e.lane & 3;
+#pragma unroll
+        for (int r0 = 0; r0 < 32; r0 += 8) {
+            const int r = r0 + (e.lane >> 2);
+            const uint4 val = lds_u4(e.staging + r * 64 + ((q ^ ((r >> 1) & 3)) * 16));
+            const int m = by + r, n = bx + q * 8;
+            if (m < a.M && n < a.N) *reinterpret_cast<uint4*>(cb + (size_t)m * a.N + n) = val;
         }
     }
 }
@@ -236,54 +288,69 @@ __device__ __forceinline__ void tmem_store_slice(uint32_t taddr, const uint32_t 
         tmem_st16(taddr, r);
 }
 
-// Split-K: write this unit's segment value for slice j to the workspace.
+// Split-K workspace: [tile][segment][slice][SW/4 column groups][128 lanes]
+// 16-byte vectors, so the 32 lanes of a warp touch 512 contiguous bytes per
+// access.  partial_ptr returns this lane's first vector; group q is 128
+// vectors further on.
 template <int SW>
-__device__ __forceinline__ uint32_t* partial_ptr(const GemmArgs& a, int tile, int seg, int j, int nslice,
-                                                 int row_lane) {
-    return a.partials + ((((size_t)tile * a.S + seg) * nslice + j) * 128 + row_lane) * SW;
+__device__ __forceinline__ uint4* partial_ptr(const GemmArgs& a, int tile, int seg, int j, int nslice,
+                                              int row_lane) {
+    return reinterpret_cast<uint4*>(a.partials) + (((size_t)tile * a.S + seg) * nslice + j) * (SW / 4) * 128 +
+           row_lane;
 }
 
 template <int SW>
-__device__ __forceinline__ void store_partial(uint32_t* p, const uint32_t (&v)[SW]) {
+__device__ __forceinline__ void store_partial(uint4* p, const uint32_t (&v)[SW]) {
 #pragma unroll
-    for (int q = 0; q < SW / 4; ++q)
-        reinterpret_cast<uint4*>(p)[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    for (int q = 0; q < SW / 4; ++q) p[q * 128] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
 // Split-K: after every segment of a tile has been written, the last CTA to
-// arrive adds them in segment order and runs the final epilogue.
+// arrive adds them in segment order and runs the final epilogue.  One thread
+// publishes the CTA's partial (release) and takes the ticket (acquire).
 template <int FMT, bool SWAP, int BN>
-__device__ __forceinline__ void splitk_finish(const GemmArgs& a, const Unit& un, int row_lane, int* bcast) {
+__device__ __forceinline__ void splitk_finish(const GemmArgs& a, const Unit& un, EpiCtx& e, int* bcast) {
     using C = Cfg<FMT, SWAP, BN>;
     constexpr int SW = C::SW;
-    __threadfence();
-    named_bar_sync(1, 128);
+    named_bar_sync(1, kEpiThreads);
     if (threadIdx.x == 0) {
-        const int old = atomicAdd(a.tickets + un.tile, 1);
+        // acq_rel: releases this CTA's partial stores (ordered before it by the
+        // barrier above) and, for the last arriver, acquires everyone else's
+        const int old = atom_add_acq_rel_gpu(a.tickets + un.tile, 1);
         *bcast = (old == a.S - 1) ? 1 : 0;
     }
-    named_bar_sync(1, 128);
+    named_bar_sync(1, kEpiThreads);
     const bool last = *(volatile int*)bcast != 0;
     if (!last) return;
-    __threadfence();
 #pragma unroll 1
-    for (int j = 0; j < C::NSLICE; ++j) {
+    for (int j = e.half; j < C::NSLICE; j += 2) {
         uint32_t acc[SW];
         if constexpr (C::INT8) {
             int32_t t[SW];
 #pragma unroll
             for (int c = 0; c < SW; ++c) t[c] = 0;
 #pragma unroll 1
-            for (int s = 0; s < a.S; ++s) {
-                const uint4* p = reinterpret_cast<const uint4*>(partial_ptr<SW>(a, un.tile, s, j, C::NSLICE, row_lane));
+            for (int s0 = 0; s0 < a.S; s0 += 2) {
+                uint4 w[2][SW / 4];
 #pragma unroll
-                for (int q = 0; q < SW / 4; ++q) {
-                    const uint4 w = __ldcg(p + q);
-                    t[4 * q] += (int32_t)w.x;
-                    t[4 * q + 1] += (int32_t)w.y;
-                    t[4 * q + 2] += (int32_t)w.z;
-                    t[4 * q + 3] += (int32_t)w.w;
-                }
+                for (int i = 0; i < 2; ++i)
+                    if (s0 + i < a.S) {
+                        const uint4* p =
+                            reinterpret_cast<const uint4*>(partial_ptr<SW>(a, un.tile, s0 + i, j, C::NSLICE, e.row_lane));
+#pragma unroll
+                        for (int q = 0; q < SW / 4; ++q) w[i][q] = __ldcg(p + q * 128);
+                    }
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    if (s0 + i < a.S) {
+#pragma unroll
+                        for (int q = 0; q < SW / 4; ++q) {
+                            t[4 * q] += (int32_t)w[i][q].x;
+                            t[4 * q + 1] += (int32_t)w[i][q].y;
+                            t[4 * q + 2] += (int32_t)w[i][q].z;
+                            t[4 * q + 3] += (int32_t)w[i][q].w;
+                        }
+                    }
             }
 #pragma unroll
             for (int c = 0; c < SW; ++c) acc[c] = (uint32_t)t[c];
@@ -292,22 +359,34 @@ __device__ __forceinline__ void splitk_finish(const GemmArgs& a, const Unit& un,
 #pragma unroll
             for (int c = 0; c < SW; ++c) t[c] = 0.f;
 #pragma unroll 1
-            for (int s = 0; s < a.S; ++s) {
-                const uint4* p = reinterpret_cast<const uint4*>(partial_ptr<SW>(a, un.tile, s, j, C::NSLICE, row_lane));
+            for (int s0 = 0; s0 < a.S; s0 += 2) {
+                uint4 w[2][SW / 4];
 #pragma unroll
-                for (int q = 0; q < SW / 4; ++q) {
-                    const uint4 w = __ldcg(p + q);
-                    t[4 * q] = __fadd_rn(t[4 * q], __uint_as_float(w.x));
-                    t[4 * q + 1] = __fadd_rn(t[4 * q + 1], __uint_as_float(w.y));
-                    t[4 * q + 2] = __fadd_rn(t[4 * q + 2], __uint_as_float(w.z));
-                    t[4 * q + 3] = __fadd_rn(t[4 * q + 3], __uint_as_float(w.w));
-                }
+                for (int i = 0; i < 2; ++i)
+                    if (s0 + i < a.S) {
+                        const uint4* p =
+                            reinterpret_cast<const uint4*>(partial_ptr<SW>(a, un.tile, s0 + i, j, C::NSLICE, e.row_lane));
+#pragma unroll
+                        for (int q = 0; q < SW / 4; ++q) w[i][q] = __ldcg(p + q * 128);
+                    }
+#pragma unroll
+                for (int i = 0; i < 2; ++i)  // fixed segment order
+                    if (s0 + i < a.S) {
+#pragma unroll
+                        for (int q = 0; q < SW / 4; ++q) {
+                            t[4 * q] = __fadd_rn(t[4 * q], __uint_as_float(w[i][q].x));
+                            t[4 * q + 1] = __fadd_rn(t[4 * q + 1], __uint_as_float(w[i][q].y));
+                            t[4 * q + 2] = __fadd_rn(t[4 * q + 2], __uint_as_float(w[i][q].z));
+                            t[4 * q + 3] = __fadd_rn(t[4 * q + 3], __uint_as_float(w[i][q].w));
+                        }
+                    }
             }
 #pragma unroll
             for (int c = 0; c < SW; ++c) acc[c] = __float_as_uint(t[c]);
         }
-        store_slice<FMT, SWAP, BN>(a, un, j, row_lane, acc);
+        finish_slice<FMT, SWAP, BN>(a, un, j, e, acc);
     }
+    named_bar_sync(1, kEpiThreads);  // every warp has read its partials
     if (threadIdx.x == 0) a.tickets[un.tile] = 0;  // leave the ticket zeroed for the next call
 }
 
@@ -316,21 +395,18 @@ __device__ __forceinline__ void splitk_finish(const GemmArgs& a, const Unit& un,
 // segment, finishes the tile).
 template <int FMT, bool SWAP, int BN>
 __device__ __forceinline__ void consume_segment_slice(const GemmArgs& a, const Unit& un, int seg_no, int j,
-                                                      int row_lane, uint32_t t_total,
+                                                      uint32_t t_total, EpiCtx& e,
                                                       const uint32_t (&segv)[Cfg<FMT, SWAP, BN>::SW]) {
     using C = Cfg<FMT, SWAP, BN>;
     constexpr int SW = C::SW;
     if (a.spread) {
-        store_partial<SW>(partial_ptr<SW>(a, un.tile, un.seg, j, C::NSLICE, row_lane), segv);
+        store_partial<SW>(partial_ptr<SW>(a, un.tile, un.seg, j, C::NSLICE, e.row_lane), segv);
         return;
     }
-    uint32_t t[SW];
     if constexpr (C::INT8) {
-#pragma unroll
-        for (int c = 0; c < SW; ++c) t[c] = segv[c];  // exact: whole K in one accumulator
-        store_slice<FMT, SWAP, BN>(a, un, j, row_lane, t);
-        return;
+        finish_slice<FMT, SWAP, BN>(a, un, j, e, segv);  // exact: whole K in one accumulator
     } else {
+        uint32_t t[SW];
         if (seg_no == 0) {
 #pragma unroll
             for (int c = 0; c < SW; ++c) t[c] = __float_as_uint(__fadd_rn(0.f, __uint_as_float(segv[c])));
@@ -343,7 +419,7 @@ __device__ __forceinline__ void consume_segment_slice(const GemmArgs& a, const U
                 t[c] = __float_as_uint(__fadd_rn(__uint_as_float(prev[c]), __uint_as_float(segv[c])));
         }
         if (seg_no == a.S - 1) {
-            store_slice<FMT, SWAP, BN>(a, un, j, row_lane, t);
+            finish_slice<FMT, SWAP, BN>(a, un, j, e, t);
         } else {
             if constexpr (C::MULTI) tmem_store_slice<SW>(t_total + j * SW, t);
         }
@@ -362,7 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sP = smem;
     uint8_t* sQ = smem + (size_t)STAGES * C::P_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sQ + (size_t)STAGES * C::Q_BYTES);
+    float* s_col = reinterpret_cast<float*>(smem + C::SCALE_OFF);
+    float* b_col = s_col + 256;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
     const uint32_t full0 = smem_u32(bars);
     const uint32_t empty0 = smem_u32(bars + STAGES);
     const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
@@ -373,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    if (warp == 4 && lane == 0) {
+    if (warp == kProducerWarp && lane == 0) {
         prefetch_tmap(&tmap_p);
         prefetch_tmap(&tmap_q);
         for (int s = 0; s < STAGES; ++s) {
@@ -382,11 +460,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
-            mbar_init(tempty0 + 8 * b, 128);
+            mbar_init(tempty0 + 8 * b, kEpiThreads);
         }
         fence_mbarrier_init();
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -394,24 +472,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    pdl_launch_dependents();
 
-    if (warp == 4) {
+    if (warp == kProducerWarp) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t pol_w = policy_evict_first();
             const uint64_t pol_a = policy_evict_last();
-            const uint64_t pol_p = SWAP ? pol_w : pol_a;
-            const uint64_t pol_q = SWAP ? pol_a : pol_w;
+            const CUtensorMap* tm_w = SWAP ? &tmap_p : &tmap_q;
+            const CUtensorMap* tm_a = SWAP ? &tmap_q : &tmap_p;
+            // weights do not depend on the previous kernel: start streaming the
+            // first unit's weight tiles before waiting for it
+            int pre = 0;
+            if ((int)blockIdx.x < args.units) {
+                const Unit un = decode_unit<FMT>(args, blockIdx.x);
+                for (int kb = un.kb0; kb < un.kb1 && pre < STAGES; ++kb, ++pre) {
+                    mbar_arrive_expect_tx(full0 + 8 * pre, C::STAGE_BYTES);
+                    if constexpr (SWAP)
+                        tma_load_2d(smem_u32(sP + (size_t)pre * C::P_BYTES), tm_w, kb * 128, un.pt * 128,
+                                    full0 + 8 * pre, pol_w);
+                    else
+                        tma_load_2d(smem_u32(sQ + (size_t)pre * C::Q_BYTES), tm_w, kb * 128, un.qt * BN,
+                                    full0 + 8 * pre, pol_w);
+                }
+            }
+            pdl_wait();
             uint32_t stage = 0, phase = 0;
+            int it = 0;
             for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
                 const Unit un = decode_unit<FMT>(args, u);
-                for (int kb = un.kb0; kb < un.kb1; ++kb) {
-                    if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) goto done;
-                    mbar_arrive_expect_tx(full0 + 8 * stage, C::STAGE_BYTES);
-                    tma_load_2d(smem_u32(sP + (size_t)stage * C::P_BYTES), &tmap_p, kb * 128, un.pt * 128,
-                                full0 + 8 * stage, pol_p);
-                    tma_load_2d(smem_u32(sQ + (size_t)stage * C::Q_BYTES), &tmap_q, kb * 128, un.qt * BN,
-                                full0 + 8 * stage, pol_q);
+                for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
+                    const uint32_t fb = full0 + 8 * stage;
+                    if (it >= pre) {
+                        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) goto done;
+                        mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+                        if constexpr (SWAP)
+                            tma_load_2d(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_w, kb * 128, un.pt * 128,
+                                        fb, pol_w);
+                        else
+                            tma_load_2d(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_w, kb * 128, un.qt * BN,
+                                        fb, pol_w);
+                    }
+                    if constexpr (SWAP)
+                        tma_load_2d(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_a, kb * 128, un.qt * BN, fb,
+                                    pol_a);
+                    else
+                        tma_load_2d(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_a, kb * 128, un.pt * 128, fb,
+                                    pol_a);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
@@ -419,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // -------------------------------------------------------- MMA issuer
         if (lane == 0) {
             uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
@@ -452,28 +559,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        const int row_lane = warp * 32 + lane;
-        const uint32_t t_lane = tmem_base + ((uint32_t)(warp * 32) << 16);
+        pdl_wait();  // scales are written by the previous kernel; C may be read by it
+        EpiCtx e;
+        e.quad = warp & 3;
+        e.half = warp >> 2;
+        e.lane = lane;
+        e.row_lane = e.quad * 32 + lane;
+        e.s_col = smem_u32(s_col);
+        e.b_col = smem_u32(b_col);
+        e.staging = smem_u32(smem + C::STAGING_OFF) + warp * 2048;
+        e.has_bias = args.bias != nullptr;
+        e.row_scale = 0.f;
+        e.row_bias = 0.f;
+        const uint32_t t_lane = tmem_base + ((uint32_t)(e.quad * 32) << 16);
         const uint32_t t_total = t_lane + C::TOTAL_COL;
         uint32_t abuf = 0, aphase = 0;
         for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
             const Unit un = decode_unit<FMT>(args, u);
+            if constexpr (!C::BLOCK) {
+                // stage the tile's column scales (and bias) once; row values in registers
+                named_bar_sync(1, kEpiThreads);
+                for (int c = threadIdx.x; c < BN; c += kEpiThreads) {
+                    const int q = un.qt * BN + c;
+                    if constexpr (!SWAP) {
+                        s_col[c] = q < args.N ? __ldg(args.s_w + q) : 0.f;
+                        b_col[c] = (e.has_bias && q < args.N) ? bf16_to_f32(__ldg(args.bias + q)) : 0.f;
+                    } else {
+                        s_col[c] = q < args.M ? __ldg(args.s_a + q) : 0.f;
+                    }
+                }
+                if constexpr (!SWAP) {
+                    const int m = un.pt * 128 + e.row_lane;
+                    e.row_scale = m < args.M ? __ldg(args.s_a + m) : 0.f;
+                } else {
+                    const int n = un.pt * 128 + e.row_lane;
+                    e.row_scale = n < args.N ? __ldg(args.s_w + n) : 0.f;
+                    e.row_bias = (e.has_bias && n < args.N) ? bf16_to_f32(__ldg(args.bias + n)) : 0.f;
+                }
+                named_bar_sync(1, kEpiThreads);
+            }
             const int nchunks = (un.kb1 - un.kb0) / un.chunk_kb;
             if (nchunks == 1 && !C::BLOCK) {
-                // one accumulator holds the whole unit: stream it slice by slice
+                // one accumulator holds the whole unit: stream this warp's slices
                 if (!mbar_wait(tfull0 + 8 * abuf, aphase)) goto done;
                 tc_fence_after();
                 const uint32_t tacc = t_lane + abuf * C::ACC_COLS;
+                if (e.half >= C::NSLICE) {  // no slice for this warp: hand the buffer back
+                    tc_fence_before();
+                    mbar_arrive(tempty0 + 8 * abuf);
+                }
 #pragma unroll 1
-                for (int j = 0; j < C::NSLICE; ++j) {
+                for (int j = e.half; j < C::NSLICE; j += 2) {
                     uint32_t v[SW];
                     tmem_load_slice<SW>(tacc + j * SW, v);
                     tc_wait_ld();
-                    if (j == C::NSLICE - 1) {  // accumulator fully read: hand it back
+                    if (j + 2 >= C::NSLICE) {  // this warp's last read of the accumulator
                         tc_fence_before();
                         mbar_arrive(tempty0 + 8 * abuf);
                     }
-                    consume_segment_slice<FMT, SWAP, BN>(args, un, un.seg, j, row_lane, t_total, v);
+                    consume_segment_slice<FMT, SWAP, BN>(args, un, un.seg, j, t_total, e, v);
                 }
                 abuf ^= 1;
                 if (abuf == 0) aphase ^= 1;
@@ -481,44 +625,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if constexpr (C::BLOCK) {
                     // Block-FP8: promote every 128-wide K block into the fp32
                     // segment sum: seg = fma(P_kb, s_a[m,kb] * s_w[n/128,kb], seg)
-                    float seg[BN];
+                    float seg[C::MY_SLICES * SW];
                     for (int c0 = un.kb0; c0 < un.kb1; ++c0) {
                         const int rel = c0 - (args.spread ? un.kb0 : 0);
                         const int seg_no = args.spread ? un.seg : rel / args.kb_per_seg;
                         const bool seg_start = (rel % args.kb_per_seg) == 0;
                         const bool seg_end = ((rel + 1) % args.kb_per_seg) == 0;
-                        float row_scale = 0.f, swv;
+                        float row_scale = 0.f;
+                        float colscale[(BN + 31) / 32];  // Swap-AB: lane l holds columns l, l+32
                         if constexpr (!SWAP) {
-                            const int m = un.pt * 128 + row_lane;
-                            swv = __ldg(args.s_w + (size_t)((un.qt * BN) >> 7) * args.kblocks + c0);
-                            if (m < args.M) row_scale = __fmul_rn(__ldg(args.s_a + (size_t)m * args.kblocks + c0), swv);
+                            const int m = un.pt * 128 + e.row_lane;
+                            const float swv = __ldg(args.s_w + (size_t)((un.qt * BN) >> 7) * args.kblocks + c0);
+                            if (m < args.M)
+                                row_scale = __fmul_rn(__ldg(args.s_a + (size_t)m * args.kblocks + c0), swv);
                         } else {
-                            swv = __ldg(args.s_w + (size_t)un.pt * args.kblocks + c0);
+                            const float swv = __ldg(args.s_w + (size_t)un.pt * args.kblocks + c0);
+#pragma unroll
+                            for (int i = 0; i < (BN + 31) / 32; ++i) {
+                                const int cc = i * 32 + lane;
+                                const int m = un.qt * BN + cc;
+                                colscale[i] = (cc < BN && m < args.M)
+                                                  ? __fmul_rn(__ldg(args.s_a + (size_t)m * args.kblocks + c0), swv)
+                                                  : 0.f;
+                            }
                         }
                         if (seg_start) {
 #pragma unroll
-                            for (int c = 0; c < BN; ++c) seg[c] = 0.f;
+                            for (int c = 0; c < C::MY_SLICES * SW; ++c) seg[c] = 0.f;
                         }
                         if (!mbar_wait(tfull0 + 8 * abuf, aphase)) goto done;
                         tc_fence_after();
                         const uint32_t tacc = t_lane + abuf * C::ACC_COLS;
 #pragma unroll
-                        for (int j = 0; j < C::NSLICE; ++j) {
-                            uint32_t v[SW];
-                            tmem_load_slice<SW>(tacc + j * SW, v);
-                            tc_wait_ld();
+                        for (int js = 0; js < C::MY_SLICES; ++js) {
+                            const int j = 2 * js + e.half;
+                            if (j < C::NSLICE) {
+                                uint32_t v[SW];
+                                tmem_load_slice<SW>(tacc + j * SW, v);
+                                tc_wait_ld();
 #pragma unroll
-                            for (int c = 0; c < SW; ++c) {
-                                float sc;
-                                if constexpr (!SWAP) {
-                                    sc = row_scale;
-                                } else {
-                                    const int m = un.qt * BN + j * SW + c;
-                                    sc = (m < args.M)
-                                             ? __fmul_rn(__ldg(args.s_a + (size_t)m * args.kblocks + c0), swv)
-                                             : 0.f;
+                                for (int c = 0; c < SW; ++c) {
+                                    float sc;
+                                    if constexpr (!SWAP) {
+                                        sc = row_scale;
+                                    } else {
+                                        const int cc = j * SW + c;
+                                        sc = __shfl_sync(0xffffffffu, colscale[cc >> 5], cc & 31);
+                                    }
+                                    seg[js * SW + c] = __fmaf_rn(__uint_as_float(v[c]), sc, seg[js * SW + c]);
                                 }
-                                seg[j * SW + c] = __fmaf_rn(__uint_as_float(v[c]), sc, seg[j * SW + c]);
                             }
                         }
                         tc_fence_before();
@@ -527,11 +682,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (abuf == 0) aphase ^= 1;
                         if (seg_end) {
 #pragma unroll
-                            for (int j = 0; j < C::NSLICE; ++j) {
-                                uint32_t sv[SW];
+                            for (int js = 0; js < C::MY_SLICES; ++js) {
+                                const int j = 2 * js + e.half;
+                                if (j < C::NSLICE) {
+                                    uint32_t sv[SW];
 #pragma unroll
-                                for (int c = 0; c < SW; ++c) sv[c] = __float_as_uint(seg[j * SW + c]);
-                                consume_segment_slice<FMT, SWAP, BN>(args, un, seg_no, j, row_lane, t_total, sv);
+                                    for (int c = 0; c < SW; ++c) sv[c] = __float_as_uint(seg[js * SW + c]);
+                                    consume_segment_slice<FMT, SWAP, BN>(args, un, seg_no, j, t_total, e, sv);
+                                }
                             }
                             tc_wait_st();
                         }
@@ -545,11 +703,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_after();
                         const uint32_t tacc = t_lane + abuf * C::ACC_COLS;
 #pragma unroll 1
-                        for (int j = 0; j < C::NSLICE; ++j) {
+                        for (int j = e.half; j < C::NSLICE; j += 2) {
                             uint32_t v[SW];
                             tmem_load_slice<SW>(tacc + j * SW, v);
                             tc_wait_ld();
-                            consume_segment_slice<FMT, SWAP, BN>(args, un, seg_no, j, row_lane, t_total, v);
+                            consume_segment_slice<FMT, SWAP, BN>(args, un, seg_no, j, t_total, e, v);
                         }
                         tc_wait_st();
                         tc_fence_before();
@@ -559,14 +717,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (args.spread) splitk_finish<FMT, SWAP, BN>(args, un, row_lane, bcast);
+            if (args.spread) splitk_finish<FMT, SWAP, BN>(args, un, e, bcast);
         }
     }
 done:
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 5) tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if (warp == kMmaWarp) tmem_dealloc(tmem_base, C::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------ host side
@@ -583,7 +741,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// K-major 8-bit operand [rows, K] as a 2-D tensor map with a (128 B x box_rows) box.
+// K-major 8-bit operand [rows, K] as a 2-D tensor map with a (128 B x box_rows)
+// box, 128-byte swizzle (the layout the MMA descriptors describe).
 bool make_operand_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -601,7 +760,6 @@ template <int FMT, bool SWAP, int BN>
 qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaStream_t st) {
     using C = Cfg<FMT, SWAP, BN>;
     auto kern = qlin_gemm_kernel<FMT, SWAP, BN>;
-    // one attribute set per device is enough; repeating it is cheap and safe
     static int configured_device = -1;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return QLIN_ERR_CUDA;
@@ -632,8 +790,19 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     a.units = (int)plan.units;
     a.spread = plan.spread ? 1 : 0;
     a.out_i32 = ops.out_i32 ? 1 : 0;
-    kern<<<plan.grid, kThreads, C::SMEM, st>>>(tp, tq, a);
-    return cudaGetLastError() == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)plan.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = ops.pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tp, tq, a);
+    return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
 }
 
 template <int FMT>
@@ -659,12 +828,12 @@ qlin_status launch_fmt(const GemmPlan& p, const GemmOperands& ops, cudaStream_t 
 
 int gemm_stages_for(int tile_n) {
     const int stage = 128 * 128 + tile_n * 128;
-    const int s = kSmemBudget / stage;
+    const int s = kStageBudget / stage;
     return s > 12 ? 12 : s;
 }
 
 size_t gemm_smem_bytes_for(int tile_n) {
-    return 1024 + (size_t)gemm_stages_for(tile_n) * (128 * 128 + tile_n * 128) + 256;
+    return 1024 + (size_t)gemm_stages_for(tile_n) * (128 * 128 + tile_n * 128) + kStagingBytes + kScaleBytes + 256;
 }
 
 cudaError_t device_status_read_clear(int* value) {

@@ -11,12 +11,16 @@
 namespace qlin {
 
 constexpr int kNumSMsB200 = 148;
+// Split-K tickets live in a fixed-size prefix of the workspace, so that no
+// call's partial tiles ever overlap another call's ticket words.
+constexpr size_t kTicketBytes = 65536;
+constexpr int64_t kMaxSplitTiles = kTicketBytes / 4;
 
 // ---------------------------------------------------------------- quantise
 cudaError_t launch_quantize_per_token(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld, void* q,
-                                      float* s, cudaStream_t st);
+                                      float* s, bool pdl, cudaStream_t st);
 cudaError_t launch_quantize_block(const void* x, int64_t rows, int64_t cols, int64_t ld, int block_rows, void* q,
-                                  float* s, cudaStream_t st);
+                                  float* s, bool pdl, cudaStream_t st);
 
 // ------------------------------------------------------------------- GEMM
 // A fully resolved GEMM launch: which operand feeds the 128-row MMA side
@@ -58,6 +62,7 @@ struct GemmOperands {
     void* c;
     bool out_i32;
     void* workspace;
+    bool pdl;  // launch as a programmatic dependent of the previous kernel
 };
 
 qlin_status launch_gemm(const GemmPlan& plan, const GemmOperands& ops, cudaStream_t st);

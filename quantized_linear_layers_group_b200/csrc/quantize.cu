@@ -20,6 +20,7 @@
 #include <cstdint>
 
 #include "internal.h"
+#include "pdl.cuh"
 
 namespace qlin {
 
@@ -102,6 +103,8 @@ template <int FMT, int VPL>
 __global__ void __launch_bounds__(kQuantWarps * 32)
     quantize_per_token_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                               uint8_t* __restrict__ q, float* __restrict__ s) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
     if (row >= rows) return;
@@ -137,6 +140,8 @@ template <int FMT>
 __global__ void __launch_bounds__(kQuantWarps * 32)
     quantize_per_token_long_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                                    uint8_t* __restrict__ q, float* __restrict__ s) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
     if (row >= rows) return;
@@ -161,6 +166,8 @@ template <int VPL>
 __global__ void __launch_bounds__(kQuantWarps * 32)
     quantize_group128_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                              uint8_t* __restrict__ q, float* __restrict__ s) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
     if (row >= rows) return;
@@ -205,6 +212,8 @@ __global__ void __launch_bounds__(256)
     quantize_block128_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                              uint8_t* __restrict__ q, float* __restrict__ s) {
     __shared__ float warp_max[8];
+    pdl_wait();
+    pdl_launch_dependents();
     const int t = threadIdx.x;
     const int64_t br = blockIdx.y, bc = blockIdx.x;
     const int64_t nbc = cols >> 7;
@@ -235,58 +244,62 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Launch with the programmatic-stream-serialization attribute when `pdl`.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, bool pdl, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <int FMT>
 cudaError_t launch_per_token_fmt(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* q, float* s,
-                                 cudaStream_t st) {
+                                 bool pdl, cudaStream_t st) {
     const int64_t nvec = cols >> 3;
     const dim3 grid((unsigned)((rows + kQuantWarps - 1) / kQuantWarps)), block(kQuantWarps * 32);
-    if (nvec <= 32)
-        quantize_per_token_kernel<FMT, 1><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
-    else if (nvec <= 64)
-        quantize_per_token_kernel<FMT, 2><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
-    else if (nvec <= 128)
-        quantize_per_token_kernel<FMT, 4><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
-    else if (nvec <= 256)
-        quantize_per_token_kernel<FMT, 8><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
-    else if (nvec <= 512)
-        quantize_per_token_kernel<FMT, 16><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
-    else if (nvec <= 768)
-        quantize_per_token_kernel<FMT, 24><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
-    else if (nvec <= 1024)
-        quantize_per_token_kernel<FMT, 32><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
-    else
-        quantize_per_token_long_kernel<FMT><<<grid, block, 0, st>>>(x, rows, cols, ld, q, s);
-    return cudaGetLastError();
+    if (nvec <= 32) return launch_k(quantize_per_token_kernel<FMT, 1>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (nvec <= 64) return launch_k(quantize_per_token_kernel<FMT, 2>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (nvec <= 128) return launch_k(quantize_per_token_kernel<FMT, 4>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (nvec <= 256) return launch_k(quantize_per_token_kernel<FMT, 8>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (nvec <= 512)
+        return launch_k(quantize_per_token_kernel<FMT, 16>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (nvec <= 768)
+        return launch_k(quantize_per_token_kernel<FMT, 24>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (nvec <= 1024)
+        return launch_k(quantize_per_token_kernel<FMT, 32>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    return launch_k(quantize_per_token_long_kernel<FMT>, grid, block, pdl, st, x, rows, cols, ld, q, s);
 }
 
 }  // namespace
 
 cudaError_t launch_quantize_per_token(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld, void* q,
-                                      float* s, cudaStream_t st) {
+                                      float* s, bool pdl, cudaStream_t st) {
     const auto* xb = static_cast<const uint16_t*>(x);
     auto* qb = static_cast<uint8_t*>(q);
-    if (fmt == QLIN_FMT_INT8) return launch_per_token_fmt<QLIN_FMT_INT8>(xb, rows, cols, ld, qb, s, st);
-    return launch_per_token_fmt<QLIN_FMT_FP8>(xb, rows, cols, ld, qb, s, st);
+    if (fmt == QLIN_FMT_INT8) return launch_per_token_fmt<QLIN_FMT_INT8>(xb, rows, cols, ld, qb, s, pdl, st);
+    return launch_per_token_fmt<QLIN_FMT_FP8>(xb, rows, cols, ld, qb, s, pdl, st);
 }
 
 cudaError_t launch_quantize_block(const void* x, int64_t rows, int64_t cols, int64_t ld, int block_rows, void* q,
-                                  float* s, cudaStream_t st) {
+                                  float* s, bool pdl, cudaStream_t st) {
     const auto* xb = static_cast<const uint16_t*>(x);
     auto* qb = static_cast<uint8_t*>(q);
     if (block_rows == 1) {
         const dim3 grid((unsigned)((rows + kQuantWarps - 1) / kQuantWarps)), block(kQuantWarps * 32);
         const int64_t nvec = cols >> 3;
-        if (nvec <= 64)
-            quantize_group128_kernel<2><<<grid, block, 0, st>>>(xb, rows, cols, ld, qb, s);
-        else if (nvec <= 256)
-            quantize_group128_kernel<8><<<grid, block, 0, st>>>(xb, rows, cols, ld, qb, s);
-        else
-            quantize_group128_kernel<24><<<grid, block, 0, st>>>(xb, rows, cols, ld, qb, s);
-    } else {
-        const dim3 grid((unsigned)(cols >> 7), (unsigned)((rows + 127) / 128));
-        quantize_block128_kernel<<<grid, 256, 0, st>>>(xb, rows, cols, ld, qb, s);
+        if (nvec <= 64) return launch_k(quantize_group128_kernel<2>, grid, block, pdl, st, xb, rows, cols, ld, qb, s);
+        if (nvec <= 256) return launch_k(quantize_group128_kernel<8>, grid, block, pdl, st, xb, rows, cols, ld, qb, s);
+        return launch_k(quantize_group128_kernel<24>, grid, block, pdl, st, xb, rows, cols, ld, qb, s);
     }
-    return cudaGetLastError();
+    const dim3 grid((unsigned)(cols >> 7), (unsigned)((rows + 127) / 128));
+    return launch_k(quantize_block128_kernel, grid, dim3(256), pdl, st, xb, rows, cols, ld, qb, s);
 }
 
 }  // namespace qlin

@@ -47,39 +47,44 @@ def quantize_weight(fmt: int, weight: torch.Tensor, stream=None):
     return w_q, s_w
 
 
-def quantize_activation(fmt: int, x: torch.Tensor, stream=None):
+def quantize_activation(fmt: int, x: torch.Tensor, stream=None, flags: int = 0):
     """Dynamic activation quantisation; returns (a_q uint8 [M, K], s_a fp32)."""
     M, K = x.shape
     a_q = torch.empty(M, K, dtype=torch.uint8, device=x.device)
     if fmt == qlin.QLIN_FMT_FP8_BLOCK:
         s_a = torch.empty(M, K // 128, dtype=torch.float32, device=x.device)
-        qlin.qlin_quantize_block(x, 1, a_q, s_a, stream)
+        qlin.qlin_quantize_block(x, 1, a_q, s_a, stream, flags=flags)
     else:
         s_a = torch.empty(M, dtype=torch.float32, device=x.device)
-        qlin.qlin_quantize_per_token(fmt, x, a_q, s_a, stream)
+        qlin.qlin_quantize_per_token(fmt, x, a_q, s_a, stream, flags=flags)
     return a_q, s_a
 
 
 class QuantizedLinear:
     """y = x W^T + b with W8A8 INT8, FP8 per-token/per-channel or Block-FP8 arithmetic."""
 
-    def __init__(self, fmt: int, weight: torch.Tensor, bias: torch.Tensor | None = None, workspace=None):
+    def __init__(self, fmt: int, weight: torch.Tensor, bias: torch.Tensor | None = None, workspace=None,
+                 pdl: bool = True):
         self.fmt = fmt
         self.N, self.K = weight.shape
         self.w_q, self.s_w = quantize_weight(fmt, weight)
+        # the weights are final once this returns, so later launches may read
+        # them early (programmatic dependent launch)
+        torch.cuda.current_stream(weight.device).synchronize()
         self.bias = bias
+        self.flags = qlin.QLIN_PDL if pdl else 0
         self.workspace = workspace if workspace is not None else Workspace(device=weight.device)
 
     def forward(self, x: torch.Tensor, stream=None, variant: int = qlin.QLIN_VAR_AUTO, tile_n: int = 0,
                 k_segments: int = 0, out: torch.Tensor | None = None) -> torch.Tensor:
         assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.shape[1] == self.K
         M = x.shape[0]
-        a_q, s_a = quantize_activation(self.fmt, x, stream)
+        a_q, s_a = quantize_activation(self.fmt, x, stream, self.flags)
         c = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
         nbytes = qlin.qlin_scaled_mm_workspace_size(self.fmt, M, self.N, self.K, variant, tile_n, k_segments)
         ws = self.workspace.ensure(nbytes) if nbytes else None
         qlin.qlin_scaled_mm(self.fmt, a_q, s_a, self.w_q, self.s_w, self.bias, c, ws, stream, variant=variant,
-                            tile_n=tile_n, k_segments=k_segments)
+                            tile_n=tile_n, k_segments=k_segments, flags=self.flags)
         return c
 
     __call__ = forward

@@ -42,6 +42,7 @@ QLIN_VAR_SWAPAB = 3
 QLIN_VAR_SWAPAB_SPLITK = 4
 
 QLIN_OUT_I32ACC = 1
+QLIN_PDL = 2
 
 VARIANT_NAMES = {QLIN_VAR_AUTO: "auto", QLIN_VAR_PLAIN: "plain", QLIN_VAR_SPLITK: "splitk",
                  QLIN_VAR_SWAPAB: "swapab", QLIN_VAR_SWAPAB_SPLITK: "swapab_splitk"}
@@ -72,8 +73,8 @@ if not os.path.exists(LIB_PATH):
 
 lib = ctypes.CDLL(LIB_PATH)
 _vp, _i64, _i32, _u32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint32, ctypes.c_size_t
-lib.qlin_quantize_per_token.argtypes = [_i32, _vp, _i64, _i64, _i64, _vp, _vp, _vp]
-lib.qlin_quantize_block.argtypes = [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp]
+lib.qlin_quantize_per_token.argtypes = [_i32, _vp, _i64, _i64, _i64, _vp, _vp, _u32, _vp]
+lib.qlin_quantize_block.argtypes = [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _u32, _vp]
 lib.qlin_scaled_mm.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _u32, _vp,
                                _sz, _vp]
 lib.qlin_scaled_mm_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, ctypes.POINTER(_sz)]
@@ -115,23 +116,24 @@ def _stream(stream) -> int | None:
 
 
 # ------------------------------------------------------------- entry points
-def qlin_quantize_per_token(fmt: int, x, q_out, scale_out, stream=None, *, rows=None, cols=None, ld_x=None):
+def qlin_quantize_per_token(fmt: int, x, q_out, scale_out, stream=None, *, flags: int = 0, rows=None, cols=None,
+                            ld_x=None):
     """Per-token INT8/FP8 quantisation of bf16 x [rows, cols] into q_out / scale_out."""
     rows = x.shape[0] if rows is None else rows
     cols = x.shape[1] if cols is None else cols
     ld_x = (x.stride(0) if x.dim() == 2 else cols) if ld_x is None else ld_x
-    _check(lib.qlin_quantize_per_token(fmt, _ptr(x), rows, cols, ld_x, _ptr(q_out), _ptr(scale_out),
+    _check(lib.qlin_quantize_per_token(fmt, _ptr(x), rows, cols, ld_x, _ptr(q_out), _ptr(scale_out), flags,
                                        _stream(stream)), "qlin_quantize_per_token")
 
 
-def qlin_quantize_block(x, block_rows: int, q_out, scale_out, stream=None, *, block_cols: int = 128, rows=None,
-                        cols=None, ld_x=None):
+def qlin_quantize_block(x, block_rows: int, q_out, scale_out, stream=None, *, flags: int = 0, block_cols: int = 128,
+                        rows=None, cols=None, ld_x=None):
     """Block-FP8 quantisation (1x128 activation groups or 128x128 weight blocks)."""
     rows = x.shape[0] if rows is None else rows
     cols = x.shape[1] if cols is None else cols
     ld_x = (x.stride(0) if x.dim() == 2 else cols) if ld_x is None else ld_x
     _check(lib.qlin_quantize_block(_ptr(x), rows, cols, ld_x, block_rows, block_cols, _ptr(q_out), _ptr(scale_out),
-                                   _stream(stream)), "qlin_quantize_block")
+                                   flags, _stream(stream)), "qlin_quantize_block")
 
 
 def qlin_scaled_mm_workspace_size(fmt: int, M: int, N: int, K: int, variant: int = QLIN_VAR_AUTO, tile_n: int = 0,

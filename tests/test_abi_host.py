@@ -65,7 +65,7 @@ def test_scaled_mm_rejects_bad_arguments_before_launch(q):
     assert _mm(q, fmt=2, N=320) == q.QLIN_ERR_UNSUPPORTED
     assert _mm(q, M=-1) == q.QLIN_ERR_INVALID_ARG
     assert _mm(q, variant=9) == q.QLIN_ERR_INVALID_ARG
-    assert _mm(q, flags=2) == q.QLIN_ERR_INVALID_ARG
+    assert _mm(q, flags=4) == q.QLIN_ERR_INVALID_ARG
     assert _mm(q, flags=1) == q.QLIN_ERR_INVALID_ARG          # I32 accumulators are INT8 only
     assert _mm(q, fmt=2, bias=16) == q.QLIN_ERR_INVALID_ARG   # Block-FP8 takes no bias
     assert _mm(q, a=None) == q.QLIN_ERR_INVALID_ARG
@@ -77,21 +77,23 @@ def test_scaled_mm_rejects_bad_arguments_before_launch(q):
 
 def test_quantize_rejects_bad_arguments(q):
     L = q.lib
-    assert L.qlin_quantize_per_token(2, 16, 4, 64, 64, 16, 16, None) == q.QLIN_ERR_INVALID_ARG
-    assert L.qlin_quantize_per_token(1, 16, 4, 60, 64, 16, 16, None) == q.QLIN_ERR_ALIGNMENT
-    assert L.qlin_quantize_per_token(1, 16, 4, 64, 32, 16, 16, None) == q.QLIN_ERR_INVALID_ARG
-    assert L.qlin_quantize_per_token(1, 8, 4, 64, 64, 16, 16, None) == q.QLIN_ERR_ALIGNMENT
-    assert L.qlin_quantize_per_token(1, None, 4, 64, 64, 16, 16, None) == q.QLIN_ERR_INVALID_ARG
-    assert L.qlin_quantize_per_token(1, None, 0, 64, 64, None, None, None) == q.QLIN_OK
-    assert L.qlin_quantize_block(16, 4, 256, 256, 2, 128, 16, 16, None) == q.QLIN_ERR_UNSUPPORTED
-    assert L.qlin_quantize_block(16, 4, 256, 256, 1, 64, 16, 16, None) == q.QLIN_ERR_UNSUPPORTED
-    assert L.qlin_quantize_block(16, 4, 200, 200, 1, 128, 16, 16, None) == q.QLIN_ERR_UNSUPPORTED
-    assert L.qlin_quantize_block(16, 4, 256, 256, 1, 128, 16, 17, None) == q.QLIN_ERR_ALIGNMENT
+    assert L.qlin_quantize_per_token(2, 16, 4, 64, 64, 16, 16, 0, None) == q.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_per_token(1, 16, 4, 60, 64, 16, 16, 0, None) == q.QLIN_ERR_ALIGNMENT
+    assert L.qlin_quantize_per_token(1, 16, 4, 64, 32, 16, 16, 0, None) == q.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_per_token(1, 8, 4, 64, 64, 16, 16, 0, None) == q.QLIN_ERR_ALIGNMENT
+    assert L.qlin_quantize_per_token(1, None, 4, 64, 64, 16, 16, 0, None) == q.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_per_token(1, 16, 4, 64, 64, 16, 16, 4, None) == q.QLIN_ERR_INVALID_ARG  # bad flag
+    assert L.qlin_quantize_per_token(1, None, 0, 64, 64, None, None, 0, None) == q.QLIN_OK
+    assert L.qlin_quantize_block(16, 4, 256, 256, 2, 128, 16, 16, 0, None) == q.QLIN_ERR_UNSUPPORTED
+    assert L.qlin_quantize_block(16, 4, 256, 256, 1, 64, 16, 16, 0, None) == q.QLIN_ERR_UNSUPPORTED
+    assert L.qlin_quantize_block(16, 4, 200, 200, 1, 128, 16, 16, 0, None) == q.QLIN_ERR_UNSUPPORTED
+    assert L.qlin_quantize_block(16, 4, 256, 256, 1, 128, 16, 17, 0, None) == q.QLIN_ERR_ALIGNMENT
+    assert L.qlin_quantize_block(16, 4, 256, 256, 1, 128, 16, 16, 8, None) == q.QLIN_ERR_INVALID_ARG
 
 
 def test_workspace_sizes(q):
     # Swap-AB + Split-K, FP8 N=4096 K=2048 M=16: S=4 segments of 32 tiles of 128x16
-    assert q.qlin_scaled_mm_workspace_size(1, 16, 4096, 2048) == 256 + 4 * 32 * 128 * 16 * 4
+    assert q.qlin_scaled_mm_workspace_size(1, 16, 4096, 2048) == 65536 + 4 * 32 * 128 * 16 * 4
     # plain variants need none
     assert q.qlin_scaled_mm_workspace_size(1, 2048, 151936, 2048) == 0
     assert q.qlin_scaled_mm_workspace_size(1, 16, 256, 256, variant=q.QLIN_VAR_PLAIN, tile_n=128,
