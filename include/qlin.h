@@ -191,6 +191,36 @@ QLIN_API qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segm
                            size_t workspace_bytes, qlin_stream_t stream);
 
 /*
+ * qlin_scaled_mm_noalloc -- qlin_scaled_mm for callers that cannot allocate
+ * device memory and so cannot pass a workspace (the paper has no counterpart;
+ * this is a library convenience).  Typical callers: a plugin inside a serving
+ * engine that owns the whole device-memory pool and forbids allocations it
+ * does not make itself, or code reached while a CUDA graph is being captured,
+ * where an allocation is not a capturable operation.
+ *
+ * Same arguments, arithmetic and results as qlin_scaled_mm, without the
+ * workspace: the Split-K ticket words and partial tiles live in a device
+ * array of QLIN_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that
+ * loads the library holds until the process exits.  The entry point allocates
+ * nothing and calls no allocating routine.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Each call clears the ticket words on `stream` before its launch (the
+ *     array keeps the previous call's contents).
+ *   - All calls share the one array: calls whose kernels overlap in time on the
+ *     GPU (e.g. on two streams) race on it and must be avoided.
+ * Errors: as qlin_scaled_mm; QLIN_ERR_WORKSPACE when the resolved configuration
+ * needs more scratch than QLIN_NOALLOC_SCRATCH_BYTES (force a smaller
+ * k_segments or a non-Split-K variant).
+ */
+#define QLIN_NOALLOC_SCRATCH_BYTES (8u << 20) /* 8 MiB: 64 KiB of tickets + partial tiles */
+QLIN_API qlin_status qlin_scaled_mm_noalloc(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N,
+                                            int64_t K, const void* a_q, const float* s_a, const void* w_q,
+                                            const float* s_w, const void* bias, void* c_out, uint32_t flags,
+                                            qlin_stream_t stream);
+
+/*
  * qlin_scaled_mm_workspace_size -- bytes of workspace qlin_scaled_mm needs for
  * the same (fmt, variant, tile_n, k_segments, M, N, K): the Split-K partial
  * tiles plus one ticket word per output tile (0 for the other variants).

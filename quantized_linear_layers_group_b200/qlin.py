@@ -48,9 +48,10 @@ VARIANT_NAMES = {QLIN_VAR_AUTO: "auto", QLIN_VAR_PLAIN: "plain", QLIN_VAR_SPLITK
                  QLIN_VAR_SWAPAB: "swapab", QLIN_VAR_SWAPAB_SPLITK: "swapab_splitk"}
 
 # every symbol include/qlin.h declares
-EXPORTS = ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_scaled_mm_workspace_size",
-           "qlin_dispatch_table_load", "qlin_dispatch_table_clear", "qlin_dispatch_query", "qlin_status_string",
-           "qlin_sync_status", "qlin_abi_version")
+EXPORTS = ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_scaled_mm_noalloc",
+           "qlin_scaled_mm_workspace_size", "qlin_dispatch_table_load", "qlin_dispatch_table_clear",
+           "qlin_dispatch_query", "qlin_status_string", "qlin_sync_status", "qlin_abi_version")
+QLIN_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class qlin_config(ctypes.Structure):
@@ -77,6 +78,8 @@ lib.qlin_quantize_per_token.argtypes = [_i32, _vp, _i64, _i64, _i64, _vp, _vp, _
 lib.qlin_quantize_block.argtypes = [_vp, _i64, _i64, _i64, _i32, _i32, _vp, _vp, _u32, _vp]
 lib.qlin_scaled_mm.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _u32, _vp,
                                _sz, _vp]
+lib.qlin_scaled_mm_noalloc.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       _u32, _vp]
 lib.qlin_scaled_mm_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, ctypes.POINTER(_sz)]
 lib.qlin_dispatch_table_load.argtypes = [ctypes.c_char_p]
 lib.qlin_dispatch_table_clear.argtypes = []
@@ -156,6 +159,18 @@ def qlin_scaled_mm(fmt: int, a_q, s_a, w_q, s_w, bias, c_out, workspace=None, st
     _check(lib.qlin_scaled_mm(fmt, variant, tile_n, k_segments, M, N, K, _ptr(a_q), _ptr(s_a), _ptr(w_q), _ptr(s_w),
                               _ptr(bias), _ptr(c_out), flags, _ptr(workspace), workspace_bytes, _stream(stream)),
            "qlin_scaled_mm")
+
+
+def qlin_scaled_mm_noalloc(fmt: int, a_q, s_a, w_q, s_w, bias, c_out, stream=None, *, variant: int = QLIN_VAR_AUTO,
+                           tile_n: int = 0, k_segments: int = 0, flags: int = 0, M=None, N=None, K=None):
+    """qlin_scaled_mm without a workspace, for callers that cannot allocate
+    device memory: Split-K scratch comes from the library's fixed device array."""
+    M = a_q.shape[0] if M is None else M
+    N = w_q.shape[0] if N is None else N
+    K = a_q.shape[1] if K is None else K
+    _check(lib.qlin_scaled_mm_noalloc(fmt, variant, tile_n, k_segments, M, N, K, _ptr(a_q), _ptr(s_a), _ptr(w_q),
+                                      _ptr(s_w), _ptr(bias), _ptr(c_out), flags, _stream(stream)),
+           "qlin_scaled_mm_noalloc")
 
 
 def qlin_dispatch_table_load(path: str):
