@@ -84,6 +84,31 @@ def quant_bytes(M, K, fmt):
     return 2 * M * K + M * K + (M * (K // 128) if fmt == 2 else M) * 4
 
 
+def measured_traffic(workload, fmt, M, N, K, cfg):
+    """DRAM bytes (read + write) of one GEMM launch from the committed ncu
+    record, or None when there is none for this launch or the kernel source
+    has changed since it was taken."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    src = os.path.join(ROOT, "quantized_linear_layers_group_b200", "csrc", "gemm.cu")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    if rec.get("gemm_source_sha256_16") != sha:
+        return None
+    from quantized_linear_layers_group_b200 import qlin
+
+    for e in rec.get("entries", []):
+        if (e["workload"], e["M"], e["N"], e["K"], e["format"]) == (workload, M, N, K, FMT_NAME[fmt]) and \
+                e["variant"] == qlin.VARIANT_NAMES[cfg["variant"]] and e["tile_n"] == cfg["tile_n"]:
+            return e["dram_read_bytes"] + e["dram_write_bytes"]
+    return None
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons with nvidia-smi during the timed region."""
@@ -370,52 +395,67 @@ def main(argv=None):
         # ---------------------------------------------- device-timed steps
         # Each step is one CUDA graph (the launch sequence of the hot path,
         # as a serving engine replays it); G graphs use different weight
-        # copies so the rotation defeats L2.  Timing events are graph nodes.
+        # copies so the rotation defeats L2.  Events bracket each replay.
         n_graphs = max(1, math.ceil(hp.n_copies / len(ms))) if args.graph else 1
-        ev_sets, graphs = [], []
-        for _ in range(n_graphs):
-            ev = {M: [torch.cuda.Event(enable_timing=True, external=args.graph) for _ in range(3)] for M in ms}
-            ev_sets.append(ev)
-            if args.graph:
+        graphs = []
+        if args.graph:
+            for _ in range(n_graphs):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=stream):
-                    hp.step(stream, ev)
+                    hp.step(stream)
                 graphs.append(g)
         torch.cuda.synchronize()
         for i in range(args.warmup):
             if args.graph:
                 graphs[i % n_graphs].replay()
             else:
-                hp.step(stream, ev_sets[0])
+                hp.step(stream)
         torch.cuda.synchronize()
-        per_m_q = {M: [] for M in ms}
-        per_m_g = {M: [] for M in ms}
         clocks = ClockSampler(local)
         clocks.start()
         time.sleep(0.3)
         barrier(world)
         torch.cuda.synchronize()
-        step_ms = []
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
         for i in range(args.steps):
-            ev = ev_sets[i % n_graphs]
-            s0 = torch.cuda.Event(enable_timing=True)
-            s1 = torch.cuda.Event(enable_timing=True)
-            s0.record(stream)
+            evs[i][0].record(stream)
             if args.graph:
                 graphs[i % n_graphs].replay()
             else:
-                hp.step(stream, ev)
-            s1.record(stream)
-            s1.synchronize()
-            step_ms.append(s0.elapsed_time(s1))
-            for M in ms:
-                per_m_q[M].append(ev[M][0].elapsed_time(ev[M][1]))
-                per_m_g[M].append(ev[M][1].elapsed_time(ev[M][2]))
+                hp.step(stream)
+            evs[i][1].record(stream)
         torch.cuda.synchronize()
+        step_ms = [a.elapsed_time(b) for a, b in evs]
         barrier(world)
         clk = clocks.stop()
         elapsed_s = max_over_ranks(sum(step_ms) / 1e3, world)
         del graphs
+
+        # ------------------------------------------- per-kernel launch times
+        # For each M: a graph of R back-to-back launches of one kernel (the
+        # GEMM rotates weight copies), timed with events on the launching
+        # stream; per-launch time = graph time / R (median of a few replays).
+        per_m_q, per_m_g = {}, {}
+        reps = 8
+        for M in ms:
+            for kind, fn in (("q", hp.launch_quant), ("g", hp.launch_gemm)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for _ in range(reps):
+                        fn(M, stream)
+                for _ in range(2):
+                    g.replay()
+                ts = []
+                for _ in range(5):
+                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    a0.record(stream)
+                    g.replay()
+                    a1.record(stream)
+                    a1.synchronize()
+                    ts.append(a0.elapsed_time(a1) / reps)
+                (per_m_q if kind == "q" else per_m_g)[M] = [statistics.median(ts)]
+                del g
+        torch.cuda.synchronize()
 
         # ------------------------------------------------- end-to-end steps
         for _ in range(2):
@@ -472,7 +512,8 @@ def main(argv=None):
     else:
         roof = {"bound": "hbm", "achieved": abd / tgd / 1e9, "peak": hbm, "unit": "GB/s",
                 "frac": abd / tgd / 1e9 / hbm}
-    roof.update({"traffic": None, "kernel": f"qlin_gemm_kernel M={Md} N={N} K={K} {FMT_NAME[fmt]}",
+    roof.update({"traffic": measured_traffic(workload.name, fmt, Md, N, K, hp.configs[Md]),
+                 "kernel": f"qlin_gemm_kernel M={Md} N={N} K={K} {FMT_NAME[fmt]}",
                  "peak_source": f"{peaks['source']}: " + ("2 x bf16_tflops_sustained (8-bit = 2x bf16 nominal)"
                                                           if bound == "tensor" else "hbm_gbs copy")})
 

@@ -65,7 +65,27 @@ def build(verbose: bool = False, force: bool = False, extra: list[str] | None = 
     return LIB
 
 
+
+
+SWEEP_SRC = os.path.join(HERE, "sweep", "qlin_sweep.cu")
+SWEEP_BIN = os.path.join(HERE, "qlin_sweep")
+
+
+def build_sweep(verbose: bool = False) -> str:
+    """Build the offline dispatch-table sweep (links libqlin.so through the C ABI)."""
+    lib = build(verbose=verbose)
+    if not os.path.exists(SWEEP_BIN) or _stale(SWEEP_BIN, [SWEEP_SRC, lib, os.path.join(INCLUDE, "qlin.h")]):
+        cmd = [NVCC, *ARCH, "-O2", "-std=c++17", "-I", INCLUDE, SWEEP_SRC, "-o", SWEEP_BIN, "-L", HERE, "-lqlin",
+               "-Xlinker", "-rpath,$ORIGIN"]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"nvcc failed:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
+    return SWEEP_BIN
+
+
 if __name__ == "__main__":
     build(verbose="-v" in sys.argv, force="-f" in sys.argv,
           extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None)
     print(LIB)
+    if "--sweep" in sys.argv:
+        print(build_sweep(verbose="-v" in sys.argv))

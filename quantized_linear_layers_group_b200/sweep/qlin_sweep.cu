@@ -1,0 +1,320 @@
+// qlin_sweep.cu -- offline sweep that writes the per-shape dispatch table.
+//
+// The page "Helion in vLLM: A Unified Route to Tunable Linear Kernels"
+// ("Algorithm choice becomes part of tuning") has the GEMM variant chosen per
+// shape by an ahead-of-time search, and "[Kernel][Perf] Add Hopper (SM90) tuned
+// config for batch-invariant persistent matmul" keys such tables by device and
+// M bucket.  This program is that search for this library, over a bounded grid
+// (minutes, not hours):
+//
+//   for each (format, N, K):
+//     for each K segmentation S dividing K/128 (S in {1,2,3,4,6,8}):
+//       for each M bucket: time every variant / tile the library offers,
+//         keep only those whose output is bitwise equal to the plain variant
+//         with the same S (every variant must sum segments in the same order)
+//     pick the S with the smallest summed best time over the buckets (one S
+//     per shape, so results never depend on the batch size), and for each
+//     bucket the fastest variant under that S
+//
+// Timing: a CUDA graph of `iters` launches (each reading a different weight
+// copy, with enough copies that the bytes between two uses of one copy exceed
+// 2x L2), launched with QLIN_PDL as the hot path runs, CUDA events around the
+// graph, median of `reps` replays.
+//
+// Usage: qlin_sweep <out.qlt> [shape ...]   shape = fmt:N:K (fmt int8|fp8|fp8_block)
+// Without shapes it sweeps the five workload shapes.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "qlin.h"
+
+#define CK(x)                                                                                     \
+    do {                                                                                          \
+        cudaError_t e_ = (x);                                                                     \
+        if (e_ != cudaSuccess) {                                                                  \
+            std::fprintf(stderr, "CUDA error %s at %s:%d\n", cudaGetErrorString(e_), __FILE__, __LINE__); \
+            std::exit(2);                                                                         \
+        }                                                                                         \
+    } while (0)
+
+namespace {
+
+struct Shape {
+    int fmt;
+    int64_t N, K;
+};
+
+struct Cand {
+    int variant, tile_n;
+};
+
+const char* fmt_name(int f) { return f == QLIN_FMT_INT8 ? "int8" : (f == QLIN_FMT_FP8 ? "fp8" : "fp8_block"); }
+const char* var_name(int v) {
+    switch (v) {
+        case QLIN_VAR_PLAIN: return "plain";
+        case QLIN_VAR_SPLITK: return "splitk";
+        case QLIN_VAR_SWAPAB: return "swapab";
+        case QLIN_VAR_SWAPAB_SPLITK: return "swapab_splitk";
+    }
+    return "auto";
+}
+
+// Deterministic filler: int8 bytes, or finite e4m3 codes (no 0x7F / 0xFF NaNs).
+__global__ void fill_codes(uint8_t* p, size_t n, uint32_t seed, int e4m3) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        uint32_t h = (uint32_t)i * 2654435761u ^ seed;
+        h ^= h >> 13;
+        h *= 0x5bd1e995u;
+        h ^= h >> 15;
+        uint8_t v = (uint8_t)h;
+        if (e4m3) v = (uint8_t)((v & 0x80) | ((v & 0x7F) % 0x77));  // |code| <= 0x76 (240)
+        p[i] = v;
+    }
+}
+
+__global__ void fill_scales(float* p, size_t n, uint32_t seed) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        uint32_t h = (uint32_t)i * 747796405u + seed;
+        h ^= h >> 16;
+        p[i] = 1e-3f * (1.0f + (float)(h & 1023) / 1024.0f);
+    }
+}
+
+struct Problem {
+    Shape s;
+    int64_t M;
+    uint8_t* a_q = nullptr;
+    float* s_a = nullptr;
+    std::vector<uint8_t*> w_q;
+    std::vector<float*> s_w;
+    uint16_t* c = nullptr;
+    uint16_t* c_ref = nullptr;
+    void* ws = nullptr;
+    size_t ws_bytes = 0;
+};
+
+std::vector<int> segment_choices(int64_t K) {
+    std::vector<int> out;
+    const int kb = (int)(K / 128);
+    for (int s : {1, 2, 3, 4, 6, 8})
+        if (kb % s == 0 && kb / s >= 1) out.push_back(s);
+    return out;
+}
+
+std::vector<Cand> candidates(int fmt, int64_t M) {
+    std::vector<Cand> c;
+    for (int t : {16, 32, 64}) {
+        if (t >= 2 * M && t > 16) continue;  // a tile more than twice M only wastes the narrow side
+        if (M > 64 && t < 64) continue;
+        c.push_back({QLIN_VAR_SWAPAB, t});
+        c.push_back({QLIN_VAR_SWAPAB_SPLITK, t});
+    }
+    if (M >= 16) {
+        for (int t : {128, 256}) {
+            if (fmt == QLIN_FMT_FP8_BLOCK && t == 256) continue;
+            c.push_back({QLIN_VAR_PLAIN, t});
+            c.push_back({QLIN_VAR_SPLITK, t});
+        }
+    }
+    return c;
+}
+
+float time_config(Problem& P, int variant, int tile, int S, int iters, int reps, cudaStream_t st, bool* ok) {
+    *ok = false;
+    size_t need = 0;
+    if (qlin_scaled_mm_workspace_size(P.s.fmt, variant, tile, S, P.M, P.s.N, P.s.K, &need) != QLIN_OK) return -1.f;
+    if (need > P.ws_bytes) return -1.f;
+    const void* bias = nullptr;
+    // correctness / warm-up launch on copy 0
+    if (qlin_scaled_mm(P.s.fmt, variant, tile, S, P.M, P.s.N, P.s.K, P.a_q, P.s_a, P.w_q[0], P.s_w[0], bias, P.c,
+                       QLIN_PDL, P.ws, P.ws_bytes, st) != QLIN_OK)
+        return -1.f;
+    cudaGraph_t graph;
+    cudaGraphExec_t exec;
+    CK(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+    for (int i = 0; i < iters; ++i) {
+        const size_t w = (size_t)(i + 1) % P.w_q.size();
+        if (qlin_scaled_mm(P.s.fmt, variant, tile, S, P.M, P.s.N, P.s.K, P.a_q, P.s_a, P.w_q[w], P.s_w[w], bias,
+                           P.c, QLIN_PDL, P.ws, P.ws_bytes, st) != QLIN_OK) {
+            cudaStreamEndCapture(st, &graph);
+            cudaGraphDestroy(graph);
+            return -1.f;
+        }
+    }
+    CK(cudaStreamEndCapture(st, &graph));
+    CK(cudaGraphInstantiate(&exec, graph, 0));
+    cudaEvent_t e0, e1;
+    CK(cudaEventCreate(&e0));
+    CK(cudaEventCreate(&e1));
+    CK(cudaGraphLaunch(exec, st));
+    std::vector<float> ts;
+    for (int r = 0; r < reps; ++r) {
+        CK(cudaEventRecord(e0, st));
+        CK(cudaGraphLaunch(exec, st));
+        CK(cudaEventRecord(e1, st));
+        CK(cudaEventSynchronize(e1));
+        float ms = 0.f;
+        CK(cudaEventElapsedTime(&ms, e0, e1));
+        ts.push_back(ms * 1000.f / iters);
+    }
+    CK(cudaEventDestroy(e0));
+    CK(cudaEventDestroy(e1));
+    CK(cudaGraphExecDestroy(exec));
+    CK(cudaGraphDestroy(graph));
+    if (qlin_sync_status(st) != QLIN_OK) return -1.f;
+    std::sort(ts.begin(), ts.end());
+    *ok = true;
+    return ts[ts.size() / 2];
+}
+
+bool same_output(Problem& P, int variant, int tile, int S, cudaStream_t st) {
+    if (qlin_scaled_mm(P.s.fmt, variant, tile, S, P.M, P.s.N, P.s.K, P.a_q, P.s_a, P.w_q[0], P.s_w[0], nullptr,
+                       P.c, 0, P.ws, P.ws_bytes, st) != QLIN_OK)
+        return false;
+    CK(cudaStreamSynchronize(st));
+    const size_t bytes = (size_t)P.M * P.s.N * 2;
+    std::vector<uint16_t> a(bytes / 2), b(bytes / 2);
+    CK(cudaMemcpy(a.data(), P.c, bytes, cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(b.data(), P.c_ref, bytes, cudaMemcpyDeviceToHost));
+    return std::memcmp(a.data(), b.data(), bytes) == 0;
+}
+
+}  // namespace
+
+int main(int argc, char** argv) {
+    if (argc < 2) {
+        std::fprintf(stderr, "usage: %s out.qlt [fmt:N:K ...]\n", argv[0]);
+        return 1;
+    }
+    std::vector<Shape> shapes;
+    for (int i = 2; i < argc; ++i) {
+        char f[32];
+        long long n, k;
+        if (std::sscanf(argv[i], "%31[^:]:%lld:%lld", f, &n, &k) != 3) return 1;
+        const std::string fs(f);
+        shapes.push_back({fs == "int8" ? QLIN_FMT_INT8 : (fs == "fp8" ? QLIN_FMT_FP8 : QLIN_FMT_FP8_BLOCK), n, k});
+    }
+    if (shapes.empty())
+        shapes = {{QLIN_FMT_FP8, 4096, 2048},
+                  {QLIN_FMT_FP8_BLOCK, 2048, 6144},
+                  {QLIN_FMT_FP8, 151936, 2048},
+                  {QLIN_FMT_FP8, 12288, 2048},
+                  {QLIN_FMT_INT8, 2048, 2048}};
+    const std::vector<int64_t> buckets = {1, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048};
+    int dev = 0;
+    CK(cudaGetDevice(&dev));
+    cudaDeviceProp prop;
+    CK(cudaGetDeviceProperties(&prop, dev));
+    qlin_dispatch_table_clear();
+    cudaStream_t st;
+    CK(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
+    const size_t l2 = (size_t)prop.l2CacheSize;
+
+    FILE* out = std::fopen(argv[1], "w");
+    if (!out) return 1;
+    std::fprintf(out, "qlin-dispatch 1\n");
+    std::fprintf(out, "device %d %d %d %s\n", prop.multiProcessorCount, prop.major, prop.minor, prop.name);
+    std::fprintf(out, "# written by qlin_sweep; per bucket: fmt N K m_max variant tile_n k_segments\n");
+
+    for (const Shape& s : shapes) {
+        const int64_t M_max = buckets.back();
+        Problem P;
+        P.s = s;
+        const size_t wbytes = (size_t)s.N * s.K;
+        const size_t ncopy = std::max<size_t>(2, (2 * l2 + wbytes - 1) / wbytes + 1);
+        const size_t sw_elems = s.fmt == QLIN_FMT_FP8_BLOCK ? (size_t)((s.N + 127) / 128) * (s.K / 128) : (size_t)s.N;
+        const size_t sa_elems = s.fmt == QLIN_FMT_FP8_BLOCK ? (size_t)M_max * (s.K / 128) : (size_t)M_max;
+        CK(cudaMalloc(&P.a_q, (size_t)M_max * s.K));
+        CK(cudaMalloc(&P.s_a, sa_elems * 4));
+        fill_codes<<<1024, 256, 0, st>>>(P.a_q, (size_t)M_max * s.K, 17u, s.fmt != QLIN_FMT_INT8);
+        fill_scales<<<256, 256, 0, st>>>(P.s_a, sa_elems, 5u);
+        for (size_t i = 0; i < ncopy; ++i) {
+            uint8_t* w;
+            float* sw;
+            CK(cudaMalloc(&w, wbytes));
+            CK(cudaMalloc(&sw, sw_elems * 4));
+            fill_codes<<<2048, 256, 0, st>>>(w, wbytes, 1000u + (uint32_t)i, s.fmt != QLIN_FMT_INT8);
+            fill_scales<<<256, 256, 0, st>>>(sw, sw_elems, 77u);
+            P.w_q.push_back(w);
+            P.s_w.push_back(sw);
+        }
+        CK(cudaMalloc(&P.c, (size_t)M_max * s.N * 2));
+        CK(cudaMalloc(&P.c_ref, (size_t)M_max * s.N * 2));
+        P.ws_bytes = 256u << 20;
+        CK(cudaMalloc(&P.ws, P.ws_bytes));
+        CK(cudaMemsetAsync(P.ws, 0, P.ws_bytes, st));
+        CK(cudaStreamSynchronize(st));
+
+        const std::vector<int> segs = segment_choices(s.K);
+        // best[si][bi] = (time, cand)
+        std::vector<std::vector<std::pair<float, Cand>>> best(segs.size(),
+                                                              std::vector<std::pair<float, Cand>>(buckets.size()));
+        for (size_t si = 0; si < segs.size(); ++si) {
+            const int S = segs[si];
+            for (size_t bi = 0; bi < buckets.size(); ++bi) {
+                P.M = buckets[bi];
+                const int iters = std::max(4, std::min(40, (int)(40 * 64 / std::max<int64_t>(P.M, 64))));
+                // reference output: plain tile 128 with this S (the canonical order)
+                bool have_ref = qlin_scaled_mm(s.fmt, QLIN_VAR_PLAIN, 128, S, P.M, s.N, s.K, P.a_q, P.s_a, P.w_q[0],
+                                               P.s_w[0], nullptr, P.c_ref, 0, P.ws, P.ws_bytes, st) == QLIN_OK;
+                CK(cudaStreamSynchronize(st));
+                float bt = 1e30f;
+                Cand bc{0, 0};
+                for (const Cand& c : candidates(s.fmt, P.M)) {
+                    if (S == 1 && (c.variant == QLIN_VAR_SPLITK || c.variant == QLIN_VAR_SWAPAB_SPLITK)) continue;
+                    bool ok = false;
+                    const float t = time_config(P, c.variant, c.tile_n, S, iters, 5, st, &ok);
+                    if (!ok) continue;
+                    const bool same = !have_ref || s.fmt == QLIN_FMT_INT8 || same_output(P, c.variant, c.tile_n, S, st);
+                    std::printf("%s N=%lld K=%lld S=%d M=%lld %-14s tile=%3d  %9.2f us%s\n", fmt_name(s.fmt),
+                                (long long)s.N, (long long)s.K, S, (long long)P.M, var_name(c.variant), c.tile_n, t,
+                                same ? "" : "  (NOT bitwise equal: rejected)");
+                    std::fflush(stdout);
+                    if (same && t < bt) {
+                        bt = t;
+                        bc = c;
+                    }
+                }
+                best[si][bi] = {bt, bc};
+            }
+        }
+        // one segmentation per shape: smallest summed best time over the buckets
+        size_t bs = 0;
+        double bsum = 1e300;
+        for (size_t si = 0; si < segs.size(); ++si) {
+            double sum = 0;
+            for (size_t bi = 0; bi < buckets.size(); ++bi) sum += best[si][bi].first;
+            std::printf("%s N=%lld K=%lld: S=%d total %.2f us\n", fmt_name(s.fmt), (long long)s.N, (long long)s.K,
+                        segs[si], sum);
+            if (sum < bsum) {
+                bsum = sum;
+                bs = si;
+            }
+        }
+        for (size_t bi = 0; bi < buckets.size(); ++bi) {
+            const auto& b = best[bs][bi];
+            if (b.second.variant == 0) continue;
+            std::fprintf(out, "entry %s %lld %lld %lld %s %d %d   # %.2f us\n", fmt_name(s.fmt), (long long)s.N,
+                         (long long)s.K, (long long)buckets[bi], var_name(b.second.variant), b.second.tile_n,
+                         segs[bs], b.first);
+        }
+        std::fflush(out);
+        cudaFree(P.a_q);
+        cudaFree(P.s_a);
+        for (auto p : P.w_q) cudaFree(p);
+        for (auto p : P.s_w) cudaFree(p);
+        cudaFree(P.c);
+        cudaFree(P.c_ref);
+        cudaFree(P.ws);
+    }
+    std::fclose(out);
+    CK(cudaStreamDestroy(st));
+    return 0;
+}
