@@ -118,7 +118,8 @@ qlin_config default_config(int fmt, int64_t M, int64_t N, int64_t K, int num_sms
         const int64_t tiles = ((M + 127) / 128) * ((N + c.tile_n - 1) / c.tile_n);
         c.variant = (c.k_segments > 1 && tiles * 2 <= num_sms) ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN;
     }
-    c.stages = gemm_stages_for(c.tile_n);
+    size_t smem = 0;
+    gemm_kernel_info(fmt, is_swap(c.variant), c.tile_n, &c.stages, &smem);
     return c;
 }
 
@@ -136,7 +137,8 @@ bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, qlin_config* out) {
     out->variant = best->variant;
     out->tile_n = best->tile_n;
     out->k_segments = best->k_segments;
-    out->stages = gemm_stages_for(best->tile_n);
+    size_t smem = 0;
+    gemm_kernel_info(fmt, is_swap(best->variant), best->tile_n, &out->stages, &smem);
     out->m_max = best->m_max;
     out->from_table = 1;
     return true;
@@ -169,7 +171,9 @@ qlin_status resolve_config(int fmt, int variant, int tile_n, int k_segments, int
     }
     if (tile_n) base.tile_n = tile_n;
     if (k_segments) base.k_segments = k_segments;
-    base.stages = gemm_stages_for(base.tile_n);
+    size_t smem = 0;
+    base.stages = 0;
+    gemm_kernel_info(fmt, is_swap(base.variant), base.tile_n, &base.stages, &smem);
     *cfg = base;
     return QLIN_OK;
 }
@@ -216,8 +220,7 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     const bool multi_chunk = (fmt == QLIN_FMT_FP8_BLOCK && (p.spread ? p.kb_per_seg : p.kblocks) > 1) ||
                              (fmt == QLIN_FMT_FP8 && !p.spread && p.k_segments > 1);
     if (multi_chunk && p.tile_n > 128) return QLIN_ERR_UNSUPPORTED;
-    p.stages = gemm_stages_for(p.tile_n);
-    p.smem_bytes = gemm_smem_bytes_for(p.tile_n);
+    if (!gemm_kernel_info(fmt, p.swap, p.tile_n, &p.stages, &p.smem_bytes)) return QLIN_ERR_UNSUPPORTED;
     p.p_rows = p.swap ? N : M;
     p.q_rows = p.swap ? M : N;
     p.p_tiles = (p.p_rows + 127) / 128;
@@ -430,7 +433,13 @@ qlin_status qlin_dispatch_table_load(const char* path) {
         t_name != std::string(prop.name))
         return QLIN_ERR_TABLE_DEVICE;
     for (const auto& e : entries)
-        if (gemm_smem_bytes_for(e.tile_n) > prop.sharedMemPerBlockOptin) return QLIN_ERR_TABLE_FORMAT;
+    for (const auto& e : entries) {
+        int stages = 0;
+        size_t smem = 0;
+        if (!gemm_kernel_info(e.fmt, is_swap(e.variant), e.tile_n, &stages, &smem) ||
+            smem > prop.sharedMemPerBlockOptin)
+            return QLIN_ERR_TABLE_FORMAT;
+    }
     std::sort(entries.begin(), entries.end(), [](const TableEntry& a, const TableEntry& b) {
         if (a.fmt != b.fmt) return a.fmt < b.fmt;
         if (a.N != b.N) return a.N < b.N;

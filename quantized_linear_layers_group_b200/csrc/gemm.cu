@@ -92,19 +92,26 @@ struct Cfg {
     static constexpr int P_BYTES = BM * BK;
     static constexpr int Q_BYTES = BN * BK;
     static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES;
-    static constexpr int STAGES_FIT = kStageBudget / STAGE_BYTES;
+    // Block-FP8: per-unit table of scale products s_a*s_w, [K block][P row or Q column]
+    static constexpr int BS_KB = 48;                           // K blocks per staged window
+    static constexpr int BS_PITCH = (SWAP ? BN : 128) + 1;     // floats; 1 mod 32: no bank conflicts
+    static constexpr int BSCALE_BYTES = BLOCK ? ((BS_KB * BS_PITCH * 4 + 1023) / 1024) * 1024 : 0;
+    static constexpr int STAGES_FIT = (kStageBudget - BSCALE_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
     static constexpr int SW = BN < 32 ? BN : 32;   // columns per TMEM load / per store box
     static constexpr int NSLICE = BN / SW;
     static constexpr int MY_SLICES = (NSLICE + 1) / 2;  // slices per epilogue warp (at most)
     static constexpr int ACC_COLS = BN < 32 ? 32 : BN;
     static constexpr bool MULTI = BN <= 128;       // may run multi-chunk units
-    static constexpr int TOTAL_COL = 2 * ACC_COLS; // running-total region
-    static constexpr int TMEM_COLS = pow2_at_least(2 * ACC_COLS + (MULTI ? ACC_COLS : 0));
+    static constexpr int SEG_COL = 2 * ACC_COLS;   // Block-FP8: running segment sum
+    static constexpr int TOTAL_COL = (BLOCK ? 3 : 2) * ACC_COLS;  // running total over segments
+    static constexpr int TMEM_COLS =
+        pow2_at_least(2 * ACC_COLS + (MULTI ? ACC_COLS : 0) + (BLOCK ? ACC_COLS : 0));
     static constexpr uint32_t IDESC = make_idesc(INT8, 128, BN);
     static constexpr size_t STAGING_OFF = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t SCALE_OFF = STAGING_OFF + kStagingBytes;
-    static constexpr size_t BAR_OFF = SCALE_OFF + kScaleBytes;
+    static constexpr size_t BSCALE_OFF = SCALE_OFF + kScaleBytes;
+    static constexpr size_t BAR_OFF = BSCALE_OFF + BSCALE_BYTES;
     static constexpr size_t SMEM = 1024 + BAR_OFF + 256;
     static_assert(TMEM_COLS <= 512, "TMEM overflow");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
@@ -161,6 +168,21 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
                  : "memory");
     return v;
+}
+
+// Warp-level mbarrier use by the epilogue: one lane polls and the warp then
+// proceeds together; one lane arrives for the whole warp once every lane is
+// done (the barrier counts warps).  256 threads polling or arriving one by
+// one on the same barrier serialise on it.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // Per-thread epilogue context.
@@ -460,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
-            mbar_init(tempty0 + 8 * b, kEpiThreads);
+            mbar_init(tempty0 + 8 * b, kEpiWarps);  // one arrival per epilogue warp
         }
         fence_mbarrier_init();
     }
@@ -573,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         e.row_bias = 0.f;
         const uint32_t t_lane = tmem_base + ((uint32_t)(e.quad * 32) << 16);
         const uint32_t t_total = t_lane + C::TOTAL_COL;
+        const uint32_t t_seg = t_lane + C::SEG_COL;
         uint32_t abuf = 0, aphase = 0;
         for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
             const Unit un = decode_unit<FMT>(args, u);
@@ -601,12 +624,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nchunks = (un.kb1 - un.kb0) / un.chunk_kb;
             if (nchunks == 1 && !C::BLOCK) {
                 // one accumulator holds the whole unit: stream this warp's slices
-                if (!mbar_wait(tfull0 + 8 * abuf, aphase)) goto done;
+                if (!warp_wait(tfull0 + 8 * abuf, aphase)) goto done;
                 tc_fence_after();
                 const uint32_t tacc = t_lane + abuf * C::ACC_COLS;
                 if (e.half >= C::NSLICE) {  // no slice for this warp: hand the buffer back
                     tc_fence_before();
-                    mbar_arrive(tempty0 + 8 * abuf);
+                    warp_arrive(tempty0 + 8 * abuf);
                 }
 #pragma unroll 1
                 for (int j = e.half; j < C::NSLICE; j += 2) {
@@ -615,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_wait_ld();
                     if (j + 2 >= C::NSLICE) {  // this warp's last read of the accumulator
                         tc_fence_before();
-                        mbar_arrive(tempty0 + 8 * abuf);
+                        warp_arrive(tempty0 + 8 * abuf);
                     }
                     consume_segment_slice<FMT, SWAP, BN>(args, un, un.seg, j, t_total, e, v);
                 }
@@ -625,81 +648,97 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if constexpr (C::BLOCK) {
                     // Block-FP8: promote every 128-wide K block into the fp32
                     // segment sum: seg = fma(P_kb, s_a[m,kb] * s_w[n/128,kb], seg)
-                    float seg[C::MY_SLICES * SW];
+                    // The products s_a[m,kb] * s_w[n/128,kb] of a window of up to
+                    // BS_KB K blocks are staged in shared memory, [kb][row] (plain)
+                    // or [kb][column] (Swap-AB), by coalesced cooperative loads.
+                    const uint32_t bsc = smem_u32(smem + C::BSCALE_OFF);
+                    int win0 = -C::BS_KB;
                     for (int c0 = un.kb0; c0 < un.kb1; ++c0) {
                         const int rel = c0 - (args.spread ? un.kb0 : 0);
                         const int seg_no = args.spread ? un.seg : rel / args.kb_per_seg;
                         const bool seg_start = (rel % args.kb_per_seg) == 0;
                         const bool seg_end = ((rel + 1) % args.kb_per_seg) == 0;
-                        float row_scale = 0.f;
-                        float colscale[(BN + 31) / 32];  // Swap-AB: lane l holds columns l, l+32
-                        if constexpr (!SWAP) {
-                            const int m = un.pt * 128 + e.row_lane;
-                            const float swv = __ldg(args.s_w + (size_t)((un.qt * BN) >> 7) * args.kblocks + c0);
-                            if (m < args.M)
-                                row_scale = __fmul_rn(__ldg(args.s_a + (size_t)m * args.kblocks + c0), swv);
-                        } else {
-                            const float swv = __ldg(args.s_w + (size_t)un.pt * args.kblocks + c0);
+                        if (c0 - win0 >= C::BS_KB) {
+                            win0 = c0;
+                            const int kbc = min(C::BS_KB, un.kb1 - win0);
+                            constexpr int NIDX = SWAP ? BN : 128;
+                            const int nb = SWAP ? un.pt : ((un.qt * BN) >> 7);
+                            const int mbase = SWAP ? un.qt * BN : un.pt * 128;
+                            named_bar_sync(1, kEpiThreads);  // the previous window is no longer read
+                            constexpr int BATCH = 8;             // loads in flight per thread
+                            for (int i0 = threadIdx.x; i0 < NIDX * kbc; i0 += kEpiThreads * BATCH) {
+                                float va[BATCH], vw[BATCH];
+                                int off[BATCH];
 #pragma unroll
-                            for (int i = 0; i < (BN + 31) / 32; ++i) {
-                                const int cc = i * 32 + lane;
-                                const int m = un.qt * BN + cc;
-                                colscale[i] = (cc < BN && m < args.M)
-                                                  ? __fmul_rn(__ldg(args.s_a + (size_t)m * args.kblocks + c0), swv)
-                                                  : 0.f;
+                                for (int b = 0; b < BATCH; ++b) {
+                                    const int i = i0 + b * kEpiThreads;
+                                    const int idx = i / kbc, kbl = i - idx * kbc;
+                                    const int m = mbase + idx, kb = win0 + kbl;
+                                    off[b] = -1;
+                                    va[b] = 0.f;
+                                    vw[b] = 0.f;
+                                    if (i < NIDX * kbc) {
+                                        off[b] = kbl * C::BS_PITCH + idx;
+                                        if (m < args.M) {
+                                            va[b] = __ldg(args.s_a + (size_t)m * args.kblocks + kb);
+                                            vw[b] = __ldg(args.s_w + (size_t)nb * args.kblocks + kb);
+                                        }
+                                    }
+                                }
+#pragma unroll
+                                for (int b = 0; b < BATCH; ++b)
+                                    if (off[b] >= 0)
+                                        asm volatile("st.shared.f32 [%0], %1;" ::"r"(bsc + (uint32_t)off[b] * 4u),
+                                                     "f"(__fmul_rn(va[b], vw[b]))
+                                                     : "memory");
                             }
+                            named_bar_sync(1, kEpiThreads);
                         }
-                        if (seg_start) {
-#pragma unroll
-                            for (int c = 0; c < C::MY_SLICES * SW; ++c) seg[c] = 0.f;
-                        }
-                        if (!mbar_wait(tfull0 + 8 * abuf, aphase)) goto done;
+                        const uint32_t bsrow = bsc + (uint32_t)((c0 - win0) * C::BS_PITCH) * 4u;
+                        float row_scale = 0.f;
+                        if constexpr (!SWAP)
+                            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(row_scale) : "r"(bsrow + e.row_lane * 4u));
+                        if (!warp_wait(tfull0 + 8 * abuf, aphase)) goto done;
                         tc_fence_after();
                         const uint32_t tacc = t_lane + abuf * C::ACC_COLS;
+#pragma unroll 1
+                        for (int j = e.half; j < C::NSLICE; j += 2) {
+                            // this K block's accumulator and (after the first block of
+                            // the segment) the segment's running sum, both from TMEM
+                            uint32_t v[SW], sg[SW];
+                            tmem_load_slice<SW>(tacc + j * SW, v);
+                            if (!seg_start) tmem_load_slice<SW>(t_seg + j * SW, sg);
+                            tc_wait_ld();
 #pragma unroll
-                        for (int js = 0; js < C::MY_SLICES; ++js) {
-                            const int j = 2 * js + e.half;
-                            if (j < C::NSLICE) {
-                                uint32_t v[SW];
-                                tmem_load_slice<SW>(tacc + j * SW, v);
-                                tc_wait_ld();
-#pragma unroll
-                                for (int c = 0; c < SW; ++c) {
-                                    float sc;
-                                    if constexpr (!SWAP) {
-                                        sc = row_scale;
-                                    } else {
-                                        const int cc = j * SW + c;
-                                        sc = __shfl_sync(0xffffffffu, colscale[cc >> 5], cc & 31);
-                                    }
-                                    seg[js * SW + c] = __fmaf_rn(__uint_as_float(v[c]), sc, seg[js * SW + c]);
+                            for (int c = 0; c < SW; ++c) {
+                                float sc;
+                                if constexpr (!SWAP) {
+                                    sc = row_scale;
+                                } else {  // column scale, same address for the whole warp
+                                    asm volatile("ld.shared.f32 %0, [%1];"
+                                                 : "=f"(sc)
+                                                 : "r"(bsrow + (uint32_t)(j * SW + c) * 4u));
                                 }
+                                const float prev = seg_start ? 0.f : __uint_as_float(sg[c]);
+                                sg[c] = __float_as_uint(__fmaf_rn(__uint_as_float(v[c]), sc, prev));
                             }
+                            if (seg_end)
+                                consume_segment_slice<FMT, SWAP, BN>(args, un, seg_no, j, t_total, e, sg);
+                            else
+                                tmem_store_slice<SW>(t_seg + j * SW, sg);
                         }
+                        tc_wait_st();
                         tc_fence_before();
-                        mbar_arrive(tempty0 + 8 * abuf);
+                        warp_arrive(tempty0 + 8 * abuf);
                         abuf ^= 1;
                         if (abuf == 0) aphase ^= 1;
-                        if (seg_end) {
-#pragma unroll
-                            for (int js = 0; js < C::MY_SLICES; ++js) {
-                                const int j = 2 * js + e.half;
-                                if (j < C::NSLICE) {
-                                    uint32_t sv[SW];
-#pragma unroll
-                                    for (int c = 0; c < SW; ++c) sv[c] = __float_as_uint(seg[js * SW + c]);
-                                    consume_segment_slice<FMT, SWAP, BN>(args, un, seg_no, j, t_total, e, sv);
-                                }
-                            }
-                            tc_wait_st();
-                        }
                     }
                 } else {
                     // FP8 per-token, plain variant with S > 1: one chunk per
                     // segment, summed into the TMEM running total in order.
                     int seg_no = 0;
                     for (int c0 = un.kb0; c0 < un.kb1; c0 += un.chunk_kb, ++seg_no) {
-                        if (!mbar_wait(tfull0 + 8 * abuf, aphase)) goto done;
+                        if (!warp_wait(tfull0 + 8 * abuf, aphase)) goto done;
                         tc_fence_after();
                         const uint32_t tacc = t_lane + abuf * C::ACC_COLS;
 #pragma unroll 1
@@ -711,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         tc_wait_st();
                         tc_fence_before();
-                        mbar_arrive(tempty0 + 8 * abuf);
+                        warp_arrive(tempty0 + 8 * abuf);
                         abuf ^= 1;
                         if (abuf == 0) aphase ^= 1;
                     }
@@ -826,14 +865,44 @@ qlin_status launch_fmt(const GemmPlan& p, const GemmOperands& ops, cudaStream_t 
 
 }  // namespace
 
-int gemm_stages_for(int tile_n) {
-    const int stage = 128 * 128 + tile_n * 128;
-    const int s = kStageBudget / stage;
-    return s > 12 ? 12 : s;
+namespace {
+template <int FMT, bool SWAP, int BN>
+void cfg_info(int* stages, size_t* smem) {
+    *stages = Cfg<FMT, SWAP, BN>::STAGES;
+    *smem = Cfg<FMT, SWAP, BN>::SMEM;
 }
 
-size_t gemm_smem_bytes_for(int tile_n) {
-    return 1024 + (size_t)gemm_stages_for(tile_n) * (128 * 128 + tile_n * 128) + kStagingBytes + kScaleBytes + 256;
+template <int FMT>
+bool cfg_info_fmt(bool swap, int tile_n, int* stages, size_t* smem) {
+    if (swap) {
+        switch (tile_n) {
+            case 16: cfg_info<FMT, true, 16>(stages, smem); return true;
+            case 32: cfg_info<FMT, true, 32>(stages, smem); return true;
+            case 64: cfg_info<FMT, true, 64>(stages, smem); return true;
+        }
+        return false;
+    }
+    if (tile_n == 128) {
+        cfg_info<FMT, false, 128>(stages, smem);
+        return true;
+    }
+    if constexpr (FMT != QLIN_FMT_FP8_BLOCK) {
+        if (tile_n == 256) {
+            cfg_info<FMT, false, 256>(stages, smem);
+            return true;
+        }
+    }
+    return false;
+}
+}  // namespace
+
+bool gemm_kernel_info(int fmt, bool swap, int tile_n, int* stages, size_t* smem_bytes) {
+    switch (fmt) {
+        case QLIN_FMT_INT8: return cfg_info_fmt<QLIN_FMT_INT8>(swap, tile_n, stages, smem_bytes);
+        case QLIN_FMT_FP8: return cfg_info_fmt<QLIN_FMT_FP8>(swap, tile_n, stages, smem_bytes);
+        case QLIN_FMT_FP8_BLOCK: return cfg_info_fmt<QLIN_FMT_FP8_BLOCK>(swap, tile_n, stages, smem_bytes);
+    }
+    return false;
 }
 
 cudaError_t device_status_read_clear(int* value) {

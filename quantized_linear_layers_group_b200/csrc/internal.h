@@ -49,9 +49,9 @@ struct GemmPlan {
 qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
                            int num_sms, GemmPlan* plan);
 
-// Shared-memory pipeline depth and dynamic smem size for a tile_n.
-int gemm_stages_for(int tile_n);
-size_t gemm_smem_bytes_for(int tile_n);
+// Shared-memory pipeline depth and dynamic smem size of the GEMM kernel
+// instantiation for (fmt, orientation, tile_n); false if none exists.
+bool gemm_kernel_info(int fmt, bool swap, int tile_n, int* stages, size_t* smem_bytes);
 
 struct GemmOperands {
     const void* a_q;

@@ -9,7 +9,8 @@
 //
 // Arithmetic (bit-exact by construction, no fast-math anywhere):
 //   scale = amax / Qmax          IEEE binary32 division (__fdiv_rn)
-//   v     = x / scale            IEEE binary32 division (__fdiv_rn)
+//   v     = x / scale            correctly rounded quotient (Markstein-corrected
+//                                reciprocal, or __fdiv_rn; see quotient())
 //   INT8: q = clamp(rint_half_even(v), -127, 127)
 //   FP8 : q = e4m3_rn_satfinite(clamp(v, -448, 448))
 //   amax == 0 -> scale = 0, q = 0.
@@ -49,13 +50,46 @@ __device__ __forceinline__ float absmax8(const uint4& v) {
     return m;
 }
 
-__device__ __forceinline__ uint32_t quant_int8_x4(const float* f, float s) {
+// The quotient x / s, correctly rounded (IEEE binary32 division) for every x
+// whose code can be non-zero.  One scale serves a whole row (or group), so its
+// reciprocal r = RN(1/s) is formed once and each element takes Markstein's
+// correction step (P. Markstein, "Computation of elementary functions on the
+// IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with
+// q0 = RN(x r) within an ulp of x/s, the residual x - q0 s is exact as an fma
+// and RN(q0 + residual * r) is the correctly rounded quotient, barring
+// underflow or overflow.  For s in [2^-68, 2^92] neither can touch a quotient
+// of magnitude >= 2^-33, and anything smaller than that quantises to a zero
+// code under either rounding; copysign keeps the sign of a zero x.  Other
+// scales use the IEEE division itself.
+struct Divisor {
+    float s, r;
+    bool fast;
+};
+
+__device__ __forceinline__ Divisor make_divisor(float s) {
+    Divisor d;
+    d.s = s;
+    d.fast = (s >= 0x1p-68f && s <= 0x1p92f);
+    d.r = d.fast ? __frcp_rn(s) : 0.f;
+    return d;
+}
+
+__device__ __forceinline__ float quotient(float x, const Divisor& d) {
+    if (d.fast) {
+        const float q0 = __fmul_rn(x, d.r);
+        const float rem = __fmaf_rn(-q0, d.s, x);
+        return copysignf(__fmaf_rn(rem, d.r, q0), x);
+    }
+    return __fdiv_rn(x, d.s);
+}
+
+__device__ __forceinline__ uint32_t quant_int8_x4(const float* f, const Divisor& d) {
     uint32_t out = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         int r = 0;
-        if (s != 0.f) {
-            r = __float2int_rn(__fdiv_rn(f[i], s));
+        if (d.s != 0.f) {
+            r = __float2int_rn(quotient(f[i], d));
             r = max(-127, min(127, r));
         }
         out |= (uint32_t)(r & 0xFF) << (8 * i);
@@ -63,27 +97,27 @@ __device__ __forceinline__ uint32_t quant_int8_x4(const float* f, float s) {
     return out;
 }
 
-__device__ __forceinline__ uint32_t quant_e4m3_x4(const float* f, float s) {
-    if (s == 0.f) return 0u;
+__device__ __forceinline__ uint32_t quant_e4m3_x4(const float* f, const Divisor& d) {
+    if (d.s == 0.f) return 0u;
     float v[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = fminf(fmaxf(__fdiv_rn(f[i], s), -448.f), 448.f);
+    for (int i = 0; i < 4; ++i) v[i] = fminf(fmaxf(quotient(f[i], d), -448.f), 448.f);
     const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v[0], v[1]), __NV_SATFINITE, __NV_E4M3);
     const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(v[2], v[3]), __NV_SATFINITE, __NV_E4M3);
     return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
 template <int FMT>
-__device__ __forceinline__ uint2 quant8(const uint4& v, float s) {
+__device__ __forceinline__ uint2 quant8(const uint4& v, const Divisor& d) {
     float f[8];
     unpack8(v, f);
     uint2 r;
     if constexpr (FMT == QLIN_FMT_INT8) {
-        r.x = quant_int8_x4(f, s);
-        r.y = quant_int8_x4(f + 4, s);
+        r.x = quant_int8_x4(f, d);
+        r.y = quant_int8_x4(f + 4, d);
     } else {
-        r.x = quant_e4m3_x4(f, s);
-        r.y = quant_e4m3_x4(f + 4, s);
+        r.x = quant_e4m3_x4(f, d);
+        r.y = quant_e4m3_x4(f + 4, d);
     }
     return r;
 }
@@ -97,18 +131,24 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 }
 
 // ----------------------------------------------------------------------------
-// Per-token: one warp per row; lane l owns vectors l, l+32, l+64, ... of the
-// row (16 bytes = 8 bf16 each), all held in registers (VPL vectors per lane).
-template <int FMT, int VPL>
+// Per-token: WPR warps per row (WPR = 1, 2 or 8; 8 / WPR rows per 256-thread
+// CTA).  Thread t of a row's group owns vectors t, t + 32*WPR, ... (16 bytes =
+// 8 bf16 each), held in registers (VPL per thread).  The row maximum is a warp
+// shuffle reduction, then (WPR > 1) a reduction over the row's warps through
+// shared memory.
+template <int FMT, int VPL, int WPR>
 __global__ void __launch_bounds__(kQuantWarps * 32)
     quantize_per_token_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                               uint8_t* __restrict__ q, float* __restrict__ s) {
+    __shared__ float warp_max[kQuantWarps];
     pdl_wait();
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
-    if (row >= rows) return;
-    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
+    const int warp = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * (kQuantWarps / WPR) + warp / WPR;
+    const int t = (warp % WPR) * 32 + lane;
+    const bool live = row < rows;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (live ? row : 0) * ld);
     const int nvec = (int)(cols >> 3);
     constexpr float QMAX = (FMT == QLIN_FMT_INT8) ? 127.f : 448.f;
 
@@ -116,26 +156,35 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
     float amax = 0.f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-        const int idx = i * 32 + lane;
-        if (idx < nvec) {
+        const int idx = i * 32 * WPR + t;
+        if (live && idx < nvec) {
             v[i] = ld_stream(xr + idx);
             amax = fmaxf(amax, absmax8(v[i]));
         }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if constexpr (WPR > 1) {
+        if (lane == 0) warp_max[warp] = amax;
+        __syncthreads();
+        const int w0 = (warp / WPR) * WPR;
+#pragma unroll
+        for (int w = 0; w < WPR; ++w) amax = fmaxf(amax, warp_max[w0 + w]);
+    }
+    if (!live) return;
     const float sc = __fdiv_rn(amax, QMAX);
-    if (lane == 0) s[row] = sc;
+    if (t == 0) s[row] = sc;
+    const Divisor dv = make_divisor(sc);
     uint2* qr = reinterpret_cast<uint2*>(q + row * cols);
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-        const int idx = i * 32 + lane;
-        if (idx < nvec) qr[idx] = quant8<FMT>(v[i], sc);
+        const int idx = i * 32 * WPR + t;
+        if (idx < nvec) qr[idx] = quant8<FMT>(v[i], dv);
     }
 }
 
 // Per-token, rows too long to hold in registers: two passes over the row
-// (the second one hits L2).
+// (the second one hits L2), one warp per row.
 template <int FMT>
 __global__ void __launch_bounds__(kQuantWarps * 32)
     quantize_per_token_long_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
@@ -154,34 +203,38 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float sc = __fdiv_rn(amax, QMAX);
     if (lane == 0) s[row] = sc;
+    const Divisor dv = make_divisor(sc);
     uint2* qr = reinterpret_cast<uint2*>(q + row * cols);
-    for (int64_t idx = lane; idx < nvec; idx += 32) qr[idx] = quant8<FMT>(xr[idx], sc);
+    for (int64_t idx = lane; idx < nvec; idx += 32) qr[idx] = quant8<FMT>(xr[idx], dv);
 }
 
 // ----------------------------------------------------------------------------
-// Block-FP8 activations, 1x128 groups: one warp per row.  In step i, lanes
-// 0-15 hold group 2i and lanes 16-31 group 2i+1 (16 vectors x 8 = 128), so the
+// Block-FP8 activations, 1x128 groups: WPR warps per row.  Thread t of the
+// row's group owns vectors t, t + 32*WPR, ...; in each step lanes 0-15 and
+// 16-31 of a warp hold one whole group each (16 vectors x 8 = 128), so the
 // group maximum is a 16-lane shuffle reduction.
-template <int VPL>
+template <int VPL, int WPR>
 __global__ void __launch_bounds__(kQuantWarps * 32)
     quantize_group128_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                              uint8_t* __restrict__ q, float* __restrict__ s) {
     pdl_wait();
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * kQuantWarps + (threadIdx.x >> 5);
+    const int warp = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * (kQuantWarps / WPR) + warp / WPR;
+    const int t = (warp % WPR) * 32 + lane;
     if (row >= rows) return;
     const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
     const int nvec = (int)(cols >> 3);  // multiple of 16
     const int ngroups = (int)(cols >> 7);
     uint2* qr = reinterpret_cast<uint2*>(q + row * cols);
     float* sr = s + row * ngroups;
-    for (int base = 0; base < nvec; base += VPL * 32) {
+    for (int base = 0; base < nvec; base += VPL * 32 * WPR) {
         uint4 v[VPL];
         float gmax[VPL];
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
-            const int idx = base + i * 32 + lane;
+            const int idx = base + i * 32 * WPR + t;
             gmax[i] = 0.f;
             if (idx < nvec) {
                 v[i] = ld_stream(xr + idx);
@@ -195,15 +248,15 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
         }
 #pragma unroll
         for (int i = 0; i < VPL; ++i) {
-            const int idx = base + i * 32 + lane;
+            const int idx = base + i * 32 * WPR + t;
             if (idx < nvec) {
                 const float sc = __fdiv_rn(gmax[i], 448.f);
                 if ((lane & 15) == 0) sr[idx >> 4] = sc;
-                qr[idx] = quant8<QLIN_FMT_FP8>(v[i], sc);
+                const Divisor dv = make_divisor(sc);
+                qr[idx] = quant8<QLIN_FMT_FP8>(v[i], dv);
             }
         }
     }
-    (void)ngroups;
 }
 
 // Block-FP8 weights, 128x128 blocks: one CTA (256 threads) per block.  Thread
@@ -237,10 +290,11 @@ __global__ void __launch_bounds__(256)
     for (int w = 1; w < 8; ++w) amax = fmaxf(amax, warp_max[w]);
     const float sc = __fdiv_rn(amax, 448.f);
     if (t == 0) s[br * nbc + bc] = sc;
+    const Divisor dv = make_divisor(sc);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t r = br * 128 + (t >> 4) + 16 * i;
-        if (r < rows) reinterpret_cast<uint2*>(q + r * cols + bc * 128)[cv] = quant8<QLIN_FMT_FP8>(v[i], sc);
+        if (r < rows) reinterpret_cast<uint2*>(q + r * cols + bc * 128)[cv] = quant8<QLIN_FMT_FP8>(v[i], dv);
     }
 }
 
@@ -259,22 +313,42 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, bool pdl, cu
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// Warps per row: wide rows over few tokens get more threads per row.
+int warps_per_row(int64_t rows) { return rows <= 512 ? 8 : (rows <= 2048 ? 2 : 1); }
+
+template <int FMT, int WPR>
+cudaError_t launch_per_token_wpr(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* q, float* s,
+                                 bool pdl, cudaStream_t st) {
+    const int64_t per_thread = ((cols >> 3) + 32 * WPR - 1) / (32 * WPR);
+    const dim3 grid((unsigned)((rows + (kQuantWarps / WPR) - 1) / (kQuantWarps / WPR))), block(kQuantWarps * 32);
+    if (per_thread <= 1) return launch_k(quantize_per_token_kernel<FMT, 1, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (per_thread <= 2) return launch_k(quantize_per_token_kernel<FMT, 2, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (per_thread <= 4) return launch_k(quantize_per_token_kernel<FMT, 4, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (per_thread <= 8) return launch_k(quantize_per_token_kernel<FMT, 8, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (per_thread <= 16) return launch_k(quantize_per_token_kernel<FMT, 16, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (per_thread <= 32) return launch_k(quantize_per_token_kernel<FMT, 32, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    const dim3 g1((unsigned)((rows + kQuantWarps - 1) / kQuantWarps));
+    return launch_k(quantize_per_token_long_kernel<FMT>, g1, block, pdl, st, x, rows, cols, ld, q, s);
+}
+
 template <int FMT>
 cudaError_t launch_per_token_fmt(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* q, float* s,
                                  bool pdl, cudaStream_t st) {
-    const int64_t nvec = cols >> 3;
-    const dim3 grid((unsigned)((rows + kQuantWarps - 1) / kQuantWarps)), block(kQuantWarps * 32);
-    if (nvec <= 32) return launch_k(quantize_per_token_kernel<FMT, 1>, grid, block, pdl, st, x, rows, cols, ld, q, s);
-    if (nvec <= 64) return launch_k(quantize_per_token_kernel<FMT, 2>, grid, block, pdl, st, x, rows, cols, ld, q, s);
-    if (nvec <= 128) return launch_k(quantize_per_token_kernel<FMT, 4>, grid, block, pdl, st, x, rows, cols, ld, q, s);
-    if (nvec <= 256) return launch_k(quantize_per_token_kernel<FMT, 8>, grid, block, pdl, st, x, rows, cols, ld, q, s);
-    if (nvec <= 512)
-        return launch_k(quantize_per_token_kernel<FMT, 16>, grid, block, pdl, st, x, rows, cols, ld, q, s);
-    if (nvec <= 768)
-        return launch_k(quantize_per_token_kernel<FMT, 24>, grid, block, pdl, st, x, rows, cols, ld, q, s);
-    if (nvec <= 1024)
-        return launch_k(quantize_per_token_kernel<FMT, 32>, grid, block, pdl, st, x, rows, cols, ld, q, s);
-    return launch_k(quantize_per_token_long_kernel<FMT>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    switch (warps_per_row(rows)) {
+        case 8: return launch_per_token_wpr<FMT, 8>(x, rows, cols, ld, q, s, pdl, st);
+        case 2: return launch_per_token_wpr<FMT, 2>(x, rows, cols, ld, q, s, pdl, st);
+        default: return launch_per_token_wpr<FMT, 1>(x, rows, cols, ld, q, s, pdl, st);
+    }
+}
+
+template <int WPR>
+cudaError_t launch_group_wpr(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* q, float* s,
+                             bool pdl, cudaStream_t st) {
+    const int64_t per_thread = ((cols >> 3) + 32 * WPR - 1) / (32 * WPR);
+    const dim3 grid((unsigned)((rows + (kQuantWarps / WPR) - 1) / (kQuantWarps / WPR))), block(kQuantWarps * 32);
+    if (per_thread <= 1) return launch_k(quantize_group128_kernel<1, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (per_thread <= 4) return launch_k(quantize_group128_kernel<4, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    return launch_k(quantize_group128_kernel<8, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
 }
 
 }  // namespace
@@ -292,11 +366,11 @@ cudaError_t launch_quantize_block(const void* x, int64_t rows, int64_t cols, int
     const auto* xb = static_cast<const uint16_t*>(x);
     auto* qb = static_cast<uint8_t*>(q);
     if (block_rows == 1) {
-        const dim3 grid((unsigned)((rows + kQuantWarps - 1) / kQuantWarps)), block(kQuantWarps * 32);
-        const int64_t nvec = cols >> 3;
-        if (nvec <= 64) return launch_k(quantize_group128_kernel<2>, grid, block, pdl, st, xb, rows, cols, ld, qb, s);
-        if (nvec <= 256) return launch_k(quantize_group128_kernel<8>, grid, block, pdl, st, xb, rows, cols, ld, qb, s);
-        return launch_k(quantize_group128_kernel<24>, grid, block, pdl, st, xb, rows, cols, ld, qb, s);
+        switch (warps_per_row(rows)) {
+            case 8: return launch_group_wpr<8>(xb, rows, cols, ld, qb, s, pdl, st);
+            case 2: return launch_group_wpr<2>(xb, rows, cols, ld, qb, s, pdl, st);
+            default: return launch_group_wpr<1>(xb, rows, cols, ld, qb, s, pdl, st);
+        }
     }
     const dim3 grid((unsigned)(cols >> 7), (unsigned)((rows + 127) / 128));
     return launch_k(quantize_block128_kernel, grid, dim3(256), pdl, st, xb, rows, cols, ld, qb, s);

@@ -129,3 +129,54 @@ def test_block128_weights(lib, rows, cols):
     qr, sr = oracle.quantize_block(x, 128, 128)
     _assert_same(qg, sg, qr, sr, f"block128 {rows}x{cols}")
     check_status()
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_INT8, oracle.FMT_FP8])
+def test_per_token_division_across_scale_magnitudes(lib, fmt):
+    # rows whose amax spans 2^-100 .. 2^120 (both sides of the fast-quotient
+    # range of scales), filled with values concentrated near the target grid's
+    # rounding boundaries; codes and scales must equal the oracle's, which
+    # divides with IEEE binary32 division.
+    g = torch.Generator().manual_seed(99)
+    rows, cols = 2048, 136
+    e = torch.linspace(-100, 120, rows)
+    amax = torch.exp2(e.round())[:, None] * (1 + torch.rand(rows, 1, generator=g))
+    qmax = 127.0 if fmt == oracle.FMT_INT8 else 448.0
+    # quotients near half-integers (INT8) / e4m3 midpoints (FP8) and plain random ones
+    u = torch.rand(rows, cols, generator=g)
+    near = (torch.floor(u * qmax) + 0.5) / qmax
+    mix = torch.where(torch.rand(rows, cols, generator=g) < 0.5, near, u)
+    sign = torch.where(torch.rand(rows, cols, generator=g) < 0.5, -1.0, 1.0)
+    x = (sign * mix * amax).to(torch.bfloat16)
+    x[:, 0] = amax[:, 0].to(torch.bfloat16)
+    qg, sg = _gpu_per_token(lib, fmt, x)
+    qr, sr = oracle.quantize_per_token(fmt, x)
+    _assert_same(qg, sg, qr, sr, "division sweep")
+
+
+def test_group128_division_across_scale_magnitudes(lib):
+    g = torch.Generator().manual_seed(7)
+    rows, cols = 512, 1024
+    grp = torch.exp2(torch.randint(-90, 110, (rows, cols // 128), generator=g).float())
+    x = (torch.randn(rows, cols, generator=g) * grp.repeat_interleave(128, dim=1)).to(torch.bfloat16)
+    qg, sg = _gpu_block(lib, x, 1)
+    qr, sr = oracle.quantize_block(x, 1, 128)
+    _assert_same(qg, sg, qr, sr, "group division sweep")
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_INT8, oracle.FMT_FP8])
+@pytest.mark.parametrize("rows", [1, 511, 513, 2049, 4100])
+def test_per_token_every_row_split(lib, fmt, rows):
+    # 8, 2 and 1 warps per row are chosen by the row count: cover each and the edges
+    x = synth.normal((rows, 2048), 1.0, rows)
+    qg, sg = _gpu_per_token(lib, fmt, x)
+    qr, sr = oracle.quantize_per_token(fmt, x)
+    _assert_same(qg, sg, qr, sr, f"rows={rows}")
+
+
+@pytest.mark.parametrize("rows", [1, 600, 3000])
+def test_group128_every_row_split(lib, rows):
+    x = synth.normal((rows, 6144), 2.0, rows + 1)
+    qg, sg = _gpu_block(lib, x, 1)
+    qr, sr = oracle.quantize_block(x, 1, 128)
+    _assert_same(qg, sg, qr, sr, f"group rows={rows}")
