@@ -90,6 +90,14 @@ typedef enum {
  * immediately precedes the call in the stream.  Accepted by every launching
  * entry point. */
 #define QLIN_PDL 2u
+/* Swap-AB Split-K with at most 8 (tile_n 16) or 4 (tile_n 32, 64) segments:
+ * run the S segment CTAs of each tile as one thread-block cluster and reduce
+ * in the shared memory of the first of them, over distributed shared memory,
+ * instead of through the workspace (none is needed then).  Both paths add the
+ * segments in the same order and give bitwise the same C.  Not the default:
+ * in back-to-back launches the clusters start later than single CTAs and the
+ * workspace reduction finishes first.  qlin_scaled_mm only. */
+#define QLIN_SPLITK_CLUSTER 4u
 
 /* A resolved GEMM configuration (what qlin_dispatch_query returns). */
 typedef struct {
@@ -174,9 +182,10 @@ QLIN_API qlin_status qlin_quantize_block(const void* x, int64_t rows, int64_t co
  *   a_q, w_q            int8 / e4m3 [M,K] and [N,K] (device)
  *   bias                bf16 [N] (device) or NULL
  *   c_out               bf16 [M,N] (device); int32 [M,N] with QLIN_OUT_I32ACC
- *   flags               QLIN_OUT_I32ACC (INT8 only) and / or QLIN_PDL
+ *   flags               QLIN_OUT_I32ACC (INT8 only), QLIN_PDL, QLIN_SPLITK_CLUSTER
  *   workspace           device buffer of at least qlin_scaled_mm_workspace_size()
- *                       bytes (may be NULL when that size is 0).  Its first
+ *                       bytes (may be NULL when that size is 0, and for a
+ *                       Split-K run as a cluster).  Its first
  *                       64 KiB hold the Split-K ticket words: they must be
  *                       zero-filled once when the buffer is allocated, and every
  *                       call leaves them at zero again; the rest holds partial
@@ -223,7 +232,8 @@ QLIN_API qlin_status qlin_scaled_mm_noalloc(int fmt, int variant, int tile_n, in
 /*
  * qlin_scaled_mm_workspace_size -- bytes of workspace qlin_scaled_mm needs for
  * the same (fmt, variant, tile_n, k_segments, M, N, K): the Split-K partial
- * tiles plus one ticket word per output tile (0 for the other variants).
+ * tiles plus one ticket word per output tile (0 for the other variants).  A
+ * call with QLIN_SPLITK_CLUSTER that can run as a cluster needs none.
  * Host-only; resolves AUTO through the table exactly as qlin_scaled_mm does.
  * Errors: INVALID_ARG, UNSUPPORTED.
  */

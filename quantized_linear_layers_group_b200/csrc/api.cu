@@ -84,6 +84,10 @@ int parse_variant(const std::string& s) {
 
 bool is_swap(int v) { return v == QLIN_VAR_SWAPAB || v == QLIN_VAR_SWAPAB_SPLITK; }
 bool is_spread(int v) { return v == QLIN_VAR_SPLITK || v == QLIN_VAR_SWAPAB_SPLITK; }
+// Swap-AB Split-K whose segments fit one cluster may reduce through it.
+bool runs_as_cluster(int variant, int tile_n, int S) {
+    return variant == QLIN_VAR_SWAPAB_SPLITK && S > 1 && S <= cluster_split_max(tile_n);
+}
 
 bool tile_supported(int fmt, bool swap, int tile_n) {
     if (swap) return tile_n == 16 || tile_n == 32 || tile_n == 64;
@@ -119,7 +123,7 @@ qlin_config default_config(int fmt, int64_t M, int64_t N, int64_t K, int num_sms
         c.variant = (c.k_segments > 1 && tiles * 2 <= num_sms) ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN;
     }
     size_t smem = 0;
-    gemm_kernel_info(fmt, is_swap(c.variant), c.tile_n, &c.stages, &smem);
+    gemm_kernel_info(fmt, is_swap(c.variant), c.tile_n, false, &c.stages, &smem);
     return c;
 }
 
@@ -138,7 +142,7 @@ bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, qlin_config* out) {
     out->tile_n = best->tile_n;
     out->k_segments = best->k_segments;
     size_t smem = 0;
-    gemm_kernel_info(fmt, is_swap(best->variant), best->tile_n, &out->stages, &smem);
+    gemm_kernel_info(fmt, is_swap(best->variant), best->tile_n, false, &out->stages, &smem);
     out->m_max = best->m_max;
     out->from_table = 1;
     return true;
@@ -173,7 +177,7 @@ qlin_status resolve_config(int fmt, int variant, int tile_n, int k_segments, int
     if (k_segments) base.k_segments = k_segments;
     size_t smem = 0;
     base.stages = 0;
-    gemm_kernel_info(fmt, is_swap(base.variant), base.tile_n, &base.stages, &smem);
+    gemm_kernel_info(fmt, is_swap(base.variant), base.tile_n, false, &base.stages, &smem);
     *cfg = base;
     return QLIN_OK;
 }
@@ -194,7 +198,7 @@ int current_device_sms() {
 }
 
 qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
-                           int num_sms, GemmPlan* plan) {
+                           int num_sms, bool cluster_split, GemmPlan* plan) {
     qlin_status st = check_fmt_shape(fmt, M, N, K);
     if (st != QLIN_OK) return st;
     if (num_sms <= 0) num_sms = kNumSMsB200;
@@ -220,7 +224,8 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     const bool multi_chunk = (fmt == QLIN_FMT_FP8_BLOCK && (p.spread ? p.kb_per_seg : p.kblocks) > 1) ||
                              (fmt == QLIN_FMT_FP8 && !p.spread && p.k_segments > 1);
     if (multi_chunk && p.tile_n > 128) return QLIN_ERR_UNSUPPORTED;
-    if (!gemm_kernel_info(fmt, p.swap, p.tile_n, &p.stages, &p.smem_bytes)) return QLIN_ERR_UNSUPPORTED;
+    p.cluster = p.spread && cluster_split && runs_as_cluster(cfg.variant, p.tile_n, p.k_segments);
+    if (!gemm_kernel_info(fmt, p.swap, p.tile_n, p.cluster, &p.stages, &p.smem_bytes)) return QLIN_ERR_UNSUPPORTED;
     p.p_rows = p.swap ? N : M;
     p.q_rows = p.swap ? M : N;
     p.p_tiles = (p.p_rows + 127) / 128;
@@ -229,9 +234,11 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     p.units = p.num_tiles * (p.spread ? p.k_segments : 1);
     if (p.units > (int64_t)INT32_MAX / 2) return QLIN_ERR_UNSUPPORTED;
     p.grid = (int)std::min<int64_t>(p.units, num_sms);
+    if (p.cluster)  // whole clusters; the launcher also caps them by co-residency
+        p.grid = (int)std::min<int64_t>(p.num_tiles, std::max(1, num_sms / p.k_segments)) * p.k_segments;
     if (p.grid < 1) p.grid = 1;
-    if (p.spread && p.num_tiles > kMaxSplitTiles) return QLIN_ERR_UNSUPPORTED;
-    if (p.spread) {
+    if (p.spread && !p.cluster && p.num_tiles > kMaxSplitTiles) return QLIN_ERR_UNSUPPORTED;
+    if (p.spread && !p.cluster) {
         p.ticket_bytes = kTicketBytes;
         p.workspace_bytes = p.ticket_bytes + (size_t)p.k_segments * p.num_tiles * 128 * p.tile_n * 4;
     } else {
@@ -309,7 +316,7 @@ qlin_status qlin_scaled_mm_workspace_size(int fmt, int variant, int tile_n, int 
         return s;
     }
     GemmPlan p;
-    qlin_status st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, current_device_sms(), &p);
+    qlin_status st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, current_device_sms(), false, &p);
     if (st != QLIN_OK) return st;
     *bytes_out = p.workspace_bytes;
     return QLIN_OK;
@@ -321,7 +328,7 @@ qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int
                            qlin_stream_t stream) {
     qlin_status st = check_fmt_shape(fmt, M, N, K);
     if (st != QLIN_OK) return st;
-    if (flags & ~(QLIN_OUT_I32ACC | QLIN_PDL)) return QLIN_ERR_INVALID_ARG;
+    if (flags & ~(QLIN_OUT_I32ACC | QLIN_PDL | QLIN_SPLITK_CLUSTER)) return QLIN_ERR_INVALID_ARG;
     const bool out_i32 = (flags & QLIN_OUT_I32ACC) != 0;
     if (out_i32 && fmt != QLIN_FMT_INT8) return QLIN_ERR_INVALID_ARG;
     if (fmt == QLIN_FMT_FP8_BLOCK && bias) return QLIN_ERR_INVALID_ARG;
@@ -336,18 +343,18 @@ qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int
     const int sms = current_device_sms();
     if (sms <= 0) return QLIN_ERR_NO_DEVICE;
     GemmPlan p;
-    st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, sms, &p);
+    st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, sms, (flags & QLIN_SPLITK_CLUSTER) != 0, &p);
     if (st != QLIN_OK) return st;
     if (p.workspace_bytes) {
         if (!workspace || workspace_bytes < p.workspace_bytes) return QLIN_ERR_WORKSPACE;
         if (!aligned16(workspace)) return QLIN_ERR_ALIGNMENT;
     }
     if (g_log)
-        std::fprintf(stderr, "[qlin] scaled_mm %s M=%lld N=%lld K=%lld -> %s tile_n=%d S=%d grid=%d\n",
+        std::fprintf(stderr, "[qlin] scaled_mm %s M=%lld N=%lld K=%lld -> %s%s tile_n=%d S=%d grid=%d\n",
                      fmt_name(fmt), (long long)M, (long long)N, (long long)K,
                      variant_name(p.swap ? (p.spread ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB)
                                          : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
-                     p.tile_n, p.k_segments, p.grid);
+                     p.cluster ? " (cluster)" : "", p.tile_n, p.k_segments, p.grid);
     GemmOperands ops{a_q, s_a, w_q, s_w, bias, c_out, out_i32, workspace, (flags & QLIN_PDL) != 0};
     return launch_gemm(p, ops, static_cast<cudaStream_t>(stream));
 }
@@ -420,8 +427,8 @@ qlin_status qlin_dispatch_table_load(const char* path) {
     // every entry must be launchable (validates tile / segmentation / chunking)
     for (const auto& e : entries) {
         GemmPlan p;
-        if (make_gemm_plan(e.fmt, e.variant, e.tile_n, e.k_segments, e.m_max, e.N, e.K, t_sms > 0 ? t_sms : 148, &p) !=
-            QLIN_OK)
+        if (make_gemm_plan(e.fmt, e.variant, e.tile_n, e.k_segments, e.m_max, e.N, e.K, t_sms > 0 ? t_sms : 148, false,
+                           &p) != QLIN_OK)
             return QLIN_ERR_TABLE_FORMAT;
     }
     // device guard: the table must have been measured on this kind of device
@@ -432,11 +439,10 @@ qlin_status qlin_dispatch_table_load(const char* path) {
     if (prop.multiProcessorCount != t_sms || prop.major != t_major || prop.minor != t_minor ||
         t_name != std::string(prop.name))
         return QLIN_ERR_TABLE_DEVICE;
-    for (const auto& e : entries)
     for (const auto& e : entries) {
         int stages = 0;
         size_t smem = 0;
-        if (!gemm_kernel_info(e.fmt, is_swap(e.variant), e.tile_n, &stages, &smem) ||
+        if (!gemm_kernel_info(e.fmt, is_swap(e.variant), e.tile_n, false, &stages, &smem) ||
             smem > prop.sharedMemPerBlockOptin)
             return QLIN_ERR_TABLE_FORMAT;
     }

@@ -26,7 +26,11 @@
 // added in order s = 0..S-1 starting from +0.  The plain variant keeps the
 // running total in a third TMEM region, the Split-K variant writes each
 // segment to a workspace and the last CTA to arrive on the tile's ticket adds
-// them in the same order; so every variant gives bitwise the same C, and a
+// them in the same order (Swap-AB Split-K with few segments instead runs the
+// S segment CTAs of a tile as one thread-block cluster: ranks 1..S-1 store
+// their segments into rank 0's shared memory over the cluster's distributed
+// shared memory and rank 0 adds them in order); so every variant gives
+// bitwise the same C, and a
 // row of C never depends on the other rows.  INT8 sums are exact, so the
 // plain INT8 variant simply accumulates all of K in one TMEM buffer.
 //
@@ -40,6 +44,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -83,8 +88,13 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
     return p;
 }
 
-template <int FMT, bool SWAP, int BN>
+template <int FMT, bool SWAP, int BN, bool CSK = false>
 struct Cfg {
+    // CSK: cluster Split-K (Swap-AB tiles): the K segments of a tile run on the
+    // CTAs of one cluster and are reduced in the leader's shared memory.
+    static_assert(!CSK || SWAP, "cluster Split-K is built for Swap-AB tiles");
+    static constexpr int CSK_MAXS = CSK ? cluster_split_max(BN) : 1;  // segments per cluster
+    static constexpr int RECV_BYTES = CSK ? (CSK_MAXS - 1) * 128 * BN * 4 : 0;
     static constexpr bool INT8 = (FMT == QLIN_FMT_INT8);
     static constexpr bool BLOCK = (FMT == QLIN_FMT_FP8_BLOCK);
     static constexpr int BM = 128;                 // P rows per tile (MMA M)
@@ -96,7 +106,7 @@ struct Cfg {
     static constexpr int BS_KB = 48;                           // K blocks per staged window
     static constexpr int BS_PITCH = (SWAP ? BN : 128) + 1;     // floats; 1 mod 32: no bank conflicts
     static constexpr int BSCALE_BYTES = BLOCK ? ((BS_KB * BS_PITCH * 4 + 1023) / 1024) * 1024 : 0;
-    static constexpr int STAGES_FIT = (kStageBudget - BSCALE_BYTES) / STAGE_BYTES;
+    static constexpr int STAGES_FIT = (kStageBudget - BSCALE_BYTES - RECV_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
     static constexpr int SW = BN < 32 ? BN : 32;   // columns per TMEM load / per store box
     static constexpr int NSLICE = BN / SW;
@@ -111,7 +121,8 @@ struct Cfg {
     static constexpr size_t STAGING_OFF = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t SCALE_OFF = STAGING_OFF + kStagingBytes;
     static constexpr size_t BSCALE_OFF = SCALE_OFF + kScaleBytes;
-    static constexpr size_t BAR_OFF = BSCALE_OFF + BSCALE_BYTES;
+    static constexpr size_t RECV_OFF = BSCALE_OFF + BSCALE_BYTES;
+    static constexpr size_t BAR_OFF = RECV_OFF + RECV_BYTES;
     static constexpr size_t SMEM = 1024 + BAR_OFF + 256;
     static_assert(TMEM_COLS <= 512, "TMEM overflow");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
@@ -194,7 +205,23 @@ struct EpiCtx {
     uint32_t b_col;                  // shared address of the tile's column bias
     uint32_t staging;                // shared address of this warp's 2 KB transpose buffer
     bool has_bias;
+    // cluster Split-K only
+    int rank;                        // CTA rank in the cluster = K segment
+    uint32_t recv;                   // this CTA's receive area (read by rank 0)
+    uint32_t recv_remote;            // rank 0's receive area, cluster address
+    uint32_t recv_full, recv_free;   // local mbarriers
+    uint32_t xphase;                 // phase of the per-tile exchange
 };
+
+// Warp-level wait on an mbarrier that other CTAs of the cluster arrive on.
+// The __syncwarp extends lane 0's acquire to the whole warp.
+__device__ __forceinline__ bool warp_wait_cluster(uint32_t bar, uint32_t parity) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_cluster(bar, parity) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
 
 // Final epilogue of one slice of SW accumulator columns.  `v` holds fp32 bits
 // (FP8 formats: the summed value) or int32 (INT8: the exact accumulator).
@@ -412,18 +439,84 @@ __device__ __forceinline__ void splitk_finish(const GemmArgs& a, const Unit& un,
     if (threadIdx.x == 0) a.tickets[un.tile] = 0;  // leave the ticket zeroed for the next call
 }
 
-// Hand one segment value (slice j, SW columns) to the running sum: Split-K
-// writes it out; the plain variant adds it to the TMEM total (or, on the last
-// segment, finishes the tile).
+// Cluster Split-K: the S CTAs of a cluster hold the S segments of one tile
+// (rank = segment).  Ranks 1..S-1 store their segment values into rank 0's
+// shared memory, [rank-1][slice][SW/4 column groups][128 lanes] 16-byte
+// vectors; rank 0 adds them to its own in segment order, exactly as the
+// workspace Split-K reducer does, and runs the final epilogue.
 template <int FMT, bool SWAP, int BN>
-__device__ __forceinline__ void consume_segment_slice(const GemmArgs& a, const Unit& un, int seg_no, int j,
+__device__ __forceinline__ bool csk_slice(const GemmArgs& a, const Unit& un, int j, EpiCtx& e,
+                                          const uint32_t (&segv)[Cfg<FMT, SWAP, BN>::SW]) {
+    using C = Cfg<FMT, SWAP, BN>;
+    constexpr int SW = C::SW;
+    constexpr uint32_t kGroup = 128u * 16u;  // bytes between column groups
+    if (e.rank != 0) {
+        // the receive slot is free once rank 0 has read the previous tile
+        if (!warp_wait_cluster(e.recv_free, e.xphase ^ 1u)) return false;
+        const uint32_t dst =
+            e.recv_remote + ((uint32_t)((e.rank - 1) * C::NSLICE + j) * (SW / 4)) * kGroup + (uint32_t)e.row_lane * 16u;
+#pragma unroll
+        for (int q = 0; q < SW / 4; ++q)
+            st_cluster_v4(dst + q * kGroup, make_uint4(segv[4 * q], segv[4 * q + 1], segv[4 * q + 2], segv[4 * q + 3]));
+        return true;
+    }
+    if (!warp_wait_cluster(e.recv_full, e.xphase)) return false;
+    uint32_t acc[SW];
+    if constexpr (C::INT8) {
+        int32_t t[SW];
+#pragma unroll
+        for (int c = 0; c < SW; ++c) t[c] = (int32_t)segv[c];
+#pragma unroll 1
+        for (int r = 1; r < a.S; ++r) {
+            const uint32_t src = e.recv + ((uint32_t)((r - 1) * C::NSLICE + j) * (SW / 4)) * kGroup + e.row_lane * 16u;
+#pragma unroll
+            for (int q = 0; q < SW / 4; ++q) {
+                const uint4 w = lds_u4(src + q * kGroup);
+                t[4 * q] += (int32_t)w.x;
+                t[4 * q + 1] += (int32_t)w.y;
+                t[4 * q + 2] += (int32_t)w.z;
+                t[4 * q + 3] += (int32_t)w.w;
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < SW; ++c) acc[c] = (uint32_t)t[c];
+    } else {
+        float t[SW];
+#pragma unroll
+        for (int c = 0; c < SW; ++c) t[c] = __fadd_rn(0.f, __uint_as_float(segv[c]));
+#pragma unroll 1
+        for (int r = 1; r < a.S; ++r) {  // fixed segment order
+            const uint32_t src = e.recv + ((uint32_t)((r - 1) * C::NSLICE + j) * (SW / 4)) * kGroup + e.row_lane * 16u;
+#pragma unroll
+            for (int q = 0; q < SW / 4; ++q) {
+                const uint4 w = lds_u4(src + q * kGroup);
+                t[4 * q] = __fadd_rn(t[4 * q], __uint_as_float(w.x));
+                t[4 * q + 1] = __fadd_rn(t[4 * q + 1], __uint_as_float(w.y));
+                t[4 * q + 2] = __fadd_rn(t[4 * q + 2], __uint_as_float(w.z));
+                t[4 * q + 3] = __fadd_rn(t[4 * q + 3], __uint_as_float(w.w));
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < SW; ++c) acc[c] = __float_as_uint(t[c]);
+    }
+    finish_slice<FMT, SWAP, BN>(a, un, j, e, acc);
+    return true;
+}
+
+// Hand one segment value (slice j, SW columns) to the running sum: Split-K
+// writes it out (workspace, or rank 0's shared memory); the plain variant adds
+// it to the TMEM total (or, on the last segment, finishes the tile).  False
+// only when a bounded wait gave up.
+template <int FMT, bool SWAP, int BN, bool CSK>
+__device__ __forceinline__ bool consume_segment_slice(const GemmArgs& a, const Unit& un, int seg_no, int j,
                                                       uint32_t t_total, EpiCtx& e,
                                                       const uint32_t (&segv)[Cfg<FMT, SWAP, BN>::SW]) {
     using C = Cfg<FMT, SWAP, BN>;
     constexpr int SW = C::SW;
     if (a.spread) {
+        if constexpr (CSK) return csk_slice<FMT, SWAP, BN>(a, un, j, e, segv);
         store_partial<SW>(partial_ptr<SW>(a, un.tile, un.seg, j, C::NSLICE, e.row_lane), segv);
-        return;
+        return true;
     }
     if constexpr (C::INT8) {
         finish_slice<FMT, SWAP, BN>(a, un, j, e, segv);  // exact: whole K in one accumulator
@@ -446,13 +539,14 @@ __device__ __forceinline__ void consume_segment_slice(const GemmArgs& a, const U
             if constexpr (C::MULTI) tmem_store_slice<SW>(t_total + j * SW, t);
         }
     }
+    return true;
 }
 
-template <int FMT, bool SWAP, int BN>
+template <int FMT, bool SWAP, int BN, bool CSK>
 __global__ void __launch_bounds__(kThreads, 1)
     qlin_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ GemmArgs args) {
-    using C = Cfg<FMT, SWAP, BN>;
+    using C = Cfg<FMT, SWAP, BN, CSK>;
     constexpr int STAGES = C::STAGES;
     constexpr int SW = C::SW;
 
@@ -467,7 +561,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t empty0 = smem_u32(bars + STAGES);
     const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
     const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+    const uint32_t recv_full = smem_u32(bars + 2 * STAGES + 4);  // cluster Split-K, rank 0
+    const uint32_t recv_free = smem_u32(bars + 2 * STAGES + 5);  // cluster Split-K, ranks > 0
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
     int* bcast = reinterpret_cast<int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -484,6 +580,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(tfull0 + 8 * b, 1);
             mbar_init(tempty0 + 8 * b, kEpiWarps);  // one arrival per epilogue warp
         }
+        if constexpr (CSK) {
+            mbar_init(recv_full, (args.S - 1) * kEpiWarps);  // every epilogue warp of every other rank
+            mbar_init(recv_free, 1);                         // rank 0's thread 0
+        }
         fence_mbarrier_init();
     }
     if (warp == kMmaWarp) {
@@ -493,6 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if constexpr (CSK) cluster_sync();  // every rank's barriers are initialised before any remote arrive
     const uint32_t tmem_base = *tmem_holder;
     pdl_launch_dependents();
 
@@ -593,6 +694,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         e.has_bias = args.bias != nullptr;
         e.row_scale = 0.f;
         e.row_bias = 0.f;
+        e.rank = 0;
+        e.recv = smem_u32(smem + C::RECV_OFF);
+        e.recv_remote = 0;
+        e.recv_full = recv_full;
+        e.recv_free = recv_free;
+        e.xphase = 0;
+        if constexpr (CSK) {
+            e.rank = (int)cluster_ctarank();
+            e.recv_remote = mapa_shared(e.recv, 0);
+        }
         const uint32_t t_lane = tmem_base + ((uint32_t)(e.quad * 32) << 16);
         const uint32_t t_total = t_lane + C::TOTAL_COL;
         const uint32_t t_seg = t_lane + C::SEG_COL;
@@ -640,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_before();
                         warp_arrive(tempty0 + 8 * abuf);
                     }
-                    consume_segment_slice<FMT, SWAP, BN>(args, un, un.seg, j, t_total, e, v);
+                    if (!consume_segment_slice<FMT, SWAP, BN, CSK>(args, un, un.seg, j, t_total, e, v)) goto done;
                 }
                 abuf ^= 1;
                 if (abuf == 0) aphase ^= 1;
@@ -722,10 +833,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const float prev = seg_start ? 0.f : __uint_as_float(sg[c]);
                                 sg[c] = __float_as_uint(__fmaf_rn(__uint_as_float(v[c]), sc, prev));
                             }
-                            if (seg_end)
-                                consume_segment_slice<FMT, SWAP, BN>(args, un, seg_no, j, t_total, e, sg);
-                            else
+                            if (seg_end) {
+                                if (!consume_segment_slice<FMT, SWAP, BN, CSK>(args, un, seg_no, j, t_total, e, sg))
+                                    goto done;
+                            } else {
                                 tmem_store_slice<SW>(t_seg + j * SW, sg);
+                            }
                         }
                         tc_wait_st();
                         tc_fence_before();
@@ -746,7 +859,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             uint32_t v[SW];
                             tmem_load_slice<SW>(tacc + j * SW, v);
                             tc_wait_ld();
-                            consume_segment_slice<FMT, SWAP, BN>(args, un, seg_no, j, t_total, e, v);
+                            if (!consume_segment_slice<FMT, SWAP, BN, CSK>(args, un, seg_no, j, t_total, e, v))
+                                goto done;
                         }
                         tc_wait_st();
                         tc_fence_before();
@@ -756,7 +870,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (args.spread) splitk_finish<FMT, SWAP, BN>(args, un, e, bcast);
+            if constexpr (CSK) {
+                // per-tile exchange: ranks > 0 tell rank 0 their slices are in
+                // place; rank 0 hands the receive area back once it has read it
+                if (e.rank != 0) {
+                    if (e.half >= C::NSLICE && !warp_wait_cluster(e.recv_free, e.xphase ^ 1u)) goto done;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(mapa_shared(e.recv_full, 0));
+                } else {
+                    // warps without a slice wait too, so that a wait that gives
+                    // up sends every epilogue warp out together
+                    if (e.half >= C::NSLICE && !warp_wait_cluster(e.recv_full, e.xphase)) goto done;
+                    named_bar_sync(1, kEpiThreads);
+                    if (threadIdx.x == 0)
+                        for (int r = 1; r < args.S; ++r) mbar_arrive_remote(mapa_shared(e.recv_free, (uint32_t)r));
+                }
+                e.xphase ^= 1u;
+            } else {
+                if (args.spread) splitk_finish<FMT, SWAP, BN>(args, un, e, bcast);
+            }
         }
     }
 done:
@@ -764,6 +896,9 @@ done:
     __syncthreads();
     tc_fence_after();
     if (warp == kMmaWarp) tmem_dealloc(tmem_base, C::TMEM_COLS);
+    // no CTA leaves while another rank may still arrive on its barriers or
+    // store into its shared memory
+    if constexpr (CSK) cluster_sync();
 }
 
 // ------------------------------------------------------------------ host side
@@ -795,16 +930,20 @@ bool make_operand_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool SWAP, int BN>
+template <int FMT, bool SWAP, int BN, bool CSK>
 qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaStream_t st) {
-    using C = Cfg<FMT, SWAP, BN>;
-    auto kern = qlin_gemm_kernel<FMT, SWAP, BN>;
+    using C = Cfg<FMT, SWAP, BN, CSK>;
+    auto kern = qlin_gemm_kernel<FMT, SWAP, BN, CSK>;
     static int configured_device = -1;
+    static int max_clusters[QLIN_MAX_CLUSTER + 1];  // co-resident clusters per cluster size, this device
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return QLIN_ERR_CUDA;
+    const int S = plan.k_segments;
+    if (CSK && (S < 2 || S > C::CSK_MAXS)) return QLIN_ERR_UNSUPPORTED;
     if (configured_device != dev) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) != cudaSuccess)
             return QLIN_ERR_CUDA;
+        for (int& m : max_clusters) m = -1;
         configured_device = dev;
     }
     alignas(64) CUtensorMap tp, tq;
@@ -817,13 +956,15 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     a.s_w = ops.s_w;
     a.bias = static_cast<const uint16_t*>(ops.bias);
     a.c = ops.c;
-    a.tickets = plan.spread ? static_cast<int32_t*>(ops.workspace) : nullptr;
-    a.partials = plan.spread ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ops.workspace) + plan.ticket_bytes)
-                             : nullptr;
+    const bool global_split = plan.spread && !CSK;
+    a.tickets = global_split ? static_cast<int32_t*>(ops.workspace) : nullptr;
+    a.partials = global_split
+                     ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ops.workspace) + plan.ticket_bytes)
+                     : nullptr;
     a.M = (int)plan.M;
     a.N = (int)plan.N;
     a.kblocks = plan.kblocks;
-    a.S = plan.k_segments;
+    a.S = S;
     a.kb_per_seg = plan.kb_per_seg;
     a.p_tiles = (int)plan.p_tiles;
     a.units = (int)plan.units;
@@ -835,11 +976,33 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int nattr = 0;
+    if (CSK) {
+        attr[nattr].id = cudaLaunchAttributeClusterDimension;
+        attr[nattr].val.clusterDim.x = (unsigned)S;
+        attr[nattr].val.clusterDim.y = 1;
+        attr[nattr].val.clusterDim.z = 1;
+        ++nattr;
+        cfg.attrs = attr;
+        cfg.numAttrs = nattr;
+        if (max_clusters[S] < 0) {
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return QLIN_ERR_CUDA;
+            max_clusters[S] = n;
+        }
+        if (max_clusters[S] < 1) return QLIN_ERR_UNSUPPORTED;
+        // every CTA of a cluster walks the same tiles: grid = clusters x S
+        const int64_t clusters = std::min<int64_t>(plan.num_tiles, max_clusters[S]);
+        cfg.gridDim = dim3((unsigned)(clusters * S));
+    }
+    if (ops.pdl) {
+        attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[nattr].val.programmaticStreamSerializationAllowed = 1;
+        ++nattr;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = ops.pdl ? 1 : 0;
+    cfg.numAttrs = nattr;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tp, tq, a);
     return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
 }
@@ -847,17 +1010,26 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
 template <int FMT>
 qlin_status launch_fmt(const GemmPlan& p, const GemmOperands& ops, cudaStream_t st) {
     if (p.swap) {
+        if (p.cluster) {
+            switch (p.tile_n) {
+                case 16: return launch_instance<FMT, true, 16, true>(p, ops, st);
+                case 32: return launch_instance<FMT, true, 32, true>(p, ops, st);
+                case 64: return launch_instance<FMT, true, 64, true>(p, ops, st);
+                default: return QLIN_ERR_UNSUPPORTED;
+            }
+        }
         switch (p.tile_n) {
-            case 16: return launch_instance<FMT, true, 16>(p, ops, st);
-            case 32: return launch_instance<FMT, true, 32>(p, ops, st);
-            case 64: return launch_instance<FMT, true, 64>(p, ops, st);
+            case 16: return launch_instance<FMT, true, 16, false>(p, ops, st);
+            case 32: return launch_instance<FMT, true, 32, false>(p, ops, st);
+            case 64: return launch_instance<FMT, true, 64, false>(p, ops, st);
             default: return QLIN_ERR_UNSUPPORTED;
         }
     }
+    if (p.cluster) return QLIN_ERR_UNSUPPORTED;
     switch (p.tile_n) {
-        case 128: return launch_instance<FMT, false, 128>(p, ops, st);
+        case 128: return launch_instance<FMT, false, 128, false>(p, ops, st);
         case 256:
-            if constexpr (FMT != QLIN_FMT_FP8_BLOCK) return launch_instance<FMT, false, 256>(p, ops, st);
+            if constexpr (FMT != QLIN_FMT_FP8_BLOCK) return launch_instance<FMT, false, 256, false>(p, ops, st);
             return QLIN_ERR_UNSUPPORTED;
         default: return QLIN_ERR_UNSUPPORTED;
     }
@@ -866,22 +1038,26 @@ qlin_status launch_fmt(const GemmPlan& p, const GemmOperands& ops, cudaStream_t 
 }  // namespace
 
 namespace {
-template <int FMT, bool SWAP, int BN>
+template <int FMT, bool SWAP, int BN, bool CSK = false>
 void cfg_info(int* stages, size_t* smem) {
-    *stages = Cfg<FMT, SWAP, BN>::STAGES;
-    *smem = Cfg<FMT, SWAP, BN>::SMEM;
+    *stages = Cfg<FMT, SWAP, BN, CSK>::STAGES;
+    *smem = Cfg<FMT, SWAP, BN, CSK>::SMEM;
 }
 
 template <int FMT>
-bool cfg_info_fmt(bool swap, int tile_n, int* stages, size_t* smem) {
+bool cfg_info_fmt(bool swap, int tile_n, bool cluster, int* stages, size_t* smem) {
     if (swap) {
         switch (tile_n) {
-            case 16: cfg_info<FMT, true, 16>(stages, smem); return true;
-            case 32: cfg_info<FMT, true, 32>(stages, smem); return true;
-            case 64: cfg_info<FMT, true, 64>(stages, smem); return true;
+            case 16: cluster ? cfg_info<FMT, true, 16, true>(stages, smem) : cfg_info<FMT, true, 16>(stages, smem);
+                     return true;
+            case 32: cluster ? cfg_info<FMT, true, 32, true>(stages, smem) : cfg_info<FMT, true, 32>(stages, smem);
+                     return true;
+            case 64: cluster ? cfg_info<FMT, true, 64, true>(stages, smem) : cfg_info<FMT, true, 64>(stages, smem);
+                     return true;
         }
         return false;
     }
+    if (cluster) return false;
     if (tile_n == 128) {
         cfg_info<FMT, false, 128>(stages, smem);
         return true;
@@ -896,14 +1072,16 @@ bool cfg_info_fmt(bool swap, int tile_n, int* stages, size_t* smem) {
 }
 }  // namespace
 
-bool gemm_kernel_info(int fmt, bool swap, int tile_n, int* stages, size_t* smem_bytes) {
+bool gemm_kernel_info(int fmt, bool swap, int tile_n, bool cluster, int* stages, size_t* smem_bytes) {
     switch (fmt) {
-        case QLIN_FMT_INT8: return cfg_info_fmt<QLIN_FMT_INT8>(swap, tile_n, stages, smem_bytes);
-        case QLIN_FMT_FP8: return cfg_info_fmt<QLIN_FMT_FP8>(swap, tile_n, stages, smem_bytes);
-        case QLIN_FMT_FP8_BLOCK: return cfg_info_fmt<QLIN_FMT_FP8_BLOCK>(swap, tile_n, stages, smem_bytes);
+        case QLIN_FMT_INT8: return cfg_info_fmt<QLIN_FMT_INT8>(swap, tile_n, cluster, stages, smem_bytes);
+        case QLIN_FMT_FP8: return cfg_info_fmt<QLIN_FMT_FP8>(swap, tile_n, cluster, stages, smem_bytes);
+        case QLIN_FMT_FP8_BLOCK:
+            return cfg_info_fmt<QLIN_FMT_FP8_BLOCK>(swap, tile_n, cluster, stages, smem_bytes);
     }
     return false;
 }
+
 
 cudaError_t device_status_read_clear(int* value) {
     cudaError_t e = cudaMemcpyFromSymbol(value, g_device_status, sizeof(int));

@@ -15,6 +15,13 @@ constexpr int kNumSMsB200 = 148;
 // call's partial tiles ever overlap another call's ticket words.
 constexpr size_t kTicketBytes = 65536;
 constexpr int64_t kMaxSplitTiles = kTicketBytes / 4;
+// Cluster Split-K (Swap-AB): the S segments of a tile run on the S CTAs of a
+// thread-block cluster and meet in rank 0's shared memory; the receive area
+// holds S-1 segments, so S is bounded per tile width.
+#define QLIN_MAX_CLUSTER 8
+__host__ __device__ constexpr int cluster_split_max(int tile_n) {
+    return tile_n == 16 ? 8 : (tile_n == 32 || tile_n == 64) ? 4 : 0;
+}
 
 // ---------------------------------------------------------------- quantise
 cudaError_t launch_quantize_per_token(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld, void* q,
@@ -30,6 +37,7 @@ struct GemmPlan {
     int fmt = 0;
     bool swap = false;    // P = W (rows of N), Q = A (rows of M)
     bool spread = false;  // Split-K: one work unit per (tile, segment)
+    bool cluster = false; // Split-K through a thread-block cluster (no workspace)
     int tile_n = 0;       // Q rows per tile (MMA N)
     int k_segments = 1;   // S
     int stages = 0;
@@ -45,13 +53,16 @@ struct GemmPlan {
 };
 
 // Validates the (fmt, tile_n, S, variant) combination and fills the plan.
-// Returns QLIN_OK or an error status; touches no device state.
+// With cluster_split, a Swap-AB Split-K whose S fits one cluster reduces
+// through the cluster instead of the workspace.  Returns QLIN_OK or an error
+// status; touches no device state.
 qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
-                           int num_sms, GemmPlan* plan);
+                           int num_sms, bool cluster_split, GemmPlan* plan);
 
 // Shared-memory pipeline depth and dynamic smem size of the GEMM kernel
-// instantiation for (fmt, orientation, tile_n); false if none exists.
-bool gemm_kernel_info(int fmt, bool swap, int tile_n, int* stages, size_t* smem_bytes);
+// instantiation for (fmt, orientation, tile_n, cluster Split-K); false if none
+// exists.
+bool gemm_kernel_info(int fmt, bool swap, int tile_n, bool cluster, int* stages, size_t* smem_bytes);
 
 struct GemmOperands {
     const void* a_q;

@@ -43,6 +43,7 @@ QLIN_VAR_SWAPAB_SPLITK = 4
 
 QLIN_OUT_I32ACC = 1
 QLIN_PDL = 2
+QLIN_SPLITK_CLUSTER = 4  # Swap-AB Split-K: reduce through a thread-block cluster instead of the workspace
 
 VARIANT_NAMES = {QLIN_VAR_AUTO: "auto", QLIN_VAR_PLAIN: "plain", QLIN_VAR_SPLITK: "splitk",
                  QLIN_VAR_SWAPAB: "swapab", QLIN_VAR_SWAPAB_SPLITK: "swapab_splitk"}

@@ -56,7 +56,7 @@ def gpu_quantize(fmt: int, x_dev: torch.Tensor, is_weight: bool):
 
 
 def gpu_gemm(fmt, a_q, s_a, w_q, s_w, bias_dev, variant=0, tile_n=0, k_segments=0, out_i32=False,
-             workspace=None):
+             workspace=None, flags=0):
     from quantized_linear_layers_group_b200 import qlin
 
     M, K = a_q.shape
@@ -71,7 +71,7 @@ def gpu_gemm(fmt, a_q, s_a, w_q, s_w, bias_dev, variant=0, tile_n=0, k_segments=
         ws = workspace if workspace is not None and workspace.numel() >= nbytes else \
             torch.zeros(nbytes, dtype=torch.uint8, device=a_q.device)
     qlin.qlin_scaled_mm(fmt, a_q, s_a, w_q, s_w, bias_dev, c, ws, variant=variant, tile_n=tile_n,
-                        k_segments=k_segments, flags=qlin.QLIN_OUT_I32ACC if out_i32 else 0)
+                        k_segments=k_segments, flags=flags | (qlin.QLIN_OUT_I32ACC if out_i32 else 0))
     return c
 
 

@@ -65,7 +65,7 @@ def test_scaled_mm_rejects_bad_arguments_before_launch(q):
     assert _mm(q, fmt=2, N=320) == q.QLIN_ERR_UNSUPPORTED
     assert _mm(q, M=-1) == q.QLIN_ERR_INVALID_ARG
     assert _mm(q, variant=9) == q.QLIN_ERR_INVALID_ARG
-    assert _mm(q, flags=4) == q.QLIN_ERR_INVALID_ARG
+    assert _mm(q, flags=8) == q.QLIN_ERR_INVALID_ARG           # undefined flag bit
     assert _mm(q, flags=1) == q.QLIN_ERR_INVALID_ARG          # I32 accumulators are INT8 only
     assert _mm(q, fmt=2, bias=16) == q.QLIN_ERR_INVALID_ARG   # Block-FP8 takes no bias
     assert _mm(q, a=None) == q.QLIN_ERR_INVALID_ARG

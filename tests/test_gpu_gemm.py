@@ -48,9 +48,9 @@ class Prepared:
         return oracle.scaled_mm(self.fmt, self.ra_q, self.rs_a, self.rw_q, self.rs_w, self.b, m_idx=m_idx,
                                 n_idx=n_idx, want_acc=want_acc)
 
-    def run(self, variant=0, tile_n=0, k_segments=0, out_i32=False):
+    def run(self, variant=0, tile_n=0, k_segments=0, out_i32=False, flags=0):
         c = gpu_gemm(self.fmt, self.a_q, self.s_a, self.w_q, self.s_w, self.b_dev, variant, tile_n, k_segments,
-                     out_i32)
+                     out_i32, flags=flags)
         torch.cuda.synchronize()
         return c
 
@@ -115,6 +115,43 @@ def test_variants_bitwise_identical_for_fixed_segmentation(fmt):
         keys = list(outs)
         for k in keys[1:]:
             assert np.array_equal(outs[keys[0]], outs[k]), f"S={s}: {keys[0]} vs {k}"
+
+
+CLUSTER_MAX = {16: 8, 32: 4, 64: 4}
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M,N,K", [(3, 640, 1024), (40, 3072, 3072), (64, 25600, 1024)])
+def test_cluster_splitk_matches_workspace_splitk_and_oracle(fmt, M, N, K):
+    # Swap-AB Split-K through a thread-block cluster (segments reduced in the
+    # shared memory of rank 0) against the workspace reduction: bitwise equal,
+    # and within the parity bar of the oracle.  N=25600 gives every cluster
+    # several tiles (the per-tile exchange runs through many phases); M=40
+    # gives several tiles along M for the narrow tiles.
+    from quantized_linear_layers_group_b200 import qlin
+
+    p = Prepared(fmt, *_problem(fmt, M, N, K, seed=M + N + fmt))
+    rows = np.unique(np.r_[0, M - 1, np.arange(0, M, 5)])
+    ref = p.reference(m_idx=rows)
+    racc = p.reference(m_idx=rows, want_acc=True)[1] if fmt == oracle.FMT_INT8 else None
+    kb = K // 128
+    checked = 0
+    for tile in (16, 32, 64):
+        for s in range(2, CLUSTER_MAX[tile] + 1):
+            if kb % s:
+                continue
+            got = bits_u16(p.run(SWAPAB_SPLITK, tile, s, flags=qlin.QLIN_SPLITK_CLUSTER))
+            want = bits_u16(p.run(SWAPAB_SPLITK, tile, s))
+            assert np.array_equal(got, want), f"cluster vs workspace: fmt={fmt} tile={tile} S={s}"
+            same_s = bits_u16(p.run(PLAIN, 128, s))
+            assert np.array_equal(got, same_s), f"cluster vs plain: fmt={fmt} tile={tile} S={s}"
+            if fmt == oracle.FMT_INT8:
+                acc = p.run(SWAPAB_SPLITK, tile, s, out_i32=True, flags=qlin.QLIN_SPLITK_CLUSTER).cpu().numpy()
+                assert np.array_equal(acc[rows], racc), f"INT8 accumulators tile={tile} S={s}"
+            assert_parity(fmt, got[rows], ref, f"cluster fmt={fmt} M={M} N={N} K={K} tile={tile} S={s}")
+            checked += 1
+    assert checked >= 3
+    check_status()
 
 
 @pytest.mark.parametrize("fmt", FMTS)
