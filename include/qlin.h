@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define QLIN_ABI_VERSION 1
+#define QLIN_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define QLIN_API __attribute__((visibility("default")))
@@ -98,6 +98,12 @@ typedef enum {
  * in back-to-back launches the clusters start later than single CTAs and the
  * workspace reduction finishes first.  qlin_scaled_mm only. */
 #define QLIN_SPLITK_CLUSTER 4u
+/* qlin_linear: where the configuration allows, let the GEMM quantise its own
+ * activation rows (one kernel) instead of running the stand-alone quantiser
+ * first.  Not the default: measured on B200 the in-GEMM quantisation sits on
+ * the MMA's critical path and the two-kernel sequence finishes first for the
+ * per-token formats; for Block-FP8 at M = 1 the one kernel is ~3% faster. */
+#define QLIN_FUSED 8u
 
 /* A resolved GEMM configuration (what qlin_dispatch_query returns). */
 typedef struct {
@@ -228,6 +234,34 @@ QLIN_API qlin_status qlin_scaled_mm_noalloc(int fmt, int variant, int tile_n, in
                                             int64_t K, const void* a_q, const float* s_a, const void* w_q,
                                             const float* s_w, const void* bias, void* c_out, uint32_t flags,
                                             qlin_stream_t stream);
+
+/*
+ * qlin_linear -- the whole quantized linear layer: dynamic activation
+ * quantisation of bf16 x (per token for INT8 / FP8, 1x128 groups for
+ * FP8_BLOCK, exactly as qlin_quantize_per_token / qlin_quantize_block) followed
+ * by qlin_scaled_mm, in one call.  Results -- C, and the codes and scales
+ * written to a_q / s_a -- are bitwise those of the two calls in sequence.
+ *
+ * By default the quantiser runs first and the GEMM is launched as its
+ * programmatic dependent.  With QLIN_FUSED, Swap-AB configurations (small M)
+ * whose work units fit the kernel's resident activation operand (at most 32,
+ * 16 or 8 K blocks of 128 per unit for tile_n 16, 32, 64) run as ONE kernel:
+ * each CTA quantises the bf16 rows of its unit into shared memory itself, so
+ * the codes never make the round trip through HBM before the GEMM reads them
+ * and there is no second launch; other configurations ignore the flag.
+ *
+ *   x          bf16 [M, K] (device), row stride ld_x elements (ld_x >= K, ld_x % 8 == 0)
+ *   a_q, s_a   outputs: the activation codes [M, K] and scales (fp32 [M], or
+ *              [M, K/128] for FP8_BLOCK), as the quantisers write them
+ *   others     as qlin_scaled_mm (workspace: qlin_scaled_mm_workspace_size)
+ *   flags      QLIN_PDL (applies to the first kernel), QLIN_FUSED,
+ *              QLIN_OUT_I32ACC (INT8 only)
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_linear(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
+                                 const void* x, int64_t ld_x, void* a_q, float* s_a, const void* w_q,
+                                 const float* s_w, const void* bias, void* c_out, uint32_t flags, void* workspace,
+                                 size_t workspace_bytes, qlin_stream_t stream);
 
 /*
  * qlin_scaled_mm_workspace_size -- bytes of workspace qlin_scaled_mm needs for

@@ -26,7 +26,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr"]
 SOURCES = ["quantize.cu", "gemm.cu", "api.cu", "noalloc.cu"]
-HEADERS = ["ptx.cuh", "internal.h"]
+HEADERS = ["ptx.cuh", "internal.h", "pdl.cuh", "quant_math.cuh"]
 
 
 def _stale(out: str, deps: list[str]) -> bool:

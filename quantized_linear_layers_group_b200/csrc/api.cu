@@ -123,7 +123,7 @@ qlin_config default_config(int fmt, int64_t M, int64_t N, int64_t K, int num_sms
         c.variant = (c.k_segments > 1 && tiles * 2 <= num_sms) ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN;
     }
     size_t smem = 0;
-    gemm_kernel_info(fmt, is_swap(c.variant), c.tile_n, false, &c.stages, &smem);
+    gemm_kernel_info(fmt, is_swap(c.variant), c.tile_n, kModeStd, &c.stages, &smem);
     return c;
 }
 
@@ -142,7 +142,7 @@ bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, qlin_config* out) {
     out->tile_n = best->tile_n;
     out->k_segments = best->k_segments;
     size_t smem = 0;
-    gemm_kernel_info(fmt, is_swap(best->variant), best->tile_n, false, &out->stages, &smem);
+    gemm_kernel_info(fmt, is_swap(best->variant), best->tile_n, kModeStd, &out->stages, &smem);
     out->m_max = best->m_max;
     out->from_table = 1;
     return true;
@@ -177,7 +177,7 @@ qlin_status resolve_config(int fmt, int variant, int tile_n, int k_segments, int
     if (k_segments) base.k_segments = k_segments;
     size_t smem = 0;
     base.stages = 0;
-    gemm_kernel_info(fmt, is_swap(base.variant), base.tile_n, false, &base.stages, &smem);
+    gemm_kernel_info(fmt, is_swap(base.variant), base.tile_n, kModeStd, &base.stages, &smem);
     *cfg = base;
     return QLIN_OK;
 }
@@ -198,7 +198,7 @@ int current_device_sms() {
 }
 
 qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
-                           int num_sms, bool cluster_split, GemmPlan* plan) {
+                           int num_sms, int want_mode, GemmPlan* plan) {
     qlin_status st = check_fmt_shape(fmt, M, N, K);
     if (st != QLIN_OK) return st;
     if (num_sms <= 0) num_sms = kNumSMsB200;
@@ -224,8 +224,12 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     const bool multi_chunk = (fmt == QLIN_FMT_FP8_BLOCK && (p.spread ? p.kb_per_seg : p.kblocks) > 1) ||
                              (fmt == QLIN_FMT_FP8 && !p.spread && p.k_segments > 1);
     if (multi_chunk && p.tile_n > 128) return QLIN_ERR_UNSUPPORTED;
-    p.cluster = p.spread && cluster_split && runs_as_cluster(cfg.variant, p.tile_n, p.k_segments);
-    if (!gemm_kernel_info(fmt, p.swap, p.tile_n, p.cluster, &p.stages, &p.smem_bytes)) return QLIN_ERR_UNSUPPORTED;
+    p.kb_per_unit = p.spread ? p.kb_per_seg : p.kblocks;
+    p.mode = kModeStd;
+    if (want_mode == kModeCluster && p.spread && runs_as_cluster(cfg.variant, p.tile_n, p.k_segments))
+        p.mode = kModeCluster;
+    if (want_mode == kModeFused && p.swap && p.kb_per_unit <= fused_max_kblocks(p.tile_n)) p.mode = kModeFused;
+    if (!gemm_kernel_info(fmt, p.swap, p.tile_n, p.mode, &p.stages, &p.smem_bytes)) return QLIN_ERR_UNSUPPORTED;
     p.p_rows = p.swap ? N : M;
     p.q_rows = p.swap ? M : N;
     p.p_tiles = (p.p_rows + 127) / 128;
@@ -234,11 +238,12 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     p.units = p.num_tiles * (p.spread ? p.k_segments : 1);
     if (p.units > (int64_t)INT32_MAX / 2) return QLIN_ERR_UNSUPPORTED;
     p.grid = (int)std::min<int64_t>(p.units, num_sms);
-    if (p.cluster)  // whole clusters; the launcher also caps them by co-residency
+    if (p.mode == kModeCluster)  // whole clusters; the launcher also caps them by co-residency
         p.grid = (int)std::min<int64_t>(p.num_tiles, std::max(1, num_sms / p.k_segments)) * p.k_segments;
     if (p.grid < 1) p.grid = 1;
-    if (p.spread && !p.cluster && p.num_tiles > kMaxSplitTiles) return QLIN_ERR_UNSUPPORTED;
-    if (p.spread && !p.cluster) {
+    const bool workspace_split = p.spread && p.mode != kModeCluster;
+    if (workspace_split && p.num_tiles > kMaxSplitTiles) return QLIN_ERR_UNSUPPORTED;
+    if (workspace_split) {
         p.ticket_bytes = kTicketBytes;
         p.workspace_bytes = p.ticket_bytes + (size_t)p.k_segments * p.num_tiles * 128 * p.tile_n * 4;
     } else {
@@ -316,7 +321,7 @@ qlin_status qlin_scaled_mm_workspace_size(int fmt, int variant, int tile_n, int 
         return s;
     }
     GemmPlan p;
-    qlin_status st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, current_device_sms(), false, &p);
+    qlin_status st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, current_device_sms(), kModeStd, &p);
     if (st != QLIN_OK) return st;
     *bytes_out = p.workspace_bytes;
     return QLIN_OK;
@@ -343,7 +348,8 @@ qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int
     const int sms = current_device_sms();
     if (sms <= 0) return QLIN_ERR_NO_DEVICE;
     GemmPlan p;
-    st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, sms, (flags & QLIN_SPLITK_CLUSTER) != 0, &p);
+    st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, sms,
+                        (flags & QLIN_SPLITK_CLUSTER) ? kModeCluster : kModeStd, &p);
     if (st != QLIN_OK) return st;
     if (p.workspace_bytes) {
         if (!workspace || workspace_bytes < p.workspace_bytes) return QLIN_ERR_WORKSPACE;
@@ -354,9 +360,61 @@ qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int
                      fmt_name(fmt), (long long)M, (long long)N, (long long)K,
                      variant_name(p.swap ? (p.spread ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB)
                                          : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
-                     p.cluster ? " (cluster)" : "", p.tile_n, p.k_segments, p.grid);
+                     p.mode == kModeCluster ? " (cluster)" : "", p.tile_n, p.k_segments, p.grid);
     GemmOperands ops{a_q, s_a, w_q, s_w, bias, c_out, out_i32, workspace, (flags & QLIN_PDL) != 0};
     return launch_gemm(p, ops, static_cast<cudaStream_t>(stream));
+}
+
+qlin_status qlin_linear(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
+                        const void* x, int64_t ld_x, void* a_q, float* s_a, const void* w_q, const float* s_w,
+                        const void* bias, void* c_out, uint32_t flags, void* workspace, size_t workspace_bytes,
+                        qlin_stream_t stream) {
+    qlin_status st = check_fmt_shape(fmt, M, N, K);
+    if (st != QLIN_OK) return st;
+    if (flags & ~(QLIN_OUT_I32ACC | QLIN_PDL | QLIN_FUSED)) return QLIN_ERR_INVALID_ARG;
+    const bool out_i32 = (flags & QLIN_OUT_I32ACC) != 0;
+    if (out_i32 && fmt != QLIN_FMT_INT8) return QLIN_ERR_INVALID_ARG;
+    if (fmt == QLIN_FMT_FP8_BLOCK && bias) return QLIN_ERR_INVALID_ARG;
+    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_SWAPAB_SPLITK || tile_n < 0 || k_segments < 0)
+        return QLIN_ERR_INVALID_ARG;
+    if (ld_x < K) return QLIN_ERR_INVALID_ARG;
+    if (M == 0) return QLIN_OK;
+    if (!x || !a_q || !s_a || !w_q || !s_w || !c_out) return QLIN_ERR_INVALID_ARG;
+    if (ld_x % 8 != 0 || !aligned16(x) || !aligned16(a_q) || !aligned16(w_q) || !aligned16(c_out))
+        return QLIN_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(s_a) & 3u) || (reinterpret_cast<uintptr_t>(s_w) & 3u) ||
+        (reinterpret_cast<uintptr_t>(bias) & 1u))
+        return QLIN_ERR_ALIGNMENT;
+    const int sms = current_device_sms();
+    if (sms <= 0) return QLIN_ERR_NO_DEVICE;
+    GemmPlan p;
+    st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, sms,
+                        (flags & QLIN_FUSED) ? kModeFused : kModeStd, &p);
+    if (st != QLIN_OK) return st;
+    if (p.workspace_bytes) {
+        if (!workspace || workspace_bytes < p.workspace_bytes) return QLIN_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return QLIN_ERR_ALIGNMENT;
+    }
+    const bool pdl = (flags & QLIN_PDL) != 0;
+    const auto cst = static_cast<cudaStream_t>(stream);
+    if (g_log)
+        std::fprintf(stderr, "[qlin] linear %s M=%lld N=%lld K=%lld -> %s%s tile_n=%d S=%d grid=%d\n", fmt_name(fmt),
+                     (long long)M, (long long)N, (long long)K,
+                     variant_name(p.swap ? (p.spread ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB)
+                                         : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
+                     p.mode == kModeFused ? " (fused)" : "", p.tile_n, p.k_segments, p.grid);
+    if (p.mode == kModeFused) {
+        GemmOperands ops{a_q, s_a, w_q, s_w, bias, c_out, out_i32, workspace, pdl, x, ld_x};
+        return launch_gemm(p, ops, cst);
+    }
+    // two kernels: the quantiser, then the GEMM as its programmatic dependent
+    // (the quantiser writes neither the weights nor anything the GEMM's
+    // early weight prefetch reads)
+    cudaError_t e = fmt == QLIN_FMT_FP8_BLOCK ? launch_quantize_block(x, M, K, ld_x, 1, a_q, s_a, pdl, cst)
+                                              : launch_quantize_per_token(fmt, x, M, K, ld_x, a_q, s_a, pdl, cst);
+    if (e != cudaSuccess) return QLIN_ERR_CUDA;
+    GemmOperands ops{a_q, s_a, w_q, s_w, bias, c_out, out_i32, workspace, true};
+    return launch_gemm(p, ops, cst);
 }
 
 qlin_status qlin_dispatch_query(int fmt, int64_t M, int64_t N, int64_t K, qlin_config* out) {
@@ -427,8 +485,8 @@ qlin_status qlin_dispatch_table_load(const char* path) {
     // every entry must be launchable (validates tile / segmentation / chunking)
     for (const auto& e : entries) {
         GemmPlan p;
-        if (make_gemm_plan(e.fmt, e.variant, e.tile_n, e.k_segments, e.m_max, e.N, e.K, t_sms > 0 ? t_sms : 148, false,
-                           &p) != QLIN_OK)
+        if (make_gemm_plan(e.fmt, e.variant, e.tile_n, e.k_segments, e.m_max, e.N, e.K, t_sms > 0 ? t_sms : 148,
+                           kModeStd, &p) != QLIN_OK)
             return QLIN_ERR_TABLE_FORMAT;
     }
     // device guard: the table must have been measured on this kind of device
@@ -442,7 +500,7 @@ qlin_status qlin_dispatch_table_load(const char* path) {
     for (const auto& e : entries) {
         int stages = 0;
         size_t smem = 0;
-        if (!gemm_kernel_info(e.fmt, is_swap(e.variant), e.tile_n, false, &stages, &smem) ||
+        if (!gemm_kernel_info(e.fmt, is_swap(e.variant), e.tile_n, kModeStd, &stages, &smem) ||
             smem > prop.sharedMemPerBlockOptin)
             return QLIN_ERR_TABLE_FORMAT;
     }

@@ -55,6 +55,7 @@ __device__ int g_device_status = 0;
 }
 
 #include "ptx.cuh"
+#include "quant_math.cuh"
 
 namespace qlin {
 
@@ -71,6 +72,12 @@ struct GemmArgs {
     int kblocks, S, kb_per_seg;
     int p_tiles, units;
     int spread, out_i32;
+    // fused activation quantisation: bf16 x [M, K] (row stride ld_x) in,
+    // codes and scales also written out (by the CTAs of the first W tile)
+    const uint16_t* x;
+    int64_t ld_x;
+    uint8_t* a_q_out;
+    float* s_a_out;
 };
 
 constexpr int kEpiWarps = 8;
@@ -88,11 +95,14 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
     return p;
 }
 
-template <int FMT, bool SWAP, int BN, bool CSK = false>
+template <int FMT, bool SWAP, int BN, bool CSK = false, bool FUSE = false>
 struct Cfg {
     // CSK: cluster Split-K (Swap-AB tiles): the K segments of a tile run on the
     // CTAs of one cluster and are reduced in the leader's shared memory.
+    // FUSE: (Swap-AB tiles) the epilogue warps quantise the unit's activation
+    // rows from bf16 into a resident shared-memory operand; no A loads.
     static_assert(!CSK || SWAP, "cluster Split-K is built for Swap-AB tiles");
+    static_assert(!FUSE || (SWAP && !CSK), "fused quantisation is built for Swap-AB tiles");
     static constexpr int CSK_MAXS = CSK ? cluster_split_max(BN) : 1;  // segments per cluster
     static constexpr int RECV_BYTES = CSK ? (CSK_MAXS - 1) * 128 * BN * 4 : 0;
     static constexpr bool INT8 = (FMT == QLIN_FMT_INT8);
@@ -101,13 +111,19 @@ struct Cfg {
     static constexpr int BK = 128;                 // K bytes per stage: one swizzle atom
     static constexpr int P_BYTES = BM * BK;
     static constexpr int Q_BYTES = BN * BK;
-    static constexpr int STAGE_BYTES = P_BYTES + Q_BYTES;
+    static constexpr int STAGE_BYTES = P_BYTES + (FUSE ? 0 : Q_BYTES);
+    // FUSE: A codes of one unit, [K block][BN rows x 128 B] in the 128-byte
+    // swizzled K-major layout, and the unit's activation scales (2 buffers)
+    static constexpr int A_BYTES = FUSE ? 65536 : 0;
+    static constexpr int A_MAXKB = FUSE ? A_BYTES / (BN * 128) : 0;  // K blocks per unit, at most
+    static constexpr int SA_FLOATS = FUSE ? (FMT == QLIN_FMT_FP8_BLOCK ? BN * A_MAXKB : BN) : 0;
+    static constexpr int SA_BYTES = FUSE ? ((2 * SA_FLOATS * 4 + BN * 4 + 1023) / 1024) * 1024 : 0;
     // Block-FP8: per-unit table of scale products s_a*s_w, [K block][P row or Q column]
     static constexpr int BS_KB = 48;                           // K blocks per staged window
     static constexpr int BS_PITCH = (SWAP ? BN : 128) + 1;     // floats; 1 mod 32: no bank conflicts
     static constexpr int BSCALE_BYTES = BLOCK ? ((BS_KB * BS_PITCH * 4 + 1023) / 1024) * 1024 : 0;
-    static constexpr int STAGES_FIT = (kStageBudget - BSCALE_BYTES - RECV_BYTES) / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
+    static constexpr int STAGES_FIT = (kStageBudget - BSCALE_BYTES - RECV_BYTES - A_BYTES - SA_BYTES) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 11 ? 11 : STAGES_FIT;
     static constexpr int SW = BN < 32 ? BN : 32;   // columns per TMEM load / per store box
     static constexpr int NSLICE = BN / SW;
     static constexpr int MY_SLICES = (NSLICE + 1) / 2;  // slices per epilogue warp (at most)
@@ -122,8 +138,13 @@ struct Cfg {
     static constexpr size_t SCALE_OFF = STAGING_OFF + kStagingBytes;
     static constexpr size_t BSCALE_OFF = SCALE_OFF + kScaleBytes;
     static constexpr size_t RECV_OFF = BSCALE_OFF + BSCALE_BYTES;
-    static constexpr size_t BAR_OFF = RECV_OFF + RECV_BYTES;
+    static constexpr size_t A_OFF = RECV_OFF + RECV_BYTES;
+    static constexpr size_t SA_OFF = A_OFF + A_BYTES;
+    static constexpr size_t BAR_OFF = SA_OFF + SA_BYTES;
     static constexpr size_t SMEM = 1024 + BAR_OFF + 256;
+    // barriers: full/empty per stage, tfull/tempty x2, recv_full/free, a_full/empty; then the TMEM holder
+    static_assert((2 * STAGES + 8) * 8 + 8 <= 256, "barrier area");
+    static_assert(!FUSE || A_MAXKB <= BS_KB, "scale window");
     static_assert(TMEM_COLS <= 512, "TMEM overflow");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
     static_assert(SMEM <= 232448, "shared memory");
@@ -542,11 +563,157 @@ __device__ __forceinline__ bool consume_segment_slice(const GemmArgs& a, const U
     return true;
 }
 
-template <int FMT, bool SWAP, int BN, bool CSK>
+// Fused activation quantisation of one Swap-AB unit (the 256 epilogue
+// threads, which all call it): rows m0..m0+BN-1 of x, K blocks kb0..kb1-1,
+// into the resident operand sA ([K block][BN rows x 128 B], 16-byte chunk c of
+// row r stored at chunk c ^ (r % 8): the 128-byte swizzle the MMA descriptors
+// describe) and the unit's scales into sa (per token: [BN]; Block-FP8:
+// [BN][MAXKB]).  The arithmetic is the stand-alone quantisers'
+// (quant_math.cuh), so codes and scales are theirs bit for bit.  Only rows
+// below M are read; the work is spread over all threads by element, not by
+// row, and every thread issues its loads before it uses them, so a batch of
+// one row costs about two L2 round trips.  Rows past M get zero codes.
+// rmax: BN words of scratch shared memory (per-token formats).
+template <int FMT, int BN, int MAXKB>
+__device__ __noinline__ void fused_quantize_unit(const GemmArgs& a, const Unit& un, uint32_t sA, float* sa,
+                                                    uint32_t* rmax) {
+    constexpr int T = kEpiThreads;
+    constexpr int UNROLL1 = 8;  // 16-byte vectors in flight per thread, pass 1
+    constexpr int UNROLL2 = 4;  // 16-element chunks in flight per thread, pass 2
+    const int tid = threadIdx.x;  // 0 .. T-1
+    const int m0 = un.qt * BN;
+    const int rows = min(BN, a.M - m0);  // >= 1
+    const int nkb = un.kb1 - un.kb0;
+    const int cpr = nkb * 8;  // 16-element chunks per row in this unit
+    const bool write_out = un.pt == 0 && a.a_q_out != nullptr;
+    const int64_t K = (int64_t)a.kblocks * 128;
+    auto sa_addr = [&](int r, int ch) -> uint32_t {
+        const int kbl = ch >> 3, c = ch & 7;
+        return sA + (uint32_t)(kbl * BN * 128 + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+    };
+    auto xrow = [&](int r) { return reinterpret_cast<const uint4*>(a.x + (size_t)(m0 + r) * a.ld_x); };
+    if constexpr (FMT != QLIN_FMT_FP8_BLOCK) {
+        constexpr float QMAX = (FMT == QLIN_FMT_INT8) ? 127.f : 448.f;
+        // TPR consecutive threads per row: the largest power of two with
+        // TPR * rows <= T (so a batch of one row has all 256 threads on it)
+        int tpr = T;
+        while (tpr * rows > T) tpr >>= 1;
+        const int r = tid / tpr, sub = tid % tpr;
+        const bool live = r < rows;
+        const uint4* xr = xrow(live ? r : 0);
+        // pass 1: the row maximum over all of K, 16-byte vectors, loads first
+        const int nvec = (int)(K >> 3);
+        float amax = 0.f;
+        if (live) {
+            for (int v0 = sub; v0 < nvec; v0 += tpr * UNROLL1) {
+                uint4 v[UNROLL1];
+#pragma unroll
+                for (int j = 0; j < UNROLL1; ++j)
+                    if (v0 + j * tpr < nvec) v[j] = __ldg(xr + v0 + j * tpr);
+#pragma unroll
+                for (int j = 0; j < UNROLL1; ++j)
+                    if (v0 + j * tpr < nvec) amax = fmaxf(amax, qm::absmax8(v[j]));
+            }
+        }
+        // within the warp (a row's lanes are consecutive), then across warps
+        // for rows wider than a warp; |x| >= 0, so float order = bit order
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float other = __shfl_xor_sync(0xffffffffu, amax, o);
+            if (o < tpr) amax = fmaxf(amax, other);
+        }
+        for (int i = tid; i < BN; i += T) rmax[i] = 0u;
+        named_bar_sync(1, T);
+        if (live && (sub & 31) == 0) atomicMax(&rmax[r], __float_as_uint(amax));
+        named_bar_sync(1, T);
+        for (int i = tid; i < BN; i += T) {
+            const float sc = i < rows ? __fdiv_rn(__uint_as_float(rmax[i]), QMAX) : 0.f;
+            sa[i] = sc;
+            if (i < rows && un.pt == 0 && un.seg == 0 && a.s_a_out) a.s_a_out[m0 + i] = sc;
+        }
+        // pass 2: the unit's K range, 16 elements -> one 16-byte chunk of codes
+        if (live) {
+            const qm::Divisor dv = qm::make_divisor(__fdiv_rn(__uint_as_float(rmax[r]), QMAX));
+            const uint4* xs = xr + (((int64_t)un.kb0 * 128) >> 3);
+            uint8_t* qout = write_out ? a.a_q_out + (size_t)(m0 + r) * K + (int64_t)un.kb0 * 128 : nullptr;
+            for (int c0 = sub; c0 < cpr; c0 += tpr * UNROLL2) {
+                uint4 v[UNROLL2][2];
+#pragma unroll
+                for (int j = 0; j < UNROLL2; ++j) {
+                    const int ch = c0 + j * tpr;
+                    if (ch < cpr) {
+                        v[j][0] = __ldg(xs + 2 * ch);
+                        v[j][1] = __ldg(xs + 2 * ch + 1);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < UNROLL2; ++j) {
+                    const int ch = c0 + j * tpr;
+                    if (ch < cpr) {
+                        const uint2 q0 = qm::quant8<FMT>(v[j][0], dv), q1 = qm::quant8<FMT>(v[j][1], dv);
+                        const uint4 codes = make_uint4(q0.x, q0.y, q1.x, q1.y);
+                        sts_u4(sa_addr(r, ch), codes);
+                        if (qout) *reinterpret_cast<uint4*>(qout + ch * 16) = codes;
+                    }
+                }
+            }
+        }
+    } else {
+        // 1x128 groups: 8 consecutive lanes per (row, K block) group, 16 elements each
+        constexpr int GPP = T / 8;  // groups per pass
+        const int ngroups = rows * nkb;
+        const int c = tid & 7;
+        for (int g0 = 0; g0 < ngroups; g0 += GPP * 2) {  // uniform trip count: the shuffles stay converged
+            uint4 v[2][2];
+            int gr[2], gk[2];
+            bool live[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int g = g0 + j * GPP + (tid >> 3);
+                live[j] = g < ngroups;
+                gr[j] = live[j] ? g / nkb : 0;
+                gk[j] = live[j] ? g % nkb : 0;
+                if (live[j]) {
+                    const uint4* src = xrow(gr[j]) + (((int64_t)(un.kb0 + gk[j]) * 128 + c * 16) >> 3);
+                    v[j][0] = __ldg(src);
+                    v[j][1] = __ldg(src + 1);
+                } else {
+                    v[j][0] = v[j][1] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                float gmax = fmaxf(qm::absmax8(v[j][0]), qm::absmax8(v[j][1]));
+#pragma unroll
+                for (int o = 4; o > 0; o >>= 1) gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, o));
+                if (!live[j]) continue;
+                const float sc = __fdiv_rn(gmax, 448.f);
+                const int r = gr[j], kbl = gk[j];
+                if (c == 0) {
+                    sa[r * MAXKB + kbl] = sc;
+                    if (un.pt == 0 && a.s_a_out) a.s_a_out[(size_t)(m0 + r) * a.kblocks + un.kb0 + kbl] = sc;
+                }
+                const qm::Divisor dv = qm::make_divisor(sc);
+                const uint2 q0 = qm::quant8<QLIN_FMT_FP8>(v[j][0], dv), q1 = qm::quant8<QLIN_FMT_FP8>(v[j][1], dv);
+                const uint4 codes = make_uint4(q0.x, q0.y, q1.x, q1.y);
+                sts_u4(sa_addr(r, kbl * 8 + c), codes);
+                if (write_out)
+                    *reinterpret_cast<uint4*>(a.a_q_out + (size_t)(m0 + r) * K + (int64_t)(un.kb0 + kbl) * 128 + c * 16) =
+                        codes;
+            }
+        }
+    }
+    // rows past M: zero codes (what the TMA's out-of-bounds fill gives)
+    for (int i = tid; i < (BN - rows) * cpr; i += T) sts_u4(sa_addr(rows + i / cpr, i % cpr), make_uint4(0u, 0u, 0u, 0u));
+    // make the generic-proxy stores visible to the tensor core, then hand over
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE>
 __global__ void __launch_bounds__(kThreads, 1)
     qlin_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ GemmArgs args) {
-    using C = Cfg<FMT, SWAP, BN, CSK>;
+    using C = Cfg<FMT, SWAP, BN, CSK, FUSE>;
     constexpr int STAGES = C::STAGES;
     constexpr int SW = C::SW;
 
@@ -563,7 +730,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
     const uint32_t recv_full = smem_u32(bars + 2 * STAGES + 4);  // cluster Split-K, rank 0
     const uint32_t recv_free = smem_u32(bars + 2 * STAGES + 5);  // cluster Split-K, ranks > 0
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 6);
+    const uint32_t a_full = smem_u32(bars + 2 * STAGES + 6);     // fused: unit's A codes written
+    const uint32_t a_empty = smem_u32(bars + 2 * STAGES + 7);    // fused: MMA done with them
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 8);
+    const uint32_t sA = smem_u32(smem + C::A_OFF);
+    float* sa_tile = reinterpret_cast<float*>(smem + C::SA_OFF);
+    uint32_t* rmax = reinterpret_cast<uint32_t*>(sa_tile + 2 * C::SA_FLOATS);  // fused per-token row maxima
     int* bcast = reinterpret_cast<int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -571,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kProducerWarp && lane == 0) {
         prefetch_tmap(&tmap_p);
-        prefetch_tmap(&tmap_q);
+        if constexpr (!FUSE) prefetch_tmap(&tmap_q);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
@@ -583,6 +755,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (CSK) {
             mbar_init(recv_full, (args.S - 1) * kEpiWarps);  // every epilogue warp of every other rank
             mbar_init(recv_free, 1);                         // rank 0's thread 0
+        }
+        if constexpr (FUSE) {
+            mbar_init(a_full, kEpiWarps);
+            mbar_init(a_empty, 1);
         }
         fence_mbarrier_init();
     }
@@ -636,7 +812,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_2d(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_w, kb * 128, un.qt * BN,
                                         fb, pol_w);
                     }
-                    if constexpr (SWAP)
+                    if constexpr (FUSE)
+                        (void)pol_a;  // the activation operand is quantised in place
+                    else if constexpr (SWAP)
                         tma_load_2d(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_a, kb * 128, un.qt * BN, fb,
                                     pol_a);
                     else
@@ -652,9 +830,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kMmaWarp) {
         // -------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
+            uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0, uphase = 0;
             for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
                 const Unit un = decode_unit<FMT>(args, u);
+                if constexpr (FUSE) {
+                    if (!mbar_wait(a_full, uphase)) goto done;
+                    tc_fence_after();
+                }
                 for (int c0 = un.kb0; c0 < un.kb1; c0 += un.chunk_kb) {
                     if (!mbar_wait(tempty0 + 8 * abuf, aphase ^ 1)) goto done;
                     tc_fence_after();
@@ -663,7 +845,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!mbar_wait(full0 + 8 * stage, phase)) goto done;
                         tc_fence_after();
                         const uint64_t adesc = smem_desc_k_sw128(smem_u32(sP + (size_t)stage * C::P_BYTES));
-                        const uint64_t bdesc = smem_desc_k_sw128(smem_u32(sQ + (size_t)stage * C::Q_BYTES));
+                        const uint64_t bdesc =
+                            FUSE ? smem_desc_k_sw128(sA + (uint32_t)((kb - un.kb0) * BN * 128))
+                                 : smem_desc_k_sw128(smem_u32(sQ + (size_t)stage * C::Q_BYTES));
 #pragma unroll
                         for (int k = 0; k < 4; ++k)  // 4 x K=32 bytes per 128-byte stage
                             tc_mma<C::INT8>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC,
@@ -677,6 +861,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_commit(tfull0 + 8 * abuf);
                     abuf ^= 1;
                     if (abuf == 0) aphase ^= 1;
+                }
+                if constexpr (FUSE) {
+                    tc_commit(a_empty);  // arrives once every MMA of the unit has read sA
+                    uphase ^= 1;
                 }
             }
         }
@@ -708,8 +896,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_total = t_lane + C::TOTAL_COL;
         const uint32_t t_seg = t_lane + C::SEG_COL;
         uint32_t abuf = 0, aphase = 0;
-        for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
+        if constexpr (FUSE) {
+            if ((int)blockIdx.x < args.units) {
+                fused_quantize_unit<FMT, BN, C::A_MAXKB>(args, decode_unit<FMT>(args, blockIdx.x), sA, sa_tile,
+                                                         rmax);
+                warp_arrive(a_full);
+            }
+        }
+        int ui = 0;  // this CTA's unit count so far (fused: scale buffer ui % 2)
+        for (int u = blockIdx.x; u < args.units; u += gridDim.x, ++ui) {
             const Unit un = decode_unit<FMT>(args, u);
+            const float* sa_cur = sa_tile + (ui & 1) * C::SA_FLOATS;
+            // Fused: the next unit's rows are quantised once the MMA is done
+            // with this unit's.  A unit whose MMAs fill one accumulator is
+            // finished before its epilogue starts, so the next unit is
+            // quantised first and its MMAs overlap this epilogue; a unit of
+            // several accumulator chunks needs this epilogue to drain them
+            // first, so its successor waits until after it.
+            const int nxt = u + (int)gridDim.x;
+            const bool quantise_next = FUSE && nxt < args.units;
+            const bool next_first = (un.kb1 - un.kb0) == un.chunk_kb;
+            if (quantise_next && next_first) {
+                if (!warp_wait(a_empty, (uint32_t)(ui & 1))) goto done;
+                fused_quantize_unit<FMT, BN, C::A_MAXKB>(args, decode_unit<FMT>(args, nxt), sA,
+                                                         sa_tile + ((ui + 1) & 1) * C::SA_FLOATS, rmax);
+                warp_arrive(a_full);
+            }
             if constexpr (!C::BLOCK) {
                 // stage the tile's column scales (and bias) once; row values in registers
                 named_bar_sync(1, kEpiThreads);
@@ -718,6 +930,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (!SWAP) {
                         s_col[c] = q < args.N ? __ldg(args.s_w + q) : 0.f;
                         b_col[c] = (e.has_bias && q < args.N) ? bf16_to_f32(__ldg(args.bias + q)) : 0.f;
+                    } else if constexpr (FUSE) {
+                        s_col[c] = sa_cur[c];
                     } else {
                         s_col[c] = q < args.M ? __ldg(args.s_a + q) : 0.f;
                     }
@@ -791,7 +1005,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     if (i < NIDX * kbc) {
                                         off[b] = kbl * C::BS_PITCH + idx;
                                         if (m < args.M) {
-                                            va[b] = __ldg(args.s_a + (size_t)m * args.kblocks + kb);
+                                            if constexpr (FUSE)
+                                                va[b] = sa_cur[idx * C::A_MAXKB + (kb - un.kb0)];
+                                            else
+                                                va[b] = __ldg(args.s_a + (size_t)m * args.kblocks + kb);
                                             vw[b] = __ldg(args.s_w + (size_t)nb * args.kblocks + kb);
                                         }
                                     }
@@ -889,6 +1106,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 if (args.spread) splitk_finish<FMT, SWAP, BN>(args, un, e, bcast);
             }
+            if (quantise_next && !next_first) {
+                if (!warp_wait(a_empty, (uint32_t)(ui & 1))) goto done;
+                fused_quantize_unit<FMT, BN, C::A_MAXKB>(args, decode_unit<FMT>(args, nxt), sA,
+                                                         sa_tile + ((ui + 1) & 1) * C::SA_FLOATS, rmax);
+                warp_arrive(a_full);
+            }
         }
     }
 done:
@@ -930,10 +1153,10 @@ bool make_operand_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool SWAP, int BN, bool CSK>
+template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE>
 qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaStream_t st) {
-    using C = Cfg<FMT, SWAP, BN, CSK>;
-    auto kern = qlin_gemm_kernel<FMT, SWAP, BN, CSK>;
+    using C = Cfg<FMT, SWAP, BN, CSK, FUSE>;
+    auto kern = qlin_gemm_kernel<FMT, SWAP, BN, CSK, FUSE>;
     static int configured_device = -1;
     static int max_clusters[QLIN_MAX_CLUSTER + 1];  // co-resident clusters per cluster size, this device
     int dev = 0;
@@ -946,11 +1169,15 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
         for (int& m : max_clusters) m = -1;
         configured_device = dev;
     }
+    if (FUSE && plan.kb_per_unit > C::A_MAXKB) return QLIN_ERR_UNSUPPORTED;
     alignas(64) CUtensorMap tp, tq;
     const void* p_base = SWAP ? ops.w_q : ops.a_q;
     const void* q_base = SWAP ? ops.a_q : ops.w_q;
     if (!make_operand_tmap(&tp, p_base, plan.p_rows, plan.K, 128)) return QLIN_ERR_CUDA;
-    if (!make_operand_tmap(&tq, q_base, plan.q_rows, plan.K, BN)) return QLIN_ERR_CUDA;
+    if (FUSE)
+        tq = tp;  // unused: the kernel quantises its activation operand in place
+    else if (!make_operand_tmap(&tq, q_base, plan.q_rows, plan.K, BN))
+        return QLIN_ERR_CUDA;
     GemmArgs a;
     a.s_a = ops.s_a;
     a.s_w = ops.s_w;
@@ -970,6 +1197,10 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     a.units = (int)plan.units;
     a.spread = plan.spread ? 1 : 0;
     a.out_i32 = ops.out_i32 ? 1 : 0;
+    a.x = FUSE ? static_cast<const uint16_t*>(ops.x) : nullptr;
+    a.ld_x = FUSE ? ops.ld_x : 0;
+    a.a_q_out = FUSE ? static_cast<uint8_t*>(const_cast<void*>(ops.a_q)) : nullptr;
+    a.s_a_out = FUSE ? const_cast<float*>(ops.s_a) : nullptr;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)plan.grid);
@@ -1007,77 +1238,71 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
 }
 
-template <int FMT>
-qlin_status launch_fmt(const GemmPlan& p, const GemmOperands& ops, cudaStream_t st) {
-    if (p.swap) {
-        if (p.cluster) {
-            switch (p.tile_n) {
-                case 16: return launch_instance<FMT, true, 16, true>(p, ops, st);
-                case 32: return launch_instance<FMT, true, 32, true>(p, ops, st);
-                case 64: return launch_instance<FMT, true, 64, true>(p, ops, st);
-                default: return QLIN_ERR_UNSUPPORTED;
-            }
-        }
-        switch (p.tile_n) {
-            case 16: return launch_instance<FMT, true, 16, false>(p, ops, st);
-            case 32: return launch_instance<FMT, true, 32, false>(p, ops, st);
-            case 64: return launch_instance<FMT, true, 64, false>(p, ops, st);
-            default: return QLIN_ERR_UNSUPPORTED;
-        }
-    }
-    if (p.cluster) return QLIN_ERR_UNSUPPORTED;
-    switch (p.tile_n) {
-        case 128: return launch_instance<FMT, false, 128, false>(p, ops, st);
-        case 256:
-            if constexpr (FMT != QLIN_FMT_FP8_BLOCK) return launch_instance<FMT, false, 256, false>(p, ops, st);
-            return QLIN_ERR_UNSUPPORTED;
-        default: return QLIN_ERR_UNSUPPORTED;
-    }
-}
-
-}  // namespace
-
-namespace {
-template <int FMT, bool SWAP, int BN, bool CSK = false>
+template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE>
 void cfg_info(int* stages, size_t* smem) {
-    *stages = Cfg<FMT, SWAP, BN, CSK>::STAGES;
-    *smem = Cfg<FMT, SWAP, BN, CSK>::SMEM;
+    *stages = Cfg<FMT, SWAP, BN, CSK, FUSE>::STAGES;
+    *smem = Cfg<FMT, SWAP, BN, CSK, FUSE>::SMEM;
 }
 
-template <int FMT>
-bool cfg_info_fmt(bool swap, int tile_n, bool cluster, int* stages, size_t* smem) {
+// One switch over every kernel instantiation: OP<FMT, SWAP, BN, CSK, FUSE>
+// is applied to the one matching (swap, tile_n, mode); false if none exists.
+template <int FMT, template <int, bool, int, bool, bool> class OP, typename... A>
+bool dispatch_instance(bool swap, int tile_n, int mode, A&&... args) {
     if (swap) {
-        switch (tile_n) {
-            case 16: cluster ? cfg_info<FMT, true, 16, true>(stages, smem) : cfg_info<FMT, true, 16>(stages, smem);
-                     return true;
-            case 32: cluster ? cfg_info<FMT, true, 32, true>(stages, smem) : cfg_info<FMT, true, 32>(stages, smem);
-                     return true;
-            case 64: cluster ? cfg_info<FMT, true, 64, true>(stages, smem) : cfg_info<FMT, true, 64>(stages, smem);
-                     return true;
+        switch (mode * 1000 + tile_n) {
+            case kModeStd * 1000 + 16: OP<FMT, true, 16, false, false>::run(args...); return true;
+            case kModeStd * 1000 + 32: OP<FMT, true, 32, false, false>::run(args...); return true;
+            case kModeStd * 1000 + 64: OP<FMT, true, 64, false, false>::run(args...); return true;
+            case kModeCluster * 1000 + 16: OP<FMT, true, 16, true, false>::run(args...); return true;
+            case kModeCluster * 1000 + 32: OP<FMT, true, 32, true, false>::run(args...); return true;
+            case kModeCluster * 1000 + 64: OP<FMT, true, 64, true, false>::run(args...); return true;
+            case kModeFused * 1000 + 16: OP<FMT, true, 16, false, true>::run(args...); return true;
+            case kModeFused * 1000 + 32: OP<FMT, true, 32, false, true>::run(args...); return true;
+            case kModeFused * 1000 + 64: OP<FMT, true, 64, false, true>::run(args...); return true;
         }
         return false;
     }
-    if (cluster) return false;
+    if (mode != kModeStd) return false;
     if (tile_n == 128) {
-        cfg_info<FMT, false, 128>(stages, smem);
+        OP<FMT, false, 128, false, false>::run(args...);
         return true;
     }
     if constexpr (FMT != QLIN_FMT_FP8_BLOCK) {
         if (tile_n == 256) {
-            cfg_info<FMT, false, 256>(stages, smem);
+            OP<FMT, false, 256, false, false>::run(args...);
             return true;
         }
     }
     return false;
 }
+
+template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE>
+struct LaunchOp {
+    static void run(const GemmPlan& p, const GemmOperands& ops, cudaStream_t st, qlin_status* out) {
+        *out = launch_instance<FMT, SWAP, BN, CSK, FUSE>(p, ops, st);
+    }
+};
+
+template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE>
+struct InfoOp {
+    static void run(int* stages, size_t* smem) { cfg_info<FMT, SWAP, BN, CSK, FUSE>(stages, smem); }
+};
+
+template <int FMT>
+qlin_status launch_fmt(const GemmPlan& p, const GemmOperands& ops, cudaStream_t st) {
+    qlin_status r = QLIN_ERR_UNSUPPORTED;
+    if (!dispatch_instance<FMT, LaunchOp>(p.swap, p.tile_n, p.mode, p, ops, st, &r)) return QLIN_ERR_UNSUPPORTED;
+    return r;
+}
+
 }  // namespace
 
-bool gemm_kernel_info(int fmt, bool swap, int tile_n, bool cluster, int* stages, size_t* smem_bytes) {
+bool gemm_kernel_info(int fmt, bool swap, int tile_n, int mode, int* stages, size_t* smem_bytes) {
     switch (fmt) {
-        case QLIN_FMT_INT8: return cfg_info_fmt<QLIN_FMT_INT8>(swap, tile_n, cluster, stages, smem_bytes);
-        case QLIN_FMT_FP8: return cfg_info_fmt<QLIN_FMT_FP8>(swap, tile_n, cluster, stages, smem_bytes);
+        case QLIN_FMT_INT8: return dispatch_instance<QLIN_FMT_INT8, InfoOp>(swap, tile_n, mode, stages, smem_bytes);
+        case QLIN_FMT_FP8: return dispatch_instance<QLIN_FMT_FP8, InfoOp>(swap, tile_n, mode, stages, smem_bytes);
         case QLIN_FMT_FP8_BLOCK:
-            return cfg_info_fmt<QLIN_FMT_FP8_BLOCK>(swap, tile_n, cluster, stages, smem_bytes);
+            return dispatch_instance<QLIN_FMT_FP8_BLOCK, InfoOp>(swap, tile_n, mode, stages, smem_bytes);
     }
     return false;
 }

@@ -23,6 +23,16 @@ __host__ __device__ constexpr int cluster_split_max(int tile_n) {
     return tile_n == 16 ? 8 : (tile_n == 32 || tile_n == 64) ? 4 : 0;
 }
 
+// Kernel variants of one (format, orientation, tile_n).
+enum GemmMode : int {
+    kModeStd = 0,      // operands from global memory by TMA; Split-K through the workspace
+    kModeCluster = 1,  // Swap-AB Split-K reduced through a thread-block cluster
+    kModeFused = 2,    // Swap-AB with the activation quantisation done by the GEMM itself
+};
+// Fused mode keeps the unit's activation codes resident: 64 KiB of shared
+// memory, so at most this many K blocks per unit.
+__host__ __device__ constexpr int fused_max_kblocks(int tile_n) { return tile_n > 0 ? 65536 / (tile_n * 128) : 0; }
+
 // ---------------------------------------------------------------- quantise
 cudaError_t launch_quantize_per_token(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld, void* q,
                                       float* s, bool pdl, cudaStream_t st);
@@ -37,7 +47,7 @@ struct GemmPlan {
     int fmt = 0;
     bool swap = false;    // P = W (rows of N), Q = A (rows of M)
     bool spread = false;  // Split-K: one work unit per (tile, segment)
-    bool cluster = false; // Split-K through a thread-block cluster (no workspace)
+    int mode = kModeStd;  // GemmMode
     int tile_n = 0;       // Q rows per tile (MMA N)
     int k_segments = 1;   // S
     int stages = 0;
@@ -46,6 +56,7 @@ struct GemmPlan {
     int64_t p_tiles = 0, q_tiles = 0, num_tiles = 0, units = 0;
     int kblocks = 0;       // K / 128
     int kb_per_seg = 0;    // kblocks / S
+    int kb_per_unit = 0;   // K blocks one work unit covers
     int grid = 0;          // persistent CTAs
     size_t smem_bytes = 0;
     size_t ticket_bytes = 0;   // workspace prefix holding the per-tile tickets
@@ -53,20 +64,21 @@ struct GemmPlan {
 };
 
 // Validates the (fmt, tile_n, S, variant) combination and fills the plan.
-// With cluster_split, a Swap-AB Split-K whose S fits one cluster reduces
-// through the cluster instead of the workspace.  Returns QLIN_OK or an error
-// status; touches no device state.
+// want_mode kModeCluster: a Swap-AB Split-K whose S fits one cluster reduces
+// through the cluster; kModeFused: a Swap-AB plan whose units fit the
+// resident activation operand quantises its own activations (otherwise the
+// plan keeps kModeStd).  Returns QLIN_OK or an error status; touches no
+// device state.
 qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
-                           int num_sms, bool cluster_split, GemmPlan* plan);
+                           int num_sms, int want_mode, GemmPlan* plan);
 
 // Shared-memory pipeline depth and dynamic smem size of the GEMM kernel
-// instantiation for (fmt, orientation, tile_n, cluster Split-K); false if none
-// exists.
-bool gemm_kernel_info(int fmt, bool swap, int tile_n, bool cluster, int* stages, size_t* smem_bytes);
+// instantiation for (fmt, orientation, tile_n, mode); false if none exists.
+bool gemm_kernel_info(int fmt, bool swap, int tile_n, int mode, int* stages, size_t* smem_bytes);
 
 struct GemmOperands {
-    const void* a_q;
-    const float* s_a;
+    const void* a_q;   // fused mode: written (codes), not read
+    const float* s_a;  // fused mode: written (scales), not read
     const void* w_q;
     const float* s_w;
     const void* bias;
@@ -74,6 +86,8 @@ struct GemmOperands {
     bool out_i32;
     void* workspace;
     bool pdl;  // launch as a programmatic dependent of the previous kernel
+    const void* x = nullptr;  // fused mode: bf16 activations [M, K], row stride ld_x elements
+    int64_t ld_x = 0;
 };
 
 qlin_status launch_gemm(const GemmPlan& plan, const GemmOperands& ops, cudaStream_t st);

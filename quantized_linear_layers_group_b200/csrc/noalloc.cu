@@ -75,7 +75,7 @@ extern "C" qlin_status qlin_scaled_mm_noalloc(int fmt, int variant, int tile_n, 
     if (M < 0) return QLIN_ERR_INVALID_ARG;
     const int sms = current_device_sms();
     GemmPlan p;
-    qlin_status st = make_gemm_plan(fmt, variant, tile_n, k_segments, M > 0 ? M : 1, N, K, sms, false, &p);
+    qlin_status st = make_gemm_plan(fmt, variant, tile_n, k_segments, M > 0 ? M : 1, N, K, sms, kModeStd, &p);
     if (st != QLIN_OK) return st;
     if (p.workspace_bytes > QLIN_NOALLOC_SCRATCH_BYTES) return QLIN_ERR_WORKSPACE;  // beyond the fixed maximum
     if (M == 0) return QLIN_OK;

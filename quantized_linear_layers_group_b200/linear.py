@@ -2,11 +2,12 @@
 
 ``QuantizedLinear(fmt, weight, bias)`` quantises the bf16 weight once
 (per output channel for INT8 / FP8, 128x128 blocks for Block-FP8) with the
-library's own kernels, and its ``forward(x)`` runs the hot path: dynamic
-activation quantisation (per token, or per 1x128 group) followed by the
-scaled GEMM with the fused scale / bias / bf16 epilogue.  Both steps run in
-libqlin.so; this module only allocates tensors (through PyTorch's caching
-allocator) and passes pointers.
+library's own kernels, and its ``forward(x)`` runs the hot path through
+``qlin_linear``: dynamic activation quantisation (per token, or per 1x128
+group) followed by the scaled GEMM with the fused scale / bias / bf16
+epilogue -- one kernel for small batches, where the GEMM quantises its own
+activation tiles.  Everything runs in libqlin.so; this module only allocates
+tensors (through PyTorch's caching allocator) and passes pointers.
 """
 from __future__ import annotations
 
@@ -78,13 +79,19 @@ class QuantizedLinear:
     def forward(self, x: torch.Tensor, stream=None, variant: int = qlin.QLIN_VAR_AUTO, tile_n: int = 0,
                 k_segments: int = 0, out: torch.Tensor | None = None) -> torch.Tensor:
         assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.shape[1] == self.K
+        assert x.stride(1) == 1
         M = x.shape[0]
-        a_q, s_a = quantize_activation(self.fmt, x, stream, self.flags)
+        a_q = torch.empty(M, self.K, dtype=torch.uint8, device=x.device)
+        if self.fmt == qlin.QLIN_FMT_FP8_BLOCK:
+            s_a = torch.empty(M, self.K // 128, dtype=torch.float32, device=x.device)
+        else:
+            s_a = torch.empty(M, dtype=torch.float32, device=x.device)
         c = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
         nbytes = qlin.qlin_scaled_mm_workspace_size(self.fmt, M, self.N, self.K, variant, tile_n, k_segments)
         ws = self.workspace.ensure(nbytes) if nbytes else None
-        qlin.qlin_scaled_mm(self.fmt, a_q, s_a, self.w_q, self.s_w, self.bias, c, ws, stream, variant=variant,
-                            tile_n=tile_n, k_segments=k_segments, flags=self.flags)
+        # quantisation + GEMM in one call (one kernel for small batches)
+        qlin.qlin_linear(self.fmt, x, a_q, s_a, self.w_q, self.s_w, self.bias, c, ws, stream, variant=variant,
+                         tile_n=tile_n, k_segments=k_segments, flags=self.flags)
         return c
 
     __call__ = forward

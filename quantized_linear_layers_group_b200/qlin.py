@@ -44,12 +44,13 @@ QLIN_VAR_SWAPAB_SPLITK = 4
 QLIN_OUT_I32ACC = 1
 QLIN_PDL = 2
 QLIN_SPLITK_CLUSTER = 4  # Swap-AB Split-K: reduce through a thread-block cluster instead of the workspace
+QLIN_FUSED = 8  # qlin_linear: the GEMM quantises its own activation rows where it can (one kernel)
 
 VARIANT_NAMES = {QLIN_VAR_AUTO: "auto", QLIN_VAR_PLAIN: "plain", QLIN_VAR_SPLITK: "splitk",
                  QLIN_VAR_SWAPAB: "swapab", QLIN_VAR_SWAPAB_SPLITK: "swapab_splitk"}
 
 # every symbol include/qlin.h declares
-EXPORTS = ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_scaled_mm_noalloc",
+EXPORTS = ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_scaled_mm_noalloc", "qlin_linear",
            "qlin_scaled_mm_workspace_size", "qlin_dispatch_table_load", "qlin_dispatch_table_clear",
            "qlin_dispatch_query", "qlin_status_string", "qlin_sync_status", "qlin_abi_version")
 QLIN_NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -81,6 +82,8 @@ lib.qlin_scaled_mm.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _v
                                _sz, _vp]
 lib.qlin_scaled_mm_noalloc.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _u32, _vp]
+lib.qlin_linear.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _u32,
+                            _vp, _sz, _vp]
 lib.qlin_scaled_mm_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, ctypes.POINTER(_sz)]
 lib.qlin_dispatch_table_load.argtypes = [ctypes.c_char_p]
 lib.qlin_dispatch_table_clear.argtypes = []
@@ -172,6 +175,23 @@ def qlin_scaled_mm_noalloc(fmt: int, a_q, s_a, w_q, s_w, bias, c_out, stream=Non
     _check(lib.qlin_scaled_mm_noalloc(fmt, variant, tile_n, k_segments, M, N, K, _ptr(a_q), _ptr(s_a), _ptr(w_q),
                                       _ptr(s_w), _ptr(bias), _ptr(c_out), flags, _stream(stream)),
            "qlin_scaled_mm_noalloc")
+
+
+def qlin_linear(fmt: int, x, a_q, s_a, w_q, s_w, bias, c_out, workspace=None, stream=None, *,
+                variant: int = QLIN_VAR_AUTO, tile_n: int = 0, k_segments: int = 0, flags: int = 0, M=None, N=None,
+                K=None, ld_x=None, workspace_bytes=None):
+    """Quantise bf16 x and run the scaled GEMM in one call (one kernel with
+    QLIN_FUSED where the configuration allows); a_q / s_a receive the
+    activation codes and scales."""
+    M = x.shape[0] if M is None else M
+    K = x.shape[1] if K is None else K
+    N = w_q.shape[0] if N is None else N
+    ld_x = (x.stride(0) if x.dim() == 2 else K) if ld_x is None else ld_x
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.qlin_linear(fmt, variant, tile_n, k_segments, M, N, K, _ptr(x), ld_x, _ptr(a_q), _ptr(s_a), _ptr(w_q),
+                           _ptr(s_w), _ptr(bias), _ptr(c_out), flags, _ptr(workspace), workspace_bytes,
+                           _stream(stream)), "qlin_linear")
 
 
 def qlin_dispatch_table_load(path: str):

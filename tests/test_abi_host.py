@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
     syms = _declared_symbols()
     for name in ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_dispatch_table_load"):
         assert name in syms
-    assert len(syms) == 11
+    assert len(syms) == 12
 
 
 def test_library_exports_every_declared_symbol(q):
@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(q):
     for name in _declared_symbols():
         assert hasattr(lib, name), name
     assert set(_declared_symbols()) == set(q.EXPORTS)
-    assert q.qlin_abi_version() == 1
+    assert q.qlin_abi_version() == 2
 
 
 def test_status_strings(q):
@@ -65,7 +65,8 @@ def test_scaled_mm_rejects_bad_arguments_before_launch(q):
     assert _mm(q, fmt=2, N=320) == q.QLIN_ERR_UNSUPPORTED
     assert _mm(q, M=-1) == q.QLIN_ERR_INVALID_ARG
     assert _mm(q, variant=9) == q.QLIN_ERR_INVALID_ARG
-    assert _mm(q, flags=8) == q.QLIN_ERR_INVALID_ARG           # undefined flag bit
+    assert _mm(q, flags=16) == q.QLIN_ERR_INVALID_ARG          # undefined flag bit
+    assert _mm(q, flags=8) == q.QLIN_ERR_INVALID_ARG           # QLIN_FUSED is for qlin_linear
     assert _mm(q, flags=1) == q.QLIN_ERR_INVALID_ARG          # I32 accumulators are INT8 only
     assert _mm(q, fmt=2, bias=16) == q.QLIN_ERR_INVALID_ARG   # Block-FP8 takes no bias
     assert _mm(q, a=None) == q.QLIN_ERR_INVALID_ARG
@@ -165,3 +166,26 @@ def test_shipped_table_parses(q, tmp_path):
         assert e.status in (q.QLIN_ERR_NO_DEVICE, q.QLIN_ERR_TABLE_DEVICE, q.QLIN_ERR_CUDA), e
     finally:
         q.qlin_dispatch_table_clear()
+
+
+def _lin(q, **kw):
+    args = dict(fmt=1, variant=0, tile_n=0, k_segments=0, M=16, N=256, K=256, x=16, ld=256, a=16, sa=16, w=16,
+                sw=16, bias=None, c=16, flags=0, ws=None, wsb=0)
+    args.update(kw)
+    return q.lib.qlin_linear(args["fmt"], args["variant"], args["tile_n"], args["k_segments"], args["M"], args["N"],
+                             args["K"], args["x"], args["ld"], args["a"], args["sa"], args["w"], args["sw"],
+                             args["bias"], args["c"], args["flags"], args["ws"], args["wsb"], None)
+
+
+def test_linear_rejects_bad_arguments_before_launch(q):
+    assert _lin(q, fmt=5) == q.QLIN_ERR_INVALID_ARG
+    assert _lin(q, ld=128) == q.QLIN_ERR_INVALID_ARG            # row stride below K
+    assert _lin(q, ld=260) == q.QLIN_ERR_ALIGNMENT              # rows not 16-byte aligned
+    assert _lin(q, x=24) == q.QLIN_ERR_ALIGNMENT
+    assert _lin(q, x=None) == q.QLIN_ERR_INVALID_ARG
+    assert _lin(q, a=None) == q.QLIN_ERR_INVALID_ARG            # the codes are an output and required
+    assert _lin(q, flags=4) == q.QLIN_ERR_INVALID_ARG           # cluster Split-K is a qlin_scaled_mm flag
+    assert _lin(q, flags=16) == q.QLIN_ERR_INVALID_ARG
+    assert _lin(q, fmt=2, bias=16) == q.QLIN_ERR_INVALID_ARG
+    assert _lin(q, K=200, ld=200) == q.QLIN_ERR_UNSUPPORTED
+    assert _lin(q, M=0) == q.QLIN_OK
