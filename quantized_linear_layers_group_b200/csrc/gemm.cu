@@ -573,13 +573,16 @@ __device__ __forceinline__ bool consume_segment_slice(const GemmArgs& a, const U
 // below M are read; the work is spread over all threads by element, not by
 // row, and every thread issues its loads before it uses them, so a batch of
 // one row costs about two L2 round trips.  Rows past M get zero codes.
-// rmax: BN words of scratch shared memory (per-token formats).
+// rmax: BN words of scratch shared memory (per-token formats).  xs: a
+// shared-memory buffer of xs_bytes; when the unit's slice of x (rows x its K
+// range in bf16) fits, pass 1 keeps that slice there and pass 2 reads it back
+// instead of going to memory a second time.
 template <int FMT, int BN, int MAXKB>
-__device__ __noinline__ void fused_quantize_unit(const GemmArgs& a, const Unit& un, uint32_t sA, float* sa,
-                                                    uint32_t* rmax) {
+__device__ __forceinline__ void fused_quantize_unit(const GemmArgs& a, const Unit& un, uint32_t sA, float* sa,
+                                                    uint32_t* rmax, uint32_t xs, int xs_bytes) {
     constexpr int T = kEpiThreads;
-    constexpr int UNROLL1 = 8;  // 16-byte vectors in flight per thread, pass 1
-    constexpr int UNROLL2 = 4;  // 16-element chunks in flight per thread, pass 2
+    constexpr int UNROLL1 = 4;  // 16-byte vectors in flight per thread, pass 1
+    constexpr int UNROLL2 = 2;  // 16-element chunks in flight per thread, pass 2
     const int tid = threadIdx.x;  // 0 .. T-1
     const int m0 = un.qt * BN;
     const int rows = min(BN, a.M - m0);  // >= 1
@@ -601,8 +604,11 @@ __device__ __noinline__ void fused_quantize_unit(const GemmArgs& a, const Unit& 
         const int r = tid / tpr, sub = tid % tpr;
         const bool live = r < rows;
         const uint4* xr = xrow(live ? r : 0);
-        // pass 1: the row maximum over all of K, 16-byte vectors, loads first
+        // pass 1: the row maximum over all of K, 16-byte vectors, loads first;
+        // the vectors of this unit's K range are kept in xs when they fit
         const int nvec = (int)(K >> 3);
+        const int uv0 = un.kb0 * 16, uvn = nkb * 16;  // the unit's vectors of a row
+        const bool staged = rows * uvn * 16 <= xs_bytes;
         float amax = 0.f;
         if (live) {
             for (int v0 = sub; v0 < nvec; v0 += tpr * UNROLL1) {
@@ -611,8 +617,14 @@ __device__ __noinline__ void fused_quantize_unit(const GemmArgs& a, const Unit& 
                 for (int j = 0; j < UNROLL1; ++j)
                     if (v0 + j * tpr < nvec) v[j] = __ldg(xr + v0 + j * tpr);
 #pragma unroll
-                for (int j = 0; j < UNROLL1; ++j)
-                    if (v0 + j * tpr < nvec) amax = fmaxf(amax, qm::absmax8(v[j]));
+                for (int j = 0; j < UNROLL1; ++j) {
+                    const int vi = v0 + j * tpr;
+                    if (vi < nvec) {
+                        amax = fmaxf(amax, qm::absmax8(v[j]));
+                        if (staged && vi >= uv0 && vi < uv0 + uvn)
+                            sts_u4(xs + (uint32_t)((r * uvn + vi - uv0) * 16), v[j]);
+                    }
+                }
             }
         }
         // within the warp (a row's lanes are consecutive), then across warps
@@ -634,7 +646,7 @@ __device__ __noinline__ void fused_quantize_unit(const GemmArgs& a, const Unit& 
         // pass 2: the unit's K range, 16 elements -> one 16-byte chunk of codes
         if (live) {
             const qm::Divisor dv = qm::make_divisor(__fdiv_rn(__uint_as_float(rmax[r]), QMAX));
-            const uint4* xs = xr + (((int64_t)un.kb0 * 128) >> 3);
+            const uint4* xsrc = xr + (((int64_t)un.kb0 * 128) >> 3);
             uint8_t* qout = write_out ? a.a_q_out + (size_t)(m0 + r) * K + (int64_t)un.kb0 * 128 : nullptr;
             for (int c0 = sub; c0 < cpr; c0 += tpr * UNROLL2) {
                 uint4 v[UNROLL2][2];
@@ -642,8 +654,13 @@ __device__ __noinline__ void fused_quantize_unit(const GemmArgs& a, const Unit& 
                 for (int j = 0; j < UNROLL2; ++j) {
                     const int ch = c0 + j * tpr;
                     if (ch < cpr) {
-                        v[j][0] = __ldg(xs + 2 * ch);
-                        v[j][1] = __ldg(xs + 2 * ch + 1);
+                        if (staged) {
+                            v[j][0] = lds_u4(xs + (uint32_t)((r * uvn + 2 * ch) * 16));
+                            v[j][1] = lds_u4(xs + (uint32_t)((r * uvn + 2 * ch + 1) * 16));
+                        } else {
+                            v[j][0] = __ldg(xsrc + 2 * ch);
+                            v[j][1] = __ldg(xsrc + 2 * ch + 1);
+                        }
                     }
                 }
 #pragma unroll
@@ -736,6 +753,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sA = smem_u32(smem + C::A_OFF);
     float* sa_tile = reinterpret_cast<float*>(smem + C::SA_OFF);
     uint32_t* rmax = reinterpret_cast<uint32_t*>(sa_tile + 2 * C::SA_FLOATS);  // fused per-token row maxima
+    // fused: the epilogue's transpose buffers (unused by Swap-AB tiles) hold x slices
+    const uint32_t xstage = smem_u32(smem + C::STAGING_OFF);
     int* bcast = reinterpret_cast<int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -899,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (FUSE) {
             if ((int)blockIdx.x < args.units) {
                 fused_quantize_unit<FMT, BN, C::A_MAXKB>(args, decode_unit<FMT>(args, blockIdx.x), sA, sa_tile,
-                                                         rmax);
+                                                         rmax, xstage, kStagingBytes);
                 warp_arrive(a_full);
             }
         }
@@ -919,7 +938,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (quantise_next && next_first) {
                 if (!warp_wait(a_empty, (uint32_t)(ui & 1))) goto done;
                 fused_quantize_unit<FMT, BN, C::A_MAXKB>(args, decode_unit<FMT>(args, nxt), sA,
-                                                         sa_tile + ((ui + 1) & 1) * C::SA_FLOATS, rmax);
+                                                         sa_tile + ((ui + 1) & 1) * C::SA_FLOATS, rmax, xstage,
+                                                         kStagingBytes);
                 warp_arrive(a_full);
             }
             if constexpr (!C::BLOCK) {
@@ -1109,7 +1129,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (quantise_next && !next_first) {
                 if (!warp_wait(a_empty, (uint32_t)(ui & 1))) goto done;
                 fused_quantize_unit<FMT, BN, C::A_MAXKB>(args, decode_unit<FMT>(args, nxt), sA,
-                                                         sa_tile + ((ui + 1) & 1) * C::SA_FLOATS, rmax);
+                                                         sa_tile + ((ui + 1) & 1) * C::SA_FLOATS, rmax, xstage,
+                                                         kStagingBytes);
                 warp_arrive(a_full);
             }
         }
