@@ -382,6 +382,7 @@ template <int FMT, bool SWAP, int BN>
 __device__ __forceinline__ void splitk_finish(const GemmArgs& a, const Unit& un, EpiCtx& e, int* bcast) {
     using C = Cfg<FMT, SWAP, BN>;
     constexpr int SW = C::SW;
+    constexpr int SB = 64 / SW;  // segments loaded per round trip: 64 registers of partials
     named_bar_sync(1, kEpiThreads);
     if (threadIdx.x == 0) {
         // acq_rel: releases this CTA's partial stores (ordered before it by the
@@ -400,10 +401,10 @@ __device__ __forceinline__ void splitk_finish(const GemmArgs& a, const Unit& un,
 #pragma unroll
             for (int c = 0; c < SW; ++c) t[c] = 0;
 #pragma unroll 1
-            for (int s0 = 0; s0 < a.S; s0 += 2) {
-                uint4 w[2][SW / 4];
+            for (int s0 = 0; s0 < a.S; s0 += SB) {
+                uint4 w[SB][SW / 4];
 #pragma unroll
-                for (int i = 0; i < 2; ++i)
+                for (int i = 0; i < SB; ++i)
                     if (s0 + i < a.S) {
                         const uint4* p =
                             reinterpret_cast<const uint4*>(partial_ptr<SW>(a, un.tile, s0 + i, j, C::NSLICE, e.row_lane));
@@ -411,7 +412,7 @@ __device__ __forceinline__ void splitk_finish(const GemmArgs& a, const Unit& un,
                         for (int q = 0; q < SW / 4; ++q) w[i][q] = __ldcg(p + q * 128);
                     }
 #pragma unroll
-                for (int i = 0; i < 2; ++i)
+                for (int i = 0; i < SB; ++i)
                     if (s0 + i < a.S) {
 #pragma unroll
                         for (int q = 0; q < SW / 4; ++q) {
@@ -429,10 +430,10 @@ __device__ __forceinline__ void splitk_finish(const GemmArgs& a, const Unit& un,
 #pragma unroll
             for (int c = 0; c < SW; ++c) t[c] = 0.f;
 #pragma unroll 1
-            for (int s0 = 0; s0 < a.S; s0 += 2) {
-                uint4 w[2][SW / 4];
+            for (int s0 = 0; s0 < a.S; s0 += SB) {
+                uint4 w[SB][SW / 4];
 #pragma unroll
-                for (int i = 0; i < 2; ++i)
+                for (int i = 0; i < SB; ++i)
                     if (s0 + i < a.S) {
                         const uint4* p =
                             reinterpret_cast<const uint4*>(partial_ptr<SW>(a, un.tile, s0 + i, j, C::NSLICE, e.row_lane));
@@ -440,7 +441,7 @@ __device__ __forceinline__ void splitk_finish(const GemmArgs& a, const Unit& un,
                         for (int q = 0; q < SW / 4; ++q) w[i][q] = __ldcg(p + q * 128);
                     }
 #pragma unroll
-                for (int i = 0; i < 2; ++i)  // fixed segment order
+                for (int i = 0; i < SB; ++i)  // fixed segment order
                     if (s0 + i < a.S) {
 #pragma unroll
                         for (int q = 0; q < SW / 4; ++q) {
