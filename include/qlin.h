@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define QLIN_ABI_VERSION 2
+#define QLIN_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define QLIN_API __attribute__((visibility("default")))
@@ -313,6 +313,17 @@ QLIN_API const char* qlin_status_string(qlin_status status);
  * QLIN_ERR_DEVICE_TIMEOUT or QLIN_ERR_CUDA.  Blocking.
  */
 QLIN_API qlin_status qlin_sync_status(qlin_stream_t stream);
+
+/*
+ * qlin_selftest_wait_timeout -- exercise the failure path of the device-side
+ * waits without faulting the GPU: enqueue a one-thread kernel that waits, for
+ * at most limit_us microseconds (1 .. 1000000), on an mbarrier that nothing
+ * arrives on.  The wait gives up, records QLIN_ERR_DEVICE_TIMEOUT and the
+ * kernel returns; the next qlin_sync_status() on the stream reports (and
+ * clears) it, and the context stays usable.  Asynchronous.
+ * Errors: INVALID_ARG, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_selftest_wait_timeout(uint32_t limit_us, qlin_stream_t stream);
 
 /* ABI version of the loaded library (QLIN_ABI_VERSION at build time). */
 QLIN_API int qlin_abi_version(void);

@@ -518,6 +518,14 @@ qlin_status qlin_dispatch_table_load(const char* path) {
     return QLIN_OK;
 }
 
+qlin_status qlin_selftest_wait_timeout(uint32_t limit_us, qlin_stream_t stream) {
+    if (limit_us == 0 || limit_us > 1000000u) return QLIN_ERR_INVALID_ARG;
+    if (current_device_sms() <= 0) return QLIN_ERR_NO_DEVICE;
+    return launch_wait_selftest((uint64_t)limit_us * 1000u, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QLIN_OK
+               : QLIN_ERR_CUDA;
+}
+
 qlin_status qlin_sync_status(qlin_stream_t stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QLIN_ERR_CUDA;
     int v = 0;

@@ -1330,6 +1330,23 @@ bool gemm_kernel_info(int fmt, bool swap, int tile_n, int mode, int* stages, siz
 }
 
 
+// Failure-path self-test: one thread waits, with the given limit, on an
+// mbarrier that nothing ever arrives on; the wait gives up, records
+// QLIN_ERR_DEVICE_TIMEOUT and the kernel returns normally.
+__global__ void qlin_wait_selftest_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbarrier_init();
+        (void)mbar_wait_for(smem_u32(&bar), 0, limit_ns);
+    }
+}
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st) {
+    qlin_wait_selftest_kernel<<<1, 32, 0, st>>>(limit_ns);
+    return cudaGetLastError();
+}
+
 cudaError_t device_status_read_clear(int* value) {
     cudaError_t e = cudaMemcpyFromSymbol(value, g_device_status, sizeof(int));
     if (e != cudaSuccess || *value == 0) return e;

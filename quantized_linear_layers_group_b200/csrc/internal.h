@@ -95,6 +95,9 @@ qlin_status launch_gemm(const GemmPlan& plan, const GemmOperands& ops, cudaStrea
 // Reads and clears the device status word that bounded waits set on timeout.
 cudaError_t device_status_read_clear(int* value);
 
+// Launches the failure-path self-test (a bounded wait that must give up).
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st);
+
 // Number of SMs of the current device (cached per device); 0 if none.
 int current_device_sms();
 

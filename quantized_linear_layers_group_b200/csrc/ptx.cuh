@@ -58,19 +58,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
-// (and records a timeout) if it has not completed within the limit.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// (and records a timeout) if it has not completed within limit_ns.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > QLIN_WAIT_LIMIT_NS) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             atomicExch(&g_device_status, 9 /* QLIN_ERR_DEVICE_TIMEOUT */);
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    return mbar_wait_for(bar, parity, QLIN_WAIT_LIMIT_NS);
 }
 
 // ----------------------------------------------------------------------- TMA

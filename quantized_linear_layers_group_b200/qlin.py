@@ -52,7 +52,8 @@ VARIANT_NAMES = {QLIN_VAR_AUTO: "auto", QLIN_VAR_PLAIN: "plain", QLIN_VAR_SPLITK
 # every symbol include/qlin.h declares
 EXPORTS = ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_scaled_mm_noalloc", "qlin_linear",
            "qlin_scaled_mm_workspace_size", "qlin_dispatch_table_load", "qlin_dispatch_table_clear",
-           "qlin_dispatch_query", "qlin_status_string", "qlin_sync_status", "qlin_abi_version")
+           "qlin_dispatch_query", "qlin_status_string", "qlin_sync_status", "qlin_abi_version",
+           "qlin_selftest_wait_timeout")
 QLIN_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -91,6 +92,7 @@ lib.qlin_dispatch_query.argtypes = [_i32, _i64, _i64, _i64, ctypes.POINTER(qlin_
 lib.qlin_status_string.argtypes = [_i32]
 lib.qlin_status_string.restype = ctypes.c_char_p
 lib.qlin_sync_status.argtypes = [_vp]
+lib.qlin_selftest_wait_timeout.argtypes = [_u32, _vp]
 lib.qlin_abi_version.argtypes = []
 for _name in EXPORTS:
     if _name != "qlin_status_string":
@@ -215,6 +217,13 @@ def qlin_status_string(status: int) -> str:
 def qlin_sync_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return lib.qlin_sync_status(_stream(stream))
+
+
+def qlin_selftest_wait_timeout(limit_us: int = 20000, stream=None):
+    """Enqueue the failure-path self-test: a device wait that must give up
+    after limit_us and record QLIN_ERR_DEVICE_TIMEOUT (read it back with
+    qlin_sync_status)."""
+    _check(lib.qlin_selftest_wait_timeout(limit_us, _stream(stream)), "qlin_selftest_wait_timeout")
 
 
 def qlin_abi_version() -> int:

@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
     syms = _declared_symbols()
     for name in ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_dispatch_table_load"):
         assert name in syms
-    assert len(syms) == 12
+    assert len(syms) == 13
 
 
 def test_library_exports_every_declared_symbol(q):
@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(q):
     for name in _declared_symbols():
         assert hasattr(lib, name), name
     assert set(_declared_symbols()) == set(q.EXPORTS)
-    assert q.qlin_abi_version() == 2
+    assert q.qlin_abi_version() == 3
 
 
 def test_status_strings(q):
@@ -189,3 +189,8 @@ def test_linear_rejects_bad_arguments_before_launch(q):
     assert _lin(q, fmt=2, bias=16) == q.QLIN_ERR_INVALID_ARG
     assert _lin(q, K=200, ld=200) == q.QLIN_ERR_UNSUPPORTED
     assert _lin(q, M=0) == q.QLIN_OK
+
+
+def test_selftest_rejects_bad_limits(q):
+    assert q.lib.qlin_selftest_wait_timeout(0, None) == q.QLIN_ERR_INVALID_ARG
+    assert q.lib.qlin_selftest_wait_timeout(2000000, None) == q.QLIN_ERR_INVALID_ARG

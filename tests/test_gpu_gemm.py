@@ -162,6 +162,21 @@ def test_auto_dispatch_matches_oracle(fmt):
         assert_parity(fmt, bits_u16(p.run()), p.reference(), f"auto M={M}")
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("M,N,K", [(3, 256, 128), (70, 384, 128), (5, 256, 8192), (140, 256, 8192)])
+def test_extreme_depths(fmt, M, N, K):
+    # one 128-wide K block (no pipelining across K), and a deep K of 64 blocks
+    # (the shared-memory ring wraps several times; up to 8 segments)
+    p = Prepared(fmt, *_problem(fmt, M, N, K, seed=K + M + fmt))
+    ref = p.reference()
+    kb = K // 128
+    for var, tile, s in [(PLAIN, 128, 1), (SWAPAB, 16, 1), (SWAPAB, 64, 1)] + \
+            ([(SPLITK, 128, 8), (SWAPAB_SPLITK, 16, 8), (PLAIN, 128, 8)] if kb % 8 == 0 else []):
+        c = p.run(var, tile, s)
+        assert_parity(fmt, bits_u16(c), ref, f"fmt={fmt} M={M} N={N} K={K} var={var} tile={tile} S={s}")
+    check_status()
+
+
 def test_zero_activation_row_gives_bias():
     fmt = oracle.FMT_FP8
     a, w, b = _problem(fmt, 9, 256, 256, seed=3)
