@@ -15,8 +15,9 @@
 
 namespace qlin {
 
-// Device status word (0 = OK, otherwise a qlin_status code set by a kernel).
-// The one translation unit that includes this header defines it first.
+// The bounded waits below write the device status word g_device_status
+// (0 = OK, otherwise a qlin_status code), which the one translation unit that
+// includes this header defines before including it.
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -232,38 +233,6 @@ __host__ __device__ constexpr uint32_t make_idesc(bool int8, int m, int n) {
     return (int8 ? (2u << 4) : (1u << 4)) | (int8 ? (1u << 7) : 0u) | (int8 ? (1u << 10) : 0u) |
            ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
-
-}  // namespace qlin
-
-namespace qlin {
-
-// --------------------------------------------------- TMA stores (bulk groups)
-__device__ __forceinline__ void fence_proxy_async_shared() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// 2-D tiled bulk tensor store shared -> global; out-of-bounds parts of the box
-// are not written.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int32_t x, int32_t y) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(m)),
-                 "r"(src), "r"(x), "r"(y)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// wait until at most N committed groups still read their shared-memory source
-template <int N>
-__device__ __forceinline__ void bulk_wait_group_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-template <int N>
-__device__ __forceinline__ void bulk_wait_group() {
-    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
-}
-
-}  // namespace qlin
-
-namespace qlin {
 
 // ------------------------------------------------------- thread-block clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
