@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define QLIN_ABI_VERSION 3
+#define QLIN_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define QLIN_API __attribute__((visibility("default")))
@@ -77,7 +77,11 @@ typedef enum {
     QLIN_VAR_PLAIN = 1,         /* one CTA per output tile, all K segments in it */
     QLIN_VAR_SPLITK = 2,        /* K segments of a tile spread over CTAs, fixed-order reduce */
     QLIN_VAR_SWAPAB = 3,        /* C^T = W A^T: N fills the 128-row MMA side, M the narrow side */
-    QLIN_VAR_SWAPAB_SPLITK = 4  /* Swap-AB with the K segments spread over CTAs */
+    QLIN_VAR_SWAPAB_SPLITK = 4, /* Swap-AB with the K segments spread over CTAs */
+    QLIN_VAR_PAIR = 5           /* plain, 256-row tiles on a pair of CTAs (a cluster of 2): each CTA
+                                   loads its 128 rows of A and half of the W tile, and one
+                                   tcgen05.mma.cta_group::2 per K step fills both CTAs' accumulators.
+                                   tile_n 256, INT8 and FP8; sums K in the plain variant's order */
 } qlin_variant;
 
 /* flags */

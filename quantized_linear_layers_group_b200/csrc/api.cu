@@ -70,6 +70,7 @@ const char* variant_name(int v) {
         case QLIN_VAR_SPLITK: return "splitk";
         case QLIN_VAR_SWAPAB: return "swapab";
         case QLIN_VAR_SWAPAB_SPLITK: return "swapab_splitk";
+        case QLIN_VAR_PAIR: return "pair";
     }
     return "auto";
 }
@@ -79,17 +80,20 @@ int parse_variant(const std::string& s) {
     if (s == "splitk") return QLIN_VAR_SPLITK;
     if (s == "swapab") return QLIN_VAR_SWAPAB;
     if (s == "swapab_splitk") return QLIN_VAR_SWAPAB_SPLITK;
+    if (s == "pair") return QLIN_VAR_PAIR;
     return -1;
 }
 
 bool is_swap(int v) { return v == QLIN_VAR_SWAPAB || v == QLIN_VAR_SWAPAB_SPLITK; }
+int base_mode(int v) { return v == QLIN_VAR_PAIR ? kModePair : kModeStd; }
 bool is_spread(int v) { return v == QLIN_VAR_SPLITK || v == QLIN_VAR_SWAPAB_SPLITK; }
 // Swap-AB Split-K whose segments fit one cluster may reduce through it.
 bool runs_as_cluster(int variant, int tile_n, int S) {
     return variant == QLIN_VAR_SWAPAB_SPLITK && S > 1 && S <= cluster_split_max(tile_n);
 }
 
-bool tile_supported(int fmt, bool swap, int tile_n) {
+bool tile_supported(int fmt, bool swap, int tile_n, bool pair = false) {
+    if (pair) return fmt != QLIN_FMT_FP8_BLOCK && tile_n == 256;
     if (swap) return tile_n == 16 || tile_n == 32 || tile_n == 64;
     if (fmt == QLIN_FMT_FP8_BLOCK) return tile_n == 128;
     return tile_n == 128 || tile_n == 256;
@@ -142,7 +146,7 @@ bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, qlin_config* out) {
     out->tile_n = best->tile_n;
     out->k_segments = best->k_segments;
     size_t smem = 0;
-    gemm_kernel_info(fmt, is_swap(best->variant), best->tile_n, kModeStd, &out->stages, &smem);
+    gemm_kernel_info(fmt, is_swap(best->variant), best->tile_n, base_mode(best->variant), &out->stages, &smem);
     out->m_max = best->m_max;
     out->from_table = 1;
     return true;
@@ -159,7 +163,7 @@ qlin_status check_fmt_shape(int fmt, int64_t M, int64_t N, int64_t K) {
 
 qlin_status resolve_config(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
                            int num_sms, qlin_config* cfg) {
-    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_SWAPAB_SPLITK) return QLIN_ERR_INVALID_ARG;
+    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_PAIR) return QLIN_ERR_INVALID_ARG;
     if (tile_n < 0 || k_segments < 0) return QLIN_ERR_INVALID_ARG;
     qlin_config base{};
     if (!lookup_table(fmt, M, N, K, &base)) base = default_config(fmt, M, N, K, num_sms);
@@ -171,13 +175,14 @@ qlin_status resolve_config(int fmt, int variant, int tile_n, int k_segments, int
         base.tile_n = same_orientation ? base.tile_n : d.tile_n;
         if (is_swap(variant) && !same_orientation)
             base.tile_n = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+        if (variant == QLIN_VAR_PAIR) base.tile_n = 256;
         base.variant = variant;
     }
     if (tile_n) base.tile_n = tile_n;
     if (k_segments) base.k_segments = k_segments;
     size_t smem = 0;
     base.stages = 0;
-    gemm_kernel_info(fmt, is_swap(base.variant), base.tile_n, kModeStd, &base.stages, &smem);
+    gemm_kernel_info(fmt, is_swap(base.variant), base.tile_n, base_mode(base.variant), &base.stages, &smem);
     *cfg = base;
     return QLIN_OK;
 }
@@ -215,7 +220,8 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     p.N = N;
     p.K = K;
     p.kblocks = (int)(K / 128);
-    if (!tile_supported(fmt, p.swap, p.tile_n)) return QLIN_ERR_UNSUPPORTED;
+    const bool pair = cfg.variant == QLIN_VAR_PAIR;
+    if (!tile_supported(fmt, p.swap, p.tile_n, pair)) return QLIN_ERR_UNSUPPORTED;
     if (p.k_segments < 1 || p.kblocks % p.k_segments != 0) return QLIN_ERR_UNSUPPORTED;
     if (p.k_segments == 1) p.spread = false;
     p.kb_per_seg = p.kblocks / p.k_segments;
@@ -225,7 +231,7 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
                              (fmt == QLIN_FMT_FP8 && !p.spread && p.k_segments > 1);
     if (multi_chunk && p.tile_n > 128) return QLIN_ERR_UNSUPPORTED;
     p.kb_per_unit = p.spread ? p.kb_per_seg : p.kblocks;
-    p.mode = kModeStd;
+    p.mode = pair ? kModePair : kModeStd;
     if (want_mode == kModeCluster && p.spread && runs_as_cluster(cfg.variant, p.tile_n, p.k_segments))
         p.mode = kModeCluster;
     if (want_mode == kModeFused && p.swap && p.kb_per_unit <= fused_max_kblocks(p.tile_n)) p.mode = kModeFused;
@@ -234,12 +240,14 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     p.q_rows = p.swap ? M : N;
     p.p_tiles = (p.p_rows + 127) / 128;
     p.q_tiles = (p.q_rows + p.tile_n - 1) / p.tile_n;
-    p.num_tiles = p.p_tiles * p.q_tiles;
+    // PAIR: one unit per 256-row tile (two 128-row halves on the two CTAs)
+    p.num_tiles = (pair ? (p.p_tiles + 1) / 2 : p.p_tiles) * p.q_tiles;
     p.units = p.num_tiles * (p.spread ? p.k_segments : 1);
     if (p.units > (int64_t)INT32_MAX / 2) return QLIN_ERR_UNSUPPORTED;
     p.grid = (int)std::min<int64_t>(p.units, num_sms);
     if (p.mode == kModeCluster)  // whole clusters; the launcher also caps them by co-residency
         p.grid = (int)std::min<int64_t>(p.num_tiles, std::max(1, num_sms / p.k_segments)) * p.k_segments;
+    if (p.mode == kModePair) p.grid = (int)std::min<int64_t>(p.num_tiles, std::max(1, num_sms / 2)) * 2;
     if (p.grid < 1) p.grid = 1;
     const bool workspace_split = p.spread && p.mode != kModeCluster;
     if (workspace_split && p.num_tiles > kMaxSplitTiles) return QLIN_ERR_UNSUPPORTED;
@@ -337,7 +345,7 @@ qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int
     const bool out_i32 = (flags & QLIN_OUT_I32ACC) != 0;
     if (out_i32 && fmt != QLIN_FMT_INT8) return QLIN_ERR_INVALID_ARG;
     if (fmt == QLIN_FMT_FP8_BLOCK && bias) return QLIN_ERR_INVALID_ARG;
-    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_SWAPAB_SPLITK || tile_n < 0 || k_segments < 0)
+    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_PAIR || tile_n < 0 || k_segments < 0)
         return QLIN_ERR_INVALID_ARG;
     if (M == 0) return QLIN_OK;
     if (!a_q || !s_a || !w_q || !s_w || !c_out) return QLIN_ERR_INVALID_ARG;
@@ -358,8 +366,9 @@ qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int
     if (g_log)
         std::fprintf(stderr, "[qlin] scaled_mm %s M=%lld N=%lld K=%lld -> %s%s tile_n=%d S=%d grid=%d\n",
                      fmt_name(fmt), (long long)M, (long long)N, (long long)K,
-                     variant_name(p.swap ? (p.spread ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB)
-                                         : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
+                     variant_name(p.mode == kModePair ? QLIN_VAR_PAIR
+                                  : p.swap ? (p.spread ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB)
+                                           : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
                      p.mode == kModeCluster ? " (cluster)" : "", p.tile_n, p.k_segments, p.grid);
     GemmOperands ops{a_q, s_a, w_q, s_w, bias, c_out, out_i32, workspace, (flags & QLIN_PDL) != 0};
     return launch_gemm(p, ops, static_cast<cudaStream_t>(stream));
@@ -375,7 +384,7 @@ qlin_status qlin_linear(int fmt, int variant, int tile_n, int k_segments, int64_
     const bool out_i32 = (flags & QLIN_OUT_I32ACC) != 0;
     if (out_i32 && fmt != QLIN_FMT_INT8) return QLIN_ERR_INVALID_ARG;
     if (fmt == QLIN_FMT_FP8_BLOCK && bias) return QLIN_ERR_INVALID_ARG;
-    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_SWAPAB_SPLITK || tile_n < 0 || k_segments < 0)
+    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_PAIR || tile_n < 0 || k_segments < 0)
         return QLIN_ERR_INVALID_ARG;
     if (ld_x < K) return QLIN_ERR_INVALID_ARG;
     if (M == 0) return QLIN_OK;
@@ -400,8 +409,9 @@ qlin_status qlin_linear(int fmt, int variant, int tile_n, int k_segments, int64_
     if (g_log)
         std::fprintf(stderr, "[qlin] linear %s M=%lld N=%lld K=%lld -> %s%s tile_n=%d S=%d grid=%d\n", fmt_name(fmt),
                      (long long)M, (long long)N, (long long)K,
-                     variant_name(p.swap ? (p.spread ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB)
-                                         : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
+                     variant_name(p.mode == kModePair ? QLIN_VAR_PAIR
+                                  : p.swap ? (p.spread ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB)
+                                           : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
                      p.mode == kModeFused ? " (fused)" : "", p.tile_n, p.k_segments, p.grid);
     if (p.mode == kModeFused) {
         GemmOperands ops{a_q, s_a, w_q, s_w, bias, c_out, out_i32, workspace, pdl, x, ld_x};

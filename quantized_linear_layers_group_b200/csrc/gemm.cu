@@ -95,7 +95,7 @@ __host__ __device__ constexpr int pow2_at_least(int v) {
     return p;
 }
 
-template <int FMT, bool SWAP, int BN, bool CSK = false, bool FUSE = false>
+template <int FMT, bool SWAP, int BN, bool CSK = false, bool FUSE = false, bool PAIR = false>
 struct Cfg {
     // CSK: cluster Split-K (Swap-AB tiles): the K segments of a tile run on the
     // CTAs of one cluster and are reduced in the leader's shared memory.
@@ -103,6 +103,11 @@ struct Cfg {
     // rows from bf16 into a resident shared-memory operand; no A loads.
     static_assert(!CSK || SWAP, "cluster Split-K is built for Swap-AB tiles");
     static_assert(!FUSE || (SWAP && !CSK), "fused quantisation is built for Swap-AB tiles");
+    // PAIR: plain tiles of 256 P rows on the two CTAs of a cluster; each CTA
+    // loads its own 128 rows of A and half (BN/2 rows) of the W tile, and CTA
+    // rank 0 issues M=256 MMAs that fill both CTAs' accumulators.
+    static_assert(!PAIR || (!SWAP && !CSK && !FUSE && BN == 256 && FMT != QLIN_FMT_FP8_BLOCK),
+                  "CTA pairs are built for plain 256-column tiles");
     static constexpr int CSK_MAXS = CSK ? cluster_split_max(BN) : 1;  // segments per cluster
     static constexpr int RECV_BYTES = CSK ? (CSK_MAXS - 1) * 128 * BN * 4 : 0;
     static constexpr bool INT8 = (FMT == QLIN_FMT_INT8);
@@ -110,7 +115,7 @@ struct Cfg {
     static constexpr int BM = 128;                 // P rows per tile (MMA M)
     static constexpr int BK = 128;                 // K bytes per stage: one swizzle atom
     static constexpr int P_BYTES = BM * BK;
-    static constexpr int Q_BYTES = BN * BK;
+    static constexpr int Q_BYTES = (PAIR ? BN / 2 : BN) * BK;
     static constexpr int STAGE_BYTES = P_BYTES + (FUSE ? 0 : Q_BYTES);
     // FUSE: A codes of one unit, [K block][BN rows x 128 B] in the 128-byte
     // swizzled K-major layout, and the unit's activation scales (2 buffers)
@@ -133,7 +138,7 @@ struct Cfg {
     static constexpr int TOTAL_COL = (BLOCK ? 3 : 2) * ACC_COLS;  // running total over segments
     static constexpr int TMEM_COLS =
         pow2_at_least(2 * ACC_COLS + (MULTI ? ACC_COLS : 0) + (BLOCK ? ACC_COLS : 0));
-    static constexpr uint32_t IDESC = make_idesc(INT8, 128, BN);
+    static constexpr uint32_t IDESC = make_idesc(INT8, PAIR ? 256 : 128, BN);
     static constexpr size_t STAGING_OFF = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t SCALE_OFF = STAGING_OFF + kStagingBytes;
     static constexpr size_t BSCALE_OFF = SCALE_OFF + kScaleBytes;
@@ -154,8 +159,9 @@ struct Unit {
     int tile, seg, pt, qt, kb0, kb1, chunk_kb;
 };
 
-template <int FMT>
-__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
+// Pair tiles (PAIR): unit = 256-row tile; pt is this CTA's 128-row half of it.
+template <int FMT, bool PAIR = false>
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int rank = 0) {
     Unit r;
     if (a.spread) {
         r.seg = u % a.S;
@@ -168,8 +174,14 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u) {
         r.kb0 = 0;
         r.kb1 = a.kblocks;
     }
-    r.pt = r.tile % a.p_tiles;
-    r.qt = r.tile / a.p_tiles;
+    if constexpr (PAIR) {
+        const int pairs = (a.p_tiles + 1) >> 1;
+        r.pt = 2 * (r.tile % pairs) + rank;
+        r.qt = r.tile / pairs;
+    } else {
+        r.pt = r.tile % a.p_tiles;
+        r.qt = r.tile / a.p_tiles;
+    }
     if (FMT == QLIN_FMT_FP8_BLOCK)
         r.chunk_kb = 1;
     else if (FMT == QLIN_FMT_INT8)
@@ -727,11 +739,11 @@ __device__ __forceinline__ void fused_quantize_unit(const GemmArgs& a, const Uni
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE>
+template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     qlin_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ GemmArgs args) {
-    using C = Cfg<FMT, SWAP, BN, CSK, FUSE>;
+    using C = Cfg<FMT, SWAP, BN, CSK, FUSE, PAIR>;
     constexpr int STAGES = C::STAGES;
     constexpr int SW = C::SW;
 
@@ -760,6 +772,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // PAIR: both CTAs of a cluster walk the same pair tiles; rank 0 leads
+    const int rank = PAIR ? (int)cluster_ctarank() : 0;
+    const int u_first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int u_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
     if (warp == kProducerWarp && lane == 0) {
         prefetch_tmap(&tmap_p);
@@ -770,7 +786,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
-            mbar_init(tempty0 + 8 * b, kEpiWarps);  // one arrival per epilogue warp
+            // one arrival per epilogue warp (PAIR: of both CTAs, on rank 0's barrier)
+            mbar_init(tempty0 + 8 * b, PAIR ? 2 * kEpiWarps : kEpiWarps);
         }
         if constexpr (CSK) {
             mbar_init(recv_full, (args.S - 1) * kEpiWarps);  // every epilogue warp of every other rank
@@ -783,13 +800,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_mbarrier_init();
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
-        tmem_relinquish();
+        if constexpr (PAIR) {
+            tmem_alloc_pair(smem_u32(tmem_holder), C::TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if constexpr (CSK) cluster_sync();  // every rank's barriers are initialised before any remote arrive
+    // every rank's barriers are initialised before any remote arrive or load signal
+    if constexpr (CSK || PAIR) cluster_sync();
     const uint32_t tmem_base = *tmem_holder;
     pdl_launch_dependents();
 
@@ -800,46 +823,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pol_a = policy_evict_last();
             const CUtensorMap* tm_w = SWAP ? &tmap_p : &tmap_q;
             const CUtensorMap* tm_a = SWAP ? &tmap_q : &tmap_p;
+            // PAIR: both CTAs' loads of a stage are counted on rank 0's full
+            // barrier, which rank 0 alone arms with the bytes of both
+            const uint32_t stage_tx = PAIR ? 2 * C::STAGE_BYTES : C::STAGE_BYTES;
+            const int w_row_off = PAIR ? rank * (BN / 2) : 0;  // this CTA's half of the W tile
+            auto arm = [&](uint32_t fb) {
+                if (!PAIR || rank == 0) mbar_arrive_expect_tx(fb, stage_tx);
+            };
+            auto load = [&](uint32_t dst, const CUtensorMap* m, int x, int y, uint32_t fb, uint64_t pol) {
+                if constexpr (PAIR)
+                    tma_load_2d_pair(dst, m, x, y, mapa_shared(fb, 0), pol);
+                else
+                    tma_load_2d(dst, m, x, y, fb, pol);
+            };
+            auto load_w = [&](uint32_t stage, const Unit& un, int kb, uint32_t fb) {
+                if constexpr (SWAP)
+                    load(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_w, kb * 128, un.pt * 128, fb, pol_w);
+                else
+                    load(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_w, kb * 128, un.qt * BN + w_row_off, fb,
+                         pol_w);
+            };
             // weights do not depend on the previous kernel: start streaming the
             // first unit's weight tiles before waiting for it
             int pre = 0;
-            if ((int)blockIdx.x < args.units) {
-                const Unit un = decode_unit<FMT>(args, blockIdx.x);
+            if (u_first < args.units) {
+                const Unit un = decode_unit<FMT, PAIR>(args, u_first, rank);
                 for (int kb = un.kb0; kb < un.kb1 && pre < STAGES; ++kb, ++pre) {
-                    mbar_arrive_expect_tx(full0 + 8 * pre, C::STAGE_BYTES);
-                    if constexpr (SWAP)
-                        tma_load_2d(smem_u32(sP + (size_t)pre * C::P_BYTES), tm_w, kb * 128, un.pt * 128,
-                                    full0 + 8 * pre, pol_w);
-                    else
-                        tma_load_2d(smem_u32(sQ + (size_t)pre * C::Q_BYTES), tm_w, kb * 128, un.qt * BN,
-                                    full0 + 8 * pre, pol_w);
+                    arm(full0 + 8 * pre);
+                    load_w(pre, un, kb, full0 + 8 * pre);
                 }
             }
             pdl_wait();
             uint32_t stage = 0, phase = 0;
             int it = 0;
-            for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
-                const Unit un = decode_unit<FMT>(args, u);
+            for (int u = u_first; u < args.units; u += u_step) {
+                const Unit un = decode_unit<FMT, PAIR>(args, u, rank);
                 for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
                     const uint32_t fb = full0 + 8 * stage;
                     if (it >= pre) {
-                        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) goto done;
-                        mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-                        if constexpr (SWAP)
-                            tma_load_2d(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_w, kb * 128, un.pt * 128,
-                                        fb, pol_w);
-                        else
-                            tma_load_2d(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_w, kb * 128, un.qt * BN,
-                                        fb, pol_w);
+                        const bool freed = PAIR ? mbar_wait_cluster(empty0 + 8 * stage, phase ^ 1)
+                                                : mbar_wait(empty0 + 8 * stage, phase ^ 1);
+                        if (!freed) goto done;
+                        arm(fb);
+                        load_w(stage, un, kb, fb);
                     }
                     if constexpr (FUSE)
                         (void)pol_a;  // the activation operand is quantised in place
                     else if constexpr (SWAP)
-                        tma_load_2d(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_a, kb * 128, un.qt * BN, fb,
-                                    pol_a);
+                        load(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_a, kb * 128, un.qt * BN, fb, pol_a);
                     else
-                        tma_load_2d(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_a, kb * 128, un.pt * 128, fb,
-                                    pol_a);
+                        load(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_a, kb * 128, un.pt * 128, fb, pol_a);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
@@ -849,36 +882,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // -------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // (PAIR: rank 0 issues for both CTAs; rank 1's MMA warp only holds TMEM)
+        if (lane == 0 && (!PAIR || rank == 0)) {
             uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0, uphase = 0;
-            for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
-                const Unit un = decode_unit<FMT>(args, u);
+            for (int u = u_first; u < args.units; u += u_step) {
+                const Unit un = decode_unit<FMT, PAIR>(args, u, rank);
                 if constexpr (FUSE) {
                     if (!mbar_wait(a_full, uphase)) goto done;
                     tc_fence_after();
                 }
                 for (int c0 = un.kb0; c0 < un.kb1; c0 += un.chunk_kb) {
-                    if (!mbar_wait(tempty0 + 8 * abuf, aphase ^ 1)) goto done;
+                    const bool acc_free = PAIR ? mbar_wait_cluster(tempty0 + 8 * abuf, aphase ^ 1)
+                                               : mbar_wait(tempty0 + 8 * abuf, aphase ^ 1);
+                    if (!acc_free) goto done;
                     tc_fence_after();
                     const uint32_t d = tmem_base + abuf * C::ACC_COLS;
                     for (int kb = c0; kb < c0 + un.chunk_kb; ++kb) {
-                        if (!mbar_wait(full0 + 8 * stage, phase)) goto done;
+                        const bool landed = PAIR ? mbar_wait_cluster(full0 + 8 * stage, phase)
+                                                 : mbar_wait(full0 + 8 * stage, phase);
+                        if (!landed) goto done;
                         tc_fence_after();
                         const uint64_t adesc = smem_desc_k_sw128(smem_u32(sP + (size_t)stage * C::P_BYTES));
                         const uint64_t bdesc =
                             FUSE ? smem_desc_k_sw128(sA + (uint32_t)((kb - un.kb0) * BN * 128))
                                  : smem_desc_k_sw128(smem_u32(sQ + (size_t)stage * C::Q_BYTES));
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)  // 4 x K=32 bytes per 128-byte stage
-                            tc_mma<C::INT8>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC,
-                                            (kb > c0 || k > 0) ? 1u : 0u);
-                        tc_commit(empty0 + 8 * stage);
+                        for (int k = 0; k < 4; ++k) {  // 4 x K=32 bytes per 128-byte stage
+                            const uint32_t accum = (kb > c0 || k > 0) ? 1u : 0u;
+                            if constexpr (PAIR)
+                                tc_mma_pair<C::INT8>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
+                            else
+                                tc_mma<C::INT8>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
+                        }
+                        if constexpr (PAIR)
+                            tc_commit_pair(empty0 + 8 * stage, 0x3);  // both CTAs may refill the stage
+                        else
+                            tc_commit(empty0 + 8 * stage);
                         if (++stage == STAGES) {
                             stage = 0;
                             phase ^= 1;
                         }
                     }
-                    tc_commit(tfull0 + 8 * abuf);
+                    if constexpr (PAIR)
+                        tc_commit_pair(tfull0 + 8 * abuf, 0x3);  // both CTAs' accumulators are ready
+                    else
+                        tc_commit(tfull0 + 8 * abuf);
                     abuf ^= 1;
                     if (abuf == 0) aphase ^= 1;
                 }
@@ -916,16 +964,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_total = t_lane + C::TOTAL_COL;
         const uint32_t t_seg = t_lane + C::SEG_COL;
         uint32_t abuf = 0, aphase = 0;
+        // accumulator hand-over; PAIR: rank 0's MMAs fill both CTAs' TMEM and
+        // both CTAs' epilogue warps hand the buffer back on rank 0's barrier
+        auto acc_wait = [&](uint32_t bar, uint32_t parity) {
+            return PAIR ? warp_wait_cluster(bar, parity) : warp_wait(bar, parity);
+        };
+        auto acc_release = [&](uint32_t bar) {
+            if constexpr (PAIR) {
+                __syncwarp();
+                if (lane == 0) {
+                    if (rank == 0)
+                        mbar_arrive(bar);
+                    else
+                        mbar_arrive_remote(mapa_shared(bar, 0));
+                }
+            } else {
+                warp_arrive(bar);
+            }
+        };
         if constexpr (FUSE) {
-            if ((int)blockIdx.x < args.units) {
-                fused_quantize_unit<FMT, BN, C::A_MAXKB>(args, decode_unit<FMT>(args, blockIdx.x), sA, sa_tile,
+            if (u_first < args.units) {
+                fused_quantize_unit<FMT, BN, C::A_MAXKB>(args, decode_unit<FMT>(args, u_first), sA, sa_tile,
                                                          rmax, xstage, kStagingBytes);
                 warp_arrive(a_full);
             }
         }
         int ui = 0;  // this CTA's unit count so far (fused: scale buffer ui % 2)
-        for (int u = blockIdx.x; u < args.units; u += gridDim.x, ++ui) {
-            const Unit un = decode_unit<FMT>(args, u);
+        for (int u = u_first; u < args.units; u += u_step, ++ui) {
+            const Unit un = decode_unit<FMT, PAIR>(args, u, rank);
             const float* sa_cur = sa_tile + (ui & 1) * C::SA_FLOATS;
             // Fused: the next unit's rows are quantised once the MMA is done
             // with this unit's.  A unit whose MMAs fill one accumulator is
@@ -933,7 +999,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // quantised first and its MMAs overlap this epilogue; a unit of
             // several accumulator chunks needs this epilogue to drain them
             // first, so its successor waits until after it.
-            const int nxt = u + (int)gridDim.x;
+            const int nxt = u + u_step;
             const bool quantise_next = FUSE && nxt < args.units;
             const bool next_first = (un.kb1 - un.kb0) == un.chunk_kb;
             if (quantise_next && next_first) {
@@ -970,12 +1036,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nchunks = (un.kb1 - un.kb0) / un.chunk_kb;
             if (nchunks == 1 && !C::BLOCK) {
                 // one accumulator holds the whole unit: stream this warp's slices
-                if (!warp_wait(tfull0 + 8 * abuf, aphase)) goto done;
+                if (!acc_wait(tfull0 + 8 * abuf, aphase)) goto done;
                 tc_fence_after();
                 const uint32_t tacc = t_lane + abuf * C::ACC_COLS;
                 if (e.half >= C::NSLICE) {  // no slice for this warp: hand the buffer back
                     tc_fence_before();
-                    warp_arrive(tempty0 + 8 * abuf);
+                    acc_release(tempty0 + 8 * abuf);
                 }
 #pragma unroll 1
                 for (int j = e.half; j < C::NSLICE; j += 2) {
@@ -984,7 +1050,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_wait_ld();
                     if (j + 2 >= C::NSLICE) {  // this warp's last read of the accumulator
                         tc_fence_before();
-                        warp_arrive(tempty0 + 8 * abuf);
+                        acc_release(tempty0 + 8 * abuf);
                     }
                     if (!consume_segment_slice<FMT, SWAP, BN, CSK>(args, un, un.seg, j, t_total, e, v)) goto done;
                 }
@@ -1047,7 +1113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float row_scale = 0.f;
                         if constexpr (!SWAP)
                             asm volatile("ld.shared.f32 %0, [%1];" : "=f"(row_scale) : "r"(bsrow + e.row_lane * 4u));
-                        if (!warp_wait(tfull0 + 8 * abuf, aphase)) goto done;
+                        if (!acc_wait(tfull0 + 8 * abuf, aphase)) goto done;
                         tc_fence_after();
                         const uint32_t tacc = t_lane + abuf * C::ACC_COLS;
 #pragma unroll 1
@@ -1080,7 +1146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         tc_wait_st();
                         tc_fence_before();
-                        warp_arrive(tempty0 + 8 * abuf);
+                        acc_release(tempty0 + 8 * abuf);
                         abuf ^= 1;
                         if (abuf == 0) aphase ^= 1;
                     }
@@ -1089,7 +1155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // segment, summed into the TMEM running total in order.
                     int seg_no = 0;
                     for (int c0 = un.kb0; c0 < un.kb1; c0 += un.chunk_kb, ++seg_no) {
-                        if (!warp_wait(tfull0 + 8 * abuf, aphase)) goto done;
+                        if (!acc_wait(tfull0 + 8 * abuf, aphase)) goto done;
                         tc_fence_after();
                         const uint32_t tacc = t_lane + abuf * C::ACC_COLS;
 #pragma unroll 1
@@ -1102,7 +1168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         tc_wait_st();
                         tc_fence_before();
-                        warp_arrive(tempty0 + 8 * abuf);
+                        acc_release(tempty0 + 8 * abuf);
                         abuf ^= 1;
                         if (abuf == 0) aphase ^= 1;
                     }
@@ -1140,10 +1206,18 @@ done:
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kMmaWarp) tmem_dealloc(tmem_base, C::TMEM_COLS);
-    // no CTA leaves while another rank may still arrive on its barriers or
-    // store into its shared memory
-    if constexpr (CSK) cluster_sync();
+    if constexpr (PAIR) {
+        // both CTAs are done with the TMEM that rank 0's MMAs wrote, and with
+        // each other's barriers, before the pair frees its columns
+        cluster_sync();
+        tc_fence_after();
+        if (warp == kMmaWarp) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    } else {
+        if (warp == kMmaWarp) tmem_dealloc(tmem_base, C::TMEM_COLS);
+        // no CTA leaves while another rank may still arrive on its barriers or
+        // store into its shared memory
+        if constexpr (CSK) cluster_sync();
+    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -1175,10 +1249,10 @@ bool make_operand_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE>
+template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE, bool PAIR>
 qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaStream_t st) {
-    using C = Cfg<FMT, SWAP, BN, CSK, FUSE>;
-    auto kern = qlin_gemm_kernel<FMT, SWAP, BN, CSK, FUSE>;
+    using C = Cfg<FMT, SWAP, BN, CSK, FUSE, PAIR>;
+    auto kern = qlin_gemm_kernel<FMT, SWAP, BN, CSK, FUSE, PAIR>;
     static int configured_device = -1;
     static int max_clusters[QLIN_MAX_CLUSTER + 1];  // co-resident clusters per cluster size, this device
     int dev = 0;
@@ -1198,7 +1272,7 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     if (!make_operand_tmap(&tp, p_base, plan.p_rows, plan.K, 128)) return QLIN_ERR_CUDA;
     if (FUSE)
         tq = tp;  // unused: the kernel quantises its activation operand in place
-    else if (!make_operand_tmap(&tq, q_base, plan.q_rows, plan.K, BN))
+    else if (!make_operand_tmap(&tq, q_base, plan.q_rows, plan.K, PAIR ? BN / 2 : BN))  // PAIR: half a W tile
         return QLIN_ERR_CUDA;
     GemmArgs a;
     a.s_a = ops.s_a;
@@ -1231,23 +1305,24 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     int nattr = 0;
-    if (CSK) {
+    const int csize = PAIR ? 2 : S;  // CTAs per cluster
+    if (CSK || PAIR) {
         attr[nattr].id = cudaLaunchAttributeClusterDimension;
-        attr[nattr].val.clusterDim.x = (unsigned)S;
+        attr[nattr].val.clusterDim.x = (unsigned)csize;
         attr[nattr].val.clusterDim.y = 1;
         attr[nattr].val.clusterDim.z = 1;
         ++nattr;
         cfg.attrs = attr;
         cfg.numAttrs = nattr;
-        if (max_clusters[S] < 0) {
+        if (max_clusters[csize] < 0) {
             int n = 0;
             if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) return QLIN_ERR_CUDA;
-            max_clusters[S] = n;
+            max_clusters[csize] = n;
         }
-        if (max_clusters[S] < 1) return QLIN_ERR_UNSUPPORTED;
-        // every CTA of a cluster walks the same tiles: grid = clusters x S
-        const int64_t clusters = std::min<int64_t>(plan.num_tiles, max_clusters[S]);
-        cfg.gridDim = dim3((unsigned)(clusters * S));
+        if (max_clusters[csize] < 1) return QLIN_ERR_UNSUPPORTED;
+        // every CTA of a cluster walks the same tiles: grid = clusters x cluster size
+        const int64_t clusters = std::min<int64_t>(plan.num_tiles, max_clusters[csize]);
+        cfg.gridDim = dim3((unsigned)(clusters * csize));
     }
     if (ops.pdl) {
         attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1260,54 +1335,63 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
 }
 
-template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE>
+template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE, bool PAIR>
 void cfg_info(int* stages, size_t* smem) {
-    *stages = Cfg<FMT, SWAP, BN, CSK, FUSE>::STAGES;
-    *smem = Cfg<FMT, SWAP, BN, CSK, FUSE>::SMEM;
+    *stages = Cfg<FMT, SWAP, BN, CSK, FUSE, PAIR>::STAGES;
+    *smem = Cfg<FMT, SWAP, BN, CSK, FUSE, PAIR>::SMEM;
 }
 
-// One switch over every kernel instantiation: OP<FMT, SWAP, BN, CSK, FUSE>
+// One switch over every kernel instantiation: OP<FMT, SWAP, BN, CSK, FUSE, PAIR>
 // is applied to the one matching (swap, tile_n, mode); false if none exists.
-template <int FMT, template <int, bool, int, bool, bool> class OP, typename... A>
+template <int FMT, template <int, bool, int, bool, bool, bool> class OP, typename... A>
 bool dispatch_instance(bool swap, int tile_n, int mode, A&&... args) {
     if (swap) {
         switch (mode * 1000 + tile_n) {
-            case kModeStd * 1000 + 16: OP<FMT, true, 16, false, false>::run(args...); return true;
-            case kModeStd * 1000 + 32: OP<FMT, true, 32, false, false>::run(args...); return true;
-            case kModeStd * 1000 + 64: OP<FMT, true, 64, false, false>::run(args...); return true;
-            case kModeCluster * 1000 + 16: OP<FMT, true, 16, true, false>::run(args...); return true;
-            case kModeCluster * 1000 + 32: OP<FMT, true, 32, true, false>::run(args...); return true;
-            case kModeCluster * 1000 + 64: OP<FMT, true, 64, true, false>::run(args...); return true;
-            case kModeFused * 1000 + 16: OP<FMT, true, 16, false, true>::run(args...); return true;
-            case kModeFused * 1000 + 32: OP<FMT, true, 32, false, true>::run(args...); return true;
-            case kModeFused * 1000 + 64: OP<FMT, true, 64, false, true>::run(args...); return true;
+            case kModeStd * 1000 + 16: OP<FMT, true, 16, false, false, false>::run(args...); return true;
+            case kModeStd * 1000 + 32: OP<FMT, true, 32, false, false, false>::run(args...); return true;
+            case kModeStd * 1000 + 64: OP<FMT, true, 64, false, false, false>::run(args...); return true;
+            case kModeCluster * 1000 + 16: OP<FMT, true, 16, true, false, false>::run(args...); return true;
+            case kModeCluster * 1000 + 32: OP<FMT, true, 32, true, false, false>::run(args...); return true;
+            case kModeCluster * 1000 + 64: OP<FMT, true, 64, true, false, false>::run(args...); return true;
+            case kModeFused * 1000 + 16: OP<FMT, true, 16, false, true, false>::run(args...); return true;
+            case kModeFused * 1000 + 32: OP<FMT, true, 32, false, true, false>::run(args...); return true;
+            case kModeFused * 1000 + 64: OP<FMT, true, 64, false, true, false>::run(args...); return true;
+        }
+        return false;
+    }
+    if (mode == kModePair) {
+        if constexpr (FMT != QLIN_FMT_FP8_BLOCK) {
+            if (tile_n == 256) {
+                OP<FMT, false, 256, false, false, true>::run(args...);
+                return true;
+            }
         }
         return false;
     }
     if (mode != kModeStd) return false;
     if (tile_n == 128) {
-        OP<FMT, false, 128, false, false>::run(args...);
+        OP<FMT, false, 128, false, false, false>::run(args...);
         return true;
     }
     if constexpr (FMT != QLIN_FMT_FP8_BLOCK) {
         if (tile_n == 256) {
-            OP<FMT, false, 256, false, false>::run(args...);
+            OP<FMT, false, 256, false, false, false>::run(args...);
             return true;
         }
     }
     return false;
 }
 
-template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE>
+template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE, bool PAIR>
 struct LaunchOp {
     static void run(const GemmPlan& p, const GemmOperands& ops, cudaStream_t st, qlin_status* out) {
-        *out = launch_instance<FMT, SWAP, BN, CSK, FUSE>(p, ops, st);
+        *out = launch_instance<FMT, SWAP, BN, CSK, FUSE, PAIR>(p, ops, st);
     }
 };
 
-template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE>
+template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE, bool PAIR>
 struct InfoOp {
-    static void run(int* stages, size_t* smem) { cfg_info<FMT, SWAP, BN, CSK, FUSE>(stages, smem); }
+    static void run(int* stages, size_t* smem) { cfg_info<FMT, SWAP, BN, CSK, FUSE, PAIR>(stages, smem); }
 };
 
 template <int FMT>

@@ -28,6 +28,7 @@ enum GemmMode : int {
     kModeStd = 0,      // operands from global memory by TMA; Split-K through the workspace
     kModeCluster = 1,  // Swap-AB Split-K reduced through a thread-block cluster
     kModeFused = 2,    // Swap-AB with the activation quantisation done by the GEMM itself
+    kModePair = 3,     // plain 256-row tiles on a pair of CTAs (cluster of 2, cta_group::2 MMA)
 };
 // Fused mode keeps the unit's activation codes resident: 64 KiB of shared
 // memory, so at most this many K blocks per unit.

@@ -70,7 +70,7 @@ extern "C" qlin_status qlin_scaled_mm_noalloc(int fmt, int variant, int tile_n, 
     const bool out_i32 = (flags & QLIN_OUT_I32ACC) != 0;
     if (out_i32 && fmt != QLIN_FMT_INT8) return QLIN_ERR_INVALID_ARG;
     if (fmt == QLIN_FMT_FP8_BLOCK && bias) return QLIN_ERR_INVALID_ARG;
-    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_SWAPAB_SPLITK || tile_n < 0 || k_segments < 0)
+    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_PAIR || tile_n < 0 || k_segments < 0)
         return QLIN_ERR_INVALID_ARG;
     if (M < 0) return QLIN_ERR_INVALID_ARG;
     const int sms = current_device_sms();

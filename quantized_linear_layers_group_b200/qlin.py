@@ -40,6 +40,7 @@ QLIN_VAR_PLAIN = 1
 QLIN_VAR_SPLITK = 2
 QLIN_VAR_SWAPAB = 3
 QLIN_VAR_SWAPAB_SPLITK = 4
+QLIN_VAR_PAIR = 5
 
 QLIN_OUT_I32ACC = 1
 QLIN_PDL = 2
@@ -47,7 +48,7 @@ QLIN_SPLITK_CLUSTER = 4  # Swap-AB Split-K: reduce through a thread-block cluste
 QLIN_FUSED = 8  # qlin_linear: the GEMM quantises its own activation rows where it can (one kernel)
 
 VARIANT_NAMES = {QLIN_VAR_AUTO: "auto", QLIN_VAR_PLAIN: "plain", QLIN_VAR_SPLITK: "splitk",
-                 QLIN_VAR_SWAPAB: "swapab", QLIN_VAR_SWAPAB_SPLITK: "swapab_splitk"}
+                 QLIN_VAR_SWAPAB: "swapab", QLIN_VAR_SWAPAB_SPLITK: "swapab_splitk", QLIN_VAR_PAIR: "pair"}
 
 # every symbol include/qlin.h declares
 EXPORTS = ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_scaled_mm_noalloc", "qlin_linear",

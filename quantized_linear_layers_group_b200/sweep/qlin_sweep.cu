@@ -62,6 +62,7 @@ const char* var_name(int v) {
         case QLIN_VAR_SPLITK: return "splitk";
         case QLIN_VAR_SWAPAB: return "swapab";
         case QLIN_VAR_SWAPAB_SPLITK: return "swapab_splitk";
+        case QLIN_VAR_PAIR: return "pair";
     }
     return "auto";
 }
@@ -122,6 +123,8 @@ std::vector<Cand> candidates(int fmt, int64_t M) {
             c.push_back({QLIN_VAR_PLAIN, t});
             c.push_back({QLIN_VAR_SPLITK, t});
         }
+        // 256-row tiles on CTA pairs: only worth a try once M fills two 128-row halves
+        if (fmt != QLIN_FMT_FP8_BLOCK && M >= 256) c.push_back({QLIN_VAR_PAIR, 256});
     }
     return c;
 }

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(q):
     for name in _declared_symbols():
         assert hasattr(lib, name), name
     assert set(_declared_symbols()) == set(q.EXPORTS)
-    assert q.qlin_abi_version() == 3
+    assert q.qlin_abi_version() == 4
 
 
 def test_status_strings(q):
@@ -106,6 +106,14 @@ def test_workspace_sizes(q):
                                         k_segments=4)                            # multi-chunk on a 256 tile
     with pytest.raises(q.QlinError):
         q.qlin_scaled_mm_workspace_size(1, 16, 256, 256, variant=q.QLIN_VAR_SWAPAB, tile_n=128)
+    # CTA-pair tiles: 256 columns, INT8 / FP8 only, no workspace, no multi-chunk FP8
+    assert q.qlin_scaled_mm_workspace_size(1, 2048, 4096, 2048, variant=q.QLIN_VAR_PAIR, k_segments=1) == 0
+    assert q.qlin_scaled_mm_workspace_size(0, 300, 2048, 2048, variant=q.QLIN_VAR_PAIR, k_segments=4) == 0
+    for fmt, kw in ((1, dict(tile_n=128)), (2, {}), (1, dict(k_segments=2))):
+        with pytest.raises(q.QlinError):
+            q.qlin_scaled_mm_workspace_size(fmt, 2048, 4096, 2048, variant=q.QLIN_VAR_PAIR, **kw)
+    with pytest.raises(q.QlinError):
+        q.qlin_scaled_mm_workspace_size(1, 16, 256, 256, variant=6)
 
 
 def test_builtin_dispatch_rule(q):

@@ -15,7 +15,7 @@ from helpers import assert_parity, bits_u8, bits_u16, check_status, gpu_gemm, gp
 
 pytestmark = pytest.mark.gpu
 
-PLAIN, SPLITK, SWAPAB, SWAPAB_SPLITK = 1, 2, 3, 4
+PLAIN, SPLITK, SWAPAB, SWAPAB_SPLITK, PAIR = 1, 2, 3, 4, 5
 FMTS = [oracle.FMT_INT8, oracle.FMT_FP8, oracle.FMT_FP8_BLOCK]
 
 
@@ -64,6 +64,7 @@ def _variants(fmt, K):
         out.append((PLAIN, 128, s))
         if fmt != oracle.FMT_FP8_BLOCK and (fmt == oracle.FMT_INT8 or s == 1):
             out.append((PLAIN, 256, s))
+            out.append((PAIR, 256, s))
         for t in (16, 32, 64):
             out.append((SWAPAB, t, s))
         if s > 1:
@@ -171,6 +172,7 @@ def test_extreme_depths(fmt, M, N, K):
     ref = p.reference()
     kb = K // 128
     for var, tile, s in [(PLAIN, 128, 1), (SWAPAB, 16, 1), (SWAPAB, 64, 1)] + \
+            ([(PAIR, 256, 1)] if fmt != oracle.FMT_FP8_BLOCK else []) + \
             ([(SPLITK, 128, 8), (SWAPAB_SPLITK, 16, 8), (PLAIN, 128, 8)] if kb % 8 == 0 else []):
         c = p.run(var, tile, s)
         assert_parity(fmt, bits_u16(c), ref, f"fmt={fmt} M={M} N={N} K={K} var={var} tile={tile} S={s}")
@@ -197,3 +199,27 @@ def test_empty_batch_is_a_no_op():
     a = torch.empty(0, 256, dtype=torch.uint8, device="cuda")
     qlin.qlin_scaled_mm(qlin.QLIN_FMT_FP8, a, s, w, s, None, c, M=0)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_INT8, oracle.FMT_FP8])
+@pytest.mark.parametrize("M,N,K", [(300, 25600, 1024), (1100, 4096, 2048), (2048, 4096, 2048), (129, 272, 640)])
+def test_pair_tiles_match_single_cta_tiles_and_oracle(fmt, M, N, K):
+    # 256-row tiles on CTA pairs (cta_group::2): every cluster walks several
+    # tiles (N=25600: 200 tiles on at most 74 pairs), the last pair's second
+    # CTA may hold no rows at all (M=1100, 129: an odd number of 128-row
+    # halves), and N tails inside the second CTA's half of a W tile (N=272).
+    # Bitwise equal to the one-CTA 256-column tiles with the same K
+    # segmentation, within the parity bar of the oracle on a row sample.
+    p = Prepared(fmt, *_problem(fmt, M, N, K, seed=M + N + K + 3 * fmt))
+    rows = np.unique(np.r_[0, 1, 127, 128, 255, 256, M - 1, np.arange(0, M, max(1, M // 24))])
+    rows = rows[rows < M]
+    segs = [1] if fmt == oracle.FMT_FP8 or (K // 128) % 4 else [1, 4]
+    for s in segs:
+        got = bits_u16(p.run(PAIR, 256, s))
+        want = bits_u16(p.run(PLAIN, 256, s))
+        assert np.array_equal(got, want), f"pair vs plain: fmt={fmt} M={M} N={N} K={K} S={s}"
+        assert_parity(fmt, got[rows], p.reference(m_idx=rows), f"pair fmt={fmt} M={M} N={N} K={K} S={s}")
+    if fmt == oracle.FMT_INT8:
+        acc = p.run(PAIR, 256, 1, out_i32=True).cpu().numpy()
+        assert np.array_equal(acc[rows], p.reference(m_idx=rows, want_acc=True)[1])
+    check_status()

@@ -24,7 +24,7 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 TABLE = os.path.join(ROOT, "quantized_linear_layers_group_b200", "tables", "b200.qlt")
 
-PLAIN, SPLITK, SWAPAB, SWAPAB_SPLITK = 1, 2, 3, 4
+PLAIN, SPLITK, SWAPAB, SWAPAB_SPLITK, PAIR = 1, 2, 3, 4, 5
 M_SET = [1, 2, 3, 5, 8, 15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 129, 255, 256, 257, 511, 512, 700, 1023,
          1024, 1025, 2047, 2048]
 
@@ -41,7 +41,7 @@ def table():
 def _forced(fmt):
     out = [(PLAIN, 128), (SPLITK, 128), (SWAPAB, 16), (SWAPAB, 64), (SWAPAB_SPLITK, 32)]
     if fmt != oracle.FMT_FP8_BLOCK:
-        out += [(PLAIN, 256), (SPLITK, 256)]
+        out += [(PLAIN, 256), (SPLITK, 256), (PAIR, 256)]
     return out
 
 
