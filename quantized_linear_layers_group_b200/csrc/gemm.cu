@@ -220,7 +220,7 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
 // one on the same barrier serialise on it.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
     int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_idle(bar, parity) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 

@@ -78,6 +78,33 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     return mbar_wait_for(bar, parity, QLIN_WAIT_LIMIT_NS);
 }
 
+// try_wait that lets the hardware suspend the thread for up to hint_ns while
+// the phase is incomplete, instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for threads with nothing else to do meanwhile (the epilogue):
+// suspended in the barrier rather than polling it.
+__device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait_suspend(bar, parity, 100000u)) return true;
+        if (globaltimer_ns() - t0 > QLIN_WAIT_LIMIT_NS) {
+            atomicExch(&g_device_status, 9 /* QLIN_ERR_DEVICE_TIMEOUT */);
+            return false;
+        }
+    }
+}
+
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
