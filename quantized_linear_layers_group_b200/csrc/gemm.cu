@@ -237,6 +237,7 @@ struct EpiCtx {
     uint32_t s_col;                  // shared address of the tile's column scales
     uint32_t b_col;                  // shared address of the tile's column bias
     uint32_t staging;                // shared address of this warp's 2 KB transpose buffer
+    const CUtensorMap* tmap_c;       // plain tiles: bf16 C as a tensor of 32 x 32 boxes (64-byte swizzle)
     bool has_bias;
     // cluster Split-K only
     int rank;                        // CTA rank in the cluster = K segment
@@ -328,28 +329,28 @@ __device__ __forceinline__ void finish_slice(const GemmArgs& a, const Unit& un, 
                 if (m0 + c < a.M) cb[(size_t)(m0 + c) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y[c]));
         }
     } else {
-        // The warp's 32 x 32 box of C is transposed through shared memory so that
-        // every store instruction writes whole 64-byte row segments (4 lanes per
-        // row).  Chunk q of row r sits at q ^ ((r >> 1) & 3): conflict-free both ways.
+        // The warp's 32 x 32 box of C goes to shared memory row by row (lane =
+        // row, 64 bytes, chunk q of row r at q ^ ((r >> 1) & 3): the 64-byte
+        // swizzle) and from there to global memory as one bulk tensor store,
+        // which also leaves out the rows and columns past the edges of C.
         const int bx = un.qt * BN + j * SW;
         const int by = un.pt * 128 + e.quad * 32;
         if (bx >= a.N || by >= a.M) return;  // warp-uniform: the whole box is outside C
+        (void)cb;
         uint32_t packed[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) packed[c / 2] = pack_bf16x2(y[c], y[c + 1]);
-        __syncwarp();  // every lane has read the previous box back
+        if (e.lane == 0) bulk_wait_read_all();  // the previous box has left the buffer
+        __syncwarp();
 #pragma unroll
         for (int q = 0; q < 4; ++q)
             sts_u4(e.staging + e.lane * 64 + ((q ^ ((e.lane >> 1) & 3)) * 16),
                    make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]));
+        fence_proxy_async_shared();
         __syncwarp();
-        const int q = e.lane & 3;
-#pragma unroll
-        for (int r0 = 0; r0 < 32; r0 += 8) {
-            const int r = r0 + (e.lane >> 2);
-            const uint4 val = lds_u4(e.staging + r * 64 + ((q ^ ((r >> 1) & 3)) * 16));
-            const int m = by + r, n = bx + q * 8;
-            if (m < a.M && n < a.N) *reinterpret_cast<uint4*>(cb + (size_t)m * a.N + n) = val;
+        if (e.lane == 0) {
+            tma_store_2d(e.tmap_c, bx, by, e.staging);
+            bulk_commit_group();
         }
     }
 }
@@ -742,7 +743,7 @@ __device__ __forceinline__ void fused_quantize_unit(const GemmArgs& a, const Uni
 template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     qlin_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
-                     const __grid_constant__ GemmArgs args) {
+                     const __grid_constant__ CUtensorMap tmap_c, const __grid_constant__ GemmArgs args) {
     using C = Cfg<FMT, SWAP, BN, CSK, FUSE, PAIR>;
     constexpr int STAGES = C::STAGES;
     constexpr int SW = C::SW;
@@ -947,6 +948,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         e.s_col = smem_u32(s_col);
         e.b_col = smem_u32(b_col);
         e.staging = smem_u32(smem + C::STAGING_OFF) + warp * 2048;
+        e.tmap_c = &tmap_c;
         e.has_bias = args.bias != nullptr;
         e.row_scale = 0.f;
         e.row_bias = 0.f;
@@ -1203,6 +1205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 done:
+    // the bulk stores of C have completed (and left the staging buffers)
+    if (!SWAP && warp < kEpiWarps && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1249,6 +1253,21 @@ bool make_operand_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t
     return r == CUDA_SUCCESS;
 }
 
+// bf16 C [M, N] (row stride N) as a 2-D tensor map with a 32 x 32 box and the
+// 64-byte swizzle (the layout the epilogue writes into its staging buffer).
+bool make_output_tmap(CUtensorMap* map, const void* base, int64_t M, int64_t N) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE, bool PAIR>
 qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaStream_t st) {
     using C = Cfg<FMT, SWAP, BN, CSK, FUSE, PAIR>;
@@ -1274,6 +1293,12 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
         tq = tp;  // unused: the kernel quantises its activation operand in place
     else if (!make_operand_tmap(&tq, q_base, plan.q_rows, plan.K, PAIR ? BN / 2 : BN))  // PAIR: half a W tile
         return QLIN_ERR_CUDA;
+    alignas(64) CUtensorMap tc;  // plain tiles: bf16 C in 32 x 32 boxes
+    if (!SWAP && !ops.out_i32) {
+        if (!make_output_tmap(&tc, ops.c, plan.M, plan.N)) return QLIN_ERR_CUDA;
+    } else {
+        tc = tp;  // unused (Swap-AB stores columns of C directly; int32 output stores directly)
+    }
     GemmArgs a;
     a.s_a = ops.s_a;
     a.s_w = ops.s_w;
@@ -1331,7 +1356,7 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     }
     cfg.attrs = attr;
     cfg.numAttrs = nattr;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tp, tq, a);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tp, tq, tc, a);
     return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
 }
 
