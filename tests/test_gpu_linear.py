@@ -168,3 +168,30 @@ def test_quantized_linear_module_uses_the_fused_call():
     ra_q, rs_a = oracle_quantize(fmt, x, False)
     rw_q, rs_w = oracle_quantize(fmt, w, True)
     assert_parity(fmt, bits_u16(c), oracle.scaled_mm(fmt, ra_q, rs_a, rw_q, rs_w, b), "module")
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_INT8, oracle.FMT_FP8])
+def test_layer_on_cta_pair_tiles(fmt):
+    # qlin_linear with the 256x256 CTA-pair tiles (the quantiser, then the
+    # pair GEMM; QLIN_FUSED does not apply to plain tiles and is ignored):
+    # codes and scales bit-exact, C bitwise equal to one-CTA 256-column tiles
+    # and within the parity bar of the oracle, with a strided x and a tail of
+    # rows and columns.
+    PAIR = 5
+    M, N, K = 300, 528, 1024
+    x, w, b = _inputs(fmt, M, N, K, seed=21 + fmt, pad=64)
+    layer = Layer(fmt, w, b)
+    x_dev = x.cuda()
+    rows = np.unique(np.r_[0, 127, 128, 255, 256, M - 1, np.arange(0, M, 11)])
+    c_pair, a_q, s_a = layer.run(x_dev, K, PAIR, 256, 1)
+    c_plain, _, _ = layer.run(x_dev, K, PLAIN, 256, 1)
+    assert np.array_equal(bits_u16(c_pair), bits_u16(c_plain)), "pair vs one-CTA tiles"
+    ra_q, rs_a = oracle_quantize(fmt, x[:, :K].contiguous(), False)
+    assert np.array_equal(bits_u8(a_q), ra_q)
+    assert np.array_equal(s_a.cpu().numpy().view(np.uint32), rs_a.view(np.uint32))
+    ref = oracle.scaled_mm(fmt, ra_q, rs_a, layer.rw_q, layer.rs_w, layer.b, m_idx=rows)
+    assert_parity(fmt, bits_u16(c_pair)[rows], ref, f"pair layer fmt={fmt}")
+    from quantized_linear_layers_group_b200 import qlin
+    c_fl, _, _ = layer.run(x_dev, K, PAIR, 256, 1, flags=qlin.QLIN_FUSED)
+    assert np.array_equal(bits_u16(c_fl), bits_u16(c_pair)), "QLIN_FUSED on pair tiles"
+    check_status()
