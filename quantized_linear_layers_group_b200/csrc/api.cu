@@ -510,7 +510,7 @@ qlin_status qlin_dispatch_table_load(const char* path) {
     for (const auto& e : entries) {
         int stages = 0;
         size_t smem = 0;
-        if (!gemm_kernel_info(e.fmt, is_swap(e.variant), e.tile_n, kModeStd, &stages, &smem) ||
+        if (!gemm_kernel_info(e.fmt, is_swap(e.variant), e.tile_n, base_mode(e.variant), &stages, &smem) ||
             smem > prop.sharedMemPerBlockOptin)
             return QLIN_ERR_TABLE_FORMAT;
     }

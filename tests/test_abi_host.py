@@ -156,11 +156,28 @@ def test_table_loader_rejects_bad_files(q, tmp_path):
         head + "entry fp8 4096 2048 16 swapab 16 4\nentry fp8 4096 2048 16 plain 128 4\n",  # duplicate bucket
         head + "entry fp8 4096 2048 256 plain 256 4\n",                        # multi-chunk 256 tile
         head + "entry fp8 4096 2048 16 swapab 16\n",                           # truncated
+        head + "entry fp8 4096 2048 2048 pair 128 1\n",                       # pair tiles are 256 wide
+        head + "entry fp8_block 2048 6144 2048 pair 256 4\n",                 # no Block-FP8 pair tiles
+        head + "entry fp8 4096 2048 2048 pair 256 2\n",                       # multi-chunk 256 tile
     ]
     for text in bad:
         with pytest.raises(q.QlinError) as e:
             q.qlin_dispatch_table_load(_write(tmp_path, text))
         assert e.value.status == q.QLIN_ERR_TABLE_FORMAT, text
+
+
+def test_pair_entries_pass_the_format_checks(q, tmp_path):
+    # a table with CTA-pair entries gets past every format check; only the
+    # device guard (which needs a B200) can refuse it here
+    text = ("qlin-dispatch 1\ndevice 148 10 0 NVIDIA B200\n"
+            "entry fp8 151936 2048 16 swapab 16 1\nentry fp8 151936 2048 2048 pair 256 1\n"
+            "entry int8 2048 2048 16 swapab_splitk 16 4\nentry int8 2048 2048 2048 pair 256 4\n")
+    try:
+        q.qlin_dispatch_table_load(_write(tmp_path, text))
+    except q.QlinError as e:
+        assert e.status in (q.QLIN_ERR_NO_DEVICE, q.QLIN_ERR_TABLE_DEVICE, q.QLIN_ERR_CUDA), e
+    finally:
+        q.qlin_dispatch_table_clear()
 
 
 def test_shipped_table_parses(q, tmp_path):
