@@ -109,6 +109,55 @@ def measured_traffic(workload, fmt, M, N, K, cfg):
     return None
 
 
+def kernel_of(fmt, cfg):
+    """The compiled GEMM kernel a configuration runs, named as in the ncu
+    launch list: qlin_gemm_kernel<format, swap_ab, tile_n, cluster, fused, pair>.
+    Split-K shares the kernel of its orientation (the split is a run-time
+    argument)."""
+    from quantized_linear_layers_group_b200 import qlin
+
+    v = cfg["variant"]
+    swap = int(v in (qlin.QLIN_VAR_SWAPAB, qlin.QLIN_VAR_SWAPAB_SPLITK))
+    pair = int(v == qlin.QLIN_VAR_PAIR)
+    return f"qlin_gemm_kernel<{fmt}, {swap}, {cfg['tile_n']}, 0, 0, {pair}>"
+
+
+def kernel_roofline(per_m, configs, fmt, N, K, hbm, tc_peak, total_dev_us):
+    """Roofline of the dominant GEMM kernel: launches grouped by the kernel they
+    run, the group with the largest share of the step's device time.  achieved
+    = mean algorithmic bytes (or flops) per launch / mean launch duration; the
+    bound is the larger of the group's summed HBM and tensor roofline times."""
+    groups = {}
+    for r in per_m:
+        groups.setdefault(kernel_of(fmt, configs[r["M"]]), []).append(r)
+    name, rows = max(groups.items(), key=lambda kv: sum(r["gemm_us"] for r in kv[1]))
+    ms = [r["M"] for r in rows]
+    t_mean = statistics.mean(r["gemm_us"] for r in rows) * 1e-6
+    ab = [gemm_bytes(M, N, K, fmt)[0] for M in ms]
+    fl = [gemm_flops(M, N, K) for M in ms]
+    t_hbm = sum(b / (hbm * 1e9) for b in ab)
+    t_tc = sum(f / (tc_peak * 1e12) for f in fl)
+    out = {"kernel": name, "m_values": ms, "launches_per_step": len(ms),
+           "share": sum(r["gemm_us"] for r in rows) / total_dev_us, "mean_launch_us": t_mean * 1e6}
+    if t_hbm >= t_tc:
+        a = statistics.mean(ab) / t_mean / 1e9
+        out.update({"bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm})
+    else:
+        a = statistics.mean(fl) / t_mean / 1e12
+        out.update({"bound": "tensor", "achieved": a, "peak": tc_peak, "unit": "TFLOP/s", "frac": a / tc_peak})
+    return out
+
+
+def measured_traffic_kernel(workload, fmt, N, K, configs, ms):
+    """DRAM bytes of one launch of the dominant kernel, from the committed ncu
+    record of one of its launches (the first M of the group that has one)."""
+    for M in ms:
+        t = measured_traffic(workload, fmt, M, N, K, configs[M])
+        if t is not None:
+            return t
+    return None
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons with nvidia-smi during the timed region."""
@@ -504,18 +553,19 @@ def main(argv=None):
         share = tg / (total_dev / 1e3)
         if dominant is None or share > dominant[0]:
             dominant = (share, M, tg, ab, fl)
+    roof = kernel_roofline(per_m, hp.configs, fmt, N, K, hbm, tc_peak, total_dev * 1e3)  # total_dev in ms
+    roof["traffic"] = measured_traffic_kernel(workload.name, fmt, N, K, hp.configs, roof["m_values"])
+    roof["peak_source"] = f"{peaks['source']}: " + ("2 x bf16_tflops_sustained (8-bit = 2x bf16 nominal)"
+                                                     if roof["bound"] == "tensor" else "hbm_gbs copy")
+    # for context: the single longest launch of the step
     _, Md, tgd, abd, fld = dominant
-    bound = "hbm" if abd / (hbm * 1e9) >= fld / (tc_peak * 1e12) else "tensor"
-    if bound == "tensor":
-        roof = {"bound": "tensor", "achieved": fld / tgd / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": fld / tgd / 1e12 / tc_peak}
+    largest = {"kernel": f"qlin_gemm_kernel M={Md} N={N} K={K} {FMT_NAME[fmt]}", "M": Md, "us": tgd * 1e6}
+    if abd / (hbm * 1e9) >= fld / (tc_peak * 1e12):
+        largest.update({"bound": "hbm", "achieved": abd / tgd / 1e9, "peak": hbm, "unit": "GB/s",
+                        "frac": abd / tgd / 1e9 / hbm})
     else:
-        roof = {"bound": "hbm", "achieved": abd / tgd / 1e9, "peak": hbm, "unit": "GB/s",
-                "frac": abd / tgd / 1e9 / hbm}
-    roof.update({"traffic": measured_traffic(workload.name, fmt, Md, N, K, hp.configs[Md]),
-                 "kernel": f"qlin_gemm_kernel M={Md} N={N} K={K} {FMT_NAME[fmt]}",
-                 "peak_source": f"{peaks['source']}: " + ("2 x bf16_tflops_sustained (8-bit = 2x bf16 nominal)"
-                                                          if bound == "tensor" else "hbm_gbs copy")})
+        largest.update({"bound": "tensor", "achieved": fld / tgd / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
+                        "frac": fld / tgd / 1e12 / tc_peak})
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * elapsed_s / args.steps, "higher_is_better": True,
@@ -527,6 +577,7 @@ def main(argv=None):
                        "pdl": True,
                        "table": (not args.no_table and os.path.exists(args.table))},
             "roofline": roof,
+            "roofline_largest_launch": largest,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db},
             "gpu_launches": 2 * len(ms) * args.steps,
             "clocks": clk,

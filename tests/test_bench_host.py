@@ -50,3 +50,31 @@ def test_reference_arm_prints_one_json_line():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_dominant_kernel_groups_launches_like_the_launch_list():
+    # launches of one compiled kernel (here the Swap-AB tile-16 kernel serving
+    # M <= 64) are grouped before ranking by share of the step, as ncu's
+    # launch list groups them; the roofline uses the group's mean launch
+    import bench
+    from quantized_linear_layers_group_b200 import qlin
+
+    ms = [1, 4, 8, 16, 32, 64, 256, 512, 1024, 2048]
+    cfg = {M: {"variant": qlin.QLIN_VAR_SWAPAB if M <= 64 else (qlin.QLIN_VAR_PAIR if M > 1024 else
+                                                                 qlin.QLIN_VAR_PLAIN),
+               "tile_n": 16 if M <= 64 else (128 if M <= 512 else 256), "k_segments": 1} for M in ms}
+    us = {1: 7.0, 4: 7.0, 8: 7.0, 16: 7.0, 32: 7.0, 64: 8.0, 256: 9.0, 512: 10.0, 1024: 12.0, 2048: 18.0}
+    per_m = [{"M": M, "gemm_us": us[M]} for M in ms]
+    total = sum(us.values()) + 20.0
+    r = bench.kernel_roofline(per_m, cfg, 1, 4096, 2048, 6550.4, 2751.2, total)
+    assert r["kernel"] == "qlin_gemm_kernel<1, 1, 16, 0, 0, 0>"
+    assert r["m_values"] == [1, 4, 8, 16, 32, 64] and r["launches_per_step"] == 6
+    assert abs(r["share"] - 43.0 / total) < 1e-12
+    ab = sum(M * 2048 + 4096 * 2048 for M in r["m_values"]) / 6
+    assert r["bound"] == "hbm" and abs(r["achieved"] - ab / (43.0 / 6 * 1e-6) / 1e9) < 1e-6
+    assert abs(r["frac"] - r["achieved"] / 6550.4) < 1e-12
+    # pair and plain 256 tiles are different kernels; one-CTA tiles of 128 and 256 too
+    assert bench.kernel_of(1, cfg[2048]) == "qlin_gemm_kernel<1, 0, 256, 0, 0, 1>"
+    assert bench.kernel_of(1, cfg[1024]) == "qlin_gemm_kernel<1, 0, 256, 0, 0, 0>"
+    assert bench.kernel_of(1, {"variant": qlin.QLIN_VAR_SWAPAB_SPLITK, "tile_n": 16}) == \
+        bench.kernel_of(1, cfg[16])
