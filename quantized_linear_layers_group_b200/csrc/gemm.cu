@@ -17,12 +17,16 @@
 //   warps 0-7  epilogue: warp w reads TMEM lanes 32(w%4)..32(w%4)+31 (the
 //           hardware's lane quadrant for that warp) and the 32-column slices
 //           j with j % 2 == w / 4, so two warps share each quadrant; scales
-//           and bias are staged once per tile in shared memory.
+//           and bias are staged once per tile in shared memory.  Plain tiles
+//           leave through bulk tensor stores of 32 x 32 bf16 boxes.
+// Plain 256 x 256 tiles may also run on the two CTAs of a cluster
+// (cta_group::2): each CTA loads its 128 rows of A and half of the W tile,
+// and rank 0 issues M = 256 MMAs that fill both CTAs' accumulators.
 //
 // Fixed reduction order (batch invariance).  K is cut into S segments fixed
 // per (format, N, K).  Each segment is accumulated on its own in TMEM
 // (Block-FP8: each 128-wide K block is, and is promoted into an fp32 segment
-// sum in registers with one fma per block), and the per-segment values are
+// sum kept in TMEM with one fma per block), and the per-segment values are
 // added in order s = 0..S-1 starting from +0.  The plain variant keeps the
 // running total in a third TMEM region, the Split-K variant writes each
 // segment to a workspace and the last CTA to arrive on the tile's ticket adds
