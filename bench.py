@@ -6,16 +6,26 @@ group for Block-FP8) followed by the scaled GEMM with the variant the dispatch
 table (or the built-in rule) picks for that (M, N, K, format).  Each GEMM of a
 step reads a different copy of the quantised weight, rotating through enough
 copies that the weights read between two uses of one copy exceed 2x the L2
-(126 MB), so every GEMM streams its weight from HBM.
+(126 MB), and each step reads its own set of activation copies, so every
+weight byte and every activation byte comes from HBM.
 
 Prints one JSON line (rank 0):
-  value       whole-job GEMM TFLOP/s over the device-timed steps (inputs resident)
+  value       whole-job GEMM TFLOP/s over the device-timed steps of the
+              headline workload (FP8 attention projection, M sweep), inputs
+              resident, one CUDA graph per step
   e2e         the same steps through the same C ABI calls with the bf16
               activations copied in from pinned host memory and C copied back
-  roofline    the dominant kernel (largest share of device time) against the
-              measured HBM / tensor peak
-  per_m       per (M, N, K, format): GEMM time, TFLOP/s, HBM GB/s, roofline fraction
-  cpu_baseline  the CPU oracle on a bounded sample (rank 0, N = 1 only)
+  roofline    the dominant kernel of the headline workload (largest share of
+              device time) against the measured HBM / tensor peak
+  per_m       per (M, N, K, format) of the headline workload: GEMM and
+              quantiser time, TFLOP/s, HBM GB/s, roofline fraction
+  workloads   the same per-M table, step time and dominant-kernel roofline for
+              every workload of the metric (INT8 smoke, FP8 attention,
+              Block-FP8 down projection, lm_head, FP8 12288 x 2048, INT8 2048^2)
+  tensor_peaks  dense FP8 (torch._scaled_mm) and INT8 (torch._int_mm) library
+              GEMM throughput at 8192^3 measured on this GPU (burst, best of 10)
+  cpu_baseline  the CPU oracle on a bounded sample (rank 0, N = 1 only), on one
+              thread and on every host core
 
   --impl reference  times the CPU oracle as the reference arm instead.
 
@@ -26,9 +36,11 @@ time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import json
 import math
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -48,6 +60,9 @@ METRIC = "scaled_mm TFLOPS & HBM GB/s vs roofline, per (M,N,K,format), 1×B200"
 L2_BYTES = 126 * 1024 * 1024
 FMT_NAME = {0: "int8", 1: "fp8", 2: "fp8_block"}
 DTYPE = {0: "int8 (int32 accumulate)", 1: "fp8_e4m3 (fp32 accumulate)", 2: "fp8_e4m3 block-scaled (fp32 accumulate)"}
+HEADLINE = "fp8_attn"
+# every workload of the metric: the headline plus the parity configurations
+ALL_WORKLOADS = ("fp8_attn", "int8_smoke", "fp8_block_down", "lm_head", "fp8_vocab", "int8_square")
 
 
 # ------------------------------------------------------------------ peaks
@@ -61,10 +76,49 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def tensor_peak(peaks, fmt, sustained=True):
-    """8-bit dense tensor peak = measured bf16 cuBLAS peak x 2 (nominal 4.5 vs 2.25 PF)."""
-    base = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    return 2.0 * base
+def measure_tensor_peaks(device, n=8192, reps=10):
+    """Dense 8-bit library GEMM throughput on this GPU: torch._scaled_mm (e4m3,
+    bf16 out) and torch._int_mm (int8, int32 out) at n^3, each call timed with
+    CUDA events on the current stream, best of `reps` (burst)."""
+    out = {"n": n, "reps": reps, "how": "best of 10 single calls, CUDA events, 2*n^3 flop"}
+    a8 = torch.randn(n, n, device=device).to(torch.float8_e4m3fn)
+    b8 = torch.randn(n, n, device=device).to(torch.float8_e4m3fn)
+    one = torch.ones((), device=device, dtype=torch.float32)
+    i8a = torch.randint(-127, 128, (n, n), device=device, dtype=torch.int8)
+    i8b = torch.randint(-127, 128, (n, n), device=device, dtype=torch.int8)
+    calls = {"fp8_tflops": lambda: torch._scaled_mm(a8, b8.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16),
+             "int8_tops": lambda: torch._int_mm(i8a, i8b.t())}
+    for key, fn in calls.items():
+        try:
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            best = float("inf")
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                e1.synchronize()
+                best = min(best, e0.elapsed_time(e1) / 1e3)
+            out[key] = 2.0 * n ** 3 / best / 1e12
+        except Exception as exc:  # a library without the kernel on this build: say so
+            out[key] = None
+            out[key + "_error"] = f"{type(exc).__name__}: {exc}"[:200]
+    del a8, b8, i8a, i8b
+    torch.cuda.synchronize()
+    return out
+
+
+def tensor_peak(peaks, fmt, tpk=None):
+    """Dense 8-bit tensor peak for a kernel timed in isolation (burst): the
+    measured library figure for the format when there is one, else the
+    measured bf16 burst peak x 2 (the nominal 8-bit / bf16 ratio)."""
+    if tpk is not None:
+        v = tpk.get("int8_tops" if fmt == 0 else "fp8_tflops")
+        if v:
+            return v, ("measured torch._int_mm int8" if fmt == 0 else "measured torch._scaled_mm e4m3") + " burst"
+    return 2.0 * peaks["bf16_tflops"], f"{peaks['source']} bf16 burst x 2 (nominal 8-bit / bf16 ratio)"
 
 
 def gemm_flops(M, N, K):
@@ -215,7 +269,11 @@ class ClockSampler:
 
 # --------------------------------------------------------------- the step
 class HotPath:
-    """Device buffers and the per-step launch sequence for one workload."""
+    """Device buffers and the per-step launch sequence for one workload.
+
+    Weights rotate per GEMM launch through `n_copies` copies, and each step
+    (one CUDA graph) reads its own set of activation copies, so that the bytes
+    read between two uses of one copy exceed 2x L2 for both."""
 
     def __init__(self, workload: synth.Workload, m_values, device, seed=0):
         from quantized_linear_layers_group_b200 import linear, qlin
@@ -237,8 +295,14 @@ class HotPath:
         self.n_copies = max(2, math.ceil(2 * L2_BYTES / wbytes) + 1)
         self.w_copies = [(w_q if i == 0 else w_q.clone(), s_w if i == 0 else s_w.clone())
                          for i in range(self.n_copies)]
-        self.a = {M: synth.activations(workload, M, seed=seed).to(device) for M in self.ms}
-        self.a_host = {M: self.a[M].cpu().pin_memory() for M in self.ms}
+        # graphs per rotation of the weight copies; each graph = one step with its own activation set
+        self.n_graphs = max(1, math.ceil(self.n_copies / len(self.ms)))
+        step_bytes = len(self.ms) * wbytes + sum(2 * M * K for M in self.ms)
+        self.n_act_sets = max(self.n_graphs, math.ceil(2 * L2_BYTES / step_bytes) + 1)
+        a_cpu = {M: synth.activations(workload, M, seed=seed) for M in self.ms}
+        self.a_sets = [{M: a_cpu[M].to(device) for M in self.ms} for _ in range(self.n_act_sets)]
+        self.a_host = {M: a_cpu[M].pin_memory() for M in self.ms}
+        self.act = 0  # activation set of the step being issued
         self.a_q, self.s_a, self.c, self.c_host = {}, {}, {}, {}
         ws = 0
         for M in self.ms:
@@ -257,10 +321,11 @@ class HotPath:
 
     def launch_quant(self, M, stream):
         q = self.qlin
+        x = self.a_sets[self.act][M]
         if self.fmt == 2:
-            q.qlin_quantize_block(self.a[M], 1, self.a_q[M], self.s_a[M], stream, flags=self.flags)
+            q.qlin_quantize_block(x, 1, self.a_q[M], self.s_a[M], stream, flags=self.flags)
         else:
-            q.qlin_quantize_per_token(self.fmt, self.a[M], self.a_q[M], self.s_a[M], stream, flags=self.flags)
+            q.qlin_quantize_per_token(self.fmt, x, self.a_q[M], self.s_a[M], stream, flags=self.flags)
 
     def launch_gemm(self, M, stream):
         w_q, s_w = self.w_copies[self.calls % self.n_copies]
@@ -268,23 +333,32 @@ class HotPath:
         self.qlin.qlin_scaled_mm(self.fmt, self.a_q[M], self.s_a[M], w_q, s_w, self.bias, self.c[M],
                                  self.workspace, stream, flags=self.flags)
 
-    def step(self, stream, events=None):
+    def step(self, stream, act_set=None):
+        """Issue one step: for each M, the quantiser then the GEMM (PDL)."""
+        self.act = (self.act + 1) % self.n_act_sets if act_set is None else act_set
         for M in self.ms:
-            if events is not None:
-                events[M][0].record(stream)
             self.launch_quant(M, stream)
-            if events is not None:
-                events[M][1].record(stream)
             self.launch_gemm(M, stream)
-            if events is not None:
-                events[M][2].record(stream)
+
+    def capture_graphs(self, stream):
+        """One CUDA graph per step of a rotation: graph g reads activation set
+        g and the next len(ms) weight copies.  Exactly what the timed region
+        replays."""
+        graphs = []
+        for g in range(self.n_graphs):
+            cg = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(cg, stream=stream):
+                self.step(stream, act_set=g)
+            graphs.append(cg)
+        return graphs
 
     def step_e2e(self, stream):
         """Same step with the activations copied in from pinned host memory and
         C copied back; returns (h2d bytes, d2h bytes)."""
         hb = db = 0
+        self.act = 0
         for M in self.ms:
-            self.a[M].copy_(self.a_host[M], non_blocking=True)
+            self.a_sets[0][M].copy_(self.a_host[M], non_blocking=True)
             hb += self.a_host[M].numel() * 2
             self.launch_quant(M, stream)
             self.launch_gemm(M, stream)
@@ -293,8 +367,68 @@ class HotPath:
         return hb, db
 
 
-def flush_l2(buf):
-    buf.add_(1)
+def per_kernel_times(hp: HotPath, stream, reps=8, replays=5):
+    """For each M: a graph of `reps` back-to-back launches of one kernel (the
+    quantiser rotates activation sets, the GEMM weight copies), timed with
+    events on the launching stream; per-launch time = graph time / reps,
+    median of `replays` replays.  Returns ({M: quant us}, {M: gemm us})."""
+    qt, gt = {}, {}
+    for M in hp.ms:
+        for kind in ("q", "g"):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(reps):
+                    if kind == "q":
+                        hp.act = i % hp.n_act_sets
+                        hp.launch_quant(M, stream)
+                    else:
+                        hp.launch_gemm(M, stream)
+            for _ in range(2):
+                g.replay()
+            ts = []
+            for _ in range(replays):
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record(stream)
+                g.replay()
+                a1.record(stream)
+                a1.synchronize()
+                ts.append(a0.elapsed_time(a1) * 1e3 / reps)
+            (qt if kind == "q" else gt)[M] = statistics.median(ts)
+            del g
+    torch.cuda.synchronize()
+    return qt, gt
+
+
+def workload_report(hp: HotPath, qt, gt, peaks, tpk):
+    """Per-M table and dominant-kernel roofline of one workload."""
+    from quantized_linear_layers_group_b200 import qlin
+
+    w = hp.w
+    N, K, fmt = w.N, w.K, w.fmt
+    tc_peak, tc_src = tensor_peak(peaks, fmt, tpk)
+    hbm = peaks["hbm_gbs"]
+    per_m = []
+    for M in hp.ms:
+        tg, tq = gt[M] * 1e-6, qt[M] * 1e-6
+        ab, extra = gemm_bytes(M, N, K, fmt)
+        fl = gemm_flops(M, N, K)
+        t_hbm, t_tc = ab / (hbm * 1e9), fl / (tc_peak * 1e12)
+        t_roof = max(t_hbm, t_tc)
+        cfg = hp.configs[M]
+        per_m.append({"M": M, "N": N, "K": K, "format": FMT_NAME[fmt],
+                      "variant": qlin.VARIANT_NAMES[cfg["variant"]], "tile_n": cfg["tile_n"],
+                      "k_segments": cfg["k_segments"], "gemm_us": gt[M], "quant_us": qt[M],
+                      "tflops": fl / tg / 1e12, "hbm_gbs": ab / tg / 1e9,
+                      "hbm_gbs_all_bytes": (ab + extra) / tg / 1e9,
+                      "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / tg,
+                      "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                      "quant_gbs": quant_bytes(M, K, fmt) / tq / 1e9,
+                      "quant_frac_hbm": quant_bytes(M, K, fmt) / tq / 1e9 / hbm})
+    total = sum(gt[M] + qt[M] for M in hp.ms)
+    roof = kernel_roofline(per_m, hp.configs, fmt, N, K, hbm, tc_peak, total)
+    roof["traffic"] = measured_traffic_kernel(w.name, fmt, N, K, hp.configs, roof["m_values"])
+    roof["peak_source"] = tc_src if roof["bound"] == "tensor" else f"{peaks['source']} hbm_gbs copy"
+    return per_m, roof, tc_peak, tc_src
 
 
 # ----------------------------------------------------------- distributed
@@ -343,13 +477,27 @@ def aggregate(per_rank_units: float, max_seconds: float, world: int) -> float:
 _ORACLE_WEIGHTS = {}
 
 
-def cpu_oracle_sample(workload: synth.Workload, M: int, seed=0):
-    """The CPU oracle (as it stands) on a bounded sample: quantise M activation
-    rows and compute their full C rows against the whole (offline-quantised)
-    weight.  Returns (seconds, GEMM flops, description)."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_weight(workload: synth.Workload, seed=0):
     import oracle
 
-    N, K = workload.N, workload.K
     key = (workload.name, seed)
     if key not in _ORACLE_WEIGHTS:
         w = synth.weights(workload, seed)
@@ -357,52 +505,120 @@ def cpu_oracle_sample(workload: synth.Workload, M: int, seed=0):
             _ORACLE_WEIGHTS[key] = oracle.quantize_block(w, 128, 128)
         else:
             _ORACLE_WEIGHTS[key] = oracle.quantize_per_token(workload.fmt, w)
-    wq, sw = _ORACLE_WEIGHTS[key]
-    a = synth.activations(workload, M, seed=seed)
+    return _ORACLE_WEIGHTS[key]
+
+
+def cpu_oracle_rows(workload: synth.Workload, rows_per_m, threads=1, seed=0):
+    """The CPU oracle (as it stands) on a bounded sample: for each (M, r) in
+    rows_per_m, the first r of M activation rows are quantised and their full C
+    rows computed against the whole (offline-quantised) weight.  With
+    threads > 1, row slices run concurrently on a thread pool (the oracle's C
+    code runs without the interpreter lock).  Returns (seconds, GEMM flops)."""
+    import oracle
+
+    N, K = workload.N, workload.K
+    wq, sw = _oracle_weight(workload, seed)
     b = synth.bias(workload, seed)
+    inputs = [synth.activations(workload, M, seed=seed)[:r].contiguous() for M, r in rows_per_m]
+    flops = sum(gemm_flops(r, N, K) for _, r in rows_per_m)
+
+    def job(a):
+        if workload.fmt == 2:
+            aq, sa = oracle.quantize_block(a, 1, 128)
+        else:
+            aq, sa = oracle.quantize_per_token(workload.fmt, a)
+        oracle.scaled_mm(workload.fmt, aq, sa, wq, sw, b)
+
+    # split every sample into slices of a few rows so all threads stay busy
+    slices = []
+    for a in inputs:
+        step = max(1, math.ceil(a.shape[0] / max(1, threads)))
+        slices += [a[i:i + step].contiguous() for i in range(0, a.shape[0], step)]
     t0 = time.perf_counter()
-    if workload.fmt == 2:
-        aq, sa = oracle.quantize_block(a, 1, 128)
+    if threads <= 1:
+        for s in slices:
+            job(s)
     else:
-        aq, sa = oracle.quantize_per_token(workload.fmt, a)
-    oracle.scaled_mm(workload.fmt, aq, sa, wq, sw, b)
-    dt = time.perf_counter() - t0
-    return dt, gemm_flops(M, N, K), f"{workload.name}: quantise + scaled_mm of M={M} rows x N={N} x K={K}, 1 thread"
+        with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(job, slices))
+    return time.perf_counter() - t0, flops
+
+
+def reference_rows(workload: synth.Workload, cap: int):
+    """The reference arm's per-step sample: every M of the sweep, at most `cap` rows of it."""
+    return [(M, min(M, cap)) for M in workload.m_values]
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
     w = synth.WORKLOADS[args.workload]
-    M = args.ref_rows
-    times, flops = [], 0.0
+    rows = reference_rows(w, args.ref_rows)
+    cores = host_cores()
     for _ in range(args.warmup):
-        cpu_oracle_sample(w, M)
-    desc = ""
+        cpu_oracle_rows(w, rows, threads=cores)
+    times, flops = [], 0.0
     for _ in range(args.steps):
-        dt, fl, desc = cpu_oracle_sample(w, M)
+        dt, flops = cpu_oracle_rows(w, rows, threads=cores)
         times.append(dt)
-        flops = fl
     total = sum(times)
     value = flops * len(times) / total / 1e12
+    desc = (f"{w.name}: every M of the sweep, its first min(M, {args.ref_rows}) rows quantised and their full "
+            f"C rows computed (N={w.N}, K={w.K}), {cores} threads")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE[w.fmt],
             "data": "synthetic", "config": {"workload": w.name, "format": FMT_NAME[w.fmt], "N": w.N, "K": w.K,
-                                            "m_values": [M], "parallelism": "single process"},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle", "sample": desc},
+                                            "m_values": list(w.m_values), "bias": w.bias,
+                                            "parallelism": "single process"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
+                             "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------ main
+def time_steps(hp: HotPath, stream, steps, warmup, world, local, use_graph=True):
+    """The device-timed region: `steps` graph replays of whole steps (each
+    graph reads its own activation set and rotates the weights), events on
+    the launching stream around each replay, barrier + synchronise on both
+    sides, clocks sampled meanwhile.  Returns (seconds, clocks)."""
+    graphs = hp.capture_graphs(stream) if use_graph else []
+    torch.cuda.synchronize()
+    for i in range(warmup):
+        if use_graph:
+            graphs[i % len(graphs)].replay()
+        else:
+            hp.step(stream)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        evs[i][0].record(stream)
+        if use_graph:
+            graphs[i % len(graphs)].replay()
+        else:
+            hp.step(stream)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    barrier(world)
+    clk = clocks.stop()
+    del graphs
+    return max_over_ranks(sum(step_ms) / 1e3, world), clk
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="fp8_attn", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--m", type=str, default=None, help="comma-separated M values (default: the workload's sweep)")
     ap.add_argument("--table", default=os.path.join(ROOT, "quantized_linear_layers_group_b200", "tables",
                                                     "b200.qlt"))
@@ -411,8 +627,10 @@ def main(argv=None):
                     help="replay each device-timed step as a CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-rows", type=int, default=256, help="rows per reference-arm step")
-    ap.add_argument("--baseline-rows", type=int, default=1024, help="rows of the cpu_baseline sample")
+    ap.add_argument("--no-workloads", action="store_true", help="measure the headline workload only")
+    ap.add_argument("--no-peaks", action="store_true", help="skip the 8-bit library peak measurement")
+    ap.add_argument("--ref-rows", type=int, default=64, help="rows per M in a reference-arm step")
+    ap.add_argument("--baseline-rows", type=int, default=64, help="rows per M of the cpu_baseline sample")
     args = ap.parse_args(argv)
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
 
@@ -429,11 +647,11 @@ def main(argv=None):
     workload = synth.WORKLOADS[args.workload]
     ms = [int(x) for x in args.m.split(",")] if args.m else list(workload.m_values)
     device = torch.device("cuda", local)
-    hp = HotPath(workload, ms, device)
     stream = torch.cuda.Stream(device)
     peaks = load_peaks()
 
     with torch.cuda.stream(stream):
+        hp = HotPath(workload, ms, device)
         for _ in range(args.warmup):
             hp.step(stream)
         torch.cuda.synchronize()
@@ -442,69 +660,7 @@ def main(argv=None):
             raise RuntimeError(f"device status after warm-up: {qlin.qlin_status_string(st)}")
 
         # ---------------------------------------------- device-timed steps
-        # Each step is one CUDA graph (the launch sequence of the hot path,
-        # as a serving engine replays it); G graphs use different weight
-        # copies so the rotation defeats L2.  Events bracket each replay.
-        n_graphs = max(1, math.ceil(hp.n_copies / len(ms))) if args.graph else 1
-        graphs = []
-        if args.graph:
-            for _ in range(n_graphs):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    hp.step(stream)
-                graphs.append(g)
-        torch.cuda.synchronize()
-        for i in range(args.warmup):
-            if args.graph:
-                graphs[i % n_graphs].replay()
-            else:
-                hp.step(stream)
-        torch.cuda.synchronize()
-        clocks = ClockSampler(local)
-        clocks.start()
-        time.sleep(0.3)
-        barrier(world)
-        torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        for i in range(args.steps):
-            evs[i][0].record(stream)
-            if args.graph:
-                graphs[i % n_graphs].replay()
-            else:
-                hp.step(stream)
-            evs[i][1].record(stream)
-        torch.cuda.synchronize()
-        step_ms = [a.elapsed_time(b) for a, b in evs]
-        barrier(world)
-        clk = clocks.stop()
-        elapsed_s = max_over_ranks(sum(step_ms) / 1e3, world)
-        del graphs
-
-        # ------------------------------------------- per-kernel launch times
-        # For each M: a graph of R back-to-back launches of one kernel (the
-        # GEMM rotates weight copies), timed with events on the launching
-        # stream; per-launch time = graph time / R (median of a few replays).
-        per_m_q, per_m_g = {}, {}
-        reps = 8
-        for M in ms:
-            for kind, fn in (("q", hp.launch_quant), ("g", hp.launch_gemm)):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    for _ in range(reps):
-                        fn(M, stream)
-                for _ in range(2):
-                    g.replay()
-                ts = []
-                for _ in range(5):
-                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    a0.record(stream)
-                    g.replay()
-                    a1.record(stream)
-                    a1.synchronize()
-                    ts.append(a0.elapsed_time(a1) / reps)
-                (per_m_q if kind == "q" else per_m_g)[M] = [statistics.median(ts)]
-                del g
-        torch.cuda.synchronize()
+        elapsed_s, clk = time_steps(hp, stream, args.steps, args.warmup, world, local, args.graph)
 
         # ------------------------------------------------- end-to-end steps
         for _ in range(2):
@@ -521,71 +677,86 @@ def main(argv=None):
         torch.cuda.synchronize()
         barrier(world)
         e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+
+        # ------------------------------------------- per-kernel launch times
+        tpk = None if args.no_peaks else measure_tensor_peaks(device)
+        qt, gt = per_kernel_times(hp, stream)
+        per_m, roof, tc_peak, tc_src = workload_report(hp, qt, gt, peaks, tpk)
         st = qlin.qlin_sync_status(stream)
         if st != 0:
             raise RuntimeError(f"device status: {qlin.qlin_status_string(st)}")
+        del hp
+        torch.cuda.empty_cache()
+
+        # ------------------------------ every workload of the metric, per M
+        workloads = {}
+        if not args.no_workloads and world == 1:
+            for name in ALL_WORKLOADS:
+                w = synth.WORKLOADS[name]
+                wh = HotPath(w, list(w.m_values), device)
+                for _ in range(3):
+                    wh.step(stream)
+                w_s, _ = time_steps(wh, stream, 5, 3, 1, local, args.graph)
+                wq, wg = per_kernel_times(wh, stream)
+                w_per_m, w_roof, _, _ = workload_report(wh, wq, wg, peaks, tpk)
+                fl = sum(gemm_flops(M, w.N, w.K) for M in w.m_values)
+                workloads[name] = {"format": FMT_NAME[w.fmt], "N": w.N, "K": w.K, "m_values": list(w.m_values),
+                                   "step_us": w_s / 5 * 1e6, "step_tflops": fl * 5 / w_s / 1e12,
+                                   "roofline": w_roof, "per_m": w_per_m}
+                st = qlin.qlin_sync_status(stream)
+                if st != 0:
+                    raise RuntimeError(f"device status ({name}): {qlin.qlin_status_string(st)}")
+                del wh
+                torch.cuda.empty_cache()
 
     N, K, fmt = workload.N, workload.K, workload.fmt
     flops_step = sum(gemm_flops(M, N, K) for M in ms)
     value = aggregate(flops_step * args.steps, elapsed_s, world) / 1e12
     e2e_value = aggregate(flops_step * args.steps, e2e_s, world) / 1e12
-
-    tc_peak = tensor_peak(peaks, fmt, sustained=True)
-    hbm = peaks["hbm_gbs"]
-    per_m = []
-    dominant = None
-    total_dev = sum(statistics.mean(per_m_g[M]) + statistics.mean(per_m_q[M]) for M in ms)
-    for M in ms:
-        tg = statistics.mean(per_m_g[M]) / 1e3
-        tq = statistics.mean(per_m_q[M]) / 1e3
-        ab, extra = gemm_bytes(M, N, K, fmt)
-        fl = gemm_flops(M, N, K)
-        t_roof = max(ab / (hbm * 1e9), fl / (tc_peak * 1e12))
-        cfg = hp.configs[M]
-        per_m.append({"M": M, "N": N, "K": K, "format": FMT_NAME[fmt],
-                      "variant": qlin.VARIANT_NAMES[cfg["variant"]], "tile_n": cfg["tile_n"],
-                      "k_segments": cfg["k_segments"], "gemm_us": tg * 1e6, "quant_us": tq * 1e6,
-                      "tflops": fl / tg / 1e12, "hbm_gbs": ab / tg / 1e9,
-                      "hbm_gbs_all_bytes": (ab + extra) / tg / 1e9,
-                      "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / tg,
-                      "bound": "hbm" if ab / (hbm * 1e9) >= fl / (tc_peak * 1e12) else "tensor",
-                      "quant_gbs": quant_bytes(M, K, fmt) / tq / 1e9})
-        share = tg / (total_dev / 1e3)
-        if dominant is None or share > dominant[0]:
-            dominant = (share, M, tg, ab, fl)
-    roof = kernel_roofline(per_m, hp.configs, fmt, N, K, hbm, tc_peak, total_dev * 1e3)  # total_dev in ms
-    roof["traffic"] = measured_traffic_kernel(workload.name, fmt, N, K, hp.configs, roof["m_values"])
-    roof["peak_source"] = f"{peaks['source']}: " + ("2 x bf16_tflops_sustained (8-bit = 2x bf16 nominal)"
-                                                     if roof["bound"] == "tensor" else "hbm_gbs copy")
     # for context: the single longest launch of the step
-    _, Md, tgd, abd, fld = dominant
-    largest = {"kernel": f"qlin_gemm_kernel M={Md} N={N} K={K} {FMT_NAME[fmt]}", "M": Md, "us": tgd * 1e6}
-    if abd / (hbm * 1e9) >= fld / (tc_peak * 1e12):
-        largest.update({"bound": "hbm", "achieved": abd / tgd / 1e9, "peak": hbm, "unit": "GB/s",
-                        "frac": abd / tgd / 1e9 / hbm})
+    big = max(per_m, key=lambda r: r["gemm_us"])
+    largest = {"kernel": f"qlin_gemm_kernel M={big['M']} N={N} K={K} {FMT_NAME[fmt]}", "M": big["M"],
+               "us": big["gemm_us"], "bound": big["bound"]}
+    if big["bound"] == "hbm":
+        largest.update({"achieved": big["hbm_gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": big["hbm_gbs"] / peaks["hbm_gbs"]})
     else:
-        largest.update({"bound": "tensor", "achieved": fld / tgd / 1e12, "peak": tc_peak, "unit": "TFLOP/s",
-                        "frac": fld / tgd / 1e12 / tc_peak})
+        largest.update({"achieved": big["tflops"], "peak": tc_peak, "unit": "TFLOP/s",
+                        "frac": big["tflops"] / tc_peak})
 
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * elapsed_s / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": DTYPE[fmt], "data": "synthetic",
             "config": {"workload": workload.name, "format": FMT_NAME[fmt], "N": N, "K": K, "m_values": ms,
                        "bias": workload.bias,
-                       "l2": f"{hp.n_copies} rotating weight copies ({hp.n_copies * N * K / 1e6:.0f} MB) > 2x L2",
+                       "l2": ("inputs larger than L2: weights rotate per GEMM and activations per step, "
+                              "> 2x L2 between two uses of one copy"),
                        "parallelism": "replicas" if world > 1 else "single GPU", "cuda_graph": args.graph,
                        "pdl": True,
                        "table": (not args.no_table and os.path.exists(args.table))},
             "roofline": roof,
             "roofline_largest_launch": largest,
+            "tensor_peak_used": {"value": tc_peak, "source": tc_src},
+            "tensor_peaks": tpk,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db},
             "gpu_launches": 2 * len(ms) * args.steps,
             "clocks": clk,
             "per_m": per_m}
+    if workloads:
+        line["workloads"] = workloads
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, fl, desc = cpu_oracle_sample(workload, args.baseline_rows)
-        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                                "sample": desc, "seconds": dt}
+        rows = reference_rows(workload, args.baseline_rows)
+        cores = host_cores()
+        dt1, fl1 = cpu_oracle_rows(workload, [(M, min(r, 16)) for M, r in rows], threads=1)
+        dtn, fln = cpu_oracle_rows(workload, rows, threads=cores)
+        line["cpu_baseline"] = {
+            "value": fln / dtn / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(),
+            "sample": (f"{workload.name}: every M of the sweep, its first min(M, {args.baseline_rows}) rows "
+                       f"quantised and their full C rows computed (N={N}, K={K}), {cores} threads"),
+            "seconds": dtn,
+            "one_thread": {"value": fl1 / dt1 / 1e12, "unit": "TFLOP/s", "cores": 1, "seconds": dt1,
+                           "sample": f"the same, first min(M, 16) rows, 1 thread"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -19,9 +19,10 @@
  *     keeps no pointer after a call returns.
  *   - All device work is enqueued on `stream` (a cudaStream_t; NULL = the
  *     legacy default stream) and is asynchronous: outputs are valid once the
- *     stream has reached that point.  Apart from the table loader, no entry
- *     point synchronises, allocates or compiles, so calls may be captured in a
- *     CUDA graph.
+ *     stream has reached that point.  Apart from the table loader and
+ *     qlin_sync_status, no entry point synchronises, allocates or compiles;
+ *     the quantisers, qlin_scaled_mm and qlin_linear may be captured in a
+ *     CUDA graph (the benchmark replays them that way).
  *   - Arguments are validated on the host before anything is launched; a bad
  *     argument returns an error status and launches nothing.  No entry point
  *     aborts the process.
@@ -198,9 +199,12 @@ QLIN_API qlin_status qlin_quantize_block(const void* x, int64_t rows, int64_t co
  *                       Split-K run as a cluster).  Its first
  *                       64 KiB hold the Split-K ticket words: they must be
  *                       zero-filled once when the buffer is allocated, and every
- *                       call leaves them at zero again; the rest holds partial
- *                       tiles.  Calls that overlap in time must not share a
- *                       workspace.
+ *                       call that completes leaves them at zero again; the rest
+ *                       holds partial tiles.  Calls that overlap in time must
+ *                       not share a workspace.  After qlin_sync_status() has
+ *                       reported QLIN_ERR_DEVICE_TIMEOUT, a CTA may have left a
+ *                       ticket half-counted: zero the first 64 KiB again before
+ *                       the buffer is used by another call.
  * Alignment: a_q, w_q, c_out, workspace 16-byte aligned; scales and bias 4 / 2.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, NO_DEVICE.
  */
@@ -212,26 +216,27 @@ QLIN_API qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segm
 /*
  * qlin_scaled_mm_noalloc -- qlin_scaled_mm for callers that cannot allocate
  * device memory and so cannot pass a workspace (the paper has no counterpart;
- * this is a library convenience).  Typical callers: a plugin inside a serving
+ * this is a library convenience).  Typical caller: a plugin inside a serving
  * engine that owns the whole device-memory pool and forbids allocations it
- * does not make itself, or code reached while a CUDA graph is being captured,
- * where an allocation is not a capturable operation.
+ * does not make itself, so that every byte the engine hands out is accounted
+ * for by the engine.
  *
- * Same arguments, arithmetic and results as qlin_scaled_mm, without the
- * workspace: the Split-K ticket words and partial tiles live in a device
- * array of QLIN_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that
- * loads the library holds until the process exits.  The entry point allocates
+ * Same arguments, flags (QLIN_OUT_I32ACC, QLIN_PDL, QLIN_SPLITK_CLUSTER),
+ * arithmetic and results as qlin_scaled_mm, without the workspace: the Split-K
+ * ticket words and partial tiles live in a device array of
+ * QLIN_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.  The entry point allocates
  * nothing and calls no allocating routine.
  *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any
- *     stream capture.
- *   - Each call clears the ticket words on `stream` before its launch (the
- *     array keeps the previous call's contents).
+ *     device, with that device current).
+ *   - Each call that needs the array clears its ticket words on `stream`
+ *     before the launch (the array keeps the previous call's contents).
  *   - All calls share the one array: calls whose kernels overlap in time on the
  *     GPU (e.g. on two streams) race on it and must be avoided.
+ *   - M = 0 is a no-op that returns QLIN_OK after the shape checks.
  * Errors: as qlin_scaled_mm; QLIN_ERR_WORKSPACE when the resolved configuration
  * needs more scratch than QLIN_NOALLOC_SCRATCH_BYTES (force a smaller
- * k_segments or a non-Split-K variant).
+ * k_segments, a non-Split-K variant, or QLIN_SPLITK_CLUSTER, which needs none).
  */
 #define QLIN_NOALLOC_SCRATCH_BYTES (8u << 20) /* 8 MiB: 64 KiB of tickets + partial tiles */
 QLIN_API qlin_status qlin_scaled_mm_noalloc(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N,
@@ -314,7 +319,10 @@ QLIN_API const char* qlin_status_string(qlin_status status);
 /*
  * qlin_sync_status -- synchronise `stream`, then report and clear the device
  * status word that kernels set when a bounded wait gives up.  Returns QLIN_OK,
- * QLIN_ERR_DEVICE_TIMEOUT or QLIN_ERR_CUDA.  Blocking.
+ * QLIN_ERR_DEVICE_TIMEOUT or QLIN_ERR_CUDA.  Blocking.  After
+ * QLIN_ERR_DEVICE_TIMEOUT the outputs of the calls since the previous check
+ * are undefined and any Split-K workspace they used must have its 64 KiB
+ * ticket prefix zeroed again before reuse.
  */
 QLIN_API qlin_status qlin_sync_status(qlin_stream_t stream);
 

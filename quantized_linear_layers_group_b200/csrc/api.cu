@@ -152,14 +152,6 @@ bool lookup_table(int fmt, int64_t M, int64_t N, int64_t K, qlin_config* out) {
     return true;
 }
 
-qlin_status check_fmt_shape(int fmt, int64_t M, int64_t N, int64_t K) {
-    if (fmt < QLIN_FMT_INT8 || fmt > QLIN_FMT_FP8_BLOCK) return QLIN_ERR_INVALID_ARG;
-    if (M < 0 || N < 16 || K < 128) return QLIN_ERR_INVALID_ARG;
-    if (N % 16 != 0 || K % 128 != 0) return QLIN_ERR_UNSUPPORTED;
-    if (fmt == QLIN_FMT_FP8_BLOCK && N % 128 != 0) return QLIN_ERR_UNSUPPORTED;
-    if (M > (int64_t)1 << 30 || N > (int64_t)1 << 30 || K > (int64_t)1 << 24) return QLIN_ERR_UNSUPPORTED;
-    return QLIN_OK;
-}
 
 qlin_status resolve_config(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
                            int num_sms, qlin_config* cfg) {
@@ -188,6 +180,15 @@ qlin_status resolve_config(int fmt, int variant, int tile_n, int k_segments, int
 }
 
 }  // namespace
+
+qlin_status check_fmt_shape(int fmt, int64_t M, int64_t N, int64_t K) {
+    if (fmt < QLIN_FMT_INT8 || fmt > QLIN_FMT_FP8_BLOCK) return QLIN_ERR_INVALID_ARG;
+    if (M < 0 || N < 16 || K < 128) return QLIN_ERR_INVALID_ARG;
+    if (N % 16 != 0 || K % 128 != 0) return QLIN_ERR_UNSUPPORTED;
+    if (fmt == QLIN_FMT_FP8_BLOCK && N % 128 != 0) return QLIN_ERR_UNSUPPORTED;
+    if (M > (int64_t)1 << 30 || N > (int64_t)1 << 30 || K > (int64_t)1 << 24) return QLIN_ERR_UNSUPPORTED;
+    return QLIN_OK;
+}
 
 int current_device_sms() {
     static int cached_dev = -1, cached_sms = 0;

@@ -99,6 +99,9 @@ cudaError_t device_status_read_clear(int* value);
 // Launches the failure-path self-test (a bounded wait that must give up).
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t st);
 
+// Shape / format preconditions shared by the GEMM entry points (M >= 0).
+qlin_status check_fmt_shape(int fmt, int64_t M, int64_t N, int64_t K);
+
 // Number of SMs of the current device (cached per device); 0 if none.
 int current_device_sms();
 

@@ -5,9 +5,10 @@
 library's own kernels, and its ``forward(x)`` runs the hot path through
 ``qlin_linear``: dynamic activation quantisation (per token, or per 1x128
 group) followed by the scaled GEMM with the fused scale / bias / bf16
-epilogue -- one kernel for small batches, where the GEMM quantises its own
-activation tiles.  Everything runs in libqlin.so; this module only allocates
-tensors (through PyTorch's caching allocator) and passes pointers.
+epilogue, launched as the quantiser's programmatic dependent (QLIN_PDL).  The
+one-kernel mode (QLIN_FUSED) is opt-in through ``fused=True``.  Everything runs
+in libqlin.so; this module only allocates tensors (through PyTorch's caching
+allocator) and passes pointers.
 """
 from __future__ import annotations
 
@@ -32,6 +33,27 @@ class Workspace:
         if nbytes > self.buf.numel():
             self.buf = torch.zeros(int(nbytes), dtype=torch.uint8, device=self.device)
         return self.buf
+
+    def reset_tickets(self):
+        """Zero the 64 KiB ticket prefix again (needed after a device-side
+        timeout, which can leave a tile's ticket half-counted)."""
+        self.buf[: min(self.buf.numel(), TICKET_BYTES)].zero_()
+
+
+TICKET_BYTES = 65536  # the Split-K ticket prefix of a workspace (include/qlin.h)
+
+
+def check_device_status(stream=None, workspaces=()):
+    """Synchronise and read the library's device status word.  On a device
+    timeout, re-zero the ticket prefix of the given workspaces (so the next
+    Split-K call counts its arrivals from zero) and raise QlinError."""
+    st = qlin.qlin_sync_status(stream)
+    if st == qlin.QLIN_ERR_DEVICE_TIMEOUT:
+        for ws in workspaces:
+            ws.reset_tickets()
+        torch.cuda.synchronize()
+    if st != qlin.QLIN_OK:
+        raise qlin.QlinError(st, "device status")
 
 
 def quantize_weight(fmt: int, weight: torch.Tensor, stream=None):
@@ -65,7 +87,7 @@ class QuantizedLinear:
     """y = x W^T + b with W8A8 INT8, FP8 per-token/per-channel or Block-FP8 arithmetic."""
 
     def __init__(self, fmt: int, weight: torch.Tensor, bias: torch.Tensor | None = None, workspace=None,
-                 pdl: bool = True):
+                 pdl: bool = True, fused: bool = False):
         self.fmt = fmt
         self.N, self.K = weight.shape
         self.w_q, self.s_w = quantize_weight(fmt, weight)
@@ -73,7 +95,7 @@ class QuantizedLinear:
         # them early (programmatic dependent launch)
         torch.cuda.current_stream(weight.device).synchronize()
         self.bias = bias
-        self.flags = qlin.QLIN_PDL if pdl else 0
+        self.flags = (qlin.QLIN_PDL if pdl else 0) | (qlin.QLIN_FUSED if fused else 0)
         self.workspace = workspace if workspace is not None else Workspace(device=weight.device)
 
     def forward(self, x: torch.Tensor, stream=None, variant: int = qlin.QLIN_VAR_AUTO, tile_n: int = 0,
@@ -89,7 +111,8 @@ class QuantizedLinear:
         c = out if out is not None else torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
         nbytes = qlin.qlin_scaled_mm_workspace_size(self.fmt, M, self.N, self.K, variant, tile_n, k_segments)
         ws = self.workspace.ensure(nbytes) if nbytes else None
-        # quantisation + GEMM in one call (one kernel for small batches)
+        # quantisation + GEMM in one call (the quantiser, then the GEMM as its
+        # programmatic dependent; one kernel where QLIN_FUSED applies)
         qlin.qlin_linear(self.fmt, x, a_q, s_a, self.w_q, self.s_w, self.bias, c, ws, stream, variant=variant,
                          tile_n=tile_n, k_segments=k_segments, flags=self.flags)
         return c

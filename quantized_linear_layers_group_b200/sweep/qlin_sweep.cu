@@ -21,8 +21,9 @@
 // 2x L2), launched with QLIN_PDL as the hot path runs, CUDA events around the
 // graph, median of `reps` replays.
 //
-// Usage: qlin_sweep <out.qlt> [shape ...]   shape = fmt:N:K (fmt int8|fp8|fp8_block)
-// Without shapes it sweeps the five workload shapes.
+// Usage: qlin_sweep [--quick] <out.qlt> [shape ...]   shape = fmt:N:K (fmt int8|fp8|fp8_block)
+// Without shapes it sweeps the five workload shapes.  --quick (for tests):
+// buckets {1, 16, 256} only, two weight copies, short timing loops.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -192,12 +193,19 @@ bool same_output(Problem& P, int variant, int tile, int S, cudaStream_t st) {
 }  // namespace
 
 int main(int argc, char** argv) {
-    if (argc < 2) {
-        std::fprintf(stderr, "usage: %s out.qlt [fmt:N:K ...]\n", argv[0]);
+    bool quick = false;
+    int first = 1;
+    if (argc > 1 && std::strcmp(argv[1], "--quick") == 0) {
+        quick = true;
+        first = 2;
+    }
+    if (argc < first + 1) {
+        std::fprintf(stderr, "usage: %s [--quick] out.qlt [fmt:N:K ...]\n", argv[0]);
         return 1;
     }
+    const char* out_path = argv[first];
     std::vector<Shape> shapes;
-    for (int i = 2; i < argc; ++i) {
+    for (int i = first + 1; i < argc; ++i) {
         char f[32];
         long long n, k;
         if (std::sscanf(argv[i], "%31[^:]:%lld:%lld", f, &n, &k) != 3) return 1;
@@ -210,7 +218,8 @@ int main(int argc, char** argv) {
                   {QLIN_FMT_FP8, 151936, 2048},
                   {QLIN_FMT_FP8, 12288, 2048},
                   {QLIN_FMT_INT8, 2048, 2048}};
-    const std::vector<int64_t> buckets = {1, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048};
+    const std::vector<int64_t> buckets =
+        quick ? std::vector<int64_t>{1, 16, 256} : std::vector<int64_t>{1, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048};
     int dev = 0;
     CK(cudaGetDevice(&dev));
     cudaDeviceProp prop;
@@ -220,7 +229,7 @@ int main(int argc, char** argv) {
     CK(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
     const size_t l2 = (size_t)prop.l2CacheSize;
 
-    FILE* out = std::fopen(argv[1], "w");
+    FILE* out = std::fopen(out_path, "w");
     if (!out) return 1;
     std::fprintf(out, "qlin-dispatch 1\n");
     std::fprintf(out, "device %d %d %d %s\n", prop.multiProcessorCount, prop.major, prop.minor, prop.name);
@@ -231,7 +240,7 @@ int main(int argc, char** argv) {
         Problem P;
         P.s = s;
         const size_t wbytes = (size_t)s.N * s.K;
-        const size_t ncopy = std::max<size_t>(2, (2 * l2 + wbytes - 1) / wbytes + 1);
+        const size_t ncopy = quick ? 2 : std::max<size_t>(2, (2 * l2 + wbytes - 1) / wbytes + 1);
         const size_t sw_elems = s.fmt == QLIN_FMT_FP8_BLOCK ? (size_t)((s.N + 127) / 128) * (s.K / 128) : (size_t)s.N;
         const size_t sa_elems = s.fmt == QLIN_FMT_FP8_BLOCK ? (size_t)M_max * (s.K / 128) : (size_t)M_max;
         CK(cudaMalloc(&P.a_q, (size_t)M_max * s.K));
@@ -263,7 +272,8 @@ int main(int argc, char** argv) {
             const int S = segs[si];
             for (size_t bi = 0; bi < buckets.size(); ++bi) {
                 P.M = buckets[bi];
-                const int iters = std::max(4, std::min(40, (int)(40 * 64 / std::max<int64_t>(P.M, 64))));
+                const int iters =
+                    quick ? 4 : std::max(4, std::min(40, (int)(40 * 64 / std::max<int64_t>(P.M, 64))));
                 // reference output: plain tile 128 with this S (the canonical order)
                 bool have_ref = qlin_scaled_mm(s.fmt, QLIN_VAR_PLAIN, 128, S, P.M, s.N, s.K, P.a_q, P.s_a, P.w_q[0],
                                                P.s_w[0], nullptr, P.c_ref, 0, P.ws, P.ws_bytes, st) == QLIN_OK;
@@ -273,7 +283,7 @@ int main(int argc, char** argv) {
                 for (const Cand& c : candidates(s.fmt, P.M)) {
                     if (S == 1 && (c.variant == QLIN_VAR_SPLITK || c.variant == QLIN_VAR_SWAPAB_SPLITK)) continue;
                     bool ok = false;
-                    const float t = time_config(P, c.variant, c.tile_n, S, iters, 5, st, &ok);
+                    const float t = time_config(P, c.variant, c.tile_n, S, iters, quick ? 2 : 5, st, &ok);
                     if (!ok) continue;
                     const bool same = !have_ref || s.fmt == QLIN_FMT_INT8 || same_output(P, c.variant, c.tile_n, S, st);
                     std::printf("%s N=%lld K=%lld S=%d M=%lld %-14s tile=%3d  %9.2f us%s\n", fmt_name(s.fmt),

@@ -156,7 +156,9 @@ def test_fused_layer_zero_rows_and_auto_dispatch():
     assert qlin.qlin_sync_status() == 0
 
 
-def test_quantized_linear_module_uses_the_fused_call():
+def test_quantized_linear_module_runs_quantiser_then_pdl_gemm():
+    # QuantizedLinear's default: qlin_linear with QLIN_PDL (the stand-alone
+    # quantiser, then the GEMM as its programmatic dependent)
     from quantized_linear_layers_group_b200 import linear
 
     fmt = oracle.FMT_FP8

@@ -180,3 +180,57 @@ def test_group128_every_row_split(lib, rows):
     qg, sg = _gpu_block(lib, x, 1)
     qr, sr = oracle.quantize_block(x, 1, 128)
     _assert_same(qg, sg, qr, sr, f"group rows={rows}")
+
+
+def _markstein_rows(fmt, binades):
+    """Rows [amax, x...] for every amax significand in the given binades: the
+    row's x values are every bf16 significand at every exponent from amax's
+    down to 21 binades below it (where the quotient x / s leaves the range of
+    non-zero codes), both signs, |x| <= amax; unused slots are +0."""
+    rel = 22
+    L = 8 + 2 * 128 * rel                     # a multiple of 8 (16-byte rows)
+    rows = []
+    for eb in binades:                        # unbiased exponent of amax
+        EA = eb + 127
+        for ma in range(128):
+            amax = (EA << 7) | ma
+            r = np.zeros(L, np.uint16)
+            r[0] = amax
+            i = 1
+            for d in range(rel):
+                E = EA - d
+                for mx in range(128):
+                    if d == 0 and mx > ma:
+                        continue
+                    v = (E << 7) | mx
+                    r[i] = v
+                    r[i + 1] = v | 0x8000
+                    i += 2
+            rows.append(r)
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("fmt", [oracle.FMT_INT8, oracle.FMT_FP8])
+def test_per_token_quotient_exhaustive_over_significands(lib, fmt):
+    # The quantisers form x / s as one reciprocal of s plus Markstein's
+    # correction step where s lies in [2^-68, 2^92], and as an IEEE division
+    # elsewhere.  A quotient's rounding depends only on the significands of
+    # amax (hence of s = amax / Qmax) and of x and on their exponent gap, so
+    # every amax significand x every x significand x every gap that can give a
+    # non-zero code, in the binade amax in [1, 2), covers the whole fast range
+    # up to its edges; the edges themselves are covered by every amax of the
+    # five binades around each of 2^-68 * Qmax and 2^92 * Qmax.  Codes and
+    # scales must equal the oracle's (IEEE binary32 division) bit for bit.
+    qmax = 127.0 if fmt == oracle.FMT_INT8 else 448.0
+    lo = int(np.floor(np.log2(2.0 ** -68 * qmax)))
+    hi = int(np.floor(np.log2(2.0 ** 92 * qmax)))
+    binades = [0] + list(range(lo - 2, lo + 3)) + list(range(hi - 2, hi + 3))
+    x_bits = _markstein_rows(fmt, binades)
+    x = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16)
+    qg, sg = _gpu_per_token(lib, fmt, x)
+    qr, sr = oracle.quantize_per_token(fmt, x)
+    s_edge = sr[128:]
+    assert (s_edge < 2.0 ** -68).any() and (s_edge >= 2.0 ** -68).any()      # both sides of the low edge
+    assert (s_edge > 2.0 ** 92).any() and (s_edge <= 2.0 ** 92).any()        # and of the high edge
+    _assert_same(qg, sg, qr, sr, "quotient exhaustive")
+    check_status()
