@@ -12,7 +12,9 @@ numpy arrays to it.  bf16 tensors travel as their uint16 bit patterns.
 Format codes: 0 = INT8 (W8A8), 1 = FP8 e4m3 per-token/per-channel,
 2 = Block-FP8 (1x128 activation groups, 128x128 weight blocks), the three
 formats named on the page "Helion in vLLM: A Unified Route to Tunable Linear
-Kernels", section "What the integration changes".
+Kernels", section "What the integration changes".  ``gemm_bf16`` is the bf16
+matmul of the page "[Kernel][Perf] Add Hopper (SM90) tuned config for
+batch-invariant persistent matmul" (section "Summary").
 """
 from __future__ import annotations
 
@@ -74,6 +76,8 @@ def _load():
         lib.qo_scaled_mm.argtypes = [ctypes.c_int, i64, i64, i64, u8p, f32p, u8p, f32p, u16p,
                                      i64p, i64, i64p, i64, u16p, i32p]
         lib.qo_scaled_mm.restype = ctypes.c_int
+        lib.qo_gemm_bf16.argtypes = [i64, i64, i64, u16p, u16p, u16p, i64p, i64, i64p, i64, u16p]
+        lib.qo_gemm_bf16.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -183,6 +187,28 @@ def scaled_mm(fmt: int, a_q: np.ndarray, s_a: np.ndarray, w_q: np.ndarray, s_w: 
     if rc != 0:
         raise MemoryError("oracle allocation failed")
     return (c, acc) if want_acc else c
+
+
+def gemm_bf16(a, w, bias=None, m_idx=None, n_idx=None) -> np.ndarray:
+    """C = bf16(fp32(A W^T) + bias) for bf16 A [M, K] and W [N, K] (torch bf16
+    or uint16 bit arrays), optionally on a row / column sample; returns uint16
+    bits [len(m_idx), len(n_idx)] (or [M, N])."""
+    ab, wb = _bits(a), _bits(w)
+    M, K = ab.shape
+    N, K2 = wb.shape
+    assert K == K2
+    bb = None if bias is None else _bits(bias).reshape(-1)
+    mi = None if m_idx is None else np.ascontiguousarray(m_idx, dtype=np.int64)
+    ni = None if n_idx is None else np.ascontiguousarray(n_idx, dtype=np.int64)
+    mc = M if mi is None else len(mi)
+    nc = N if ni is None else len(ni)
+    c = np.empty((mc, nc), np.uint16)
+    rc = _load().qo_gemm_bf16(M, N, K, _ptr(ab, ctypes.c_uint16), _ptr(wb, ctypes.c_uint16),
+                              _ptr(bb, ctypes.c_uint16), _ptr(mi, ctypes.c_int64), mc, _ptr(ni, ctypes.c_int64), nc,
+                              _ptr(c, ctypes.c_uint16))
+    if rc != 0:
+        raise MemoryError("oracle allocation failed")
+    return c
 
 
 def bf16_bits_to_f32(c: np.ndarray) -> np.ndarray:

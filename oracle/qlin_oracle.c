@@ -19,6 +19,9 @@
  *                             (weights) block, s = amax_block / 448
  *   scaled GEMM:              C[m,n] = bf16( (acc[m,n] * s_a[m]) * s_w[n] + bias[n] )
  *   Block-FP8 GEMM:           C[m,n] = bf16( sum_kb P_kb[m,n] * s_a[m,kb] * s_w[n/128,kb] )
+ *   bf16 GEMM:                C[m,n] = bf16( fp32(sum_k a[m,k] w[n,k]) + bias[n] ), the
+ *                             matmul of the page "[Kernel][Perf] Add Hopper (SM90)
+ *                             tuned config for batch-invariant persistent matmul"
  *
  * Every fp32 operation is a separately rounded IEEE binary32 operation
  * (compile with -O2 -fno-fast-math -ffp-contract=off; x86-64 SSE arithmetic),
@@ -273,4 +276,51 @@ int qo_scaled_mm(int fmt, int64_t M, int64_t N, int64_t K,
     free(ua);
     free(uw);
     return rc;
+}
+
+/* ------------------------------------------------------------- bf16 GEMM ---- */
+/*
+ * bf16 matmul with fp32 accumulation and bf16 output, the workload of the
+ * page "[Kernel][Perf] Add Hopper (SM90) tuned config for batch-invariant
+ * persistent matmul" (sections "Summary" and "H100 NVL Sweep Results": a
+ * bfloat16 matmul of activations [M,K] with weights [N,K]):
+ *
+ *   C[m,n] = bf16( fp32( sum_k a[m,k] * w[n,k] ) + bias[n] )
+ *
+ * The product of two bf16 values (8-bit significands) is exact in binary64;
+ * the products are summed in binary64 in k order, the sum is rounded once to
+ * binary32, the bias (if any) is added as a binary32 addition and the result
+ * is rounded to bf16.  The binary64 sum differs from the exact one by at most
+ * K * 2^-53 * sum_k |a w|, far below the bf16 output rounding, so comparing a
+ * GPU result (fp32 accumulation in any fixed order) with this one measures the
+ * GPU's accumulation error.  Row and column selection as qo_scaled_mm.
+ */
+int qo_gemm_bf16(int64_t M, int64_t N, int64_t K, const uint16_t* a, const uint16_t* w, const uint16_t* bias,
+                 const int64_t* m_idx, int64_t m_cnt, const int64_t* n_idx, int64_t n_cnt, uint16_t* c) {
+    if (!m_idx) m_cnt = M;
+    if (!n_idx) n_cnt = N;
+    double* da = (double*)malloc(sizeof(double) * (size_t)(m_cnt * K));
+    double* dw = (double*)malloc(sizeof(double) * (size_t)(n_cnt * K));
+    if (!da || !dw) { free(da); free(dw); return -2; }
+    for (int64_t i = 0; i < m_cnt; ++i) {
+        int64_t m = m_idx ? m_idx[i] : i;
+        for (int64_t k = 0; k < K; ++k) da[i * K + k] = (double)qo_bf16_to_f32(a[m * K + k]);
+    }
+    for (int64_t j = 0; j < n_cnt; ++j) {
+        int64_t n = n_idx ? n_idx[j] : j;
+        for (int64_t k = 0; k < K; ++k) dw[j * K + k] = (double)qo_bf16_to_f32(w[n * K + k]);
+    }
+    for (int64_t i = 0; i < m_cnt; ++i) {
+        for (int64_t j = 0; j < n_cnt; ++j) {
+            int64_t n = n_idx ? n_idx[j] : j;
+            double s = 0.0;
+            for (int64_t k = 0; k < K; ++k) s += da[i * K + k] * dw[j * K + k];
+            float y = (float)s;                         /* one rounding to binary32 */
+            if (bias) y = y + qo_bf16_to_f32(bias[n]);  /* binary32 addition */
+            c[i * n_cnt + j] = qo_f32_to_bf16(y);
+        }
+    }
+    free(da);
+    free(dw);
+    return 0;
 }
