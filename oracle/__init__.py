@@ -78,6 +78,10 @@ def _load():
         lib.qo_scaled_mm.restype = ctypes.c_int
         lib.qo_gemm_bf16.argtypes = [i64, i64, i64, u16p, u16p, u16p, i64p, i64, i64p, i64, u16p]
         lib.qo_gemm_bf16.restype = ctypes.c_int
+        f32p_ = f32p
+        lib.qo_moe_forward.argtypes = [i64, i64, i64, i64, i64, u16p, f32p_, u8p, f32p_, u8p, f32p_, i32p, f32p_,
+                                       i32p, i32p, u16p, u8p, f32p_, u16p, u16p]
+        lib.qo_moe_forward.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -209,6 +213,41 @@ def gemm_bf16(a, w, bias=None, m_idx=None, n_idx=None) -> np.ndarray:
     if rc != 0:
         raise MemoryError("oracle allocation failed")
     return c
+
+
+def moe_forward(x, logits: np.ndarray, w1_q: np.ndarray, s_w1: np.ndarray, w2_q: np.ndarray, s_w2: np.ndarray,
+                topk: int) -> dict:
+    """The FP8 MoE layer step by step (see qo_moe_forward): x bf16 [T, H],
+    logits fp32 [T, E], W1_q [E, 2I, H] e4m3 codes with s_w1 [E, 2I], W2_q
+    [E, H, I] with s_w2 [E, H].  Returns a dict of numpy arrays: topk_ids,
+    topk_w, rows, offsets, g (bf16 bits [R, 2I]), h_q, s_h, y (bf16 bits
+    [R, H]) and out (bf16 bits [T, H])."""
+    xb = _bits(x)
+    T, H = xb.shape
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    E = logits.shape[1]
+    w1_q = np.ascontiguousarray(w1_q, dtype=np.uint8)
+    w2_q = np.ascontiguousarray(w2_q, dtype=np.uint8)
+    s_w1 = np.ascontiguousarray(s_w1, dtype=np.float32)
+    s_w2 = np.ascontiguousarray(s_w2, dtype=np.float32)
+    I = w2_q.shape[2]
+    assert w1_q.shape == (E, 2 * I, H) and w2_q.shape == (E, H, I)
+    assert s_w1.shape == (E, 2 * I) and s_w2.shape == (E, H)
+    R = T * topk
+    o = {"topk_ids": np.zeros((T, topk), np.int32), "topk_w": np.zeros((T, topk), np.float32),
+         "rows": np.zeros((T, topk), np.int32), "offsets": np.zeros(E + 1, np.int32),
+         "g": np.zeros((R, 2 * I), np.uint16), "h_q": np.zeros((R, I), np.uint8), "s_h": np.zeros(R, np.float32),
+         "y": np.zeros((R, H), np.uint16), "out": np.zeros((T, H), np.uint16)}
+    rc = _load().qo_moe_forward(T, H, I, E, topk, _ptr(xb, ctypes.c_uint16), _ptr(logits, ctypes.c_float),
+                                _ptr(w1_q, ctypes.c_uint8), _ptr(s_w1, ctypes.c_float), _ptr(w2_q, ctypes.c_uint8),
+                                _ptr(s_w2, ctypes.c_float), _ptr(o["topk_ids"], ctypes.c_int32),
+                                _ptr(o["topk_w"], ctypes.c_float), _ptr(o["rows"], ctypes.c_int32),
+                                _ptr(o["offsets"], ctypes.c_int32), _ptr(o["g"], ctypes.c_uint16),
+                                _ptr(o["h_q"], ctypes.c_uint8), _ptr(o["s_h"], ctypes.c_float),
+                                _ptr(o["y"], ctypes.c_uint16), _ptr(o["out"], ctypes.c_uint16))
+    if rc != 0:
+        raise RuntimeError(f"oracle moe_forward failed ({rc})")
+    return o
 
 
 def bf16_bits_to_f32(c: np.ndarray) -> np.ndarray:

@@ -324,3 +324,142 @@ int qo_gemm_bf16(int64_t M, int64_t N, int64_t K, const uint16_t* a, const uint1
     free(dw);
     return 0;
 }
+
+/* ------------------------------------------------------------- FP8 MoE ---- */
+/*
+ * The FP8 MoE layer the page "vLLM and Tencent Hunyuan upstream two HPC
+ * backends for NVIDIA Hopper GPUs" describes as one execution path (section
+ * "FP8 MoE pipeline as a single execution path": routing, Gate-Up GEMM,
+ * activation, quantisation, Down GEMM, top-k reduction), written out step by
+ * step.  The page gives the order of the steps, not their arithmetic; the
+ * plainest readings, stated here:
+ *
+ *   routing   for each token t, the k experts with the largest fp32 router
+ *             logits (ties: the lower expert index first), in descending
+ *             order; weights = softmax over those k logits:
+ *               m = l_0 (the largest); e_j = fp32(exp_binary64(l_j - m));
+ *               s = e_0 + e_1 + ... (fp32, in j order); w_j = e_j / s (fp32)
+ *   rows      token t's j-th expert e gets one row of that expert's group;
+ *             within an expert the rows are ordered by token index
+ *   gate-up   x is quantised per token to FP8 (qo_quantize_per_token); the
+ *             row of expert e computes G = scaled_mm(x_q[t], W1_q[e], s_x[t],
+ *             s_w1[e]) (the per-token FP8 GEMM of qo_scaled_mm, bf16 out, no
+ *             bias); G has 2I columns, gate = G[:, :I], up = G[:, I:]
+ *   act       h = silu(gate) * up in fp32 with silu(g) = g / (1 + q),
+ *             q = fp32(exp_binary64(-g)); the row of h is quantised per
+ *             token to FP8 (H_q, s_h)
+ *   down      Y = scaled_mm(H_q, W2_q[e], s_h, s_w2[e]) (bf16, no bias)
+ *   combine   out[t, n] = bf16( sum_j w_j * Y[row(t, j), n] ), the sum in fp32
+ *             from +0, j in routing order, each product and add separately
+ *             rounded
+ *
+ * Shapes: x bf16 [T, H]; logits fp32 [T, E]; W1_q [E, 2I, H] with s_w1 [E, 2I];
+ * W2_q [E, H, I] with s_w2 [E, H]; out bf16 [T, H].  Also returned for checks:
+ * topk ids/weights [T, k], the row of each (t, j) and the expert offsets
+ * [E + 1].
+ */
+static float silu_f32(float g) {
+    float q = (float)exp(-(double)g);      /* binary64 exponential, rounded once */
+    return g / (1.0f + q);
+}
+
+/* Intermediates returned for checks (caller-allocated): g bf16 [R, 2I],
+ * hq [R, I], sh [R], y bf16 [R, H], R = T * topk.  topk <= 64. */
+int qo_moe_forward(int64_t T, int64_t H, int64_t I, int64_t E, int64_t topk, const uint16_t* x,
+                   const float* logits, const uint8_t* w1_q, const float* s_w1, const uint8_t* w2_q,
+                   const float* s_w2, int32_t* topk_ids, float* topk_w, int32_t* rows, int32_t* offsets,
+                   uint16_t* g, uint8_t* hq, float* sh, uint16_t* y, uint16_t* out) {
+    const int64_t R = T * topk;
+    int rc = 0;
+    if (topk < 1 || topk > 64 || topk > E) return -3;
+    /* routing */
+    for (int64_t t = 0; t < T; ++t) {
+        const float* l = logits + t * E;
+        for (int64_t j = 0; j < topk; ++j) {
+            int64_t best = -1;
+            for (int64_t e = 0; e < E; ++e) {
+                int taken = 0;
+                for (int64_t i = 0; i < j; ++i) taken |= topk_ids[t * topk + i] == (int32_t)e;
+                if (taken) continue;
+                if (best < 0 || l[e] > l[best]) best = e;   /* ties keep the lower index */
+            }
+            topk_ids[t * topk + j] = (int32_t)best;
+        }
+        const float m = l[topk_ids[t * topk]];
+        float ev[64];
+        float s = 0.0f;
+        for (int64_t j = 0; j < topk; ++j) {
+            ev[j] = (float)exp((double)(l[topk_ids[t * topk + j]] - m));
+            s = s + ev[j];
+        }
+        for (int64_t j = 0; j < topk; ++j) topk_w[t * topk + j] = ev[j] / s;
+    }
+    /* rows: expert groups in expert order, tokens in order inside a group */
+    offsets[0] = 0;
+    for (int64_t e = 0; e < E; ++e) {
+        int32_t n = 0;
+        for (int64_t t = 0; t < T; ++t)
+            for (int64_t j = 0; j < topk; ++j) n += topk_ids[t * topk + j] == (int32_t)e;
+        offsets[e + 1] = offsets[e] + n;
+    }
+    int32_t* fill = (int32_t*)calloc((size_t)E, sizeof(int32_t));
+    uint8_t* xq = (uint8_t*)malloc((size_t)(T * H));
+    float* sx = (float*)malloc(sizeof(float) * (size_t)T);
+    uint8_t* a1 = (uint8_t*)malloc((size_t)(R * H));
+    float* sa1 = (float*)malloc(sizeof(float) * (size_t)R);
+    if (!fill || !xq || !sx || !a1 || !sa1) { rc = -2; goto out; }
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t j = 0; j < topk; ++j) {
+            const int32_t e = topk_ids[t * topk + j];
+            rows[t * topk + j] = offsets[e] + fill[e]++;
+        }
+    /* gate-up: per-token FP8 codes of x, gathered into the expert rows */
+    qo_quantize_per_token(QO_FMT_FP8, x, T, H, H, xq, sx);
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t j = 0; j < topk; ++j) {
+            const int64_t r = rows[t * topk + j];
+            memcpy(a1 + r * H, xq + t * H, (size_t)H);
+            sa1[r] = sx[t];
+        }
+    for (int64_t e = 0; e < E; ++e) {
+        const int64_t r0 = offsets[e], n = offsets[e + 1] - offsets[e];
+        if (n == 0) continue;
+        rc |= qo_scaled_mm(QO_FMT_FP8, n, 2 * I, H, a1 + r0 * H, sa1 + r0, w1_q + e * 2 * I * H, s_w1 + e * 2 * I,
+                           NULL, NULL, n, NULL, 2 * I, g + r0 * 2 * I, NULL);
+    }
+    /* act: h = silu(gate) * up in fp32, then the row's per-token FP8
+     * quantisation (amax, scale = amax / 448, codes as quantize_one) */
+    for (int64_t r = 0; r < R; ++r) {
+        float amax = 0.0f;
+        for (int64_t i = 0; i < I; ++i) {
+            const float h = silu_f32(qo_bf16_to_f32(g[r * 2 * I + i])) * qo_bf16_to_f32(g[r * 2 * I + I + i]);
+            if (fabsf(h) > amax) amax = fabsf(h);
+        }
+        const float sc = amax / 448.0f;
+        sh[r] = sc;
+        for (int64_t i = 0; i < I; ++i) {
+            const float h = silu_f32(qo_bf16_to_f32(g[r * 2 * I + i])) * qo_bf16_to_f32(g[r * 2 * I + I + i]);
+            hq[r * I + i] = quantize_one(QO_FMT_FP8, h, sc);
+        }
+    }
+    /* down */
+    for (int64_t e = 0; e < E; ++e) {
+        const int64_t r0 = offsets[e], n = offsets[e + 1] - offsets[e];
+        if (n == 0) continue;
+        rc |= qo_scaled_mm(QO_FMT_FP8, n, H, I, hq + r0 * I, sh + r0, w2_q + e * H * I, s_w2 + e * H, NULL, NULL,
+                           n, NULL, H, y + r0 * H, NULL);
+    }
+    /* combine: top-k reduction in routing order */
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t n = 0; n < H; ++n) {
+            float acc = 0.0f;
+            for (int64_t j = 0; j < topk; ++j) {
+                const float p = topk_w[t * topk + j] * qo_bf16_to_f32(y[(int64_t)rows[t * topk + j] * H + n]);
+                acc = acc + p;
+            }
+            out[t * H + n] = qo_f32_to_bf16(acc);
+        }
+out:
+    free(fill); free(xq); free(sx); free(a1); free(sa1);
+    return rc;
+}
