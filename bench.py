@@ -58,11 +58,14 @@ import synth  # noqa: E402
 
 METRIC = "scaled_mm TFLOPS & HBM GB/s vs roofline, per (M,N,K,format), 1×B200"
 L2_BYTES = 126 * 1024 * 1024
-FMT_NAME = {0: "int8", 1: "fp8", 2: "fp8_block"}
-DTYPE = {0: "int8 (int32 accumulate)", 1: "fp8_e4m3 (fp32 accumulate)", 2: "fp8_e4m3 block-scaled (fp32 accumulate)"}
+FMT_NAME = {0: "int8", 1: "fp8", 2: "fp8_block", 3: "bf16"}
+DTYPE = {0: "int8 (int32 accumulate)", 1: "fp8_e4m3 (fp32 accumulate)", 2: "fp8_e4m3 block-scaled (fp32 accumulate)",
+         3: "bf16 (fp32 accumulate)"}
 HEADLINE = "fp8_attn"
 # every workload of the metric: the headline plus the parity configurations
 ALL_WORKLOADS = ("fp8_attn", "int8_smoke", "fp8_block_down", "lm_head", "fp8_vocab", "int8_square")
+# the bf16 batch-invariant matmul on the five shapes of its sweep (no quantisation step)
+BF16_WORKLOADS = ("bf16_vocab", "bf16_down", "bf16_attn", "bf16_lm_head", "bf16_square")
 
 
 # ------------------------------------------------------------------ peaks
@@ -111,9 +114,12 @@ def measure_tensor_peaks(device, n=8192, reps=10):
 
 
 def tensor_peak(peaks, fmt, tpk=None):
-    """Dense 8-bit tensor peak for a kernel timed in isolation (burst): the
-    measured library figure for the format when there is one, else the
-    measured bf16 burst peak x 2 (the nominal 8-bit / bf16 ratio)."""
+    """Dense tensor peak for a kernel timed in isolation (burst): bf16 the
+    measured cuBLAS bf16 burst figure; 8-bit the measured library figure for
+    the format when there is one, else the bf16 burst peak x 2 (the nominal
+    8-bit / bf16 ratio)."""
+    if fmt == 3:
+        return peaks["bf16_tflops"], f"{peaks['source']} bf16_tflops (cuBLAS bf16 burst)"
     if tpk is not None:
         v = tpk.get("int8_tops" if fmt == 0 else "fp8_tflops")
         if v:
@@ -128,13 +134,16 @@ def gemm_flops(M, N, K):
 def gemm_bytes(M, N, K, fmt):
     """Algorithmic bytes per GEMM launch: the 8-bit operands A and W (as the
     roofline is defined on), plus scales, bias and the bf16 output separately."""
-    ab = M * K + N * K
-    scales = (M * (K // 128) + (N // 128) * (K // 128)) * 4 if fmt == 2 else (M + N) * 4
+    elt = 2 if fmt == 3 else 1
+    ab = (M * K + N * K) * elt
+    scales = (M * (K // 128) + (N // 128) * (K // 128)) * 4 if fmt == 2 else (0 if fmt == 3 else (M + N) * 4)
     extra = scales + 2 * M * N
     return ab, extra
 
 
 def quant_bytes(M, K, fmt):
+    if fmt == 3:
+        return 0  # bf16: no quantisation step
     return 2 * M * K + M * K + (M * (K // 128) if fmt == 2 else M) * 4
 
 
@@ -287,13 +296,16 @@ class HotPath:
         w_cpu = synth.weights(workload, seed)
         b_cpu = synth.bias(workload, seed)
         w_dev = w_cpu.to(device)
-        w_q, s_w = linear.quantize_weight(self.fmt, w_dev)
-        del w_dev
+        if self.fmt == 3:  # bf16: the weight is used as it is
+            w_q, s_w = w_dev, None
+        else:
+            w_q, s_w = linear.quantize_weight(self.fmt, w_dev)
+            del w_dev
         self.bias = None if b_cpu is None else b_cpu.to(device)
-        wbytes = N * K
+        wbytes = N * K * (2 if self.fmt == 3 else 1)
         # enough weight copies that the bytes read between two uses of a copy exceed 2x L2
         self.n_copies = max(2, math.ceil(2 * L2_BYTES / wbytes) + 1)
-        self.w_copies = [(w_q if i == 0 else w_q.clone(), s_w if i == 0 else s_w.clone())
+        self.w_copies = [(w_q if i == 0 else w_q.clone(), s_w if i == 0 or s_w is None else s_w.clone())
                          for i in range(self.n_copies)]
         # graphs per rotation of the weight copies; each graph = one step with its own activation set
         self.n_graphs = max(1, math.ceil(self.n_copies / len(self.ms)))
@@ -301,16 +313,17 @@ class HotPath:
         self.n_act_sets = max(self.n_graphs, math.ceil(2 * L2_BYTES / step_bytes) + 1)
         a_cpu = {M: synth.activations(workload, M, seed=seed) for M in self.ms}
         self.a_sets = [{M: a_cpu[M].to(device) for M in self.ms} for _ in range(self.n_act_sets)]
-        self.a_host = {M: a_cpu[M].pin_memory() for M in self.ms}
+        self.a_cpu = a_cpu
+        self.a_host = None  # pinned copies, made by the first end-to-end step
         self.act = 0  # activation set of the step being issued
         self.a_q, self.s_a, self.c, self.c_host = {}, {}, {}, {}
         ws = 0
         for M in self.ms:
-            self.a_q[M] = torch.empty(M, K, dtype=torch.uint8, device=device)
+            self.a_q[M] = (torch.empty(M, K, dtype=torch.bfloat16, device=device) if self.fmt == 3 else
+                           torch.empty(M, K, dtype=torch.uint8, device=device))
             self.s_a[M] = torch.empty(*((M, K // 128) if self.fmt == 2 else (M,)), dtype=torch.float32,
                                       device=device)
             self.c[M] = torch.empty(M, N, dtype=torch.bfloat16, device=device)
-            self.c_host[M] = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
             ws = max(ws, qlin.qlin_scaled_mm_workspace_size(self.fmt, M, N, K))
         self.workspace = torch.zeros(max(ws, 256), dtype=torch.uint8, device=device)
         self.calls = 0
@@ -322,6 +335,8 @@ class HotPath:
     def launch_quant(self, M, stream):
         q = self.qlin
         x = self.a_sets[self.act][M]
+        if self.fmt == 3:
+            return  # bf16: the GEMM reads the activations themselves
         if self.fmt == 2:
             q.qlin_quantize_block(x, 1, self.a_q[M], self.s_a[M], stream, flags=self.flags)
         else:
@@ -330,6 +345,10 @@ class HotPath:
     def launch_gemm(self, M, stream):
         w_q, s_w = self.w_copies[self.calls % self.n_copies]
         self.calls += 1
+        if self.fmt == 3:
+            self.qlin.qlin_matmul_bf16(self.a_sets[self.act][M], w_q, self.bias, self.c[M], self.workspace, stream,
+                                       flags=self.flags)
+            return
         self.qlin.qlin_scaled_mm(self.fmt, self.a_q[M], self.s_a[M], w_q, s_w, self.bias, self.c[M],
                                  self.workspace, stream, flags=self.flags)
 
@@ -357,6 +376,9 @@ class HotPath:
         C copied back; returns (h2d bytes, d2h bytes)."""
         hb = db = 0
         self.act = 0
+        if self.a_host is None:
+            self.a_host = {M: self.a_cpu[M].pin_memory() for M in self.ms}
+            self.c_host = {M: torch.empty(M, self.w.N, dtype=torch.bfloat16).pin_memory() for M in self.ms}
         for M in self.ms:
             self.a_sets[0][M].copy_(self.a_host[M], non_blocking=True)
             hb += self.a_host[M].numel() * 2
@@ -374,7 +396,7 @@ def per_kernel_times(hp: HotPath, stream, reps=8, replays=5):
     median of `replays` replays.  Returns ({M: quant us}, {M: gemm us})."""
     qt, gt = {}, {}
     for M in hp.ms:
-        for kind in ("q", "g"):
+        for kind in (("g",) if hp.fmt == 3 else ("q", "g")):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 for i in range(reps):
@@ -395,6 +417,7 @@ def per_kernel_times(hp: HotPath, stream, reps=8, replays=5):
                 ts.append(a0.elapsed_time(a1) * 1e3 / reps)
             (qt if kind == "q" else gt)[M] = statistics.median(ts)
             del g
+        qt.setdefault(M, 0.0)
     torch.cuda.synchronize()
     return qt, gt
 
@@ -422,8 +445,8 @@ def workload_report(hp: HotPath, qt, gt, peaks, tpk):
                       "hbm_gbs_all_bytes": (ab + extra) / tg / 1e9,
                       "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / tg,
                       "bound": "hbm" if t_hbm >= t_tc else "tensor",
-                      "quant_gbs": quant_bytes(M, K, fmt) / tq / 1e9,
-                      "quant_frac_hbm": quant_bytes(M, K, fmt) / tq / 1e9 / hbm})
+                      "quant_gbs": quant_bytes(M, K, fmt) / tq / 1e9 if tq > 0 else None,
+                      "quant_frac_hbm": quant_bytes(M, K, fmt) / tq / 1e9 / hbm if tq > 0 else None})
     total = sum(gt[M] + qt[M] for M in hp.ms)
     roof = kernel_roofline(per_m, hp.configs, fmt, N, K, hbm, tc_peak, total)
     roof["traffic"] = measured_traffic_kernel(w.name, fmt, N, K, hp.configs, roof["m_values"])
@@ -630,7 +653,7 @@ def main(argv=None):
     ap.add_argument("--no-workloads", action="store_true", help="measure the headline workload only")
     ap.add_argument("--no-peaks", action="store_true", help="skip the 8-bit library peak measurement")
     ap.add_argument("--ref-rows", type=int, default=64, help="rows per M in a reference-arm step")
-    ap.add_argument("--baseline-rows", type=int, default=64, help="rows per M of the cpu_baseline sample")
+    ap.add_argument("--baseline-rows", type=int, default=1024, help="rows per M of the all-core cpu_baseline sample")
     args = ap.parse_args(argv)
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
 
@@ -691,7 +714,7 @@ def main(argv=None):
         # ------------------------------ every workload of the metric, per M
         workloads = {}
         if not args.no_workloads and world == 1:
-            for name in ALL_WORKLOADS:
+            for name in ALL_WORKLOADS + BF16_WORKLOADS:
                 w = synth.WORKLOADS[name]
                 wh = HotPath(w, list(w.m_values), device)
                 for _ in range(3):
@@ -747,7 +770,7 @@ def main(argv=None):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows = reference_rows(workload, args.baseline_rows)
         cores = host_cores()
-        dt1, fl1 = cpu_oracle_rows(workload, [(M, min(r, 16)) for M, r in rows], threads=1)
+        dt1, fl1 = cpu_oracle_rows(workload, [(M, min(r, 64)) for M, r in rows], threads=1)
         dtn, fln = cpu_oracle_rows(workload, rows, threads=cores)
         line["cpu_baseline"] = {
             "value": fln / dtn / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
@@ -756,7 +779,7 @@ def main(argv=None):
                        f"quantised and their full C rows computed (N={N}, K={K}), {cores} threads"),
             "seconds": dtn,
             "one_thread": {"value": fl1 / dt1 / 1e12, "unit": "TFLOP/s", "cores": 1, "seconds": dt1,
-                           "sample": f"the same, first min(M, 16) rows, 1 thread"}}
+                           "sample": "the same, first min(M, 64) rows, 1 thread"}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

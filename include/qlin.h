@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define QLIN_ABI_VERSION 4
+#define QLIN_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define QLIN_API __attribute__((visibility("default")))
@@ -70,7 +70,10 @@ typedef enum {
 typedef enum {
     QLIN_FMT_INT8 = 0,       /* W8A8 INT8, per-token / per-channel scales, int32 accumulate */
     QLIN_FMT_FP8 = 1,        /* e4m3, per-token / per-channel scales, fp32 accumulate */
-    QLIN_FMT_FP8_BLOCK = 2   /* e4m3, 1x128 activation groups, 128x128 weight blocks */
+    QLIN_FMT_FP8_BLOCK = 2,  /* e4m3, 1x128 activation groups, 128x128 weight blocks */
+    QLIN_FMT_BF16 = 3        /* bf16 operands, no scales, fp32 accumulate (qlin_matmul_bf16 only;
+                                also accepted by qlin_scaled_mm_workspace_size and
+                                qlin_dispatch_query) */
 } qlin_format;
 
 typedef enum {
@@ -214,6 +217,36 @@ QLIN_API qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segm
                            size_t workspace_bytes, qlin_stream_t stream);
 
 /*
+ * qlin_matmul_bf16 -- the batch-invariant persistent bf16 matmul of the page
+ * "[Kernel][Perf] Add Hopper (SM90) tuned config for batch-invariant
+ * persistent matmul" (section "Summary": a per-shape tuned persistent matmul
+ * whose outputs do not depend on the batch size; "Test Plan"), on the same
+ * kernel family, tiles, strategies and dispatch table as qlin_scaled_mm:
+ *
+ *     C[m,n] = bf16( fp32( sum_k a[m,k] * w[n,k] ) + bias[n] )
+ *
+ * Determinism and batch invariance exactly as qlin_scaled_mm: K is cut into
+ * k_segments segments fixed per (N, K) in the table; each segment is summed by
+ * the tensor core in fp32 and the segments are added in order from +0, so a
+ * row of C depends only on that row of a, never on M, the variant or CTA
+ * timing.  A K block is 64 bf16 elements (128 bytes); k_segments | K/64.
+ *
+ *   variant, tile_n, k_segments   as qlin_scaled_mm (AUTO: table entry "bf16")
+ *   M, N, K       M >= 0 (0 is a no-op), N >= 16, N % 16 == 0, K % 64 == 0
+ *   a, w          bf16 [M, K] and [N, K] row-major (device)
+ *   bias          bf16 [N] (device) or NULL
+ *   c_out         bf16 [M, N] (device)
+ *   flags         QLIN_PDL, QLIN_SPLITK_CLUSTER
+ *   workspace     as qlin_scaled_mm (size from qlin_scaled_mm_workspace_size
+ *                 with QLIN_FMT_BF16)
+ * Alignment: a, w, c_out, workspace 16-byte aligned; bias 2.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_matmul_bf16(int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
+                                      const void* a, const void* w, const void* bias, void* c_out, uint32_t flags,
+                                      void* workspace, size_t workspace_bytes, qlin_stream_t stream);
+
+/*
  * qlin_scaled_mm_noalloc -- qlin_scaled_mm for callers that cannot allocate
  * device memory and so cannot pass a workspace (the paper has no counterpart;
  * this is a library convenience).  Typical caller: a plugin inside a serving
@@ -271,6 +304,112 @@ QLIN_API qlin_status qlin_linear(int fmt, int variant, int tile_n, int k_segment
                                  const void* x, int64_t ld_x, void* a_q, float* s_a, const void* w_q,
                                  const float* s_w, const void* bias, void* c_out, uint32_t flags, void* workspace,
                                  size_t workspace_bytes, qlin_stream_t stream);
+
+/*
+ * ---------------------------------------------------------------- FP8 MoE
+ * The FP8 MoE layer run as one path of kernels chained with programmatic
+ * dependent launch, as the page "vLLM and Tencent Hunyuan upstream two HPC
+ * backends for NVIDIA Hopper GPUs" describes it (section "FP8 MoE pipeline as
+ * a single execution path": routing, Gate-Up GEMM, activation function,
+ * quantisation, Down GEMM, top-k reduction).  Dimensions: T tokens, hidden
+ * size H, expert intermediate size I, E experts (1 .. 255), top-k (1 .. 32,
+ * <= E); R = T * topk expert rows.  Each entry point below is one step; every
+ * one accepts QLIN_PDL (launch as the previous kernel's programmatic
+ * dependent) and is asynchronous on `stream`.
+ */
+
+/*
+ * qlin_moe_route -- top-k routing and the expert row layout.  For token t:
+ * the topk experts with the largest fp32 logits (descending; ties to the
+ * lower expert index) into topk_ids [T, topk], and weights into topk_w
+ * [T, topk]: w_j = e_j / (e_0 + ... ) in fp32 with e_j = fp32(exp(l_j - l_0))
+ * (the exponential in binary64).  Then offsets [E + 1] = prefix sums of the
+ * experts' row counts, and rows [T, topk] = the row of (t, j) in expert
+ * topk_ids[t, j]'s group [offsets[e], offsets[e+1]) (any order inside a group;
+ * results never depend on it).  logits fp32 [T, E]; all device pointers.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_moe_route(int64_t T, int E, int topk, const float* logits, int32_t* topk_ids,
+                                    float* topk_w, int32_t* rows, int32_t* offsets, uint32_t flags,
+                                    qlin_stream_t stream);
+
+/*
+ * qlin_moe_quantize_scatter -- per-token FP8 quantisation of x (bf16 [T, H],
+ * H % 16 == 0; as qlin_quantize_per_token) written to each of the token's
+ * expert rows: a_q [R, H] e4m3, s_a [R] fp32, rows as qlin_moe_route made them.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_moe_quantize_scatter(int64_t T, int64_t H, int topk, const void* x, const int32_t* rows,
+                                               void* a_q, float* s_a, uint32_t flags, qlin_stream_t stream);
+
+/*
+ * qlin_moe_grouped_mm -- the scaled GEMM over experts: for each expert e and
+ * each row r of its group [offsets[e], offsets[e+1]),
+ *     C[r, n] = bf16( ((float)acc * s_a[r]) * s_w[e N + n] ),
+ *     acc = sum_k A_q[r, k] W_q[e N + n, k]
+ * (INT8 or FP8 per-token / per-channel, as qlin_scaled_mm without bias).  One
+ * persistent tcgen05 kernel; the experts' tile counts are read from offsets
+ * (device) after the dependency wait.  A row's result never depends on the
+ * other rows of its tile or on the tiling (K is summed in one segment).
+ *   fmt        QLIN_FMT_INT8 or QLIN_FMT_FP8
+ *   variant    AUTO (Swap-AB when the average rows per expert is <= 64, else
+ *              plain), QLIN_VAR_SWAPAB or QLIN_VAR_PLAIN; tile_n 0 or as
+ *              qlin_scaled_mm
+ *   a_q [R, K], s_a [R]; w_q [E N, K], s_w [E N]; c_out bf16 [R, N]
+ *   N % 16 == 0, K % 128 == 0
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_moe_grouped_mm(int fmt, int variant, int tile_n, int E, int64_t R, int64_t N, int64_t K,
+                                         const void* a_q, const float* s_a, const int32_t* offsets, const void* w_q,
+                                         const float* s_w, void* c_out, uint32_t flags, qlin_stream_t stream);
+
+/*
+ * qlin_moe_act_quantize -- the activation and its quantisation: for each row
+ * r of g (bf16 [R, 2I]: gate = g[:, :I], up = g[:, I:]), h = silu(gate) * up
+ * in fp32 with silu(x) = x / (1 + fp32(exp(-x))) (the exponential in
+ * binary64), then the per-token FP8 quantisation of h into h_q [R, I] and
+ * s_h [R] (scale = amax / 448, codes as qlin_quantize_per_token).  I % 16 == 0.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_moe_act_quantize(int64_t R, int64_t I, const void* g, void* h_q, float* s_h,
+                                           uint32_t flags, qlin_stream_t stream);
+
+/*
+ * qlin_moe_combine -- the top-k reduction: out[t, n] = bf16( sum_j topk_w[t, j]
+ * * y[rows[t, j], n] ), summed in fp32 from +0 in routing order j = 0 ..
+ * topk-1, each product and add separately rounded.  y bf16 [R, H], out bf16
+ * [T, H], H % 16 == 0.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_moe_combine(int64_t T, int64_t H, int topk, const void* y, const float* topk_w,
+                                      const int32_t* rows, void* out, uint32_t flags, qlin_stream_t stream);
+
+/*
+ * qlin_moe_workspace_size -- bytes of workspace qlin_moe_forward needs.  The
+ * workspace holds, each at a 256-byte aligned offset in this order: topk_ids
+ * [R] int32, topk_w [R] fp32, rows [R] int32, offsets [E + 1] int32, a_q [R, H]
+ * e4m3, s_a [R], g [R, 2I] bf16, h_q [R, I] e4m3, s_h [R], y [R, H] bf16.
+ * Errors: INVALID_ARG.
+ */
+QLIN_API qlin_status qlin_moe_workspace_size(int64_t T, int64_t H, int64_t I, int E, int topk, size_t* bytes_out);
+
+/*
+ * qlin_moe_forward -- the whole FP8 MoE layer: route, quantise-scatter,
+ * grouped gate-up GEMM (N = 2I, K = H), activation + quantisation, grouped
+ * down GEMM (N = H, K = I), combine; seven kernels, each after the first the
+ * previous one's programmatic dependent.  x bf16 [T, H]; logits fp32 [T, E];
+ * w1_q e4m3 [E, 2I, H] with s_w1 [E, 2I]; w2_q e4m3 [E, H, I] with s_w2
+ * [E, H] (weights quantised per output channel, e.g. by
+ * qlin_quantize_per_token on the [E * rows, cols] view); out bf16 [T, H].
+ * H % 128 == 0, I % 128 == 0.  workspace: qlin_moe_workspace_size() bytes,
+ * 16-byte aligned, no initialisation needed; calls that overlap in time must
+ * not share one.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_moe_forward(int64_t T, int64_t H, int64_t I, int E, int topk, const void* x,
+                                      const float* logits, const void* w1_q, const float* s_w1, const void* w2_q,
+                                      const float* s_w2, void* out, uint32_t flags, void* workspace,
+                                      size_t workspace_bytes, qlin_stream_t stream);
 
 /*
  * qlin_scaled_mm_workspace_size -- bytes of workspace qlin_scaled_mm needs for

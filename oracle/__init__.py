@@ -82,6 +82,10 @@ def _load():
         lib.qo_moe_forward.argtypes = [i64, i64, i64, i64, i64, u16p, f32p_, u8p, f32p_, u8p, f32p_, i32p, f32p_,
                                        i32p, i32p, u16p, u8p, f32p_, u16p, u16p]
         lib.qo_moe_forward.restype = ctypes.c_int
+        lib.qo_moe_act_quantize.argtypes = [i64, i64, u16p, u8p, f32p_]
+        lib.qo_moe_act_quantize.restype = None
+        lib.qo_moe_combine.argtypes = [i64, i64, i64, u16p, f32p_, i32p, u16p]
+        lib.qo_moe_combine.restype = None
         _lib = lib
     return _lib
 
@@ -248,6 +252,29 @@ def moe_forward(x, logits: np.ndarray, w1_q: np.ndarray, s_w1: np.ndarray, w2_q:
     if rc != 0:
         raise RuntimeError(f"oracle moe_forward failed ({rc})")
     return o
+
+
+def moe_act_quantize(g: np.ndarray):
+    """The MoE activation step alone: g bf16 bits [R, 2I] -> (h_q [R, I], s_h [R])."""
+    g = np.ascontiguousarray(g, dtype=np.uint16)
+    R, I2 = g.shape
+    hq = np.zeros((R, I2 // 2), np.uint8)
+    sh = np.zeros(R, np.float32)
+    _load().qo_moe_act_quantize(R, I2 // 2, _ptr(g, ctypes.c_uint16), _ptr(hq, ctypes.c_uint8), _ptr(sh, ctypes.c_float))
+    return hq, sh
+
+
+def moe_combine(y: np.ndarray, w: np.ndarray, rows: np.ndarray) -> np.ndarray:
+    """The MoE top-k reduction alone: y bf16 bits [R, H], w [T, k], rows [T, k] -> out bits [T, H]."""
+    y = np.ascontiguousarray(y, dtype=np.uint16)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    T, k = w.shape
+    H = y.shape[1]
+    out = np.zeros((T, H), np.uint16)
+    _load().qo_moe_combine(T, H, k, _ptr(y, ctypes.c_uint16), _ptr(w, ctypes.c_float), _ptr(rows, ctypes.c_int32),
+                           _ptr(out, ctypes.c_uint16))
+    return out
 
 
 def bf16_bits_to_f32(c: np.ndarray) -> np.ndarray:

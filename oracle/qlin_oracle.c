@@ -363,6 +363,40 @@ static float silu_f32(float g) {
     return g / (1.0f + q);
 }
 
+/* act: h = silu(gate) * up in fp32 for each row of g (bf16 [R, 2I]), then
+ * the row's per-token FP8 quantisation (amax, scale = amax / 448, codes as
+ * quantize_one) into hq [R, I] and sh [R]. */
+void qo_moe_act_quantize(int64_t R, int64_t I, const uint16_t* g, uint8_t* hq, float* sh) {
+    for (int64_t r = 0; r < R; ++r) {
+        float amax = 0.0f;
+        for (int64_t i = 0; i < I; ++i) {
+            const float h = silu_f32(qo_bf16_to_f32(g[r * 2 * I + i])) * qo_bf16_to_f32(g[r * 2 * I + I + i]);
+            if (fabsf(h) > amax) amax = fabsf(h);
+        }
+        const float sc = amax / 448.0f;
+        sh[r] = sc;
+        for (int64_t i = 0; i < I; ++i) {
+            const float h = silu_f32(qo_bf16_to_f32(g[r * 2 * I + i])) * qo_bf16_to_f32(g[r * 2 * I + I + i]);
+            hq[r * I + i] = quantize_one(QO_FMT_FP8, h, sc);
+        }
+    }
+}
+
+/* combine: out[t, n] = bf16( sum_j w[t, j] * y[rows[t, j], n] ), fp32 from +0
+ * in routing order, each product and add separately rounded. */
+void qo_moe_combine(int64_t T, int64_t H, int64_t topk, const uint16_t* y, const float* w, const int32_t* rows,
+                    uint16_t* out) {
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t n = 0; n < H; ++n) {
+            float acc = 0.0f;
+            for (int64_t j = 0; j < topk; ++j) {
+                const float p = w[t * topk + j] * qo_bf16_to_f32(y[(int64_t)rows[t * topk + j] * H + n]);
+                acc = acc + p;
+            }
+            out[t * H + n] = qo_f32_to_bf16(acc);
+        }
+}
+
 /* Intermediates returned for checks (caller-allocated): g bf16 [R, 2I],
  * hq [R, I], sh [R], y bf16 [R, H], R = T * topk.  topk <= 64. */
 int qo_moe_forward(int64_t T, int64_t H, int64_t I, int64_t E, int64_t topk, const uint16_t* x,
@@ -427,21 +461,8 @@ int qo_moe_forward(int64_t T, int64_t H, int64_t I, int64_t E, int64_t topk, con
         rc |= qo_scaled_mm(QO_FMT_FP8, n, 2 * I, H, a1 + r0 * H, sa1 + r0, w1_q + e * 2 * I * H, s_w1 + e * 2 * I,
                            NULL, NULL, n, NULL, 2 * I, g + r0 * 2 * I, NULL);
     }
-    /* act: h = silu(gate) * up in fp32, then the row's per-token FP8
-     * quantisation (amax, scale = amax / 448, codes as quantize_one) */
-    for (int64_t r = 0; r < R; ++r) {
-        float amax = 0.0f;
-        for (int64_t i = 0; i < I; ++i) {
-            const float h = silu_f32(qo_bf16_to_f32(g[r * 2 * I + i])) * qo_bf16_to_f32(g[r * 2 * I + I + i]);
-            if (fabsf(h) > amax) amax = fabsf(h);
-        }
-        const float sc = amax / 448.0f;
-        sh[r] = sc;
-        for (int64_t i = 0; i < I; ++i) {
-            const float h = silu_f32(qo_bf16_to_f32(g[r * 2 * I + i])) * qo_bf16_to_f32(g[r * 2 * I + I + i]);
-            hq[r * I + i] = quantize_one(QO_FMT_FP8, h, sc);
-        }
-    }
+    /* act */
+    qo_moe_act_quantize(R, I, g, hq, sh);
     /* down */
     for (int64_t e = 0; e < E; ++e) {
         const int64_t r0 = offsets[e], n = offsets[e + 1] - offsets[e];
@@ -449,16 +470,8 @@ int qo_moe_forward(int64_t T, int64_t H, int64_t I, int64_t E, int64_t topk, con
         rc |= qo_scaled_mm(QO_FMT_FP8, n, H, I, hq + r0 * I, sh + r0, w2_q + e * H * I, s_w2 + e * H, NULL, NULL,
                            n, NULL, H, y + r0 * H, NULL);
     }
-    /* combine: top-k reduction in routing order */
-    for (int64_t t = 0; t < T; ++t)
-        for (int64_t n = 0; n < H; ++n) {
-            float acc = 0.0f;
-            for (int64_t j = 0; j < topk; ++j) {
-                const float p = topk_w[t * topk + j] * qo_bf16_to_f32(y[(int64_t)rows[t * topk + j] * H + n]);
-                acc = acc + p;
-            }
-            out[t * H + n] = qo_f32_to_bf16(acc);
-        }
+    /* combine */
+    qo_moe_combine(T, H, topk, y, topk_w, rows, out);
 out:
     free(fill); free(xq); free(sx); free(a1); free(sa1);
     return rc;

@@ -53,6 +53,7 @@ const char* fmt_name(int f) {
         case QLIN_FMT_INT8: return "int8";
         case QLIN_FMT_FP8: return "fp8";
         case QLIN_FMT_FP8_BLOCK: return "fp8_block";
+        case QLIN_FMT_BF16: return "bf16";
     }
     return "?";
 }
@@ -61,6 +62,7 @@ int parse_fmt(const std::string& s) {
     if (s == "int8") return QLIN_FMT_INT8;
     if (s == "fp8") return QLIN_FMT_FP8;
     if (s == "fp8_block") return QLIN_FMT_FP8_BLOCK;
+    if (s == "bf16") return QLIN_FMT_BF16;
     return -1;
 }
 
@@ -112,16 +114,20 @@ int default_segments(int fmt, int64_t N, int64_t K, int num_sms) {
     return best;
 }
 
+// Bytes of one operand row and 128-byte K blocks: 8-bit formats 1 B/element, bf16 2.
+int64_t row_bytes(int fmt, int64_t K) { return fmt == QLIN_FMT_BF16 ? 2 * K : K; }
+
 qlin_config default_config(int fmt, int64_t M, int64_t N, int64_t K, int num_sms) {
     qlin_config c{};
-    c.k_segments = default_segments(fmt, N, K, num_sms);
+    c.k_segments = default_segments(fmt, N, row_bytes(fmt, K), num_sms);
     c.from_table = 0;
     c.m_max = 0;
     if (M <= 64) {
         c.tile_n = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
         c.variant = c.k_segments > 1 ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB;
     } else {
-        const bool multi = fmt == QLIN_FMT_FP8_BLOCK || (fmt == QLIN_FMT_FP8 && c.k_segments > 1);
+        const bool multi =
+            fmt == QLIN_FMT_FP8_BLOCK || ((fmt == QLIN_FMT_FP8 || fmt == QLIN_FMT_BF16) && c.k_segments > 1);
         c.tile_n = multi ? 128 : 256;
         const int64_t tiles = ((M + 127) / 128) * ((N + c.tile_n - 1) / c.tile_n);
         c.variant = (c.k_segments > 1 && tiles * 2 <= num_sms) ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN;
@@ -182,9 +188,10 @@ qlin_status resolve_config(int fmt, int variant, int tile_n, int k_segments, int
 }  // namespace
 
 qlin_status check_fmt_shape(int fmt, int64_t M, int64_t N, int64_t K) {
-    if (fmt < QLIN_FMT_INT8 || fmt > QLIN_FMT_FP8_BLOCK) return QLIN_ERR_INVALID_ARG;
-    if (M < 0 || N < 16 || K < 128) return QLIN_ERR_INVALID_ARG;
-    if (N % 16 != 0 || K % 128 != 0) return QLIN_ERR_UNSUPPORTED;
+    if (fmt < QLIN_FMT_INT8 || fmt > QLIN_FMT_BF16) return QLIN_ERR_INVALID_ARG;
+    const int64_t kunit = fmt == QLIN_FMT_BF16 ? 64 : 128;  // elements per 128-byte K block
+    if (M < 0 || N < 16 || K < kunit) return QLIN_ERR_INVALID_ARG;
+    if (N % 16 != 0 || K % kunit != 0) return QLIN_ERR_UNSUPPORTED;
     if (fmt == QLIN_FMT_FP8_BLOCK && N % 128 != 0) return QLIN_ERR_UNSUPPORTED;
     if (M > (int64_t)1 << 30 || N > (int64_t)1 << 30 || K > (int64_t)1 << 24) return QLIN_ERR_UNSUPPORTED;
     return QLIN_OK;
@@ -220,7 +227,8 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     p.M = M;
     p.N = N;
     p.K = K;
-    p.kblocks = (int)(K / 128);
+    p.k_bytes = row_bytes(fmt, K);
+    p.kblocks = (int)(p.k_bytes / 128);
     const bool pair = cfg.variant == QLIN_VAR_PAIR;
     if (!tile_supported(fmt, p.swap, p.tile_n, pair)) return QLIN_ERR_UNSUPPORTED;
     if (p.k_segments < 1 || p.kblocks % p.k_segments != 0) return QLIN_ERR_UNSUPPORTED;
@@ -229,7 +237,7 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     // units with more than one accumulator chunk keep tile_n fp32 values per
     // thread and a TMEM running total: only tiles up to 128 columns do that
     const bool multi_chunk = (fmt == QLIN_FMT_FP8_BLOCK && (p.spread ? p.kb_per_seg : p.kblocks) > 1) ||
-                             (fmt == QLIN_FMT_FP8 && !p.spread && p.k_segments > 1);
+                             ((fmt == QLIN_FMT_FP8 || fmt == QLIN_FMT_BF16) && !p.spread && p.k_segments > 1);
     if (multi_chunk && p.tile_n > 128) return QLIN_ERR_UNSUPPORTED;
     p.kb_per_unit = p.spread ? p.kb_per_seg : p.kblocks;
     p.mode = pair ? kModePair : kModeStd;
@@ -259,6 +267,47 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
         p.ticket_bytes = 0;
         p.workspace_bytes = 0;
     }
+    *plan = p;
+    return QLIN_OK;
+}
+
+qlin_status make_moe_plan(int fmt, int variant, int tile_n, int64_t R, int E, int64_t N, int64_t K, int num_sms,
+                          GemmPlan* plan) {
+    if (fmt != QLIN_FMT_INT8 && fmt != QLIN_FMT_FP8) return QLIN_ERR_UNSUPPORTED;
+    if (E < 1 || E > kMoeMaxE) return QLIN_ERR_UNSUPPORTED;
+    qlin_status st = check_fmt_shape(fmt, R, N, K);
+    if (st != QLIN_OK) return st;
+    if ((int64_t)E * N > (int64_t)1 << 31) return QLIN_ERR_UNSUPPORTED;
+    if (num_sms <= 0) num_sms = kNumSMsB200;
+    const int64_t avg = (R + E - 1) / E;  // rows per expert, on average
+    if (variant == QLIN_VAR_AUTO) variant = avg <= 64 ? QLIN_VAR_SWAPAB : QLIN_VAR_PLAIN;
+    if (variant != QLIN_VAR_SWAPAB && variant != QLIN_VAR_PLAIN) return QLIN_ERR_UNSUPPORTED;
+    GemmPlan p;
+    p.fmt = fmt;
+    p.swap = variant == QLIN_VAR_SWAPAB;
+    p.spread = false;
+    p.mode = kModeStd;
+    p.tile_n = tile_n ? tile_n : (p.swap ? (avg <= 16 ? 16 : avg <= 32 ? 32 : 64) : 128);
+    if (!tile_supported(fmt, p.swap, p.tile_n)) return QLIN_ERR_UNSUPPORTED;
+    p.k_segments = 1;
+    p.M = R;
+    p.N = N;
+    p.K = K;
+    p.k_bytes = K;
+    p.kblocks = (int)(K / 128);
+    p.kb_per_seg = p.kblocks;
+    p.kb_per_unit = p.kblocks;
+    if (!gemm_kernel_info(fmt, p.swap, p.tile_n, p.mode, &p.stages, &p.smem_bytes)) return QLIN_ERR_UNSUPPORTED;
+    p.p_rows = p.swap ? (int64_t)E * N : R;
+    p.q_rows = p.swap ? R : (int64_t)E * N;
+    // upper bound on the units the device will count (each expert's last tile may be partial)
+    const int64_t bound = p.swap ? ((N + 127) / 128) * (R / p.tile_n + E) : ((N + p.tile_n - 1) / p.tile_n) * (R / 128 + E);
+    p.p_tiles = 0;
+    p.q_tiles = 0;
+    p.num_tiles = bound;
+    p.units = 0;
+    p.grid = (int)std::max<int64_t>(1, std::min<int64_t>(bound, num_sms));
+    p.moe_E = E;
     *plan = p;
     return QLIN_OK;
 }
@@ -340,6 +389,7 @@ qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int
                            const void* a_q, const float* s_a, const void* w_q, const float* s_w, const void* bias,
                            void* c_out, uint32_t flags, void* workspace, size_t workspace_bytes,
                            qlin_stream_t stream) {
+    if (fmt == QLIN_FMT_BF16) return QLIN_ERR_INVALID_ARG;  // qlin_matmul_bf16
     qlin_status st = check_fmt_shape(fmt, M, N, K);
     if (st != QLIN_OK) return st;
     if (flags & ~(QLIN_OUT_I32ACC | QLIN_PDL | QLIN_SPLITK_CLUSTER)) return QLIN_ERR_INVALID_ARG;
@@ -379,6 +429,7 @@ qlin_status qlin_linear(int fmt, int variant, int tile_n, int k_segments, int64_
                         const void* x, int64_t ld_x, void* a_q, float* s_a, const void* w_q, const float* s_w,
                         const void* bias, void* c_out, uint32_t flags, void* workspace, size_t workspace_bytes,
                         qlin_stream_t stream) {
+    if (fmt == QLIN_FMT_BF16) return QLIN_ERR_INVALID_ARG;  // no quantisation step
     qlin_status st = check_fmt_shape(fmt, M, N, K);
     if (st != QLIN_OK) return st;
     if (flags & ~(QLIN_OUT_I32ACC | QLIN_PDL | QLIN_FUSED)) return QLIN_ERR_INVALID_ARG;
@@ -426,6 +477,173 @@ qlin_status qlin_linear(int fmt, int variant, int tile_n, int k_segments, int64_
     if (e != cudaSuccess) return QLIN_ERR_CUDA;
     GemmOperands ops{a_q, s_a, w_q, s_w, bias, c_out, out_i32, workspace, true};
     return launch_gemm(p, ops, cst);
+}
+
+qlin_status qlin_matmul_bf16(int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K, const void* a,
+                             const void* w, const void* bias, void* c_out, uint32_t flags, void* workspace,
+                             size_t workspace_bytes, qlin_stream_t stream) {
+    const int fmt = QLIN_FMT_BF16;
+    qlin_status st = check_fmt_shape(fmt, M, N, K);
+    if (st != QLIN_OK) return st;
+    if (flags & ~(QLIN_PDL | QLIN_SPLITK_CLUSTER)) return QLIN_ERR_INVALID_ARG;
+    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_PAIR || tile_n < 0 || k_segments < 0)
+        return QLIN_ERR_INVALID_ARG;
+    if (M == 0) return QLIN_OK;
+    if (!a || !w || !c_out) return QLIN_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(w) || !aligned16(c_out) || (reinterpret_cast<uintptr_t>(bias) & 1u))
+        return QLIN_ERR_ALIGNMENT;
+    const int sms = current_device_sms();
+    if (sms <= 0) return QLIN_ERR_NO_DEVICE;
+    GemmPlan p;
+    st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, sms,
+                        (flags & QLIN_SPLITK_CLUSTER) ? kModeCluster : kModeStd, &p);
+    if (st != QLIN_OK) return st;
+    if (p.workspace_bytes) {
+        if (!workspace || workspace_bytes < p.workspace_bytes) return QLIN_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return QLIN_ERR_ALIGNMENT;
+    }
+    if (g_log)
+        std::fprintf(stderr, "[qlin] matmul_bf16 M=%lld N=%lld K=%lld -> %s%s tile_n=%d S=%d grid=%d\n",
+                     (long long)M, (long long)N, (long long)K,
+                     variant_name(p.mode == kModePair ? QLIN_VAR_PAIR
+                                  : p.swap ? (p.spread ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB)
+                                           : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
+                     p.mode == kModeCluster ? " (cluster)" : "", p.tile_n, p.k_segments, p.grid);
+    GemmOperands ops{a, nullptr, w, nullptr, bias, c_out, false, workspace, (flags & QLIN_PDL) != 0};
+    return launch_gemm(p, ops, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------- MoE
+namespace {
+bool moe_dims_ok(int64_t T, int E, int topk) { return T >= 0 && E >= 1 && E <= kMoeMaxE && topk >= 1 && topk <= 32 && topk <= E; }
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+struct MoeLayout {
+    size_t ids, w, rows, offsets, a_q, s_a, g, h_q, s_h, y, total;
+};
+MoeLayout moe_layout(int64_t T, int64_t H, int64_t I, int E, int topk) {
+    const size_t R = (size_t)T * topk;
+    MoeLayout l;
+    size_t o = 0;
+    l.ids = o; o = align256(o + R * 4);
+    l.w = o; o = align256(o + R * 4);
+    l.rows = o; o = align256(o + R * 4);
+    l.offsets = o; o = align256(o + ((size_t)E + 1) * 4);
+    l.a_q = o; o = align256(o + R * (size_t)H);
+    l.s_a = o; o = align256(o + R * 4);
+    l.g = o; o = align256(o + R * 2 * (size_t)I * 2);
+    l.h_q = o; o = align256(o + R * (size_t)I);
+    l.s_h = o; o = align256(o + R * 4);
+    l.y = o; o = align256(o + R * (size_t)H * 2);
+    l.total = o;
+    return l;
+}
+}  // namespace
+
+qlin_status qlin_moe_route(int64_t T, int E, int topk, const float* logits, int32_t* topk_ids, float* topk_w,
+                           int32_t* rows, int32_t* offsets, uint32_t flags, qlin_stream_t stream) {
+    if (!moe_dims_ok(T, E, topk) || (flags & ~QLIN_PDL)) return QLIN_ERR_INVALID_ARG;
+    if (T * topk > (int64_t)1 << 30) return QLIN_ERR_UNSUPPORTED;
+    if (!offsets) return QLIN_ERR_INVALID_ARG;
+    if (current_device_sms() <= 0) return QLIN_ERR_NO_DEVICE;
+    if (T == 0) return cudaMemsetAsync(offsets, 0, ((size_t)E + 1) * 4, static_cast<cudaStream_t>(stream)) == cudaSuccess
+                           ? QLIN_OK : QLIN_ERR_CUDA;
+    if (!logits || !topk_ids || !topk_w || !rows) return QLIN_ERR_INVALID_ARG;
+    return launch_moe_route(logits, (int)T, E, topk, topk_ids, topk_w, offsets, rows, (flags & QLIN_PDL) != 0,
+                            static_cast<cudaStream_t>(stream)) == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
+}
+
+qlin_status qlin_moe_quantize_scatter(int64_t T, int64_t H, int topk, const void* x, const int32_t* rows, void* a_q,
+                                      float* s_a, uint32_t flags, qlin_stream_t stream) {
+    if (T < 0 || H < 16 || topk < 1 || topk > 32 || (flags & ~QLIN_PDL)) return QLIN_ERR_INVALID_ARG;
+    if (H % 16 != 0) return QLIN_ERR_UNSUPPORTED;
+    if (T == 0) return QLIN_OK;
+    if (!x || !rows || !a_q || !s_a) return QLIN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(a_q)) return QLIN_ERR_ALIGNMENT;
+    if (current_device_sms() <= 0) return QLIN_ERR_NO_DEVICE;
+    return launch_moe_quantize_scatter(x, (int)T, (int)H, topk, rows, a_q, s_a, (flags & QLIN_PDL) != 0,
+                                       static_cast<cudaStream_t>(stream)) == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
+}
+
+qlin_status qlin_moe_grouped_mm(int fmt, int variant, int tile_n, int E, int64_t R, int64_t N, int64_t K,
+                                const void* a_q, const float* s_a, const int32_t* offsets, const void* w_q,
+                                const float* s_w, void* c_out, uint32_t flags, qlin_stream_t stream) {
+    if (flags & ~QLIN_PDL) return QLIN_ERR_INVALID_ARG;
+    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_PAIR || tile_n < 0) return QLIN_ERR_INVALID_ARG;
+    if (R < 0 || E < 1) return QLIN_ERR_INVALID_ARG;
+    if (R == 0) return QLIN_OK;
+    if (!a_q || !s_a || !offsets || !w_q || !s_w || !c_out) return QLIN_ERR_INVALID_ARG;
+    if (!aligned16(a_q) || !aligned16(w_q) || !aligned16(c_out)) return QLIN_ERR_ALIGNMENT;
+    const int sms = current_device_sms();
+    if (sms <= 0) return QLIN_ERR_NO_DEVICE;
+    GemmPlan p;
+    qlin_status st = make_moe_plan(fmt, variant, tile_n, R, E, N, K, sms, &p);
+    if (st != QLIN_OK) return st;
+    GemmOperands ops{a_q, s_a, w_q, s_w, nullptr, c_out, false, nullptr, (flags & QLIN_PDL) != 0};
+    ops.moe_offsets = offsets;
+    return launch_gemm(p, ops, static_cast<cudaStream_t>(stream));
+}
+
+qlin_status qlin_moe_act_quantize(int64_t R, int64_t I, const void* g, void* h_q, float* s_h, uint32_t flags,
+                                  qlin_stream_t stream) {
+    if (R < 0 || I < 16 || (flags & ~QLIN_PDL)) return QLIN_ERR_INVALID_ARG;
+    if (I % 16 != 0) return QLIN_ERR_UNSUPPORTED;
+    if (R == 0) return QLIN_OK;
+    if (!g || !h_q || !s_h) return QLIN_ERR_INVALID_ARG;
+    if (!aligned16(h_q) || (reinterpret_cast<uintptr_t>(g) & 3u)) return QLIN_ERR_ALIGNMENT;
+    if (current_device_sms() <= 0) return QLIN_ERR_NO_DEVICE;
+    return launch_moe_act_quantize(g, (int)R, (int)I, h_q, s_h, (flags & QLIN_PDL) != 0,
+                                   static_cast<cudaStream_t>(stream)) == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
+}
+
+qlin_status qlin_moe_combine(int64_t T, int64_t H, int topk, const void* y, const float* topk_w, const int32_t* rows,
+                             void* out, uint32_t flags, qlin_stream_t stream) {
+    if (T < 0 || H < 16 || topk < 1 || topk > 32 || (flags & ~QLIN_PDL)) return QLIN_ERR_INVALID_ARG;
+    if (H % 16 != 0) return QLIN_ERR_UNSUPPORTED;
+    if (T == 0) return QLIN_OK;
+    if (!y || !topk_w || !rows || !out) return QLIN_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(out)) return QLIN_ERR_ALIGNMENT;
+    if (current_device_sms() <= 0) return QLIN_ERR_NO_DEVICE;
+    return launch_moe_combine(y, topk_w, rows, (int)T, (int)H, topk, out, (flags & QLIN_PDL) != 0,
+                              static_cast<cudaStream_t>(stream)) == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
+}
+
+qlin_status qlin_moe_workspace_size(int64_t T, int64_t H, int64_t I, int E, int topk, size_t* bytes_out) {
+    if (!bytes_out || !moe_dims_ok(T, E, topk) || H < 16 || I < 16) return QLIN_ERR_INVALID_ARG;
+    *bytes_out = moe_layout(T, H, I, E, topk).total;
+    return QLIN_OK;
+}
+
+qlin_status qlin_moe_forward(int64_t T, int64_t H, int64_t I, int E, int topk, const void* x, const float* logits,
+                             const void* w1_q, const float* s_w1, const void* w2_q, const float* s_w2, void* out,
+                             uint32_t flags, void* workspace, size_t workspace_bytes, qlin_stream_t stream) {
+    if (!moe_dims_ok(T, E, topk) || (flags & ~QLIN_PDL)) return QLIN_ERR_INVALID_ARG;
+    if (H < 128 || I < 128) return QLIN_ERR_INVALID_ARG;
+    if (H % 128 != 0 || I % 128 != 0) return QLIN_ERR_UNSUPPORTED;
+    if (T == 0) return QLIN_OK;
+    if (!x || !logits || !w1_q || !s_w1 || !w2_q || !s_w2 || !out) return QLIN_ERR_INVALID_ARG;
+    const MoeLayout l = moe_layout(T, H, I, E, topk);
+    if (!workspace || workspace_bytes < l.total) return QLIN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QLIN_ERR_ALIGNMENT;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    auto* ids = reinterpret_cast<int32_t*>(ws + l.ids);
+    auto* w = reinterpret_cast<float*>(ws + l.w);
+    auto* rows = reinterpret_cast<int32_t*>(ws + l.rows);
+    auto* offsets = reinterpret_cast<int32_t*>(ws + l.offsets);
+    auto* s_a = reinterpret_cast<float*>(ws + l.s_a);
+    auto* s_h = reinterpret_cast<float*>(ws + l.s_h);
+    const int64_t R = T * topk;
+    const uint32_t pdl = flags & QLIN_PDL;
+    qlin_status st;
+    if ((st = qlin_moe_route(T, E, topk, logits, ids, w, rows, offsets, pdl, stream)) != QLIN_OK) return st;
+    if ((st = qlin_moe_quantize_scatter(T, H, topk, x, rows, ws + l.a_q, s_a, QLIN_PDL, stream)) != QLIN_OK) return st;
+    if ((st = qlin_moe_grouped_mm(QLIN_FMT_FP8, QLIN_VAR_AUTO, 0, E, R, 2 * I, H, ws + l.a_q, s_a, offsets, w1_q, s_w1,
+                                  ws + l.g, QLIN_PDL, stream)) != QLIN_OK)
+        return st;
+    if ((st = qlin_moe_act_quantize(R, I, ws + l.g, ws + l.h_q, s_h, QLIN_PDL, stream)) != QLIN_OK) return st;
+    if ((st = qlin_moe_grouped_mm(QLIN_FMT_FP8, QLIN_VAR_AUTO, 0, E, R, H, I, ws + l.h_q, s_h, offsets, w2_q, s_w2,
+                                  ws + l.y, QLIN_PDL, stream)) != QLIN_OK)
+        return st;
+    return qlin_moe_combine(T, H, topk, ws + l.y, w, rows, out, QLIN_PDL, stream);
 }
 
 qlin_status qlin_dispatch_query(int fmt, int64_t M, int64_t N, int64_t K, qlin_config* out) {
@@ -476,7 +694,7 @@ qlin_status qlin_dispatch_table_load(const char* path) {
             if (e.fmt < 0 || e.variant < 0 || e.m_max < 1) return QLIN_ERR_TABLE_FORMAT;
             if (check_fmt_shape(e.fmt, 1, e.N, e.K) != QLIN_OK) return QLIN_ERR_TABLE_FORMAT;
             if (!tile_supported(e.fmt, is_swap(e.variant), e.tile_n)) return QLIN_ERR_TABLE_FORMAT;
-            if (e.k_segments < 1 || (e.K / 128) % e.k_segments != 0) return QLIN_ERR_TABLE_FORMAT;
+            if (e.k_segments < 1 || (row_bytes(e.fmt, e.K) / 128) % e.k_segments != 0) return QLIN_ERR_TABLE_FORMAT;
             entries.push_back(e);
         } else {
             return QLIN_ERR_TABLE_FORMAT;

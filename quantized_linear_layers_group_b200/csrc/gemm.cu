@@ -82,16 +82,37 @@ struct GemmArgs {
     int64_t ld_x;
     uint8_t* a_q_out;
     float* s_a_out;
+    // grouped GEMM over experts (MoE): A and C rows are grouped by expert,
+    // expert e's rows [moe_offsets[e], moe_offsets[e+1]) multiply W rows
+    // [e N, e N + N); nullptr / 0 for an ordinary GEMM
+    const int32_t* moe_offsets;
+    int moe_E;
 };
 
+constexpr int kMoeMaxExperts = kMoeMaxE;
+constexpr int kMoeBytes = 2 * (kMoeMaxExperts + 1) * 4;  // expert row offsets and unit prefix sums
+
+// Three warpgroups: warps 0-7 (two warpgroups) run the epilogue; warpgroup 2
+// holds the TMA producer (warp 8), the MMA issuer (warp 9) and two idle warps.
+// After set-up the register file is rebalanced with setmaxnreg: the epilogue
+// warpgroups get kEpiRegs per thread, warpgroup 2 keeps kAuxRegs.  The sum
+// must not exceed the CTA's launch allocation (kThreads x the kernel's
+// register count), or the increase would wait forever; the host refuses to
+// launch a kernel whose register count is below kLaunchRegs.
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kProducerWarp = kEpiWarps;
 constexpr int kMmaWarp = kEpiWarps + 1;
-constexpr int kThreads = (kEpiWarps + 2) * 32;
+constexpr int kThreads = (kEpiWarps + 4) * 32;
+constexpr int kEpiRegs = 216;
+constexpr int kAuxRegs = 72;
+constexpr int kLaunchRegs = (kEpiThreads * kEpiRegs + (kThreads - kEpiThreads) * kAuxRegs + kThreads - 1) / kThreads;
+static_assert(kLaunchRegs <= 168, "register split above what a 384-thread CTA is launched with");
+static_assert(kEpiRegs % 8 == 0 && kAuxRegs % 8 == 0 && kAuxRegs >= 24 && kEpiRegs <= 256, "setmaxnreg values");
 constexpr int kStagingBytes = kEpiWarps * 2048;  // per epilogue warp: one 32x32 bf16 box
 constexpr int kScaleBytes = 2 * 256 * 4;         // column scale + column bias of one tile
-constexpr int kStageBudget = 232448 - 1024 - 256 - kStagingBytes - kScaleBytes;
+constexpr int kBarBytes = 512;                  // mbarriers and the TMEM holder
+constexpr int kStageBudget = 232448 - 1024 - kBarBytes - kStagingBytes - kScaleBytes - 2112;  // 2112: MoE table
 
 __host__ __device__ constexpr int pow2_at_least(int v) {
     int p = 32;
@@ -112,10 +133,13 @@ struct Cfg {
     // rank 0 issues M=256 MMAs that fill both CTAs' accumulators.
     static_assert(!PAIR || (!SWAP && !CSK && !FUSE && BN == 256 && FMT != QLIN_FMT_FP8_BLOCK),
                   "CTA pairs are built for plain 256-column tiles");
+    static_assert(!FUSE || FMT != QLIN_FMT_BF16, "bf16 activations need no quantisation");
     static constexpr int CSK_MAXS = CSK ? cluster_split_max(BN) : 1;  // segments per cluster
     static constexpr int RECV_BYTES = CSK ? (CSK_MAXS - 1) * 128 * BN * 4 : 0;
     static constexpr bool INT8 = (FMT == QLIN_FMT_INT8);
     static constexpr bool BLOCK = (FMT == QLIN_FMT_FP8_BLOCK);
+    static constexpr bool BF16 = (FMT == QLIN_FMT_BF16);  // bf16 operands: no scales
+    static constexpr int KIND = INT8 ? kKindI8 : (BF16 ? kKindF16 : kKindF8);
     static constexpr int BM = 128;                 // P rows per tile (MMA M)
     static constexpr int BK = 128;                 // K bytes per stage: one swizzle atom
     static constexpr int P_BYTES = BM * BK;
@@ -138,21 +162,28 @@ struct Cfg {
     static constexpr int MY_SLICES = (NSLICE + 1) / 2;  // slices per epilogue warp (at most)
     static constexpr int ACC_COLS = BN < 32 ? 32 : BN;
     static constexpr bool MULTI = BN <= 128;       // may run multi-chunk units
-    static constexpr int SEG_COL = 2 * ACC_COLS;   // Block-FP8: running segment sum
+    // TMEM accumulator buffers the MMA fills in turn.  Block-FP8 plain tiles
+    // keep their segment sum in registers and use three: the MMA runs two K
+    // blocks ahead of the promotion.
+    static constexpr int NACC = (BLOCK && !SWAP) ? 3 : 2;
+    static constexpr int SEG_COL = 2 * ACC_COLS;   // Block-FP8 Swap-AB: running segment sum
     static constexpr int TOTAL_COL = (BLOCK ? 3 : 2) * ACC_COLS;  // running total over segments
-    static constexpr int TMEM_COLS =
-        pow2_at_least(2 * ACC_COLS + (MULTI ? ACC_COLS : 0) + (BLOCK ? ACC_COLS : 0));
-    static constexpr uint32_t IDESC = make_idesc(INT8, PAIR ? 256 : 128, BN);
+    static constexpr int TMEM_COLS = pow2_at_least(NACC * ACC_COLS + (MULTI ? ACC_COLS : 0) +
+                                                   ((BLOCK && SWAP) ? ACC_COLS : 0));
+    static_assert(NACC * ACC_COLS <= TOTAL_COL, "accumulators overlap the running total");
+    static constexpr uint32_t IDESC = make_idesc(KIND, PAIR ? 256 : 128, BN);
     static constexpr size_t STAGING_OFF = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t SCALE_OFF = STAGING_OFF + kStagingBytes;
     static constexpr size_t BSCALE_OFF = SCALE_OFF + kScaleBytes;
     static constexpr size_t RECV_OFF = BSCALE_OFF + BSCALE_BYTES;
     static constexpr size_t A_OFF = RECV_OFF + RECV_BYTES;
     static constexpr size_t SA_OFF = A_OFF + A_BYTES;
-    static constexpr size_t BAR_OFF = SA_OFF + SA_BYTES;
-    static constexpr size_t SMEM = 1024 + BAR_OFF + 256;
-    // barriers: full/empty per stage, tfull/tempty x2, recv_full/free, a_full/empty; then the TMEM holder
-    static_assert((2 * STAGES + 8) * 8 + 8 <= 256, "barrier area");
+    static constexpr size_t MOE_OFF = SA_OFF + SA_BYTES;
+    static constexpr size_t BAR_OFF = MOE_OFF + ((kMoeBytes + 63) / 64) * 64;
+    static constexpr size_t SMEM = 1024 + BAR_OFF + kBarBytes;
+    // barriers: full/empty per stage, tfull/tempty per accumulator buffer,
+    // recv_full/free, a_full/empty; then the TMEM holder and a broadcast word
+    static_assert((2 * STAGES + 2 * NACC + 4) * 8 + 8 <= kBarBytes, "barrier area");
     static_assert(!FUSE || A_MAXKB <= BS_KB, "scale window");
     static_assert(TMEM_COLS <= 512, "TMEM overflow");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
@@ -161,12 +192,39 @@ struct Cfg {
 
 struct Unit {
     int tile, seg, pt, qt, kb0, kb1, chunk_kb;
+    // rows of A / C this unit's tile indexes from (row0 ..), how many exist
+    // (rows), and the first W row (wrow0): 0, M, 0 for an ordinary GEMM,
+    // the expert's group and weight slice for MoE
+    int row0, rows, wrow0;
 };
 
+// MoE: unit u lies in the expert e with pref[e] <= u < pref[e + 1] (pref =
+// prefix sums of the experts' tile counts); within it, tiles go P-side first.
+template <bool SWAP, int BN>
+__device__ __forceinline__ void decode_moe(const GemmArgs& a, int u, const int32_t* tab, Unit& r) {
+    const int32_t* off = tab;
+    const int32_t* pref = tab + kMoeMaxExperts + 1;
+    int lo = 0, hi = a.moe_E - 1;  // largest e with pref[e] <= u
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pref[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo, local = u - pref[e];
+    r.row0 = off[e];
+    r.rows = off[e + 1] - off[e];
+    r.wrow0 = e * a.N;
+    const int p_tiles = SWAP ? (a.N + 127) / 128 : (r.rows + 127) / 128;
+    r.pt = local % p_tiles;
+    r.qt = local / p_tiles;
+}
+
 // Pair tiles (PAIR): unit = 256-row tile; pt is this CTA's 128-row half of it.
-template <int FMT, bool PAIR = false>
-__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int rank = 0) {
+template <int FMT, bool PAIR = false, bool SWAP = false, int BN = 128>
+__device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int rank = 0, const int32_t* moe_tab = nullptr) {
     Unit r;
+    r.row0 = 0;
+    r.rows = a.M;
+    r.wrow0 = 0;
     if (a.spread) {
         r.seg = u % a.S;
         r.tile = u / a.S;
@@ -183,8 +241,12 @@ __device__ __forceinline__ Unit decode_unit(const GemmArgs& a, int u, int rank =
         r.pt = 2 * (r.tile % pairs) + rank;
         r.qt = r.tile / pairs;
     } else {
-        r.pt = r.tile % a.p_tiles;
-        r.qt = r.tile / a.p_tiles;
+        if (moe_tab != nullptr) {
+            decode_moe<SWAP, BN>(a, u, moe_tab, r);
+        } else {
+            r.pt = r.tile % a.p_tiles;
+            r.qt = r.tile / a.p_tiles;
+        }
     }
     if (FMT == QLIN_FMT_FP8_BLOCK)
         r.chunk_kb = 1;
@@ -226,6 +288,15 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
     int ok = 1;
     if ((threadIdx.x & 31) == 0) ok = mbar_wait_idle(bar, parity) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Next TMEM accumulator buffer (NACC in turn); the parity flips per round.
+template <int NACC>
+__device__ __forceinline__ void next_acc(uint32_t& abuf, uint32_t& aphase) {
+    if (++abuf == NACC) {
+        abuf = 0;
+        aphase ^= 1;
+    }
 }
 
 __device__ __forceinline__ void warp_arrive(uint32_t bar) {
@@ -295,7 +366,7 @@ __device__ __forceinline__ void finish_slice(const GemmArgs& a, const Unit& un, 
     for (int c4 = 0; c4 < SW; c4 += 4) {
         float4 sc = make_float4(0.f, 0.f, 0.f, 0.f), bc = make_float4(0.f, 0.f, 0.f, 0.f);
         if constexpr (!C::BLOCK) {
-            sc = lds_f4(e.s_col + (uint32_t)(j * SW + c4) * 4u);
+            if constexpr (!C::BF16) sc = lds_f4(e.s_col + (uint32_t)(j * SW + c4) * 4u);
             if (!SWAP && e.has_bias) bc = lds_f4(e.b_col + (uint32_t)(j * SW + c4) * 4u);
         }
         const float scv[4] = {sc.x, sc.y, sc.z, sc.w};
@@ -308,7 +379,9 @@ __device__ __forceinline__ void finish_slice(const GemmArgs& a, const Unit& un, 
                 t = __int2float_rn((int)v[c]);
             else
                 t = __uint_as_float(v[c]);
-            if constexpr (!C::BLOCK) {
+            if constexpr (C::BF16) {
+                if (e.has_bias) t = __fadd_rn(t, SWAP ? e.row_bias : bcv[i]);  // + bias[n]
+            } else if constexpr (!C::BLOCK) {
                 if constexpr (!SWAP) {
                     t = __fmul_rn(t, e.row_scale);  // * s_a[m]
                     t = __fmul_rn(t, scv[i]);       // * s_w[n]
@@ -330,7 +403,8 @@ __device__ __forceinline__ void finish_slice(const GemmArgs& a, const Unit& un, 
         if (n < a.N) {
 #pragma unroll
             for (int c = 0; c < SW; ++c)
-                if (m0 + c < a.M) cb[(size_t)(m0 + c) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y[c]));
+                if (m0 + c < un.rows)
+                    cb[(size_t)(un.row0 + m0 + c) * a.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y[c]));
         }
     } else {
         // The warp's 32 x 32 box of C goes to shared memory row by row (lane =
@@ -339,11 +413,23 @@ __device__ __forceinline__ void finish_slice(const GemmArgs& a, const Unit& un, 
         // which also leaves out the rows and columns past the edges of C.
         const int bx = un.qt * BN + j * SW;
         const int by = un.pt * 128 + e.quad * 32;
-        if (bx >= a.N || by >= a.M) return;  // warp-uniform: the whole box is outside C
-        (void)cb;
+        if (bx >= a.N || by >= un.rows) return;  // warp-uniform: the whole box is outside C
         uint32_t packed[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) packed[c / 2] = pack_bf16x2(y[c], y[c + 1]);
+        if (a.moe_E > 0) {
+            // MoE: the box may reach into the next expert's rows, so each
+            // thread stores its own row, 16 bytes at a time (N % 16 == 0)
+            const int m = by + e.lane;
+            if (m < un.rows) {
+                uint4* dst = reinterpret_cast<uint4*>(cb + (size_t)(un.row0 + m) * a.N + bx);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (bx + 8 * q < a.N)
+                        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+            }
+            return;
+        }
         if (e.lane == 0) bulk_wait_read_all();  // the previous box has left the buffer
         __syncwarp();
 #pragma unroll
@@ -744,6 +830,52 @@ __device__ __forceinline__ void fused_quantize_unit(const GemmArgs& a, const Uni
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Block-FP8: stage the scale products s_a[m,kb] * s_w[n/128,kb] of a window of
+// up to BS_KB K blocks from win0 into shared memory, [kb][row] (plain tiles) or
+// [kb][column] (Swap-AB), by coalesced cooperative loads of the 256 epilogue
+// threads (which all call it).  Fused mode reads s_a from the unit's own
+// scales (sa_cur).
+template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE, bool PAIR>
+__device__ __forceinline__ void stage_block_scales(const GemmArgs& args, const Unit& un, int win0, uint32_t bsc,
+                                                   const float* sa_cur) {
+    using C = Cfg<FMT, SWAP, BN, CSK, FUSE, PAIR>;
+    const int kbc = min(C::BS_KB, un.kb1 - win0);
+    constexpr int NIDX = SWAP ? BN : 128;
+    const int nb = SWAP ? un.pt : ((un.qt * BN) >> 7);
+    const int mbase = SWAP ? un.qt * BN : un.pt * 128;
+    named_bar_sync(1, kEpiThreads);  // the previous window is no longer read
+    constexpr int BATCH = 24;        // loads in flight per thread: a 128 x 48 window in one round trip
+    for (int i0 = threadIdx.x; i0 < NIDX * kbc; i0 += kEpiThreads * BATCH) {
+        float va[BATCH], vw[BATCH];
+        int off[BATCH];
+#pragma unroll
+        for (int b = 0; b < BATCH; ++b) {
+            const int i = i0 + b * kEpiThreads;
+            const int idx = i / kbc, kbl = i - idx * kbc;
+            const int m = mbase + idx, kb = win0 + kbl;
+            off[b] = -1;
+            va[b] = 0.f;
+            vw[b] = 0.f;
+            if (i < NIDX * kbc) {
+                off[b] = kbl * C::BS_PITCH + idx;
+                if (m < args.M) {
+                    if constexpr (FUSE)
+                        va[b] = sa_cur[idx * C::A_MAXKB + (kb - un.kb0)];
+                    else
+                        va[b] = __ldg(args.s_a + (size_t)m * args.kblocks + kb);
+                    vw[b] = __ldg(args.s_w + (size_t)nb * args.kblocks + kb);
+                }
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < BATCH; ++b)
+            if (off[b] >= 0)
+                asm volatile("st.shared.f32 [%0], %1;" ::"r"(bsc + (uint32_t)off[b] * 4u), "f"(__fmul_rn(va[b], vw[b]))
+                             : "memory");
+    }
+    named_bar_sync(1, kEpiThreads);
+}
+
 template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     qlin_gemm_kernel(const __grid_constant__ CUtensorMap tmap_p, const __grid_constant__ CUtensorMap tmap_q,
@@ -761,13 +893,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
     const uint32_t full0 = smem_u32(bars);
     const uint32_t empty0 = smem_u32(bars + STAGES);
+    constexpr int NACC = C::NACC;
+    uint64_t* bars_x = bars + 2 * STAGES + 2 * NACC;
     const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
-    const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
-    const uint32_t recv_full = smem_u32(bars + 2 * STAGES + 4);  // cluster Split-K, rank 0
-    const uint32_t recv_free = smem_u32(bars + 2 * STAGES + 5);  // cluster Split-K, ranks > 0
-    const uint32_t a_full = smem_u32(bars + 2 * STAGES + 6);     // fused: unit's A codes written
-    const uint32_t a_empty = smem_u32(bars + 2 * STAGES + 7);    // fused: MMA done with them
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 8);
+    const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + NACC);
+    const uint32_t recv_full = smem_u32(bars_x + 0);  // cluster Split-K, rank 0
+    const uint32_t recv_free = smem_u32(bars_x + 1);  // cluster Split-K, ranks > 0
+    const uint32_t a_full = smem_u32(bars_x + 2);     // fused: unit's A codes written
+    const uint32_t a_empty = smem_u32(bars_x + 3);    // fused: MMA done with them
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars_x + 4);
+    int32_t* moe_tab = reinterpret_cast<int32_t*>(smem + C::MOE_OFF);  // offsets [E+1], then unit prefixes
     const uint32_t sA = smem_u32(smem + C::A_OFF);
     float* sa_tile = reinterpret_cast<float*>(smem + C::SA_OFF);
     uint32_t* rmax = reinterpret_cast<uint32_t*>(sa_tile + 2 * C::SA_FLOATS);  // fused per-token row maxima
@@ -789,7 +924,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(full0 + 8 * s, 1);
             mbar_init(empty0 + 8 * s, 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < NACC; ++b) {
             mbar_init(tfull0 + 8 * b, 1);
             // one arrival per epilogue warp (PAIR: of both CTAs, on rank 0's barrier)
             mbar_init(tempty0 + 8 * b, PAIR ? 2 * kEpiWarps : kEpiWarps);
@@ -813,15 +948,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_relinquish();
         }
     }
+    if (args.moe_E > 0 && warp == kEpiWarps + 2) {
+        // MoE: the expert row offsets come from the previous kernel (routing);
+        // wait for it, then the experts' tile counts and their prefix sums
+        pdl_wait();
+        int32_t* off = moe_tab;
+        int32_t* pref = moe_tab + kMoeMaxExperts + 1;
+        const int E = args.moe_E;
+        const int per = (E + 32) / 32;  // experts per lane (E + 1 offsets)
+        int32_t sum = 0;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e <= E) off[e] = args.moe_offsets[e];
+        }
+        __syncwarp();
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) {
+                const int rows = off[e + 1] - off[e];
+                const int p_tiles = SWAP ? (args.N + 127) / 128 : (rows + 127) / 128;
+                const int q_tiles = SWAP ? (rows + BN - 1) / BN : (args.N + BN - 1) / BN;
+                sum += rows > 0 ? p_tiles * q_tiles : 0;
+            }
+        }
+        int32_t incl = sum;  // inclusive scan of the lanes' sums
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int32_t run = incl - sum;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) {
+                pref[e] = run;
+                const int rows = off[e + 1] - off[e];
+                const int p_tiles = SWAP ? (args.N + 127) / 128 : (rows + 127) / 128;
+                const int q_tiles = SWAP ? (rows + BN - 1) / BN : (args.N + BN - 1) / BN;
+                run += rows > 0 ? p_tiles * q_tiles : 0;
+            }
+        }
+        if (lane == 31) pref[E] = incl;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    const int32_t* moe = args.moe_E > 0 ? moe_tab : nullptr;
+    const int units = moe ? moe_tab[kMoeMaxExperts + 1 + args.moe_E] : args.units;
     // every rank's barriers are initialised before any remote arrive or load signal
     if constexpr (CSK || PAIR) cluster_sync();
     const uint32_t tmem_base = *tmem_holder;
     pdl_launch_dependents();
 
+    // Each role rebalances its registers first thing in its own branch (the
+    // compiler applies a warp's register limit to the code that setmaxnreg
+    // dominates, so no role's code may follow a merge of the two limits).
     if (warp == kProducerWarp) {
+        regs_decrease<kAuxRegs>();
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t pol_w = policy_evict_first();
@@ -843,16 +1026,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             auto load_w = [&](uint32_t stage, const Unit& un, int kb, uint32_t fb) {
                 if constexpr (SWAP)
-                    load(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_w, kb * 128, un.pt * 128, fb, pol_w);
-                else
-                    load(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_w, kb * 128, un.qt * BN + w_row_off, fb,
+                    load(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_w, kb * 128, un.wrow0 + un.pt * 128, fb,
                          pol_w);
+                else
+                    load(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_w, kb * 128,
+                         un.wrow0 + un.qt * BN + w_row_off, fb, pol_w);
             };
             // weights do not depend on the previous kernel: start streaming the
             // first unit's weight tiles before waiting for it
             int pre = 0;
-            if (u_first < args.units) {
-                const Unit un = decode_unit<FMT, PAIR>(args, u_first, rank);
+            if (u_first < units) {
+                const Unit un = decode_unit<FMT, PAIR, SWAP, BN>(args, u_first, rank, moe);
                 for (int kb = un.kb0; kb < un.kb1 && pre < STAGES; ++kb, ++pre) {
                     arm(full0 + 8 * pre);
                     load_w(pre, un, kb, full0 + 8 * pre);
@@ -861,8 +1045,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             pdl_wait();
             uint32_t stage = 0, phase = 0;
             int it = 0;
-            for (int u = u_first; u < args.units; u += u_step) {
-                const Unit un = decode_unit<FMT, PAIR>(args, u, rank);
+            for (int u = u_first; u < units; u += u_step) {
+                const Unit un = decode_unit<FMT, PAIR, SWAP, BN>(args, u, rank, moe);
                 for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
                     const uint32_t fb = full0 + 8 * stage;
                     if (it >= pre) {
@@ -875,9 +1059,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (FUSE)
                         (void)pol_a;  // the activation operand is quantised in place
                     else if constexpr (SWAP)
-                        load(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_a, kb * 128, un.qt * BN, fb, pol_a);
+                        load(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_a, kb * 128, un.row0 + un.qt * BN, fb,
+                             pol_a);
                     else
-                        load(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_a, kb * 128, un.pt * 128, fb, pol_a);
+                        load(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_a, kb * 128, un.row0 + un.pt * 128, fb,
+                             pol_a);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
@@ -886,12 +1072,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == kMmaWarp) {
+        regs_decrease<kAuxRegs>();
         // -------------------------------------------------------- MMA issuer
         // (PAIR: rank 0 issues for both CTAs; rank 1's MMA warp only holds TMEM)
         if (lane == 0 && (!PAIR || rank == 0)) {
             uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0, uphase = 0;
-            for (int u = u_first; u < args.units; u += u_step) {
-                const Unit un = decode_unit<FMT, PAIR>(args, u, rank);
+            for (int u = u_first; u < units; u += u_step) {
+                const Unit un = decode_unit<FMT, PAIR, SWAP, BN>(args, u, rank, moe);
                 if constexpr (FUSE) {
                     if (!mbar_wait(a_full, uphase)) goto done;
                     tc_fence_after();
@@ -915,9 +1102,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int k = 0; k < 4; ++k) {  // 4 x K=32 bytes per 128-byte stage
                             const uint32_t accum = (kb > c0 || k > 0) ? 1u : 0u;
                             if constexpr (PAIR)
-                                tc_mma_pair<C::INT8>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
+                                tc_mma_pair<C::KIND>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
                             else
-                                tc_mma<C::INT8>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
+                                tc_mma<C::KIND>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
                         }
                         if constexpr (PAIR)
                             tc_commit_pair(empty0 + 8 * stage, 0x3);  // both CTAs may refill the stage
@@ -932,8 +1119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_commit_pair(tfull0 + 8 * abuf, 0x3);  // both CTAs' accumulators are ready
                     else
                         tc_commit(tfull0 + 8 * abuf);
-                    abuf ^= 1;
-                    if (abuf == 0) aphase ^= 1;
+                    next_acc<NACC>(abuf, aphase);
                 }
                 if constexpr (FUSE) {
                     tc_commit(a_empty);  // arrives once every MMA of the unit has read sA
@@ -941,7 +1127,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else {
+    } else if (warp < kEpiWarps) {
+        regs_increase<kEpiRegs>();
         // ---------------------------------------------------------- epilogue
         pdl_wait();  // scales are written by the previous kernel; C may be read by it
         EpiCtx e;
@@ -989,15 +1176,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         if constexpr (FUSE) {
-            if (u_first < args.units) {
+            if (u_first < units) {
                 fused_quantize_unit<FMT, BN, C::A_MAXKB>(args, decode_unit<FMT>(args, u_first), sA, sa_tile,
                                                          rmax, xstage, kStagingBytes);
                 warp_arrive(a_full);
             }
         }
         int ui = 0;  // this CTA's unit count so far (fused: scale buffer ui % 2)
-        for (int u = u_first; u < args.units; u += u_step, ++ui) {
-            const Unit un = decode_unit<FMT, PAIR>(args, u, rank);
+        for (int u = u_first; u < units; u += u_step, ++ui) {
+            const Unit un = decode_unit<FMT, PAIR, SWAP, BN>(args, u, rank, moe);
             const float* sa_cur = sa_tile + (ui & 1) * C::SA_FLOATS;
             // Fused: the next unit's rows are quantised once the MMA is done
             // with this unit's.  A unit whose MMAs fill one accumulator is
@@ -1006,7 +1193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // several accumulator chunks needs this epilogue to drain them
             // first, so its successor waits until after it.
             const int nxt = u + u_step;
-            const bool quantise_next = FUSE && nxt < args.units;
+            const bool quantise_next = FUSE && nxt < units;
             const bool next_first = (un.kb1 - un.kb0) == un.chunk_kb;
             if (quantise_next && next_first) {
                 if (!warp_wait(a_empty, (uint32_t)(ui & 1))) goto done;
@@ -1021,20 +1208,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = threadIdx.x; c < BN; c += kEpiThreads) {
                     const int q = un.qt * BN + c;
                     if constexpr (!SWAP) {
-                        s_col[c] = q < args.N ? __ldg(args.s_w + q) : 0.f;
+                        if constexpr (!C::BF16) s_col[c] = q < args.N ? __ldg(args.s_w + un.wrow0 + q) : 0.f;
                         b_col[c] = (e.has_bias && q < args.N) ? bf16_to_f32(__ldg(args.bias + q)) : 0.f;
                     } else if constexpr (FUSE) {
                         s_col[c] = sa_cur[c];
-                    } else {
-                        s_col[c] = q < args.M ? __ldg(args.s_a + q) : 0.f;
+                    } else if constexpr (!C::BF16) {
+                        s_col[c] = q < un.rows ? __ldg(args.s_a + un.row0 + q) : 0.f;
                     }
                 }
                 if constexpr (!SWAP) {
                     const int m = un.pt * 128 + e.row_lane;
-                    e.row_scale = m < args.M ? __ldg(args.s_a + m) : 0.f;
+                    if constexpr (!C::BF16) e.row_scale = m < un.rows ? __ldg(args.s_a + un.row0 + m) : 0.f;
                 } else {
                     const int n = un.pt * 128 + e.row_lane;
-                    e.row_scale = n < args.N ? __ldg(args.s_w + n) : 0.f;
+                    if constexpr (!C::BF16) e.row_scale = n < args.N ? __ldg(args.s_w + un.wrow0 + n) : 0.f;
                     e.row_bias = (e.has_bias && n < args.N) ? bf16_to_f32(__ldg(args.bias + n)) : 0.f;
                 }
                 named_bar_sync(1, kEpiThreads);
@@ -1060,15 +1247,95 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (!consume_segment_slice<FMT, SWAP, BN, CSK>(args, un, un.seg, j, t_total, e, v)) goto done;
                 }
-                abuf ^= 1;
-                if (abuf == 0) aphase ^= 1;
+                next_acc<NACC>(abuf, aphase);
             } else if constexpr (C::MULTI) {
-                if constexpr (C::BLOCK) {
-                    // Block-FP8: promote every 128-wide K block into the fp32
-                    // segment sum: seg = fma(P_kb, s_a[m,kb] * s_w[n/128,kb], seg)
-                    // The products s_a[m,kb] * s_w[n/128,kb] of a window of up to
-                    // BS_KB K blocks are staged in shared memory, [kb][row] (plain)
-                    // or [kb][column] (Swap-AB), by coalesced cooperative loads.
+                if constexpr (C::BLOCK && !SWAP) {
+                    // Block-FP8, plain tiles: one 128-wide K block per
+                    // accumulator.  Each thread loads its row's 64 columns of
+                    // the K block's products P_kb (slices 2h and 2h+1 for slice
+                    // parity h), hands the buffer straight back (the MMA runs
+                    // ahead into the other buffers), and promotes them into the
+                    // segment sum it keeps in registers,
+                    //   seg = fma(P_kb, s_a[m,kb] * s_w[n/128,kb], seg)  from +0,
+                    // two lanes per instruction.  The tile's 128 columns lie in
+                    // one 128-block of N, so the scale product is one value per
+                    // row and K block, read from the staged table.
+                    static_assert(C::NSLICE == 4 && SW == 32, "128-column tiles");
+                    const uint32_t bsc = smem_u32(smem + C::BSCALE_OFF);
+                    const int kbps = args.kb_per_seg;
+                    int win0 = -C::BS_KB;
+                    int kin = 0;                          // K block within the segment
+                    int seg_no = args.spread ? un.seg : 0;
+                    float sg[2 * SW];                     // the segment sum of this thread's 64 columns
+                    for (int c0 = un.kb0; c0 < un.kb1; ++c0) {
+                        const bool seg_start = kin == 0;
+                        if (c0 - win0 >= C::BS_KB) {
+                            win0 = c0;
+                            stage_block_scales<FMT, SWAP, BN, CSK, FUSE, PAIR>(args, un, win0, bsc, nullptr);
+                        }
+                        float row_scale;
+                        asm volatile("ld.shared.f32 %0, [%1];"
+                                     : "=f"(row_scale)
+                                     : "r"(bsc + (uint32_t)((c0 - win0) * C::BS_PITCH + e.row_lane) * 4u));
+                        if (!acc_wait(tfull0 + 8 * abuf, aphase)) goto done;
+                        tc_fence_after();
+                        uint32_t v[2 * SW];
+                        tmem_ld64(t_lane + abuf * C::ACC_COLS + e.half * 2 * SW, v);
+                        tc_wait_ld();
+                        tc_fence_before();
+                        acc_release(tempty0 + 8 * abuf);
+                        next_acc<NACC>(abuf, aphase);
+                        if (seg_start) {
+#pragma unroll
+                            for (int c = 0; c < 2 * SW; c += 2)
+                                fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]), row_scale,
+                                        0.f, 0.f);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 2 * SW; c += 2)
+                                fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]), row_scale,
+                                        sg[c], sg[c + 1]);
+                        }
+                        if (++kin < kbps) continue;
+                        kin = 0;
+                        // segment end: Split-K writes the segment out; otherwise
+                        // total = total + seg in segment order from +0 (the total
+                        // lives in TMEM between segments), and the last segment
+                        // finishes the tile
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const int j = 2 * e.half + i;
+                            uint32_t out[SW];
+                            if (args.spread) {
+#pragma unroll
+                                for (int c = 0; c < SW; ++c) out[c] = __float_as_uint(sg[i * SW + c]);
+                                store_partial<SW>(partial_ptr<SW>(args, un.tile, un.seg, j, C::NSLICE, e.row_lane), out);
+                                continue;
+                            }
+                            if (seg_no == 0) {
+#pragma unroll
+                                for (int c = 0; c < SW; ++c) out[c] = __float_as_uint(__fadd_rn(0.f, sg[i * SW + c]));
+                            } else {
+                                tmem_load_slice<SW>(t_total + j * SW, out);
+                                tc_wait_ld();
+#pragma unroll
+                                for (int c = 0; c < SW; ++c)
+                                    out[c] = __float_as_uint(__fadd_rn(__uint_as_float(out[c]), sg[i * SW + c]));
+                            }
+                            if (seg_no == args.S - 1)
+                                finish_slice<FMT, SWAP, BN>(args, un, j, e, out);
+                            else
+                                tmem_store_slice<SW>(t_total + j * SW, out);
+                        }
+                        tc_wait_st();  // the running total is read again at the next segment end
+                        ++seg_no;
+                    }
+                } else if constexpr (C::BLOCK) {
+                    // Block-FP8, Swap-AB tiles: promote every 128-wide K block
+                    // into the fp32 segment sum kept in TMEM,
+                    // seg = fma(P_kb, s_a[m,kb] * s_w[n/128,kb], seg); the scale
+                    // product is one value per column m (the tile's 128 lanes
+                    // lie in one 128-block of N), read from the staged table.
                     const uint32_t bsc = smem_u32(smem + C::BSCALE_OFF);
                     int win0 = -C::BS_KB;
                     for (int c0 = un.kb0; c0 < un.kb1; ++c0) {
@@ -1078,47 +1345,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const bool seg_end = ((rel + 1) % args.kb_per_seg) == 0;
                         if (c0 - win0 >= C::BS_KB) {
                             win0 = c0;
-                            const int kbc = min(C::BS_KB, un.kb1 - win0);
-                            constexpr int NIDX = SWAP ? BN : 128;
-                            const int nb = SWAP ? un.pt : ((un.qt * BN) >> 7);
-                            const int mbase = SWAP ? un.qt * BN : un.pt * 128;
-                            named_bar_sync(1, kEpiThreads);  // the previous window is no longer read
-                            constexpr int BATCH = 8;             // loads in flight per thread
-                            for (int i0 = threadIdx.x; i0 < NIDX * kbc; i0 += kEpiThreads * BATCH) {
-                                float va[BATCH], vw[BATCH];
-                                int off[BATCH];
-#pragma unroll
-                                for (int b = 0; b < BATCH; ++b) {
-                                    const int i = i0 + b * kEpiThreads;
-                                    const int idx = i / kbc, kbl = i - idx * kbc;
-                                    const int m = mbase + idx, kb = win0 + kbl;
-                                    off[b] = -1;
-                                    va[b] = 0.f;
-                                    vw[b] = 0.f;
-                                    if (i < NIDX * kbc) {
-                                        off[b] = kbl * C::BS_PITCH + idx;
-                                        if (m < args.M) {
-                                            if constexpr (FUSE)
-                                                va[b] = sa_cur[idx * C::A_MAXKB + (kb - un.kb0)];
-                                            else
-                                                va[b] = __ldg(args.s_a + (size_t)m * args.kblocks + kb);
-                                            vw[b] = __ldg(args.s_w + (size_t)nb * args.kblocks + kb);
-                                        }
-                                    }
-                                }
-#pragma unroll
-                                for (int b = 0; b < BATCH; ++b)
-                                    if (off[b] >= 0)
-                                        asm volatile("st.shared.f32 [%0], %1;" ::"r"(bsc + (uint32_t)off[b] * 4u),
-                                                     "f"(__fmul_rn(va[b], vw[b]))
-                                                     : "memory");
-                            }
-                            named_bar_sync(1, kEpiThreads);
+                            stage_block_scales<FMT, SWAP, BN, CSK, FUSE, PAIR>(args, un, win0, bsc, sa_cur);
                         }
                         const uint32_t bsrow = bsc + (uint32_t)((c0 - win0) * C::BS_PITCH) * 4u;
-                        float row_scale = 0.f;
-                        if constexpr (!SWAP)
-                            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(row_scale) : "r"(bsrow + e.row_lane * 4u));
                         if (!acc_wait(tfull0 + 8 * abuf, aphase)) goto done;
                         tc_fence_after();
                         const uint32_t tacc = t_lane + abuf * C::ACC_COLS;
@@ -1132,14 +1361,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_wait_ld();
 #pragma unroll
                             for (int c = 0; c < SW; ++c) {
-                                float sc;
-                                if constexpr (!SWAP) {
-                                    sc = row_scale;
-                                } else {  // column scale, same address for the whole warp
-                                    asm volatile("ld.shared.f32 %0, [%1];"
-                                                 : "=f"(sc)
-                                                 : "r"(bsrow + (uint32_t)(j * SW + c) * 4u));
-                                }
+                                float sc;  // column scale, same address for the whole warp
+                                asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sc) : "r"(bsrow + (uint32_t)(j * SW + c) * 4u));
                                 const float prev = seg_start ? 0.f : __uint_as_float(sg[c]);
                                 sg[c] = __float_as_uint(__fmaf_rn(__uint_as_float(v[c]), sc, prev));
                             }
@@ -1153,8 +1376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_wait_st();
                         tc_fence_before();
                         acc_release(tempty0 + 8 * abuf);
-                        abuf ^= 1;
-                        if (abuf == 0) aphase ^= 1;
+                        next_acc<NACC>(abuf, aphase);
                     }
                 } else {
                     // FP8 per-token, plain variant with S > 1: one chunk per
@@ -1175,8 +1397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_wait_st();
                         tc_fence_before();
                         acc_release(tempty0 + 8 * abuf);
-                        abuf ^= 1;
-                        if (abuf == 0) aphase ^= 1;
+                        next_acc<NACC>(abuf, aphase);
                     }
                 }
             }
@@ -1207,6 +1428,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 warp_arrive(a_full);
             }
         }
+    } else {
+        regs_decrease<kAuxRegs>();  // warps 10 and 11: idle members of warpgroup 2
     }
 done:
     // the bulk stores of C have completed (and left the staging buffers)
@@ -1242,8 +1465,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// K-major 8-bit operand [rows, K] as a 2-D tensor map with a (128 B x box_rows)
-// box, 128-byte swizzle (the layout the MMA descriptors describe).
+// K-major operand [rows, K] (8-bit or bf16 elements) as a 2-D tensor map over
+// its bytes, K_bytes per row, with a (128 B x box_rows) box and the 128-byte
+// swizzle (the layout the MMA descriptors describe).
 bool make_operand_tmap(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -1285,6 +1509,10 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     if (configured_device != dev) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM) != cudaSuccess)
             return QLIN_ERR_CUDA;
+        // the in-kernel register split must fit the launch allocation
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return QLIN_ERR_CUDA;
+        if (fa.numRegs < kLaunchRegs) return QLIN_ERR_UNSUPPORTED;
         for (int& m : max_clusters) m = -1;
         configured_device = dev;
     }
@@ -1292,10 +1520,10 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     alignas(64) CUtensorMap tp, tq;
     const void* p_base = SWAP ? ops.w_q : ops.a_q;
     const void* q_base = SWAP ? ops.a_q : ops.w_q;
-    if (!make_operand_tmap(&tp, p_base, plan.p_rows, plan.K, 128)) return QLIN_ERR_CUDA;
+    if (!make_operand_tmap(&tp, p_base, plan.p_rows, plan.k_bytes, 128)) return QLIN_ERR_CUDA;
     if (FUSE)
         tq = tp;  // unused: the kernel quantises its activation operand in place
-    else if (!make_operand_tmap(&tq, q_base, plan.q_rows, plan.K, PAIR ? BN / 2 : BN))  // PAIR: half a W tile
+    else if (!make_operand_tmap(&tq, q_base, plan.q_rows, plan.k_bytes, PAIR ? BN / 2 : BN))  // PAIR: half a W tile
         return QLIN_ERR_CUDA;
     alignas(64) CUtensorMap tc;  // plain tiles: bf16 C in 32 x 32 boxes
     if (!SWAP && !ops.out_i32) {
@@ -1326,6 +1554,8 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     a.ld_x = FUSE ? ops.ld_x : 0;
     a.a_q_out = FUSE ? static_cast<uint8_t*>(const_cast<void*>(ops.a_q)) : nullptr;
     a.s_a_out = FUSE ? const_cast<float*>(ops.s_a) : nullptr;
+    a.moe_offsets = ops.moe_offsets;
+    a.moe_E = plan.moe_E;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)plan.grid);
@@ -1382,9 +1612,13 @@ bool dispatch_instance(bool swap, int tile_n, int mode, A&&... args) {
             case kModeCluster * 1000 + 16: OP<FMT, true, 16, true, false, false>::run(args...); return true;
             case kModeCluster * 1000 + 32: OP<FMT, true, 32, true, false, false>::run(args...); return true;
             case kModeCluster * 1000 + 64: OP<FMT, true, 64, true, false, false>::run(args...); return true;
-            case kModeFused * 1000 + 16: OP<FMT, true, 16, false, true, false>::run(args...); return true;
-            case kModeFused * 1000 + 32: OP<FMT, true, 32, false, true, false>::run(args...); return true;
-            case kModeFused * 1000 + 64: OP<FMT, true, 64, false, true, false>::run(args...); return true;
+        }
+        if constexpr (FMT != QLIN_FMT_BF16) {
+            switch (mode * 1000 + tile_n) {
+                case kModeFused * 1000 + 16: OP<FMT, true, 16, false, true, false>::run(args...); return true;
+                case kModeFused * 1000 + 32: OP<FMT, true, 32, false, true, false>::run(args...); return true;
+                case kModeFused * 1000 + 64: OP<FMT, true, 64, false, true, false>::run(args...); return true;
+            }
         }
         return false;
     }
@@ -1438,6 +1672,7 @@ bool gemm_kernel_info(int fmt, bool swap, int tile_n, int mode, int* stages, siz
         case QLIN_FMT_FP8: return dispatch_instance<QLIN_FMT_FP8, InfoOp>(swap, tile_n, mode, stages, smem_bytes);
         case QLIN_FMT_FP8_BLOCK:
             return dispatch_instance<QLIN_FMT_FP8_BLOCK, InfoOp>(swap, tile_n, mode, stages, smem_bytes);
+        case QLIN_FMT_BF16: return dispatch_instance<QLIN_FMT_BF16, InfoOp>(swap, tile_n, mode, stages, smem_bytes);
     }
     return false;
 }
@@ -1472,6 +1707,7 @@ qlin_status launch_gemm(const GemmPlan& plan, const GemmOperands& ops, cudaStrea
         case QLIN_FMT_INT8: return launch_fmt<QLIN_FMT_INT8>(plan, ops, st);
         case QLIN_FMT_FP8: return launch_fmt<QLIN_FMT_FP8>(plan, ops, st);
         case QLIN_FMT_FP8_BLOCK: return launch_fmt<QLIN_FMT_FP8_BLOCK>(plan, ops, st);
+        case QLIN_FMT_BF16: return launch_fmt<QLIN_FMT_BF16>(plan, ops, st);
         default: return QLIN_ERR_INVALID_ARG;
     }
 }

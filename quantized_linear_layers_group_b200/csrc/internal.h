@@ -55,14 +55,22 @@ struct GemmPlan {
     int64_t M = 0, N = 0, K = 0;
     int64_t p_rows = 0, q_rows = 0;
     int64_t p_tiles = 0, q_tiles = 0, num_tiles = 0, units = 0;
-    int kblocks = 0;       // K / 128
+    int64_t k_bytes = 0;   // bytes of one operand row: K (8-bit) or 2K (bf16)
+    int kblocks = 0;       // k_bytes / 128: K blocks of 128 bytes
     int kb_per_seg = 0;    // kblocks / S
     int kb_per_unit = 0;   // K blocks one work unit covers
     int grid = 0;          // persistent CTAs
     size_t smem_bytes = 0;
     size_t ticket_bytes = 0;   // workspace prefix holding the per-tile tickets
     size_t workspace_bytes = 0;
+    int moe_E = 0;             // MoE grouped GEMM: experts (units counted on the device)
 };
+
+// Grouped GEMM over experts (MoE): R rows of A / C grouped by expert, W [E N,
+// K]; the per-expert tile counts are only known on the device.
+qlin_status make_moe_plan(int fmt, int variant, int tile_n, int64_t R, int E, int64_t N, int64_t K, int num_sms,
+                          GemmPlan* plan);
+constexpr int kMoeMaxE = 255;  // experts the kernel's shared-memory table holds
 
 // Validates the (fmt, tile_n, S, variant) combination and fills the plan.
 // want_mode kModeCluster: a Swap-AB Split-K whose S fits one cluster reduces
@@ -89,7 +97,17 @@ struct GemmOperands {
     bool pdl;  // launch as a programmatic dependent of the previous kernel
     const void* x = nullptr;  // fused mode: bf16 activations [M, K], row stride ld_x elements
     int64_t ld_x = 0;
+    const int32_t* moe_offsets = nullptr;  // MoE: expert row offsets [E + 1] (device)
 };
+
+// ------------------------------------------------------------------- MoE
+cudaError_t launch_moe_route(const float* logits, int T, int E, int k, int32_t* ids, float* w, int32_t* offsets,
+                             int32_t* rows, bool pdl, cudaStream_t st);
+cudaError_t launch_moe_quantize_scatter(const void* x, int T, int H, int k, const int32_t* rows, void* a_q,
+                                        float* s_a, bool pdl, cudaStream_t st);
+cudaError_t launch_moe_act_quantize(const void* g, int R, int I, void* h_q, float* s_h, bool pdl, cudaStream_t st);
+cudaError_t launch_moe_combine(const void* y, const float* w, const int32_t* rows, int T, int H, int k, void* out,
+                               bool pdl, cudaStream_t st);
 
 qlin_status launch_gemm(const GemmPlan& plan, const GemmOperands& ops, cudaStream_t st);
 

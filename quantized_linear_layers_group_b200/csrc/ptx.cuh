@@ -58,6 +58,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of a phase: true if the phase with the given parity has
+// completed.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Returns false
 // (and records a timeout) if it has not completed within limit_ns.
 __device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
@@ -95,6 +109,7 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t par
 // Bounded wait for threads with nothing else to do meanwhile (the epilogue):
 // suspended in the barrier rather than polling it.
 __device__ __forceinline__ bool mbar_wait_idle(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;  // already complete: no timer read
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait_suspend(bar, parity, 100000u)) return true;
@@ -171,15 +186,27 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, both K-major; kind::f8f6f4 (e4m3) or kind::i8.
-template <bool INT8>
+// MMA kinds: the 8-bit float kind (e4m3 operands), the signed 8-bit integer
+// kind and the 16-bit float kind (bf16 operands).  Each consumes 32 bytes of
+// K per instruction.
+enum MmaKind : int { kKindF8 = 0, kKindI8 = 1, kKindF16 = 2 };
+
+// D[tmem] (+)= A[smem] * B[smem]^T, both K-major.
+template <int KIND>
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
-    if constexpr (INT8) {
+    if constexpr (KIND == kKindI8) {
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    } else if constexpr (KIND == kKindF16) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
             "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
             : "memory");
     } else {
@@ -217,14 +244,21 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
-template <bool INT8>
+template <int KIND>
 __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
-    if constexpr (INT8) {
+    if constexpr (KIND == kKindI8) {
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    } else if constexpr (KIND == kKindF16) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
             "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
             : "memory");
     } else {
@@ -287,6 +321,40 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr));
 }
 
+// 64 consecutive columns in one load (lane i: 64 registers).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]),
+          "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
+          "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+          "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
+          "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr));
+}
+
+// Two IEEE fp32 fused multiply-adds in one instruction (each lane rounded
+// separately, round to nearest even): (d0, d1) = (a0 * b + c0, a1 * b + c1).
+// Volatile: it stays after the tcgen05.wait::ld that makes its inputs valid.
+__device__ __forceinline__ void fma2_rn(float& d0, float& d1, float a0, float a1, float b, float c0, float c1) {
+    asm volatile("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %4};\n\t"
+        "mov.b64 rc, {%5, %6};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b), "f"(c0), "f"(c1));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -315,6 +383,19 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
     return old;
 }
 
+// Register reconfiguration per warpgroup (all four warps of a warpgroup
+// execute the same one): .dec returns registers to the CTA's pool, .inc takes
+// them from it (and waits until the pool holds them).  The pool is what the
+// CTA was launched with: threads x the kernel's register count.
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Named barrier among `count` threads (id 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -333,11 +414,13 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
 
 // Instruction descriptor (dense, K-major A and B):
 //   bits 4-5 D type (1 = f32, 2 = s32)   bits 7-9 A type   bits 10-12 B type
-//   (e4m3 = 0 for kind::f8f6f4; signed 8-bit = 1 for kind::i8)
+//   (kind::f8f6f4: e4m3 = 0; kind::i8: signed = 1; kind::f16: bf16 = 1)
 //   bits 17-22 N >> 3   bits 24-28 M >> 4
-__host__ __device__ constexpr uint32_t make_idesc(bool int8, int m, int n) {
-    return (int8 ? (2u << 4) : (1u << 4)) | (int8 ? (1u << 7) : 0u) | (int8 ? (1u << 10) : 0u) |
-           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+__host__ __device__ constexpr uint32_t make_idesc(int kind, int m, int n) {
+    const uint32_t d_type = kind == kKindI8 ? 2u : 1u;
+    const uint32_t ab_type = (kind == kKindI8 || kind == kKindF16) ? 1u : 0u;
+    return (d_type << 4) | (ab_type << 7) | (ab_type << 10) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(m >> 4) << 24);
 }
 
 // ------------------------------------------------------- thread-block clusters

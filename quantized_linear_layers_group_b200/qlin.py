@@ -34,6 +34,7 @@ QLIN_ERR_NO_DEVICE = 10
 QLIN_FMT_INT8 = 0
 QLIN_FMT_FP8 = 1
 QLIN_FMT_FP8_BLOCK = 2
+QLIN_FMT_BF16 = 3  # qlin_matmul_bf16 (and the workspace-size / dispatch queries)
 
 QLIN_VAR_AUTO = 0
 QLIN_VAR_PLAIN = 1
@@ -52,6 +53,8 @@ VARIANT_NAMES = {QLIN_VAR_AUTO: "auto", QLIN_VAR_PLAIN: "plain", QLIN_VAR_SPLITK
 
 # every symbol include/qlin.h declares
 EXPORTS = ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_scaled_mm_noalloc", "qlin_linear",
+           "qlin_matmul_bf16", "qlin_moe_route", "qlin_moe_quantize_scatter", "qlin_moe_grouped_mm",
+           "qlin_moe_act_quantize", "qlin_moe_combine", "qlin_moe_workspace_size", "qlin_moe_forward",
            "qlin_scaled_mm_workspace_size", "qlin_dispatch_table_load", "qlin_dispatch_table_clear",
            "qlin_dispatch_query", "qlin_status_string", "qlin_sync_status", "qlin_abi_version",
            "qlin_selftest_wait_timeout")
@@ -86,6 +89,14 @@ lib.qlin_scaled_mm_noalloc.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64,
                                        _u32, _vp]
 lib.qlin_linear.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _u32,
                             _vp, _sz, _vp]
+lib.qlin_matmul_bf16.argtypes = [_i32, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _u32, _vp, _sz, _vp]
+lib.qlin_moe_route.argtypes = [_i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _u32, _vp]
+lib.qlin_moe_quantize_scatter.argtypes = [_i64, _i64, _i32, _vp, _vp, _vp, _vp, _u32, _vp]
+lib.qlin_moe_grouped_mm.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _u32, _vp]
+lib.qlin_moe_act_quantize.argtypes = [_i64, _i64, _vp, _vp, _vp, _u32, _vp]
+lib.qlin_moe_combine.argtypes = [_i64, _i64, _i32, _vp, _vp, _vp, _vp, _u32, _vp]
+lib.qlin_moe_workspace_size.argtypes = [_i64, _i64, _i64, _i32, _i32, ctypes.POINTER(_sz)]
+lib.qlin_moe_forward.argtypes = [_i64, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _u32, _vp, _sz, _vp]
 lib.qlin_scaled_mm_workspace_size.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, ctypes.POINTER(_sz)]
 lib.qlin_dispatch_table_load.argtypes = [ctypes.c_char_p]
 lib.qlin_dispatch_table_clear.argtypes = []
@@ -195,6 +206,69 @@ def qlin_linear(fmt: int, x, a_q, s_a, w_q, s_w, bias, c_out, workspace=None, st
     _check(lib.qlin_linear(fmt, variant, tile_n, k_segments, M, N, K, _ptr(x), ld_x, _ptr(a_q), _ptr(s_a), _ptr(w_q),
                            _ptr(s_w), _ptr(bias), _ptr(c_out), flags, _ptr(workspace), workspace_bytes,
                            _stream(stream)), "qlin_linear")
+
+
+def qlin_matmul_bf16(a, w, bias, c_out, workspace=None, stream=None, *, variant: int = QLIN_VAR_AUTO,
+                     tile_n: int = 0, k_segments: int = 0, flags: int = 0, M=None, N=None, K=None,
+                     workspace_bytes=None):
+    """C = bf16(fp32(a w^T) + bias) for bf16 a [M, K], w [N, K] (batch-invariant)."""
+    M = a.shape[0] if M is None else M
+    N = w.shape[0] if N is None else N
+    K = a.shape[1] if K is None else K
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.qlin_matmul_bf16(variant, tile_n, k_segments, M, N, K, _ptr(a), _ptr(w), _ptr(bias), _ptr(c_out),
+                                flags, _ptr(workspace), workspace_bytes, _stream(stream)), "qlin_matmul_bf16")
+
+
+# ------------------------------------------------------------------- MoE
+def qlin_moe_route(logits, topk: int, topk_ids, topk_w, rows, offsets, stream=None, *, flags: int = 0):
+    T, E = logits.shape
+    _check(lib.qlin_moe_route(T, E, topk, _ptr(logits), _ptr(topk_ids), _ptr(topk_w), _ptr(rows), _ptr(offsets),
+                              flags, _stream(stream)), "qlin_moe_route")
+
+
+def qlin_moe_quantize_scatter(x, topk: int, rows, a_q, s_a, stream=None, *, flags: int = 0):
+    T, H = x.shape
+    _check(lib.qlin_moe_quantize_scatter(T, H, topk, _ptr(x), _ptr(rows), _ptr(a_q), _ptr(s_a), flags,
+                                         _stream(stream)), "qlin_moe_quantize_scatter")
+
+
+def qlin_moe_grouped_mm(fmt: int, E: int, a_q, s_a, offsets, w_q, s_w, c_out, stream=None, *,
+                        variant: int = QLIN_VAR_AUTO, tile_n: int = 0, flags: int = 0):
+    """Grouped scaled GEMM over experts: w_q [E * N, K], s_w [E * N], c_out [R, N]."""
+    R, K = a_q.shape
+    N = c_out.shape[1]
+    _check(lib.qlin_moe_grouped_mm(fmt, variant, tile_n, E, R, N, K, _ptr(a_q), _ptr(s_a), _ptr(offsets), _ptr(w_q),
+                                   _ptr(s_w), _ptr(c_out), flags, _stream(stream)), "qlin_moe_grouped_mm")
+
+
+def qlin_moe_act_quantize(g, h_q, s_h, stream=None, *, flags: int = 0):
+    R, I2 = g.shape
+    _check(lib.qlin_moe_act_quantize(R, I2 // 2, _ptr(g), _ptr(h_q), _ptr(s_h), flags, _stream(stream)),
+           "qlin_moe_act_quantize")
+
+
+def qlin_moe_combine(y, topk_w, rows, out, stream=None, *, flags: int = 0):
+    T, H = out.shape
+    _check(lib.qlin_moe_combine(T, H, topk_w.shape[1], _ptr(y), _ptr(topk_w), _ptr(rows), _ptr(out), flags,
+                                _stream(stream)), "qlin_moe_combine")
+
+
+def qlin_moe_workspace_size(T: int, H: int, I: int, E: int, topk: int) -> int:
+    out = _sz(0)
+    _check(lib.qlin_moe_workspace_size(T, H, I, E, topk, ctypes.byref(out)), "qlin_moe_workspace_size")
+    return out.value
+
+
+def qlin_moe_forward(x, logits, topk: int, w1_q, s_w1, w2_q, s_w2, out, workspace, stream=None, *, flags: int = 0):
+    """The whole FP8 MoE layer (x bf16 [T, H], logits [T, E], w1_q [E, 2I, H], w2_q [E, H, I])."""
+    T, H = x.shape
+    E = logits.shape[1]
+    I = w2_q.shape[-1]
+    _check(lib.qlin_moe_forward(T, H, I, E, topk, _ptr(x), _ptr(logits), _ptr(w1_q), _ptr(s_w1), _ptr(w2_q),
+                                _ptr(s_w2), _ptr(out), flags, _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream)), "qlin_moe_forward")
 
 
 def qlin_dispatch_table_load(path: str):

@@ -21,7 +21,7 @@
 // 2x L2), launched with QLIN_PDL as the hot path runs, CUDA events around the
 // graph, median of `reps` replays.
 //
-// Usage: qlin_sweep [--quick] <out.qlt> [shape ...]   shape = fmt:N:K (fmt int8|fp8|fp8_block)
+// Usage: qlin_sweep [--quick] <out.qlt> [shape ...]   shape = fmt:N:K (fmt int8|fp8|fp8_block|bf16)
 // Without shapes it sweeps the five workload shapes.  --quick (for tests):
 // buckets {1, 16, 256} only, two weight copies, short timing loops.
 #include <cuda_runtime.h>
@@ -56,7 +56,15 @@ struct Cand {
     int variant, tile_n;
 };
 
-const char* fmt_name(int f) { return f == QLIN_FMT_INT8 ? "int8" : (f == QLIN_FMT_FP8 ? "fp8" : "fp8_block"); }
+const char* fmt_name(int f) {
+    switch (f) {
+        case QLIN_FMT_INT8: return "int8";
+        case QLIN_FMT_FP8: return "fp8";
+        case QLIN_FMT_FP8_BLOCK: return "fp8_block";
+    }
+    return "bf16";
+}
+int elem_bytes(int f) { return f == QLIN_FMT_BF16 ? 2 : 1; }
 const char* var_name(int v) {
     switch (v) {
         case QLIN_VAR_PLAIN: return "plain";
@@ -81,6 +89,17 @@ __global__ void fill_codes(uint8_t* p, size_t n, uint32_t seed, int e4m3) {
     }
 }
 
+// Deterministic bf16 filler: values of magnitude below 2 (exponent field 112..127).
+__global__ void fill_bf16(uint16_t* p, size_t n, uint32_t seed) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        uint32_t h = (uint32_t)i * 2654435761u ^ seed;
+        h ^= h >> 13;
+        h *= 0x5bd1e995u;
+        h ^= h >> 15;
+        p[i] = (uint16_t)((h & 0x807Fu) | ((112u + ((h >> 8) & 15u)) << 7));
+    }
+}
+
 __global__ void fill_scales(float* p, size_t n, uint32_t seed) {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
         uint32_t h = (uint32_t)i * 747796405u + seed;
@@ -92,9 +111,9 @@ __global__ void fill_scales(float* p, size_t n, uint32_t seed) {
 struct Problem {
     Shape s;
     int64_t M;
-    uint8_t* a_q = nullptr;
+    void* a_q = nullptr;
     float* s_a = nullptr;
-    std::vector<uint8_t*> w_q;
+    std::vector<void*> w_q;
     std::vector<float*> s_w;
     uint16_t* c = nullptr;
     uint16_t* c_ref = nullptr;
@@ -102,9 +121,9 @@ struct Problem {
     size_t ws_bytes = 0;
 };
 
-std::vector<int> segment_choices(int64_t K) {
+std::vector<int> segment_choices(int fmt, int64_t K) {
     std::vector<int> out;
-    const int kb = (int)(K / 128);
+    const int kb = (int)(K * elem_bytes(fmt) / 128);
     for (int s : {1, 2, 3, 4, 6, 8})
         if (kb % s == 0 && kb / s >= 1) out.push_back(s);
     return out;
@@ -130,23 +149,29 @@ std::vector<Cand> candidates(int fmt, int64_t M) {
     return c;
 }
 
+// One GEMM call of the problem's format on weight copy w.
+qlin_status run_gemm(Problem& P, int variant, int tile, int S, size_t w, uint16_t* c, uint32_t flags,
+                     cudaStream_t st) {
+    if (P.s.fmt == QLIN_FMT_BF16)
+        return qlin_matmul_bf16(variant, tile, S, P.M, P.s.N, P.s.K, P.a_q, P.w_q[w], nullptr, c, flags, P.ws,
+                                P.ws_bytes, st);
+    return qlin_scaled_mm(P.s.fmt, variant, tile, S, P.M, P.s.N, P.s.K, P.a_q, P.s_a, P.w_q[w], P.s_w[w], nullptr, c,
+                          flags, P.ws, P.ws_bytes, st);
+}
+
 float time_config(Problem& P, int variant, int tile, int S, int iters, int reps, cudaStream_t st, bool* ok) {
     *ok = false;
     size_t need = 0;
     if (qlin_scaled_mm_workspace_size(P.s.fmt, variant, tile, S, P.M, P.s.N, P.s.K, &need) != QLIN_OK) return -1.f;
     if (need > P.ws_bytes) return -1.f;
-    const void* bias = nullptr;
     // correctness / warm-up launch on copy 0
-    if (qlin_scaled_mm(P.s.fmt, variant, tile, S, P.M, P.s.N, P.s.K, P.a_q, P.s_a, P.w_q[0], P.s_w[0], bias, P.c,
-                       QLIN_PDL, P.ws, P.ws_bytes, st) != QLIN_OK)
-        return -1.f;
+    if (run_gemm(P, variant, tile, S, 0, P.c, QLIN_PDL, st) != QLIN_OK) return -1.f;
     cudaGraph_t graph;
     cudaGraphExec_t exec;
     CK(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
     for (int i = 0; i < iters; ++i) {
         const size_t w = (size_t)(i + 1) % P.w_q.size();
-        if (qlin_scaled_mm(P.s.fmt, variant, tile, S, P.M, P.s.N, P.s.K, P.a_q, P.s_a, P.w_q[w], P.s_w[w], bias,
-                           P.c, QLIN_PDL, P.ws, P.ws_bytes, st) != QLIN_OK) {
+        if (run_gemm(P, variant, tile, S, w, P.c, QLIN_PDL, st) != QLIN_OK) {
             cudaStreamEndCapture(st, &graph);
             cudaGraphDestroy(graph);
             return -1.f;
@@ -179,9 +204,7 @@ float time_config(Problem& P, int variant, int tile, int S, int iters, int reps,
 }
 
 bool same_output(Problem& P, int variant, int tile, int S, cudaStream_t st) {
-    if (qlin_scaled_mm(P.s.fmt, variant, tile, S, P.M, P.s.N, P.s.K, P.a_q, P.s_a, P.w_q[0], P.s_w[0], nullptr,
-                       P.c, 0, P.ws, P.ws_bytes, st) != QLIN_OK)
-        return false;
+    if (run_gemm(P, variant, tile, S, 0, P.c, 0, st) != QLIN_OK) return false;
     CK(cudaStreamSynchronize(st));
     const size_t bytes = (size_t)P.M * P.s.N * 2;
     std::vector<uint16_t> a(bytes / 2), b(bytes / 2);
@@ -210,7 +233,11 @@ int main(int argc, char** argv) {
         long long n, k;
         if (std::sscanf(argv[i], "%31[^:]:%lld:%lld", f, &n, &k) != 3) return 1;
         const std::string fs(f);
-        shapes.push_back({fs == "int8" ? QLIN_FMT_INT8 : (fs == "fp8" ? QLIN_FMT_FP8 : QLIN_FMT_FP8_BLOCK), n, k});
+        shapes.push_back({fs == "int8"   ? QLIN_FMT_INT8
+                          : fs == "fp8"  ? QLIN_FMT_FP8
+                          : fs == "bf16" ? QLIN_FMT_BF16
+                                         : QLIN_FMT_FP8_BLOCK,
+                          n, k});
     }
     if (shapes.empty())
         shapes = {{QLIN_FMT_FP8, 4096, 2048},
@@ -239,20 +266,28 @@ int main(int argc, char** argv) {
         const int64_t M_max = buckets.back();
         Problem P;
         P.s = s;
-        const size_t wbytes = (size_t)s.N * s.K;
+        const size_t wbytes = (size_t)s.N * s.K * elem_bytes(s.fmt);
         const size_t ncopy = quick ? 2 : std::max<size_t>(2, (2 * l2 + wbytes - 1) / wbytes + 1);
         const size_t sw_elems = s.fmt == QLIN_FMT_FP8_BLOCK ? (size_t)((s.N + 127) / 128) * (s.K / 128) : (size_t)s.N;
         const size_t sa_elems = s.fmt == QLIN_FMT_FP8_BLOCK ? (size_t)M_max * (s.K / 128) : (size_t)M_max;
-        CK(cudaMalloc(&P.a_q, (size_t)M_max * s.K));
+        CK(cudaMalloc(&P.a_q, (size_t)M_max * s.K * elem_bytes(s.fmt)));
         CK(cudaMalloc(&P.s_a, sa_elems * 4));
-        fill_codes<<<1024, 256, 0, st>>>(P.a_q, (size_t)M_max * s.K, 17u, s.fmt != QLIN_FMT_INT8);
+        if (s.fmt == QLIN_FMT_BF16)
+            fill_bf16<<<1024, 256, 0, st>>>(static_cast<uint16_t*>(P.a_q), (size_t)M_max * s.K, 17u);
+        else
+            fill_codes<<<1024, 256, 0, st>>>(static_cast<uint8_t*>(P.a_q), (size_t)M_max * s.K, 17u,
+                                             s.fmt != QLIN_FMT_INT8);
         fill_scales<<<256, 256, 0, st>>>(P.s_a, sa_elems, 5u);
         for (size_t i = 0; i < ncopy; ++i) {
-            uint8_t* w;
+            void* w;
             float* sw;
             CK(cudaMalloc(&w, wbytes));
             CK(cudaMalloc(&sw, sw_elems * 4));
-            fill_codes<<<2048, 256, 0, st>>>(w, wbytes, 1000u + (uint32_t)i, s.fmt != QLIN_FMT_INT8);
+            if (s.fmt == QLIN_FMT_BF16)
+                fill_bf16<<<2048, 256, 0, st>>>(static_cast<uint16_t*>(w), wbytes / 2, 1000u + (uint32_t)i);
+            else
+                fill_codes<<<2048, 256, 0, st>>>(static_cast<uint8_t*>(w), wbytes, 1000u + (uint32_t)i,
+                                                 s.fmt != QLIN_FMT_INT8);
             fill_scales<<<256, 256, 0, st>>>(sw, sw_elems, 77u);
             P.w_q.push_back(w);
             P.s_w.push_back(sw);
@@ -264,7 +299,7 @@ int main(int argc, char** argv) {
         CK(cudaMemsetAsync(P.ws, 0, P.ws_bytes, st));
         CK(cudaStreamSynchronize(st));
 
-        const std::vector<int> segs = segment_choices(s.K);
+        const std::vector<int> segs = segment_choices(s.fmt, s.K);
         // best[si][bi] = (time, cand)
         std::vector<std::vector<std::pair<float, Cand>>> best(segs.size(),
                                                               std::vector<std::pair<float, Cand>>(buckets.size()));
@@ -275,8 +310,7 @@ int main(int argc, char** argv) {
                 const int iters =
                     quick ? 4 : std::max(4, std::min(40, (int)(40 * 64 / std::max<int64_t>(P.M, 64))));
                 // reference output: plain tile 128 with this S (the canonical order)
-                bool have_ref = qlin_scaled_mm(s.fmt, QLIN_VAR_PLAIN, 128, S, P.M, s.N, s.K, P.a_q, P.s_a, P.w_q[0],
-                                               P.s_w[0], nullptr, P.c_ref, 0, P.ws, P.ws_bytes, st) == QLIN_OK;
+                bool have_ref = run_gemm(P, QLIN_VAR_PLAIN, 128, S, 0, P.c_ref, 0, st) == QLIN_OK;
                 CK(cudaStreamSynchronize(st));
                 float bt = 1e30f;
                 Cand bc{0, 0};

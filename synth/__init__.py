@@ -24,6 +24,10 @@ Workloads (weights W are [N, K], nn.Linear layout; activations A are [M, K]):
   W ~ N(0, 0.02); no bias, no outliers.
 * ``fp8_vocab``    FP8 per-token/per-channel, N = 12288, K = 2048 (batch
   invariance shape); A and W as ``fp8_attn`` without bias.
+* ``bf16_*``       bf16 matmul (no quantisation) on the five (N, K) shapes of
+  the batch-invariant matmul sweep: vocab 12288 x 2048, down 2048 x 6144, attn
+  4096 x 2048, lm_head 151936 x 2048, square 2048 x 2048; M sweep as above;
+  A ~ N(0,1), W ~ N(0, 0.02), no bias.
 """
 from __future__ import annotations
 
@@ -35,6 +39,7 @@ import torch
 FMT_INT8 = 0
 FMT_FP8 = 1
 FMT_FP8_BLOCK = 2
+FMT_BF16 = 3
 
 M_SWEEP = (1, 4, 8, 16, 32, 64, 256, 512, 1024, 2048)
 LM_HEAD_M = (1, 8, 64, 256, 1024, 2048)
@@ -59,6 +64,11 @@ WORKLOADS = {
     "lm_head": Workload("lm_head", FMT_FP8, 151936, 2048, LM_HEAD_M, False, False, False),
     "fp8_vocab": Workload("fp8_vocab", FMT_FP8, 12288, 2048, M_SWEEP, True, False, False),
     "int8_square": Workload("int8_square", FMT_INT8, 2048, 2048, M_SWEEP, True, False, False),
+    "bf16_vocab": Workload("bf16_vocab", FMT_BF16, 12288, 2048, M_SWEEP, False, False, False),
+    "bf16_down": Workload("bf16_down", FMT_BF16, 2048, 6144, M_SWEEP, False, False, False),
+    "bf16_attn": Workload("bf16_attn", FMT_BF16, 4096, 2048, M_SWEEP, False, False, False),
+    "bf16_lm_head": Workload("bf16_lm_head", FMT_BF16, 151936, 2048, M_SWEEP, False, False, False),
+    "bf16_square": Workload("bf16_square", FMT_BF16, 2048, 2048, M_SWEEP, False, False, False),
 }
 
 

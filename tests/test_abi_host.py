@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
     syms = _declared_symbols()
     for name in ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_dispatch_table_load"):
         assert name in syms
-    assert len(syms) == 13
+    assert len(syms) == 21
 
 
 def test_library_exports_every_declared_symbol(q):
@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(q):
     for name in _declared_symbols():
         assert hasattr(lib, name), name
     assert set(_declared_symbols()) == set(q.EXPORTS)
-    assert q.qlin_abi_version() == 4
+    assert q.qlin_abi_version() == 6
 
 
 def test_status_strings(q):
@@ -219,3 +219,26 @@ def test_linear_rejects_bad_arguments_before_launch(q):
 def test_selftest_rejects_bad_limits(q):
     assert q.lib.qlin_selftest_wait_timeout(0, None) == q.QLIN_ERR_INVALID_ARG
     assert q.lib.qlin_selftest_wait_timeout(2000000, None) == q.QLIN_ERR_INVALID_ARG
+
+
+def test_matmul_bf16_rejects_bad_arguments_before_launch(q):
+    def mm(**kw):
+        a = dict(variant=0, tile_n=0, k_segments=0, M=16, N=256, K=256, a=16, w=16, bias=None, c=16, flags=0,
+                 ws=None, wsb=0)
+        a.update(kw)
+        return q.lib.qlin_matmul_bf16(a["variant"], a["tile_n"], a["k_segments"], a["M"], a["N"], a["K"], a["a"],
+                                      a["w"], a["bias"], a["c"], a["flags"], a["ws"], a["wsb"], None)
+
+    assert mm(K=96) == q.QLIN_ERR_UNSUPPORTED                 # K blocks are 64 bf16 elements
+    assert mm(K=32) == q.QLIN_ERR_INVALID_ARG
+    assert mm(N=250) == q.QLIN_ERR_UNSUPPORTED
+    assert mm(flags=1) == q.QLIN_ERR_INVALID_ARG              # no int32 accumulators for bf16
+    assert mm(flags=8) == q.QLIN_ERR_INVALID_ARG
+    assert mm(a=None) == q.QLIN_ERR_INVALID_ARG
+    assert mm(w=24) == q.QLIN_ERR_ALIGNMENT
+    assert mm(bias=17) == q.QLIN_ERR_ALIGNMENT
+    assert mm(M=0) == q.QLIN_OK
+    # the scaled entry points do not take the bf16 format
+    assert _mm(q, fmt=q.QLIN_FMT_BF16) == q.QLIN_ERR_INVALID_ARG
+    # K blocks of a bf16 row: K = 192 is three of them, so S = 3 divides it
+    assert q.qlin_scaled_mm_workspace_size(q.QLIN_FMT_BF16, 16, 256, 192, q.QLIN_VAR_SWAPAB_SPLITK, 16, 3) > 0
