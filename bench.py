@@ -389,6 +389,82 @@ class HotPath:
         return hb, db
 
 
+class MoEPath:
+    """The FP8 MoE layer (qlin_moe_forward: seven PDL-chained kernels) on the
+    benchmark's MoE configuration, one token count at a time."""
+
+    def __init__(self, device, seed=0):
+        from quantized_linear_layers_group_b200 import qlin
+
+        self.qlin = qlin
+        c = synth.MOE
+        self.E, self.k, self.H, self.I = c["E"], c["topk"], c["H"], c["I"]
+        E, H, I = self.E, self.H, self.I
+        self.w1 = torch.empty(E * 2 * I, H, dtype=torch.uint8, device=device)
+        self.s1 = torch.empty(E * 2 * I, dtype=torch.float32, device=device)
+        self.w2 = torch.empty(E * H, I, dtype=torch.uint8, device=device)
+        self.s2 = torch.empty(E * H, dtype=torch.float32, device=device)
+        for e0, e1, w in synth.moe_weight_chunks(E, 2 * I, H, seed + 30, device):
+            qlin.qlin_quantize_per_token(1, w, self.w1[e0 * 2 * I:e1 * 2 * I], self.s1[e0 * 2 * I:e1 * 2 * I])
+        for e0, e1, w in synth.moe_weight_chunks(E, H, I, seed + 31, device):
+            qlin.qlin_quantize_per_token(1, w, self.w2[e0 * H:e1 * H], self.s2[e0 * H:e1 * H])
+        torch.cuda.synchronize()
+        self.device = device
+
+    def time_t(self, T, stream, reps=8, replays=5):
+        """Per-layer device time (us) of qlin_moe_forward at T tokens, from a
+        CUDA graph of `reps` layers (median of `replays`), and the number of
+        experts the routing activated."""
+        q = self.qlin
+        x, logits = synth.moe_inputs(T, self.H, self.E)
+        x, logits = x.to(self.device), logits.to(self.device)
+        out = torch.empty(T, self.H, dtype=torch.bfloat16, device=self.device)
+        ws = torch.empty(q.qlin_moe_workspace_size(T, self.H, self.I, self.E, self.k), dtype=torch.uint8,
+                         device=self.device)
+        fwd = lambda: q.qlin_moe_forward(x, logits, self.k, self.w1, self.s1, self.w2, self.s2, out, ws, stream,
+                                         flags=q.QLIN_PDL)
+        for _ in range(3):
+            fwd()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                fwd()
+        g.replay()
+        ts = []
+        for _ in range(replays):
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            g.replay()
+            a1.record(stream)
+            a1.synchronize()
+            ts.append(a0.elapsed_time(a1) * 1e3 / reps)
+        # experts the routing used (offsets live in the workspace after topk ids, weights, rows)
+        R = T * self.k
+        off0 = 3 * ((R * 4 + 255) // 256 * 256)
+        offs = ws[off0:off0 + 4 * (self.E + 1)].view(torch.int32).cpu()
+        active = int((offs[1:] - offs[:-1] > 0).sum())
+        del g
+        return statistics.median(ts), active
+
+    def report(self, stream, peaks, tpk):
+        tc_peak, tc_src = tensor_peak(peaks, 1, tpk)
+        hbm = peaks["hbm_gbs"]
+        per_t = []
+        for T in synth.MOE["T"]:
+            us, active = self.time_t(T, stream)
+            R = T * self.k
+            flops = 6.0 * R * self.H * self.I
+            wbytes = active * 3 * self.H * self.I  # gate-up (2I x H) + down (H x I) of each active expert, FP8
+            t_roof = max(wbytes / (hbm * 1e9), flops / (tc_peak * 1e12))
+            per_t.append({"T": T, "rows": R, "active_experts": active, "layer_us": us,
+                          "tflops": flops / (us * 1e-6) / 1e12, "weight_gbs": wbytes / (us * 1e-6) / 1e9,
+                          "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / (us * 1e-6),
+                          "bound": "hbm" if wbytes / (hbm * 1e9) >= flops / (tc_peak * 1e12) else "tensor"})
+        return {"E": self.E, "topk": self.k, "H": self.H, "I": self.I, "kernels_per_layer": 7,
+                "peak_source": tc_src, "per_t": per_t}
+
+
 def per_kernel_times(hp: HotPath, stream, reps=8, replays=5):
     """For each M: a graph of `reps` back-to-back launches of one kernel (the
     quantiser rotates activation sets, the GEMM weight copies), timed with
@@ -731,6 +807,10 @@ def main(argv=None):
                     raise RuntimeError(f"device status ({name}): {qlin.qlin_status_string(st)}")
                 del wh
                 torch.cuda.empty_cache()
+            mp = MoEPath(device)
+            workloads["moe_fp8"] = mp.report(stream, peaks, tpk)
+            del mp
+            torch.cuda.empty_cache()
 
     N, K, fmt = workload.N, workload.K, workload.fmt
     flops_step = sum(gemm_flops(M, N, K) for M in ms)

@@ -139,6 +139,30 @@ def mixed_stream(n_calls: int = 1000, seed: int = 0):
     return out
 
 
+# FP8 MoE layer of the benchmark: the page's 192 experts with top-8 routing;
+# hidden and expert intermediate sizes are not on the page (4096 and 1536 here)
+MOE = {"E": 192, "topk": 8, "H": 4096, "I": 1536, "T": (1, 8, 64, 256, 1024)}
+
+
+def moe_inputs(T: int, H: int, E: int, seed: int = 0):
+    """x bf16 [T, H] ~ N(0,1) and router logits fp32 [T, E] ~ N(0, 4)."""
+    x = torch.randn(T, H, generator=_gen(seed + 20), dtype=torch.float32).to(torch.bfloat16)
+    logits = torch.randn(T, E, generator=_gen(seed + 21), dtype=torch.float32) * 2.0
+    return x, logits
+
+
+def moe_weight_chunks(E: int, rows: int, cols: int, seed: int, device, chunk: int = 16):
+    """Yield (e0, e1, W bf16 [(e1 - e0) * rows, cols] ~ N(0, 0.05^2)) drawn on
+    `device` from a seeded generator, a few experts at a time (the full bf16
+    weights of the benchmark's MoE would not need to exist at once)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    for e0 in range(0, E, chunk):
+        e1 = min(E, e0 + chunk)
+        w = torch.randn((e1 - e0) * rows, cols, generator=g, device=device, dtype=torch.float32) * 0.05
+        yield e0, e1, w.to(torch.bfloat16)
+
+
 def bf16_bits(t: torch.Tensor):
     """uint16 numpy view of a CPU bf16 tensor's bit patterns."""
     import numpy as np
