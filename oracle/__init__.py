@@ -27,6 +27,8 @@ import numpy as np
 FMT_INT8 = 0
 FMT_FP8 = 1
 FMT_FP8_BLOCK = 2
+FMT_MXFP8 = 4
+FMT_NVFP4 = 5
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "qlin_oracle.c")
@@ -86,6 +88,19 @@ def _load():
         lib.qo_moe_act_quantize.restype = None
         lib.qo_moe_combine.argtypes = [i64, i64, i64, u16p, f32p_, i32p, u16p]
         lib.qo_moe_combine.restype = None
+        lib.qo_e8m0_decode.argtypes = [ctypes.c_uint8]
+        lib.qo_e8m0_decode.restype = ctypes.c_double
+        lib.qo_e2m1_decode.argtypes = [ctypes.c_uint8]
+        lib.qo_e2m1_decode.restype = ctypes.c_float
+        lib.qo_e2m1_encode.argtypes = [ctypes.c_float]
+        lib.qo_e2m1_encode.restype = ctypes.c_uint8
+        lib.qo_quantize_mxfp8.argtypes = [u16p, i64, i64, i64, u8p, u8p]
+        lib.qo_quantize_mxfp8.restype = None
+        lib.qo_quantize_nvfp4.argtypes = [u16p, i64, i64, i64, ctypes.c_float, u8p, u8p]
+        lib.qo_quantize_nvfp4.restype = None
+        lib.qo_gemm_block_scaled.argtypes = [ctypes.c_int, i64, i64, i64, u8p, u8p, u8p, u8p, ctypes.c_float,
+                                             ctypes.c_float, u16p, i64p, i64, i64p, i64, u16p]
+        lib.qo_gemm_block_scaled.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -280,3 +295,75 @@ def moe_combine(y: np.ndarray, w: np.ndarray, rows: np.ndarray) -> np.ndarray:
 def bf16_bits_to_f32(c: np.ndarray) -> np.ndarray:
     """Widen bf16 bit patterns to float32 values (exact)."""
     return (c.astype(np.uint32) << 16).view(np.float32)
+
+
+# ------------------------------------------------------ block-scaled formats --
+# MXFP8 (OCP Microscaling v1.0: E4M3 elements, 32-element blocks along K, E8M0
+# scales) and NVFP4 (E2M1 elements, 16-element blocks, E4M3 block scales and a
+# per-tensor fp32 decode scale g).  NVFP4 is listed among vLLM's formats on the
+# page "Helion in vLLM: A Unified Route to Tunable Linear Kernels"
+# (introduction); the readings are stated in qlin_oracle.c.
+def e8m0_decode(code: int) -> float:
+    return _load().qo_e8m0_decode(code)
+
+
+def e2m1_decode(code: int) -> float:
+    return _load().qo_e2m1_decode(code)
+
+
+def e2m1_encode(v: float) -> int:
+    return _load().qo_e2m1_encode(v)
+
+
+def quantize_mxfp8(x) -> tuple[np.ndarray, np.ndarray]:
+    """MXFP8 codes uint8 [rows, cols] and E8M0 scale codes uint8 [rows, cols/32]."""
+    xb = _bits(x)
+    rows, cols = xb.shape
+    assert cols % 32 == 0
+    q = np.empty((rows, cols), np.uint8)
+    sf = np.empty((rows, cols // 32), np.uint8)
+    _load().qo_quantize_mxfp8(_ptr(xb, ctypes.c_uint16), rows, cols, cols, _ptr(q, ctypes.c_uint8),
+                              _ptr(sf, ctypes.c_uint8))
+    return q, sf
+
+
+def quantize_nvfp4(x, g: float) -> tuple[np.ndarray, np.ndarray]:
+    """NVFP4 packed codes uint8 [rows, cols/2] (element 2i in the low nibble) and
+    E4M3 block-scale codes uint8 [rows, cols/16], for the per-tensor decode scale g."""
+    xb = _bits(x)
+    rows, cols = xb.shape
+    assert cols % 16 == 0 and g > 0
+    q = np.empty((rows, cols // 2), np.uint8)
+    sf = np.empty((rows, cols // 16), np.uint8)
+    _load().qo_quantize_nvfp4(_ptr(xb, ctypes.c_uint16), rows, cols, cols, float(np.float32(g)),
+                              _ptr(q, ctypes.c_uint8), _ptr(sf, ctypes.c_uint8))
+    return q, sf
+
+
+def gemm_block_scaled(fmt: int, a_q: np.ndarray, a_sf: np.ndarray, w_q: np.ndarray, w_sf: np.ndarray,
+                      g_a: float = 1.0, g_w: float = 1.0, bias=None, m_idx=None, n_idx=None) -> np.ndarray:
+    """Block-scaled GEMM (FMT_MXFP8 or FMT_NVFP4) as bf16 bits [len(m_idx), len(n_idx)]."""
+    assert fmt in (FMT_MXFP8, FMT_NVFP4)
+    a_q = np.ascontiguousarray(a_q, dtype=np.uint8)
+    w_q = np.ascontiguousarray(w_q, dtype=np.uint8)
+    a_sf = np.ascontiguousarray(a_sf, dtype=np.uint8)
+    w_sf = np.ascontiguousarray(w_sf, dtype=np.uint8)
+    M, N = a_q.shape[0], w_q.shape[0]
+    K = a_q.shape[1] * (2 if fmt == FMT_NVFP4 else 1)
+    bs = 16 if fmt == FMT_NVFP4 else 32
+    assert w_q.shape[1] == a_q.shape[1] and K % bs == 0
+    assert a_sf.shape == (M, K // bs) and w_sf.shape == (N, K // bs)
+    bb = None if bias is None else _bits(bias).reshape(-1)
+    mi = None if m_idx is None else np.ascontiguousarray(m_idx, dtype=np.int64)
+    ni = None if n_idx is None else np.ascontiguousarray(n_idx, dtype=np.int64)
+    mc = M if mi is None else len(mi)
+    nc = N if ni is None else len(ni)
+    c = np.empty((mc, nc), np.uint16)
+    rc = _load().qo_gemm_block_scaled(fmt, M, N, K, _ptr(a_q, ctypes.c_uint8), _ptr(a_sf, ctypes.c_uint8),
+                                      _ptr(w_q, ctypes.c_uint8), _ptr(w_sf, ctypes.c_uint8),
+                                      float(np.float32(g_a)), float(np.float32(g_w)), _ptr(bb, ctypes.c_uint16),
+                                      _ptr(mi, ctypes.c_int64), mc, _ptr(ni, ctypes.c_int64), nc,
+                                      _ptr(c, ctypes.c_uint16))
+    if rc != 0:
+        raise MemoryError("oracle allocation failed")
+    return c

@@ -22,6 +22,8 @@
  *   bf16 GEMM:                C[m,n] = bf16( fp32(sum_k a[m,k] w[n,k]) + bias[n] ), the
  *                             matmul of the page "[Kernel][Perf] Add Hopper (SM90)
  *                             tuned config for batch-invariant persistent matmul"
+ *   MXFP8 / NVFP4:            block-scaled codecs and GEMM, at the end of this
+ *                             file with their readings
  *
  * Every fp32 operation is a separately rounded IEEE binary32 operation
  * (compile with -O2 -fno-fast-math -ffp-contract=off; x86-64 SSE arithmetic),
@@ -475,4 +477,223 @@ int qo_moe_forward(int64_t T, int64_t H, int64_t I, int64_t E, int64_t topk, con
 out:
     free(fill); free(xq); free(sx); free(a1); free(sa1);
     return rc;
+}
+
+/* ------------------------------------------------- block-scaled formats ---- */
+/*
+ * The page "Helion in vLLM: A Unified Route to Tunable Linear Kernels"
+ * (introduction) lists NVFP4 among the formats vLLM's quantized linear layers
+ * serve; the pages define neither it nor MXFP8.  The readings below follow
+ * the formats' public definitions and take the plainest arithmetic where
+ * those leave a step open:
+ *
+ * MXFP8 (OCP Microscaling Formats v1.0: E4M3 elements, blocks of 32 along K,
+ * one E8M0 scale X = 2^(code - 127) per block):
+ *   amax == 0:  scale code 0, every element +0 (as the FP8 reading above);
+ *   otherwise:  e = floor(log2(amax)) - 8 (8 = the largest E4M3 exponent),
+ *               clamped to [-127, 127]; scale code e + 127;
+ *               q = E4M3(x * 2^-e), nearest code, ties to even, saturating
+ *               at +-448 (amax * 2^-e lies in [256, 512), so the block's
+ *               largest elements may saturate: the format's own rule).
+ *   x * 2^-e is exact, so the element rounding is the only rounding.
+ *
+ * NVFP4 (E2M1 elements {0, 0.5, 1, 1.5, 2, 3, 4, 6} with sign, blocks of 16
+ * along K, one E4M3 scale per block, one fp32 decode scale g per tensor,
+ * x ~ q * s * g):
+ *   t = amax / 6 (binary32 division), t = t / g (binary32 division),
+ *   s = E4M3(t) (nearest, ties to even, saturating at 448);
+ *   d = dec(s) * g (binary32 multiply); d == 0: every element +0;
+ *   otherwise q = E2M1(x / d) (binary32 division, then the nearest E2M1
+ *   value, ties to the even code, saturating at +-6, keeping the sign of
+ *   zero).  Two elements per byte, element 2i in the low nibble.
+ *   g is an input: per-tensor amax / (6 * 448) for weights, a calibrated
+ *   constant for activations.
+ *
+ * Block-scaled GEMM, both operands K-major, bias bf16 [N] or NULL:
+ *   MXFP8: acc = sum over 32-blocks b of 2^(ea_b + eb_b) * sum_{k in b} a_k w_k,
+ *          each block sum exact (2^-18 units), the blocks added in binary64
+ *          in K order (error <= K/32 * 2^-53 * sum |terms|, far below the
+ *          binary32 rounding that follows);  C = bf16(fp32(acc) + bias).
+ *   NVFP4: acc = sum over 16-blocks b of dec(sa_b) dec(sw_b) sum_{k in b} a_k w_k,
+ *          exact in 64-bit integers (2^-20 units), rounded once to binary32;
+ *          C = bf16(((acc * g_a) * g_w) + bias), each step binary32.
+ */
+#define QO_FMT_MXFP8 4
+#define QO_FMT_NVFP4 5
+
+/* floor(log2(a)) for a finite a > 0, exact (frexp is exact). */
+static int floor_log2(double a) {
+    int e;
+    (void)frexp(a, &e);                       /* a = f * 2^e, f in [0.5, 1) */
+    return e - 1;
+}
+
+/* E8M0 scale code -> 2^(code - 127); code 0xFF is NaN. */
+double qo_e8m0_decode(uint8_t code) {
+    if (code == 0xFF) return NAN;
+    return ldexp(1.0, (int)code - 127);
+}
+
+/* E2M1 magnitudes by code (bits e1 e0 m): 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+float qo_e2m1_decode(uint8_t code) {
+    double v = kE2M1[code & 7];
+    return (float)((code & 8) ? -v : v);
+}
+
+/* Nearest E2M1 code to v: the magnitude closest to |v| (values above 6 go to
+ * 6), ties to the even code; the sign bit is v's sign, zero included. */
+uint8_t qo_e2m1_encode(float v) {
+    double a = fabs((double)v);
+    if (a > 6.0) a = 6.0;                     /* saturation (keeps the distances exact) */
+    int best = 0;
+    double bd = a;
+    for (int i = 1; i < 8; ++i) {
+        double d = fabs(a - kE2M1[i]);
+        if (d < bd || (d == bd && (i & 1) == 0)) {
+            best = i;
+            bd = d;
+        }
+    }
+    return (uint8_t)((signbit(v) ? 8 : 0) | best);
+}
+
+/*
+ * MXFP8 quantisation.  x: bf16 bits [rows][ld]; cols a multiple of 32.
+ * q: [rows][cols] E4M3 codes; sf: [rows][cols/32] E8M0 codes.
+ */
+void qo_quantize_mxfp8(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* q, uint8_t* sf) {
+    const int64_t nb = cols / 32;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < nb; ++b) {
+            const uint16_t* xb = x + r * ld + b * 32;
+            uint8_t* qb = q + r * cols + b * 32;
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float a = fabsf(qo_bf16_to_f32(xb[i]));
+                if (a > amax) amax = a;
+            }
+            if (amax == 0.0f) {
+                sf[r * nb + b] = 0;
+                memset(qb, 0, 32);
+                continue;
+            }
+            int e = floor_log2((double)amax) - 8;
+            if (e < -127) e = -127;
+            if (e > 127) e = 127;
+            sf[r * nb + b] = (uint8_t)(e + 127);
+            for (int i = 0; i < 32; ++i) {
+                double v = ldexp((double)qo_bf16_to_f32(xb[i]), -e);  /* exact */
+                qb[i] = qo_e4m3_encode((float)v);                      /* saturates at 448 */
+            }
+        }
+}
+
+/*
+ * NVFP4 quantisation with the per-tensor decode scale g > 0.  x: bf16 bits
+ * [rows][ld]; cols a multiple of 16.  q: [rows][cols/2] packed E2M1 (element
+ * 2i in the low nibble of byte i); sf: [rows][cols/16] E4M3 codes.
+ */
+void qo_quantize_nvfp4(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, float g, uint8_t* q,
+                       uint8_t* sf) {
+    const int64_t nb = cols / 16;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < nb; ++b) {
+            const uint16_t* xb = x + r * ld + b * 16;
+            uint8_t* qb = q + r * (cols / 2) + b * 8;
+            float amax = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float a = fabsf(qo_bf16_to_f32(xb[i]));
+                if (a > amax) amax = a;
+            }
+            float t = amax / 6.0f;            /* binary32 division */
+            t = t / g;                        /* binary32 division */
+            const uint8_t s = qo_e4m3_encode(t);
+            sf[r * nb + b] = s;
+            const float d = qo_e4m3_decode(s) * g;   /* binary32 multiply */
+            for (int i = 0; i < 8; ++i) {
+                uint8_t lo = 0, hi = 0;
+                if (d != 0.0f) {
+                    lo = qo_e2m1_encode(qo_bf16_to_f32(xb[2 * i]) / d);
+                    hi = qo_e2m1_encode(qo_bf16_to_f32(xb[2 * i + 1]) / d);
+                }
+                qb[i] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+}
+
+/* E2M1 element of a packed row as an integer count of 1/2. */
+static int64_t e2m1_halves(const uint8_t* row, int64_t k) {
+    const uint8_t code = (uint8_t)((row[k >> 1] >> ((k & 1) * 4)) & 0xF);
+    const int64_t h = (int64_t)(kE2M1[code & 7] * 2.0);
+    return (code & 8) ? -h : h;
+}
+
+/*
+ * Block-scaled GEMM (fmt QO_FMT_MXFP8 or QO_FMT_NVFP4), C = A W^T:
+ *   MXFP8: a_q [M][K], a_sf [M][K/32], w_q [N][K], w_sf [N][K/32]; g_a, g_w unused.
+ *   NVFP4: a_q [M][K/2] packed, a_sf [M][K/16], w_q [N][K/2], w_sf [N][K/16].
+ * K a multiple of 32 (MXFP8) or 16 (NVFP4).  Row/column selection as
+ * qo_scaled_mm.  Returns 0, or -2 if an allocation failed.
+ */
+int qo_gemm_block_scaled(int fmt, int64_t M, int64_t N, int64_t K, const uint8_t* a_q, const uint8_t* a_sf,
+                         const uint8_t* w_q, const uint8_t* w_sf, float g_a, float g_w, const uint16_t* bias,
+                         const int64_t* m_idx, int64_t m_cnt, const int64_t* n_idx, int64_t n_cnt, uint16_t* c) {
+    (void)M;
+    (void)N;
+    if (!m_idx) m_cnt = M;
+    if (!n_idx) n_cnt = N;
+    const int mx = (fmt == QO_FMT_MXFP8);
+    const int64_t bs = mx ? 32 : 16, nb = K / bs;
+    int64_t* ua = (int64_t*)malloc(sizeof(int64_t) * (size_t)(m_cnt * K));
+    int64_t* uw = (int64_t*)malloc(sizeof(int64_t) * (size_t)(n_cnt * K));
+    if (!ua || !uw) { free(ua); free(uw); return -2; }
+    /* elements as exact integers: E4M3 in 2^-9 units, E2M1 in 2^-1 units */
+    for (int64_t i = 0; i < m_cnt; ++i) {
+        const int64_t m = m_idx ? m_idx[i] : i;
+        for (int64_t k = 0; k < K; ++k)
+            ua[i * K + k] = mx ? qo_e4m3_units(a_q[m * K + k]) : e2m1_halves(a_q + m * (K / 2), k);
+    }
+    for (int64_t j = 0; j < n_cnt; ++j) {
+        const int64_t n = n_idx ? n_idx[j] : j;
+        for (int64_t k = 0; k < K; ++k)
+            uw[j * K + k] = mx ? qo_e4m3_units(w_q[n * K + k]) : e2m1_halves(w_q + n * (K / 2), k);
+    }
+    for (int64_t i = 0; i < m_cnt; ++i) {
+        const int64_t m = m_idx ? m_idx[i] : i;
+        for (int64_t j = 0; j < n_cnt; ++j) {
+            const int64_t n = n_idx ? n_idx[j] : j;
+            const int64_t* ra = ua + i * K;
+            const int64_t* rw = uw + j * K;
+            float y;
+            if (mx) {
+                double acc = 0.0;
+                for (int64_t b = 0; b < nb; ++b) {
+                    int64_t p = 0;
+                    for (int64_t k = b * 32; k < b * 32 + 32; ++k) p += ra[k] * rw[k];
+                    acc += ldexp((double)p, -18) * qo_e8m0_decode(a_sf[m * nb + b])
+                           * qo_e8m0_decode(w_sf[n * nb + b]);
+                }
+                y = (float)acc;               /* one rounding to binary32 */
+                if (bias) y = y + qo_bf16_to_f32(bias[n]);
+            } else {
+                int64_t acc = 0;              /* 2^-20 units: 2^-2 elements x 2^-18 scales */
+                for (int64_t b = 0; b < nb; ++b) {
+                    int64_t p = 0;
+                    for (int64_t k = b * 16; k < b * 16 + 16; ++k) p += ra[k] * rw[k];
+                    acc += p * qo_e4m3_units(a_sf[m * nb + b]) * qo_e4m3_units(w_sf[n * nb + b]);
+                }
+                y = (float)acc;               /* int64 -> binary32, one rounding */
+                y = y * 0x1p-20f;             /* exact power-of-two scaling */
+                y = y * g_a;
+                y = y * g_w;
+                if (bias) y = y + qo_bf16_to_f32(bias[n]);
+            }
+            c[i * n_cnt + j] = qo_f32_to_bf16(y);
+        }
+    }
+    free(ua);
+    free(uw);
+    return 0;
 }
