@@ -43,7 +43,7 @@
 extern "C" {
 #endif
 
-#define QLIN_ABI_VERSION 6
+#define QLIN_ABI_VERSION 7
 
 #if defined(__GNUC__)
 #define QLIN_API __attribute__((visibility("default")))
@@ -71,9 +71,14 @@ typedef enum {
     QLIN_FMT_INT8 = 0,       /* W8A8 INT8, per-token / per-channel scales, int32 accumulate */
     QLIN_FMT_FP8 = 1,        /* e4m3, per-token / per-channel scales, fp32 accumulate */
     QLIN_FMT_FP8_BLOCK = 2,  /* e4m3, 1x128 activation groups, 128x128 weight blocks */
-    QLIN_FMT_BF16 = 3        /* bf16 operands, no scales, fp32 accumulate (qlin_matmul_bf16 only;
+    QLIN_FMT_BF16 = 3,       /* bf16 operands, no scales, fp32 accumulate (qlin_matmul_bf16 only;
                                 also accepted by qlin_scaled_mm_workspace_size and
                                 qlin_dispatch_query) */
+    QLIN_FMT_MXFP8 = 4,      /* e4m3, one E8M0 scale per 32 elements of K (qlin_quantize_block_scaled,
+                                qlin_block_scaled_mm; also qlin_scaled_mm_workspace_size and
+                                qlin_dispatch_query) */
+    QLIN_FMT_NVFP4 = 5       /* packed e2m1, one E4M3 scale per 16 elements of K and one fp32
+                                scale per tensor (as QLIN_FMT_MXFP8) */
 } qlin_format;
 
 typedef enum {
@@ -475,6 +480,93 @@ QLIN_API qlin_status qlin_sync_status(qlin_stream_t stream);
  * Errors: INVALID_ARG, CUDA, NO_DEVICE.
  */
 QLIN_API qlin_status qlin_selftest_wait_timeout(uint32_t limit_us, qlin_stream_t stream);
+
+/*
+ * Block-scaled formats.  The page "Helion in vLLM: A Unified Route to Tunable
+ * Linear Kernels" (introduction) lists NVFP4 among the formats vLLM's quantized
+ * linear layers serve; neither it nor MXFP8 is defined there.  These entry
+ * points follow the formats' public definitions:
+ *
+ *   MXFP8 (OCP Microscaling Formats v1.0): blocks of 32 consecutive elements
+ *     along K share one E8M0 scale X = 2^(code - 127).  Quantisation: amax =
+ *     max |x| of the block; amax == 0 gives code 0 and zero elements;
+ *     otherwise e = floor(log2(amax)) - 8, clamped to [-127, 127], code e + 127,
+ *     q = e4m3(x * 2^-e) (nearest, ties to even, saturating at +-448).
+ *   NVFP4: blocks of 16 elements along K share one E4M3 scale s, and the
+ *     tensor has one fp32 decode scale g (x ~ q * s * g).  Quantisation: s =
+ *     e4m3((amax / 6) / g) (two binary32 divisions, then nearest, saturating at
+ *     448); d = s * g (binary32); d == 0 gives zero elements; otherwise q =
+ *     e2m1(x / d) (binary32 division, nearest of +-{0, .5, 1, 1.5, 2, 3, 4, 6},
+ *     ties to even, saturating at 6).  Two elements per byte, element 2i in
+ *     the low nibble.
+ *
+ * Scale-factor layout ("tiled", what the tensor cores read): rows are grouped
+ * by 128 and K by atoms of 4 scale factors (128 elements for MXFP8, 64 for
+ * NVFP4).  Each (row group, atom) is one 512-byte block, stored row group
+ * major, atom minor: sf[(r / 128) * atoms + a][512], and inside it the scale
+ * of row r and sub-block j (0..3) of the atom sits at byte
+ * (r % 32) * 16 + ((r / 32) % 4) * 4 + j.  atoms = K / 128 (MXFP8) or K / 64
+ * (NVFP4); the buffer holds ceil(rows / 128) * atoms * 512 bytes.  The bytes
+ * of rows past the last row are never written; whatever they hold only
+ * reaches outputs that are not stored.
+ */
+
+/*
+ * qlin_quantize_block_scaled -- MXFP8 or NVFP4 quantisation of a bf16 matrix
+ * (activations per call; weights once, offline), arithmetic as above.
+ *
+ *   fmt        QLIN_FMT_MXFP8 or QLIN_FMT_NVFP4
+ *   x          bf16 [rows, ld_x] (device)
+ *   rows, cols rows >= 0 (0 is a no-op); cols % 128 == 0
+ *   ld_x       row stride of x in elements, >= cols, ld_x % 8 == 0
+ *   g          NVFP4: fp32 [1] (device), the tensor's decode scale, > 0 and
+ *              finite; MXFP8: NULL
+ *   q_out      MXFP8: e4m3 [rows, cols]; NVFP4: uint8 [rows, cols / 2] (device)
+ *   sf_out     tiled scale factors, ceil(rows/128) * atoms * 512 bytes (device)
+ *   flags      0 or QLIN_PDL
+ * Inputs must be finite.  Alignment: x, q_out, sf_out 16-byte aligned; g 4.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA.
+ */
+QLIN_API qlin_status qlin_quantize_block_scaled(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                                                const float* g, void* q_out, void* sf_out, uint32_t flags,
+                                                qlin_stream_t stream);
+
+/*
+ * qlin_block_scaled_mm -- the GEMM of the block-scaled formats on the tcgen05
+ * block-scaled MMA (kind::mxf8f6f4 with E8M0 scales, kind::mxf4nvf4 with E4M3
+ * scales over 16-element blocks), which applies the scale factors inside the
+ * tensor core:
+ *
+ *   MXFP8:  C[m,n] = bf16( acc[m,n] + bias[n] )
+ *   NVFP4:  C[m,n] = bf16( ((acc[m,n] * g_a) * g_w) + bias[n] )
+ *           acc[m,n] = sum over blocks of (block scales) * sum_k a_q w_q, fp32
+ *
+ * Plain and Split-K tiles of 128 x 128 (no Swap-AB or pair tiles); K is cut
+ * into k_segments segments added in order from +0, as in qlin_scaled_mm, so
+ * rows of C do not depend on M.  The dispatch table's entries are keyed
+ * "mxfp8" / "nvfp4".
+ *
+ *   fmt                 QLIN_FMT_MXFP8 or QLIN_FMT_NVFP4
+ *   variant             AUTO, PLAIN or SPLITK;  tile_n 0 or 128;  k_segments as qlin_scaled_mm
+ *   M, N, K             M >= 0 (0 is a no-op), N >= 16, N % 16 == 0;
+ *                       K % 128 == 0 (MXFP8) or K % 256 == 0 (NVFP4)
+ *   a_q, a_sf           A codes [M, K] (NVFP4: [M, K/2] packed) and tiled scales (device)
+ *   w_q, w_sf           W codes [N, K] (NVFP4: [N, K/2]) and tiled scales (device)
+ *   g_a, g_w            NVFP4: fp32 [1] each (device), the tensors' decode scales;
+ *                       MXFP8: NULL
+ *   bias                bf16 [N] (device) or NULL
+ *   c_out               bf16 [M, N] (device)
+ *   flags               QLIN_PDL
+ *   workspace           as qlin_scaled_mm (size from qlin_scaled_mm_workspace_size
+ *                       with the same fmt)
+ * Alignment: a_q, a_sf, w_q, w_sf, c_out, workspace 16-byte aligned; g 4; bias 2.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA, NO_DEVICE.
+ */
+QLIN_API qlin_status qlin_block_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N,
+                                          int64_t K, const void* a_q, const void* a_sf, const void* w_q,
+                                          const void* w_sf, const float* g_a, const float* g_w, const void* bias,
+                                          void* c_out, uint32_t flags, void* workspace, size_t workspace_bytes,
+                                          qlin_stream_t stream);
 
 /* ABI version of the loaded library (QLIN_ABI_VERSION at build time). */
 QLIN_API int qlin_abi_version(void);

@@ -25,7 +25,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "-I", INCLUDE, "-I", CSRC, "--expt-relaxed-constexpr"]
-SOURCES = ["quantize.cu", "gemm.cu", "api.cu", "noalloc.cu", "moe.cu"]
+SOURCES = ["quantize.cu", "quantize_bs.cu", "gemm.cu", "api.cu", "noalloc.cu", "moe.cu"]
 HEADERS = ["ptx.cuh", "internal.h", "pdl.cuh", "quant_math.cuh"]
 
 

@@ -54,6 +54,8 @@ const char* fmt_name(int f) {
         case QLIN_FMT_FP8: return "fp8";
         case QLIN_FMT_FP8_BLOCK: return "fp8_block";
         case QLIN_FMT_BF16: return "bf16";
+        case QLIN_FMT_MXFP8: return "mxfp8";
+        case QLIN_FMT_NVFP4: return "nvfp4";
     }
     return "?";
 }
@@ -63,6 +65,8 @@ int parse_fmt(const std::string& s) {
     if (s == "fp8") return QLIN_FMT_FP8;
     if (s == "fp8_block") return QLIN_FMT_FP8_BLOCK;
     if (s == "bf16") return QLIN_FMT_BF16;
+    if (s == "mxfp8") return QLIN_FMT_MXFP8;
+    if (s == "nvfp4") return QLIN_FMT_NVFP4;
     return -1;
 }
 
@@ -95,6 +99,7 @@ bool runs_as_cluster(int variant, int tile_n, int S) {
 }
 
 bool tile_supported(int fmt, bool swap, int tile_n, bool pair = false) {
+    if (is_block_scaled(fmt)) return !swap && !pair && tile_n == 128;
     if (pair) return fmt != QLIN_FMT_FP8_BLOCK && tile_n == 256;
     if (swap) return tile_n == 16 || tile_n == 32 || tile_n == 64;
     if (fmt == QLIN_FMT_FP8_BLOCK) return tile_n == 128;
@@ -114,20 +119,21 @@ int default_segments(int fmt, int64_t N, int64_t K, int num_sms) {
     return best;
 }
 
-// Bytes of one operand row and 128-byte K blocks: 8-bit formats 1 B/element, bf16 2.
-int64_t row_bytes(int fmt, int64_t K) { return fmt == QLIN_FMT_BF16 ? 2 * K : K; }
+// Bytes of one operand row and 128-byte K blocks: 8-bit formats 1 B/element,
+// bf16 2, packed NVFP4 1/2.
+int64_t row_bytes(int fmt, int64_t K) { return fmt == QLIN_FMT_BF16 ? 2 * K : (fmt == QLIN_FMT_NVFP4 ? K / 2 : K); }
 
 qlin_config default_config(int fmt, int64_t M, int64_t N, int64_t K, int num_sms) {
     qlin_config c{};
     c.k_segments = default_segments(fmt, N, row_bytes(fmt, K), num_sms);
     c.from_table = 0;
     c.m_max = 0;
-    if (M <= 64) {
+    if (M <= 64 && !is_block_scaled(fmt)) {
         c.tile_n = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
         c.variant = c.k_segments > 1 ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB;
     } else {
-        const bool multi =
-            fmt == QLIN_FMT_FP8_BLOCK || ((fmt == QLIN_FMT_FP8 || fmt == QLIN_FMT_BF16) && c.k_segments > 1);
+        const bool multi = fmt == QLIN_FMT_FP8_BLOCK || is_block_scaled(fmt) ||
+                           ((fmt == QLIN_FMT_FP8 || fmt == QLIN_FMT_BF16) && c.k_segments > 1);
         c.tile_n = multi ? 128 : 256;
         const int64_t tiles = ((M + 127) / 128) * ((N + c.tile_n - 1) / c.tile_n);
         c.variant = (c.k_segments > 1 && tiles * 2 <= num_sms) ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN;
@@ -188,8 +194,9 @@ qlin_status resolve_config(int fmt, int variant, int tile_n, int k_segments, int
 }  // namespace
 
 qlin_status check_fmt_shape(int fmt, int64_t M, int64_t N, int64_t K) {
-    if (fmt < QLIN_FMT_INT8 || fmt > QLIN_FMT_BF16) return QLIN_ERR_INVALID_ARG;
-    const int64_t kunit = fmt == QLIN_FMT_BF16 ? 64 : 128;  // elements per 128-byte K block
+    if (fmt < QLIN_FMT_INT8 || fmt > QLIN_FMT_NVFP4) return QLIN_ERR_INVALID_ARG;
+    // elements per 128-byte K block
+    const int64_t kunit = fmt == QLIN_FMT_BF16 ? 64 : (fmt == QLIN_FMT_NVFP4 ? 256 : 128);
     if (M < 0 || N < 16 || K < kunit) return QLIN_ERR_INVALID_ARG;
     if (N % 16 != 0 || K % kunit != 0) return QLIN_ERR_UNSUPPORTED;
     if (fmt == QLIN_FMT_FP8_BLOCK && N % 128 != 0) return QLIN_ERR_UNSUPPORTED;
@@ -236,8 +243,9 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     p.kb_per_seg = p.kblocks / p.k_segments;
     // units with more than one accumulator chunk keep tile_n fp32 values per
     // thread and a TMEM running total: only tiles up to 128 columns do that
-    const bool multi_chunk = (fmt == QLIN_FMT_FP8_BLOCK && (p.spread ? p.kb_per_seg : p.kblocks) > 1) ||
-                             ((fmt == QLIN_FMT_FP8 || fmt == QLIN_FMT_BF16) && !p.spread && p.k_segments > 1);
+    const bool multi_chunk =
+        (fmt == QLIN_FMT_FP8_BLOCK && (p.spread ? p.kb_per_seg : p.kblocks) > 1) ||
+        ((fmt == QLIN_FMT_FP8 || fmt == QLIN_FMT_BF16 || is_block_scaled(fmt)) && !p.spread && p.k_segments > 1);
     if (multi_chunk && p.tile_n > 128) return QLIN_ERR_UNSUPPORTED;
     p.kb_per_unit = p.spread ? p.kb_per_seg : p.kblocks;
     p.mode = pair ? kModePair : kModeStd;
@@ -389,7 +397,7 @@ qlin_status qlin_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int
                            const void* a_q, const float* s_a, const void* w_q, const float* s_w, const void* bias,
                            void* c_out, uint32_t flags, void* workspace, size_t workspace_bytes,
                            qlin_stream_t stream) {
-    if (fmt == QLIN_FMT_BF16) return QLIN_ERR_INVALID_ARG;  // qlin_matmul_bf16
+    if (fmt == QLIN_FMT_BF16 || is_block_scaled(fmt)) return QLIN_ERR_INVALID_ARG;  // qlin_matmul_bf16 / _block_scaled_mm
     qlin_status st = check_fmt_shape(fmt, M, N, K);
     if (st != QLIN_OK) return st;
     if (flags & ~(QLIN_OUT_I32ACC | QLIN_PDL | QLIN_SPLITK_CLUSTER)) return QLIN_ERR_INVALID_ARG;
@@ -429,7 +437,7 @@ qlin_status qlin_linear(int fmt, int variant, int tile_n, int k_segments, int64_
                         const void* x, int64_t ld_x, void* a_q, float* s_a, const void* w_q, const float* s_w,
                         const void* bias, void* c_out, uint32_t flags, void* workspace, size_t workspace_bytes,
                         qlin_stream_t stream) {
-    if (fmt == QLIN_FMT_BF16) return QLIN_ERR_INVALID_ARG;  // no quantisation step
+    if (fmt == QLIN_FMT_BF16 || is_block_scaled(fmt)) return QLIN_ERR_INVALID_ARG;  // per-token / Block-FP8 only
     qlin_status st = check_fmt_shape(fmt, M, N, K);
     if (st != QLIN_OK) return st;
     if (flags & ~(QLIN_OUT_I32ACC | QLIN_PDL | QLIN_FUSED)) return QLIN_ERR_INVALID_ARG;
@@ -510,6 +518,64 @@ qlin_status qlin_matmul_bf16(int variant, int tile_n, int k_segments, int64_t M,
                                            : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
                      p.mode == kModeCluster ? " (cluster)" : "", p.tile_n, p.k_segments, p.grid);
     GemmOperands ops{a, nullptr, w, nullptr, bias, c_out, false, workspace, (flags & QLIN_PDL) != 0};
+    return launch_gemm(p, ops, static_cast<cudaStream_t>(stream));
+}
+
+qlin_status qlin_quantize_block_scaled(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                                       const float* g, void* q_out, void* sf_out, uint32_t flags,
+                                       qlin_stream_t stream) {
+    if (!is_block_scaled(fmt)) return QLIN_ERR_INVALID_ARG;
+    if (flags & ~QLIN_PDL) return QLIN_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 1 || ld_x < cols) return QLIN_ERR_INVALID_ARG;
+    if ((fmt == QLIN_FMT_NVFP4) != (g != nullptr)) return QLIN_ERR_INVALID_ARG;
+    if (cols % 128 != 0) return QLIN_ERR_UNSUPPORTED;
+    if (rows > (int64_t)1 << 34 || cols > (int64_t)1 << 24) return QLIN_ERR_UNSUPPORTED;
+    if (rows == 0) return QLIN_OK;
+    if (!x || !q_out || !sf_out) return QLIN_ERR_INVALID_ARG;
+    if (ld_x % 8 != 0 || !aligned16(x) || !aligned16(q_out) || !aligned16(sf_out) ||
+        (reinterpret_cast<uintptr_t>(g) & 3u))
+        return QLIN_ERR_ALIGNMENT;
+    cudaError_t e = launch_quantize_block_scaled(fmt, x, rows, cols, ld_x, g, q_out, sf_out, (flags & QLIN_PDL) != 0,
+                                                 static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? QLIN_OK : QLIN_ERR_CUDA;
+}
+
+qlin_status qlin_block_scaled_mm(int fmt, int variant, int tile_n, int k_segments, int64_t M, int64_t N, int64_t K,
+                                 const void* a_q, const void* a_sf, const void* w_q, const void* w_sf,
+                                 const float* g_a, const float* g_w, const void* bias, void* c_out, uint32_t flags,
+                                 void* workspace, size_t workspace_bytes, qlin_stream_t stream) {
+    if (!is_block_scaled(fmt)) return QLIN_ERR_INVALID_ARG;
+    qlin_status st = check_fmt_shape(fmt, M, N, K);
+    if (st != QLIN_OK) return st;
+    if (flags & ~QLIN_PDL) return QLIN_ERR_INVALID_ARG;
+    if (variant != QLIN_VAR_AUTO && variant != QLIN_VAR_PLAIN && variant != QLIN_VAR_SPLITK)
+        return variant < QLIN_VAR_AUTO || variant > QLIN_VAR_PAIR ? QLIN_ERR_INVALID_ARG : QLIN_ERR_UNSUPPORTED;
+    if (tile_n < 0 || k_segments < 0) return QLIN_ERR_INVALID_ARG;
+    const bool nv = fmt == QLIN_FMT_NVFP4;
+    if (nv != (g_a != nullptr) || nv != (g_w != nullptr)) return QLIN_ERR_INVALID_ARG;
+    if (M == 0) return QLIN_OK;
+    if (!a_q || !a_sf || !w_q || !w_sf || !c_out) return QLIN_ERR_INVALID_ARG;
+    if (!aligned16(a_q) || !aligned16(a_sf) || !aligned16(w_q) || !aligned16(w_sf) || !aligned16(c_out))
+        return QLIN_ERR_ALIGNMENT;
+    if ((reinterpret_cast<uintptr_t>(g_a) & 3u) || (reinterpret_cast<uintptr_t>(g_w) & 3u) ||
+        (reinterpret_cast<uintptr_t>(bias) & 1u))
+        return QLIN_ERR_ALIGNMENT;
+    const int sms = current_device_sms();
+    if (sms <= 0) return QLIN_ERR_NO_DEVICE;
+    GemmPlan p;
+    st = make_gemm_plan(fmt, variant, tile_n, k_segments, M, N, K, sms, kModeStd, &p);
+    if (st != QLIN_OK) return st;
+    if (p.workspace_bytes) {
+        if (!workspace || workspace_bytes < p.workspace_bytes) return QLIN_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return QLIN_ERR_ALIGNMENT;
+    }
+    if (g_log)
+        std::fprintf(stderr, "[qlin] block_scaled_mm %s M=%lld N=%lld K=%lld -> %s tile_n=%d S=%d grid=%d\n",
+                     fmt_name(fmt), (long long)M, (long long)N, (long long)K,
+                     variant_name(p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN), p.tile_n, p.k_segments, p.grid);
+    GemmOperands ops{a_q, g_a, w_q, g_w, bias, c_out, false, workspace, (flags & QLIN_PDL) != 0};
+    ops.sf_a = a_sf;
+    ops.sf_w = w_sf;
     return launch_gemm(p, ops, static_cast<cudaStream_t>(stream));
 }
 

@@ -87,6 +87,11 @@ struct GemmArgs {
     // [e N, e N + N); nullptr / 0 for an ordinary GEMM
     const int32_t* moe_offsets;
     int moe_E;
+    // block-scaled formats (MXFP8, NVFP4): tiled scale factors of A and W,
+    // 512-byte atoms [row group][atom], sf_atoms atoms per 128-row group
+    const uint8_t* sf_a;
+    const uint8_t* sf_w;
+    int sf_atoms;
 };
 
 constexpr int kMoeMaxExperts = kMoeMaxE;
@@ -139,12 +144,23 @@ struct Cfg {
     static constexpr bool INT8 = (FMT == QLIN_FMT_INT8);
     static constexpr bool BLOCK = (FMT == QLIN_FMT_FP8_BLOCK);
     static constexpr bool BF16 = (FMT == QLIN_FMT_BF16);  // bf16 operands: no scales
-    static constexpr int KIND = INT8 ? kKindI8 : (BF16 ? kKindF16 : kKindF8);
+    // block-scaled (MXFP8, NVFP4): the tensor core applies per-block scale
+    // factors that the MMA thread copies from shared memory into TMEM
+    static constexpr bool BS = is_block_scaled(FMT);
+    static_assert(!BS || (!SWAP && !CSK && !FUSE && !PAIR && BN == 128), "block-scaled formats: plain 128 x 128 tiles");
+    static constexpr int KIND =
+        BS ? (FMT == QLIN_FMT_MXFP8 ? kKindMXF8 : kKindNVF4) : (INT8 ? kKindI8 : (BF16 ? kKindF16 : kKindF8));
+    // scale-factor atoms (512 B: 128 rows x 4 scales) per 128-byte K block of
+    // one 128-row group: MXFP8 1 (128 elements), NVFP4 4 (256 elements)
+    static constexpr int SF_APK = FMT == QLIN_FMT_NVFP4 ? 4 : 1;
+    static constexpr int SFA_BYTES = BS ? 512 * SF_APK : 0;
+    static constexpr int SFB_BYTES = BS ? 512 * SF_APK * (BN / 128) : 0;
+    static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;
     static constexpr int BM = 128;                 // P rows per tile (MMA M)
     static constexpr int BK = 128;                 // K bytes per stage: one swizzle atom
     static constexpr int P_BYTES = BM * BK;
     static constexpr int Q_BYTES = (PAIR ? BN / 2 : BN) * BK;
-    static constexpr int STAGE_BYTES = P_BYTES + (FUSE ? 0 : Q_BYTES);
+    static constexpr int STAGE_BYTES = P_BYTES + (FUSE ? 0 : Q_BYTES) + SF_BYTES;
     // FUSE: A codes of one unit, [K block][BN rows x 128 B] in the 128-byte
     // swizzled K-major layout, and the unit's activation scales (2 buffers)
     static constexpr int A_BYTES = FUSE ? 65536 : 0;
@@ -168,10 +184,13 @@ struct Cfg {
     static constexpr int NACC = (BLOCK && !SWAP) ? 3 : 2;
     static constexpr int SEG_COL = 2 * ACC_COLS;   // Block-FP8 Swap-AB: running segment sum
     static constexpr int TOTAL_COL = (BLOCK ? 3 : 2) * ACC_COLS;  // running total over segments
-    static constexpr int TMEM_COLS = pow2_at_least(NACC * ACC_COLS + (MULTI ? ACC_COLS : 0) +
-                                                   ((BLOCK && SWAP) ? ACC_COLS : 0));
+    // block-scaled: two copies (alternate K blocks) of one K block's scale
+    // factors, 4 columns per atom, after the accumulators and running total
+    static constexpr int SF_COL = NACC * ACC_COLS + (MULTI ? ACC_COLS : 0) + ((BLOCK && SWAP) ? ACC_COLS : 0);
+    static constexpr int SF_COLS = BS ? 4 * SF_APK * (1 + BN / 128) : 0;
+    static constexpr int TMEM_COLS = pow2_at_least(SF_COL + 2 * SF_COLS);
     static_assert(NACC * ACC_COLS <= TOTAL_COL, "accumulators overlap the running total");
-    static constexpr uint32_t IDESC = make_idesc(KIND, PAIR ? 256 : 128, BN);
+    static constexpr uint32_t IDESC = BS ? make_idesc_bs(KIND, 128, BN) : make_idesc(KIND, PAIR ? 256 : 128, BN);
     static constexpr size_t STAGING_OFF = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t SCALE_OFF = STAGING_OFF + kStagingBytes;
     static constexpr size_t BSCALE_OFF = SCALE_OFF + kScaleBytes;
@@ -888,6 +907,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sP = smem;
     uint8_t* sQ = smem + (size_t)STAGES * C::P_BYTES;
+    uint8_t* sF = sQ + (size_t)STAGES * C::Q_BYTES;  // block-scaled: per stage, A's then W's scale atoms
     float* s_col = reinterpret_cast<float*>(smem + C::SCALE_OFF);
     float* b_col = s_col + 256;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
@@ -1025,12 +1045,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(dst, m, x, y, fb, pol);
             };
             auto load_w = [&](uint32_t stage, const Unit& un, int kb, uint32_t fb) {
-                if constexpr (SWAP)
+                if constexpr (SWAP) {
                     load(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_w, kb * 128, un.wrow0 + un.pt * 128, fb,
                          pol_w);
-                else
+                } else {
                     load(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_w, kb * 128,
                          un.wrow0 + un.qt * BN + w_row_off, fb, pol_w);
+                    if constexpr (C::BS) {  // the W tile's scale atoms of this K block
+#pragma unroll
+                        for (int j = 0; j < BN / 128; ++j)
+                            bulk_load(smem_u32(sF + (size_t)stage * C::SF_BYTES + C::SFA_BYTES + j * 512 * C::SF_APK),
+                                      args.sf_w + ((size_t)(un.qt * (BN / 128) + j) * args.sf_atoms +
+                                                   (size_t)kb * C::SF_APK) * 512u,
+                                      512u * C::SF_APK, fb, pol_w);
+                    }
+                }
             };
             // weights do not depend on the previous kernel: start streaming the
             // first unit's weight tiles before waiting for it
@@ -1064,6 +1093,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     else
                         load(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_a, kb * 128, un.row0 + un.pt * 128, fb,
                              pol_a);
+                    if constexpr (C::BS)  // the A tile's scale atoms of this K block
+                        bulk_load(smem_u32(sF + (size_t)stage * C::SF_BYTES),
+                                  args.sf_a + ((size_t)un.pt * args.sf_atoms + (size_t)kb * C::SF_APK) * 512u,
+                                  (uint32_t)C::SFA_BYTES, fb, pol_a);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1;
@@ -1077,6 +1110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (PAIR: rank 0 issues for both CTAs; rank 1's MMA warp only holds TMEM)
         if (lane == 0 && (!PAIR || rank == 0)) {
             uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0, uphase = 0;
+            uint32_t sfi = 0;  // block-scaled: K blocks issued, picks the TMEM copy of the scale factors
             for (int u = u_first; u < units; u += u_step) {
                 const Unit un = decode_unit<FMT, PAIR, SWAP, BN>(args, u, rank, moe);
                 if constexpr (FUSE) {
@@ -1098,13 +1132,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint64_t bdesc =
                             FUSE ? smem_desc_k_sw128(sA + (uint32_t)((kb - un.kb0) * BN * 128))
                                  : smem_desc_k_sw128(smem_u32(sQ + (size_t)stage * C::Q_BYTES));
+                        if constexpr (C::BS) {
+                            // this K block's scale factors into TMEM (the tensor pipe runs the
+                            // copies and the MMAs in issue order); A's atoms, then W's, 4
+                            // columns each: [atom][row group]
+                            constexpr int RG = BN / 128;
+                            const uint32_t sfa_t = tmem_base + C::SF_COL + (sfi & 1u) * C::SF_COLS;
+                            const uint32_t sfb_t = sfa_t + 4 * C::SF_APK;
+                            const uint32_t sfs = smem_u32(sF + (size_t)stage * C::SF_BYTES);
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {  // 4 x K=32 bytes per 128-byte stage
-                            const uint32_t accum = (kb > c0 || k > 0) ? 1u : 0u;
-                            if constexpr (PAIR)
-                                tc_mma_pair<C::KIND>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
-                            else
-                                tc_mma<C::KIND>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
+                            for (int at = 0; at < C::SF_APK; ++at) {
+                                tc_cp_sf(sfa_t + 4 * at, smem_desc_sf(sfs + 512 * at));
+#pragma unroll
+                                for (int j = 0; j < RG; ++j)
+                                    tc_cp_sf(sfb_t + 4 * (at * RG + j),
+                                             smem_desc_sf(sfs + C::SFA_BYTES + 512 * (j * C::SF_APK + at)));
+                            }
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const uint32_t accum = (kb > c0 || k > 0) ? 1u : 0u;
+                                if constexpr (C::KIND == kKindMXF8)  // byte k of the atom's column: sub-block k
+                                    tc_mma_bs<C::KIND>(d, adesc + 2 * k, bdesc + 2 * k,
+                                                       idesc_sf_ids(C::IDESC, (uint32_t)k, (uint32_t)k), sfa_t, sfb_t,
+                                                       accum);
+                                else  // one atom (four 16-element blocks) per MMA
+                                    tc_mma_bs<C::KIND>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, sfa_t + 4 * k,
+                                                       sfb_t + 4 * k * RG, accum);
+                            }
+                            ++sfi;
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {  // 4 x K=32 bytes per 128-byte stage
+                                const uint32_t accum = (kb > c0 || k > 0) ? 1u : 0u;
+                                if constexpr (PAIR)
+                                    tc_mma_pair<C::KIND>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
+                                else
+                                    tc_mma<C::KIND>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
+                            }
                         }
                         if constexpr (PAIR)
                             tc_commit_pair(empty0 + 8 * stage, 0x3);  // both CTAs may refill the stage
@@ -1208,7 +1272,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = threadIdx.x; c < BN; c += kEpiThreads) {
                     const int q = un.qt * BN + c;
                     if constexpr (!SWAP) {
-                        if constexpr (!C::BF16) s_col[c] = q < args.N ? __ldg(args.s_w + un.wrow0 + q) : 0.f;
+                        if constexpr (C::BS)  // NVFP4: W's decode scale; MXFP8: none (exact * 1)
+                            s_col[c] = FMT == QLIN_FMT_NVFP4 ? __ldg(args.s_w) : 1.f;
+                        else if constexpr (!C::BF16)
+                            s_col[c] = q < args.N ? __ldg(args.s_w + un.wrow0 + q) : 0.f;
                         b_col[c] = (e.has_bias && q < args.N) ? bf16_to_f32(__ldg(args.bias + q)) : 0.f;
                     } else if constexpr (FUSE) {
                         s_col[c] = sa_cur[c];
@@ -1218,7 +1285,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if constexpr (!SWAP) {
                     const int m = un.pt * 128 + e.row_lane;
-                    if constexpr (!C::BF16) e.row_scale = m < un.rows ? __ldg(args.s_a + un.row0 + m) : 0.f;
+                    if constexpr (C::BS)
+                        e.row_scale = FMT == QLIN_FMT_NVFP4 ? __ldg(args.s_a) : 1.f;
+                    else if constexpr (!C::BF16)
+                        e.row_scale = m < un.rows ? __ldg(args.s_a + un.row0 + m) : 0.f;
                 } else {
                     const int n = un.pt * 128 + e.row_lane;
                     if constexpr (!C::BF16) e.row_scale = n < args.N ? __ldg(args.s_w + un.wrow0 + n) : 0.f;
@@ -1556,6 +1626,9 @@ qlin_status launch_instance(const GemmPlan& plan, const GemmOperands& ops, cudaS
     a.s_a_out = FUSE ? const_cast<float*>(ops.s_a) : nullptr;
     a.moe_offsets = ops.moe_offsets;
     a.moe_E = plan.moe_E;
+    a.sf_a = static_cast<const uint8_t*>(ops.sf_a);
+    a.sf_w = static_cast<const uint8_t*>(ops.sf_w);
+    a.sf_atoms = plan.kblocks * C::SF_APK;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)plan.grid);
@@ -1604,6 +1677,11 @@ void cfg_info(int* stages, size_t* smem) {
 // is applied to the one matching (swap, tile_n, mode); false if none exists.
 template <int FMT, template <int, bool, int, bool, bool, bool> class OP, typename... A>
 bool dispatch_instance(bool swap, int tile_n, int mode, A&&... args) {
+    if constexpr (is_block_scaled(FMT)) {  // plain / Split-K 128 x 128 tiles only
+        if (swap || mode != kModeStd || tile_n != 128) return false;
+        OP<FMT, false, 128, false, false, false>::run(args...);
+        return true;
+    } else {
     if (swap) {
         switch (mode * 1000 + tile_n) {
             case kModeStd * 1000 + 16: OP<FMT, true, 16, false, false, false>::run(args...); return true;
@@ -1643,6 +1721,7 @@ bool dispatch_instance(bool swap, int tile_n, int mode, A&&... args) {
         }
     }
     return false;
+    }
 }
 
 template <int FMT, bool SWAP, int BN, bool CSK, bool FUSE, bool PAIR>
@@ -1673,6 +1752,8 @@ bool gemm_kernel_info(int fmt, bool swap, int tile_n, int mode, int* stages, siz
         case QLIN_FMT_FP8_BLOCK:
             return dispatch_instance<QLIN_FMT_FP8_BLOCK, InfoOp>(swap, tile_n, mode, stages, smem_bytes);
         case QLIN_FMT_BF16: return dispatch_instance<QLIN_FMT_BF16, InfoOp>(swap, tile_n, mode, stages, smem_bytes);
+        case QLIN_FMT_MXFP8: return dispatch_instance<QLIN_FMT_MXFP8, InfoOp>(swap, tile_n, mode, stages, smem_bytes);
+        case QLIN_FMT_NVFP4: return dispatch_instance<QLIN_FMT_NVFP4, InfoOp>(swap, tile_n, mode, stages, smem_bytes);
     }
     return false;
 }
@@ -1708,6 +1789,8 @@ qlin_status launch_gemm(const GemmPlan& plan, const GemmOperands& ops, cudaStrea
         case QLIN_FMT_FP8: return launch_fmt<QLIN_FMT_FP8>(plan, ops, st);
         case QLIN_FMT_FP8_BLOCK: return launch_fmt<QLIN_FMT_FP8_BLOCK>(plan, ops, st);
         case QLIN_FMT_BF16: return launch_fmt<QLIN_FMT_BF16>(plan, ops, st);
+        case QLIN_FMT_MXFP8: return launch_fmt<QLIN_FMT_MXFP8>(plan, ops, st);
+        case QLIN_FMT_NVFP4: return launch_fmt<QLIN_FMT_NVFP4>(plan, ops, st);
         default: return QLIN_ERR_INVALID_ARG;
     }
 }

@@ -39,6 +39,10 @@ cudaError_t launch_quantize_per_token(int fmt, const void* x, int64_t rows, int6
                                       float* s, bool pdl, cudaStream_t st);
 cudaError_t launch_quantize_block(const void* x, int64_t rows, int64_t cols, int64_t ld, int block_rows, void* q,
                                   float* s, bool pdl, cudaStream_t st);
+// MXFP8 / NVFP4 codes and tiled scale factors (g: NVFP4's device-side decode scale)
+cudaError_t launch_quantize_block_scaled(int fmt, const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                         const float* g, void* q, void* sf, bool pdl, cudaStream_t st);
+__host__ __device__ constexpr bool is_block_scaled(int fmt) { return fmt == QLIN_FMT_MXFP8 || fmt == QLIN_FMT_NVFP4; }
 
 // ------------------------------------------------------------------- GEMM
 // A fully resolved GEMM launch: which operand feeds the 128-row MMA side
@@ -98,6 +102,10 @@ struct GemmOperands {
     const void* x = nullptr;  // fused mode: bf16 activations [M, K], row stride ld_x elements
     int64_t ld_x = 0;
     const int32_t* moe_offsets = nullptr;  // MoE: expert row offsets [E + 1] (device)
+    // block-scaled formats: tiled scale factors of A and W (s_a / s_w then
+    // point at the NVFP4 per-tensor decode scales, or are null for MXFP8)
+    const void* sf_a = nullptr;
+    const void* sf_w = nullptr;
 };
 
 // ------------------------------------------------------------------- MoE

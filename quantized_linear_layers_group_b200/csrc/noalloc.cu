@@ -62,7 +62,7 @@ extern "C" qlin_status qlin_scaled_mm_noalloc(int fmt, int variant, int tile_n, 
                                               int64_t K, const void* a_q, const float* s_a, const void* w_q,
                                               const float* s_w, const void* bias, void* c_out, uint32_t flags,
                                               qlin_stream_t stream) {
-    if (fmt == QLIN_FMT_BF16) return QLIN_ERR_INVALID_ARG;  // scaled formats only, as qlin_scaled_mm
+    if (fmt == QLIN_FMT_BF16 || is_block_scaled(fmt)) return QLIN_ERR_INVALID_ARG;  // as qlin_scaled_mm
     qlin_status st = check_fmt_shape(fmt, M, N, K);
     if (st != QLIN_OK) return st;
     if (flags & ~(QLIN_OUT_I32ACC | QLIN_PDL | QLIN_SPLITK_CLUSTER)) return QLIN_ERR_INVALID_ARG;

@@ -136,6 +136,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
         : "memory");
 }
 
+// Contiguous bulk load global -> shared (no tensor map): both addresses
+// 16-byte aligned, bytes a multiple of 16; completion counted on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                          uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+
 // 2-D tiled bulk tensor store shared -> global (bulk-group completion).
 // Elements of the box outside the tensor are not written.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, int32_t x, int32_t y, uint32_t src) {
@@ -223,6 +233,65 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
+}
+
+// ------------------------------------------------------ block-scaled MMAs
+// Block-scaled kinds: MXFP8 (e4m3 operands, one E8M0 scale per 32 elements of
+// K, kind::mxf8f6f4) and NVFP4 (packed e2m1 operands, one E4M3 scale per 16
+// elements, kind::mxf4nvf4 with 16-element blocks).  Both consume 32 bytes of
+// K per instruction, as the dense 8-bit kinds do.  The scale factors are read
+// from tensor memory: sfa / sfb are TMEM addresses (lane 0, a column), and
+// row r of A (column n of B) takes its scale from column base + r / 32 (n /
+// 32); the instruction descriptor's scale-factor ids pick the byte of that
+// 32-bit column for MXFP8, whose four K sub-blocks of one 128-byte K block
+// share a column.
+enum BlockScaledKind : int { kKindMXF8 = 3, kKindNVF4 = 4 };
+
+template <int KIND>
+__device__ __forceinline__ void tc_mma_bs(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    if constexpr (KIND == kKindMXF8) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                d_tmem),
+            "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    }
+}
+
+// Instruction descriptor of the block-scaled kinds (dense, K-major A and B,
+// fp32 D):  bits 4-5 B scale-factor id, 7-9 A type, 10-12 B type (mxf8f6f4:
+// e4m3 = 0; mxf4nvf4: e2m1 = 1), 17-22 N >> 3, 23 scale type (E8M0 = 1,
+// UE4M3 = 0), 24-28 M >> 4, 29-30 A scale-factor id.
+__host__ __device__ constexpr uint32_t make_idesc_bs(int kind, int m, int n) {
+    const uint32_t ab = kind == kKindNVF4 ? 1u : 0u;
+    const uint32_t e8m0 = kind == kKindMXF8 ? 1u : 0u;
+    return (ab << 7) | (ab << 10) | ((uint32_t)(n >> 3) << 17) | (e8m0 << 23) | ((uint32_t)(m >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_sf_ids(uint32_t idesc, uint32_t a_id, uint32_t b_id) {
+    return idesc | (a_id << 29) | (b_id << 4);
+}
+
+// Copy 32 rows x 16 bytes of scale factors from shared memory into TMEM
+// columns taddr .. taddr + 3 of lanes 0-31, replicated into all four lane
+// quadrants.  The source is described like an MMA operand without swizzle:
+// 8-row core matrices of 16-byte rows, 128 bytes apart.
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) | ((uint64_t)(128u >> 4) << 32) |
+           ((uint64_t)1u << 46);
 }
 
 // ------------------------------------------------- CTA pairs (cta_group::2)

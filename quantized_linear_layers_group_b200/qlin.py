@@ -35,6 +35,8 @@ QLIN_FMT_INT8 = 0
 QLIN_FMT_FP8 = 1
 QLIN_FMT_FP8_BLOCK = 2
 QLIN_FMT_BF16 = 3  # qlin_matmul_bf16 (and the workspace-size / dispatch queries)
+QLIN_FMT_MXFP8 = 4  # block-scaled: qlin_quantize_block_scaled / qlin_block_scaled_mm
+QLIN_FMT_NVFP4 = 5
 
 QLIN_VAR_AUTO = 0
 QLIN_VAR_PLAIN = 1
@@ -57,7 +59,7 @@ EXPORTS = ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "
            "qlin_moe_act_quantize", "qlin_moe_combine", "qlin_moe_workspace_size", "qlin_moe_forward",
            "qlin_scaled_mm_workspace_size", "qlin_dispatch_table_load", "qlin_dispatch_table_clear",
            "qlin_dispatch_query", "qlin_status_string", "qlin_sync_status", "qlin_abi_version",
-           "qlin_selftest_wait_timeout")
+           "qlin_selftest_wait_timeout", "qlin_quantize_block_scaled", "qlin_block_scaled_mm")
 QLIN_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -90,6 +92,9 @@ lib.qlin_scaled_mm_noalloc.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64,
 lib.qlin_linear.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _u32,
                             _vp, _sz, _vp]
 lib.qlin_matmul_bf16.argtypes = [_i32, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _u32, _vp, _sz, _vp]
+lib.qlin_quantize_block_scaled.argtypes = [_i32, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _u32, _vp]
+lib.qlin_block_scaled_mm.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                     _vp, _u32, _vp, _sz, _vp]
 lib.qlin_moe_route.argtypes = [_i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _u32, _vp]
 lib.qlin_moe_quantize_scatter.argtypes = [_i64, _i64, _i32, _vp, _vp, _vp, _vp, _u32, _vp]
 lib.qlin_moe_grouped_mm.argtypes = [_i32, _i32, _i32, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _u32, _vp]
@@ -219,6 +224,37 @@ def qlin_matmul_bf16(a, w, bias, c_out, workspace=None, stream=None, *, variant:
         workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib.qlin_matmul_bf16(variant, tile_n, k_segments, M, N, K, _ptr(a), _ptr(w), _ptr(bias), _ptr(c_out),
                                 flags, _ptr(workspace), workspace_bytes, _stream(stream)), "qlin_matmul_bf16")
+
+
+def block_scaled_sf_bytes(fmt: int, rows: int, cols: int) -> int:
+    """Bytes of the tiled scale-factor buffer for a [rows, cols] operand."""
+    atoms = cols // (128 if fmt == QLIN_FMT_MXFP8 else 64)
+    return -(-rows // 128) * atoms * 512
+
+
+def qlin_quantize_block_scaled(fmt: int, x, q_out, sf_out, g=None, stream=None, *, flags: int = 0, rows=None,
+                               cols=None, ld_x=None):
+    """MXFP8 / NVFP4 quantisation of bf16 x [rows, cols]: codes into q_out, tiled
+    scale factors into sf_out (NVFP4: g is the fp32 [1] decode scale on the device)."""
+    rows = x.shape[0] if rows is None else rows
+    cols = x.shape[1] if cols is None else cols
+    ld_x = (x.stride(0) if x.dim() == 2 else cols) if ld_x is None else ld_x
+    _check(lib.qlin_quantize_block_scaled(fmt, _ptr(x), rows, cols, ld_x, _ptr(g), _ptr(q_out), _ptr(sf_out), flags,
+                                          _stream(stream)), "qlin_quantize_block_scaled")
+
+
+def qlin_block_scaled_mm(fmt: int, a_q, a_sf, w_q, w_sf, bias, c_out, g_a=None, g_w=None, workspace=None,
+                         stream=None, *, variant: int = QLIN_VAR_AUTO, tile_n: int = 0, k_segments: int = 0,
+                         flags: int = 0, M=None, N=None, K=None, workspace_bytes=None):
+    """Block-scaled GEMM: C = bf16(acc + bias) (MXFP8) or bf16((acc*g_a)*g_w + bias) (NVFP4)."""
+    M = a_q.shape[0] if M is None else M
+    N = w_q.shape[0] if N is None else N
+    K = a_q.shape[1] * (2 if fmt == QLIN_FMT_NVFP4 else 1) if K is None else K
+    if workspace_bytes is None:
+        workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.qlin_block_scaled_mm(fmt, variant, tile_n, k_segments, M, N, K, _ptr(a_q), _ptr(a_sf), _ptr(w_q),
+                                    _ptr(w_sf), _ptr(g_a), _ptr(g_w), _ptr(bias), _ptr(c_out), flags,
+                                    _ptr(workspace), workspace_bytes, _stream(stream)), "qlin_block_scaled_mm")
 
 
 # ------------------------------------------------------------------- MoE

@@ -80,3 +80,41 @@ def check_status():
 
     st = qlin.qlin_sync_status()
     assert st == 0, f"device status {st}: {qlin.qlin_status_string(st)}"
+
+
+# ------------------------------------------------------ block-scaled formats
+# The GPU keeps scale factors in the tiled layout its tensor cores read (512-byte
+# atoms of 128 rows x 4 scales, row r's four bytes at (r%32)*16 + ((r/32)%4)*4);
+# the oracle keeps them plain, [rows][K / block].  These two functions only move
+# bytes between the layouts.
+def _sf_index(rows: int, nsf: int) -> np.ndarray:
+    atoms = nsf // 4
+    r = np.arange(rows)[:, None]
+    j = np.arange(nsf)[None, :]
+    return ((r // 128) * atoms + j // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + j % 4
+
+
+def sf_tile(plain: np.ndarray) -> np.ndarray:
+    rows, nsf = plain.shape
+    out = np.zeros(-(-rows // 128) * (nsf // 4) * 512, np.uint8)
+    out[_sf_index(rows, nsf)] = plain
+    return out
+
+
+def sf_untile(tiled: np.ndarray, rows: int, nsf: int) -> np.ndarray:
+    return tiled[_sf_index(rows, nsf)]
+
+
+def gpu_block_scaled_mm(fmt, a_q, a_sf, w_q, w_sf, bias_dev=None, g_a=None, g_w=None, variant=0, tile_n=0,
+                        k_segments=0, flags=0):
+    from quantized_linear_layers_group_b200 import qlin
+
+    M = a_q.shape[0]
+    N = w_q.shape[0]
+    K = a_q.shape[1] * (2 if fmt == qlin.QLIN_FMT_NVFP4 else 1)
+    c = torch.empty(M, N, dtype=torch.bfloat16, device=a_q.device)
+    nbytes = qlin.qlin_scaled_mm_workspace_size(fmt, M, N, K, variant, tile_n, k_segments)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=a_q.device) if nbytes else None
+    qlin.qlin_block_scaled_mm(fmt, a_q, a_sf, w_q, w_sf, bias_dev, c, g_a, g_w, ws, variant=variant, tile_n=tile_n,
+                              k_segments=k_segments, flags=flags)
+    return c

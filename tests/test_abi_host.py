@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
     syms = _declared_symbols()
     for name in ("qlin_quantize_per_token", "qlin_quantize_block", "qlin_scaled_mm", "qlin_dispatch_table_load"):
         assert name in syms
-    assert len(syms) == 21
+    assert len(syms) == 23
 
 
 def test_library_exports_every_declared_symbol(q):
@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(q):
     for name in _declared_symbols():
         assert hasattr(lib, name), name
     assert set(_declared_symbols()) == set(q.EXPORTS)
-    assert q.qlin_abi_version() == 6
+    assert q.qlin_abi_version() == 7
 
 
 def test_status_strings(q):
@@ -242,3 +242,50 @@ def test_matmul_bf16_rejects_bad_arguments_before_launch(q):
     assert _mm(q, fmt=q.QLIN_FMT_BF16) == q.QLIN_ERR_INVALID_ARG
     # K blocks of a bf16 row: K = 192 is three of them, so S = 3 divides it
     assert q.qlin_scaled_mm_workspace_size(q.QLIN_FMT_BF16, 16, 256, 192, q.QLIN_VAR_SWAPAB_SPLITK, 16, 3) > 0
+
+
+def _bsmm(q, **kw):
+    args = dict(fmt=4, variant=0, tile_n=0, k_segments=0, M=16, N=256, K=256, a=16, asf=16, w=16, wsf=16, ga=None,
+                gw=None, bias=None, c=16, flags=0, ws=None, wsb=0)
+    args.update(kw)
+    return q.lib.qlin_block_scaled_mm(args["fmt"], args["variant"], args["tile_n"], args["k_segments"], args["M"],
+                                      args["N"], args["K"], args["a"], args["asf"], args["w"], args["wsf"],
+                                      args["ga"], args["gw"], args["bias"], args["c"], args["flags"], args["ws"],
+                                      args["wsb"], None)
+
+
+def test_block_scaled_entry_points_reject_bad_arguments_before_launch(q):
+    assert _bsmm(q, fmt=1) == q.QLIN_ERR_INVALID_ARG                 # per-token formats: qlin_scaled_mm
+    assert _bsmm(q, K=192) == q.QLIN_ERR_UNSUPPORTED                 # MXFP8: K % 128
+    assert _bsmm(q, fmt=5, K=384, ga=16, gw=16) == q.QLIN_ERR_UNSUPPORTED   # NVFP4: K % 256
+    assert _bsmm(q, fmt=5) == q.QLIN_ERR_INVALID_ARG                 # NVFP4 needs both decode scales
+    assert _bsmm(q, ga=16, gw=16) == q.QLIN_ERR_INVALID_ARG          # MXFP8 takes none
+    assert _bsmm(q, variant=q.QLIN_VAR_SWAPAB) == q.QLIN_ERR_UNSUPPORTED
+    assert _bsmm(q, variant=q.QLIN_VAR_PAIR) == q.QLIN_ERR_UNSUPPORTED
+    assert _bsmm(q, variant=9) == q.QLIN_ERR_INVALID_ARG
+    assert _bsmm(q, flags=q.QLIN_SPLITK_CLUSTER) == q.QLIN_ERR_INVALID_ARG
+    assert _bsmm(q, asf=None) == q.QLIN_ERR_INVALID_ARG
+    assert _bsmm(q, asf=24) == q.QLIN_ERR_ALIGNMENT
+    assert _bsmm(q, M=0) == q.QLIN_OK
+    # the per-token entry points refuse the block-scaled formats
+    assert _mm(q, fmt=4) == q.QLIN_ERR_INVALID_ARG
+    assert _mm(q, fmt=5) == q.QLIN_ERR_INVALID_ARG
+    L = q.lib
+    assert L.qlin_quantize_block_scaled(1, 16, 4, 256, 256, None, 16, 16, 0, None) == q.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_block_scaled(4, 16, 4, 192, 192, None, 16, 16, 0, None) == q.QLIN_ERR_UNSUPPORTED
+    assert L.qlin_quantize_block_scaled(5, 16, 4, 256, 256, None, 16, 16, 0, None) == q.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_block_scaled(4, 16, 4, 256, 256, 16, 16, 16, 0, None) == q.QLIN_ERR_INVALID_ARG
+    assert L.qlin_quantize_block_scaled(4, 16, 4, 256, 256, None, 16, 24, 0, None) == q.QLIN_ERR_ALIGNMENT
+    assert L.qlin_quantize_block_scaled(4, 16, 0, 256, 256, None, 16, 16, 0, None) == q.QLIN_OK
+
+
+def test_block_scaled_dispatch_uses_plain_128_tiles(q):
+    for fmt in (q.QLIN_FMT_MXFP8, q.QLIN_FMT_NVFP4):
+        for M in (1, 16, 64, 256, 2048):
+            c = q.qlin_dispatch_query(fmt, M, 4096, 2048)
+            assert c["variant"] in (q.QLIN_VAR_PLAIN, q.QLIN_VAR_SPLITK) and c["tile_n"] == 128, (fmt, M, c)
+        assert q.qlin_scaled_mm_workspace_size(fmt, 64, 4096, 2048, q.QLIN_VAR_PLAIN) == 0
+        ws = q.qlin_scaled_mm_workspace_size(fmt, 64, 4096, 2048, q.QLIN_VAR_SPLITK, 0, 4)
+        assert ws == 65536 + 4 * 32 * 128 * 128 * 4
+    assert q.block_scaled_sf_bytes(q.QLIN_FMT_MXFP8, 130, 256) == 2 * 2 * 512
+    assert q.block_scaled_sf_bytes(q.QLIN_FMT_NVFP4, 130, 256) == 2 * 4 * 512
