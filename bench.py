@@ -58,14 +58,18 @@ import synth  # noqa: E402
 
 METRIC = "scaled_mm TFLOPS & HBM GB/s vs roofline, per (M,N,K,format), 1×B200"
 L2_BYTES = 126 * 1024 * 1024
-FMT_NAME = {0: "int8", 1: "fp8", 2: "fp8_block", 3: "bf16"}
+FMT_NAME = {0: "int8", 1: "fp8", 2: "fp8_block", 3: "bf16", 4: "mxfp8", 5: "nvfp4"}
 DTYPE = {0: "int8 (int32 accumulate)", 1: "fp8_e4m3 (fp32 accumulate)", 2: "fp8_e4m3 block-scaled (fp32 accumulate)",
-         3: "bf16 (fp32 accumulate)"}
+         3: "bf16 (fp32 accumulate)", 4: "mxfp8 e4m3 / e8m0 (fp32 accumulate)",
+         5: "nvfp4 e2m1 / e4m3 (fp32 accumulate)"}
+BS_FMTS = (4, 5)  # block-scaled formats: scale factors applied inside the tensor core
 HEADLINE = "fp8_attn"
 # every workload of the metric: the headline plus the parity configurations
 ALL_WORKLOADS = ("fp8_attn", "int8_smoke", "fp8_block_down", "lm_head", "fp8_vocab", "int8_square")
 # the bf16 batch-invariant matmul on the five shapes of its sweep (no quantisation step)
 BF16_WORKLOADS = ("bf16_vocab", "bf16_down", "bf16_attn", "bf16_lm_head", "bf16_square")
+# the block-scaled formats MXFP8 / NVFP4 on the attention, down-projection and lm_head shapes
+BS_WORKLOADS = ("mxfp8_attn", "nvfp4_attn", "mxfp8_down", "nvfp4_lm_head")
 
 
 # ------------------------------------------------------------------ peaks
@@ -120,6 +124,9 @@ def tensor_peak(peaks, fmt, tpk=None):
     8-bit / bf16 ratio)."""
     if fmt == 3:
         return peaks["bf16_tflops"], f"{peaks['source']} bf16_tflops (cuBLAS bf16 burst)"
+    if fmt == 5:  # fp4 operands: twice the 8-bit rate (nominal 9 / 4.5 PFLOP/s dense)
+        p8, src8 = tensor_peak(peaks, 1, tpk)
+        return 2.0 * p8, src8 + " x 2 (nominal fp4 / fp8 ratio)"
     if tpk is not None:
         v = tpk.get("int8_tops" if fmt == 0 else "fp8_tflops")
         if v:
@@ -134,9 +141,12 @@ def gemm_flops(M, N, K):
 def gemm_bytes(M, N, K, fmt):
     """Algorithmic bytes per GEMM launch: the 8-bit operands A and W (as the
     roofline is defined on), plus scales, bias and the bf16 output separately."""
-    elt = 2 if fmt == 3 else 1
-    ab = (M * K + N * K) * elt
-    scales = (M * (K // 128) + (N // 128) * (K // 128)) * 4 if fmt == 2 else (0 if fmt == 3 else (M + N) * 4)
+    elt = {3: 2.0, 5: 0.5}.get(fmt, 1.0)
+    ab = int((M * K + N * K) * elt)
+    if fmt in BS_FMTS:  # one scale byte per 32 (MXFP8) or 16 (NVFP4) elements
+        scales = (M + N) * K // (32 if fmt == 4 else 16)
+    else:
+        scales = (M * (K // 128) + (N // 128) * (K // 128)) * 4 if fmt == 2 else (0 if fmt == 3 else (M + N) * 4)
     extra = scales + 2 * M * N
     return ab, extra
 
@@ -144,6 +154,10 @@ def gemm_bytes(M, N, K, fmt):
 def quant_bytes(M, K, fmt):
     if fmt == 3:
         return 0  # bf16: no quantisation step
+    if fmt == 4:
+        return 2 * M * K + M * K + M * K // 32
+    if fmt == 5:
+        return 2 * M * K + M * K // 2 + M * K // 16
     return 2 * M * K + M * K + (M * (K // 128) if fmt == 2 else M) * 4
 
 
@@ -296,13 +310,21 @@ class HotPath:
         w_cpu = synth.weights(workload, seed)
         b_cpu = synth.bias(workload, seed)
         w_dev = w_cpu.to(device)
+        self.g_w = self.g_a = None
         if self.fmt == 3:  # bf16: the weight is used as it is
             w_q, s_w = w_dev, None
+        elif self.fmt in BS_FMTS:  # offline: codes and tiled scale factors (NVFP4: decode scale amax / (6 * 448))
+            if self.fmt == 5:
+                self.g_w = (w_dev.float().abs().max() / 2688.0).reshape(1).contiguous()
+            w_q = torch.empty(N, K // 2 if self.fmt == 5 else K, dtype=torch.uint8, device=device)
+            s_w = torch.empty(qlin.block_scaled_sf_bytes(self.fmt, N, K), dtype=torch.uint8, device=device)
+            qlin.qlin_quantize_block_scaled(self.fmt, w_dev, w_q, s_w, self.g_w)
+            del w_dev
         else:
             w_q, s_w = linear.quantize_weight(self.fmt, w_dev)
             del w_dev
         self.bias = None if b_cpu is None else b_cpu.to(device)
-        wbytes = N * K * (2 if self.fmt == 3 else 1)
+        wbytes = N * K * {3: 2, 5: 0.5}.get(self.fmt, 1)
         # enough weight copies that the bytes read between two uses of a copy exceed 2x L2
         self.n_copies = max(2, math.ceil(2 * L2_BYTES / wbytes) + 1)
         self.w_copies = [(w_q if i == 0 else w_q.clone(), s_w if i == 0 or s_w is None else s_w.clone())
@@ -313,16 +335,24 @@ class HotPath:
         self.n_act_sets = max(self.n_graphs, math.ceil(2 * L2_BYTES / step_bytes) + 1)
         a_cpu = {M: synth.activations(workload, M, seed=seed) for M in self.ms}
         self.a_sets = [{M: a_cpu[M].to(device) for M in self.ms} for _ in range(self.n_act_sets)]
+        if self.fmt == 5:  # NVFP4 activations: a static decode scale, calibrated once on these inputs
+            amax = max(float(a.float().abs().max()) for a in a_cpu.values())
+            self.g_a = torch.tensor([amax / 2688.0], dtype=torch.float32, device=device)
         self.a_cpu = a_cpu
         self.a_host = None  # pinned copies, made by the first end-to-end step
         self.act = 0  # activation set of the step being issued
         self.a_q, self.s_a, self.c, self.c_host = {}, {}, {}, {}
         ws = 0
         for M in self.ms:
-            self.a_q[M] = (torch.empty(M, K, dtype=torch.bfloat16, device=device) if self.fmt == 3 else
-                           torch.empty(M, K, dtype=torch.uint8, device=device))
-            self.s_a[M] = torch.empty(*((M, K // 128) if self.fmt == 2 else (M,)), dtype=torch.float32,
-                                      device=device)
+            if self.fmt in BS_FMTS:
+                self.a_q[M] = torch.empty(M, K // 2 if self.fmt == 5 else K, dtype=torch.uint8, device=device)
+                self.s_a[M] = torch.empty(qlin.block_scaled_sf_bytes(self.fmt, M, K), dtype=torch.uint8,
+                                          device=device)
+            else:
+                self.a_q[M] = (torch.empty(M, K, dtype=torch.bfloat16, device=device) if self.fmt == 3 else
+                               torch.empty(M, K, dtype=torch.uint8, device=device))
+                self.s_a[M] = torch.empty(*((M, K // 128) if self.fmt == 2 else (M,)), dtype=torch.float32,
+                                          device=device)
             self.c[M] = torch.empty(M, N, dtype=torch.bfloat16, device=device)
             ws = max(ws, qlin.qlin_scaled_mm_workspace_size(self.fmt, M, N, K))
         self.workspace = torch.zeros(max(ws, 256), dtype=torch.uint8, device=device)
@@ -337,7 +367,9 @@ class HotPath:
         x = self.a_sets[self.act][M]
         if self.fmt == 3:
             return  # bf16: the GEMM reads the activations themselves
-        if self.fmt == 2:
+        if self.fmt in BS_FMTS:
+            q.qlin_quantize_block_scaled(self.fmt, x, self.a_q[M], self.s_a[M], self.g_a, stream, flags=self.flags)
+        elif self.fmt == 2:
             q.qlin_quantize_block(x, 1, self.a_q[M], self.s_a[M], stream, flags=self.flags)
         else:
             q.qlin_quantize_per_token(self.fmt, x, self.a_q[M], self.s_a[M], stream, flags=self.flags)
@@ -348,6 +380,10 @@ class HotPath:
         if self.fmt == 3:
             self.qlin.qlin_matmul_bf16(self.a_sets[self.act][M], w_q, self.bias, self.c[M], self.workspace, stream,
                                        flags=self.flags)
+            return
+        if self.fmt in BS_FMTS:
+            self.qlin.qlin_block_scaled_mm(self.fmt, self.a_q[M], self.s_a[M], w_q, s_w, self.bias, self.c[M],
+                                           self.g_a, self.g_w, self.workspace, stream, flags=self.flags)
             return
         self.qlin.qlin_scaled_mm(self.fmt, self.a_q[M], self.s_a[M], w_q, s_w, self.bias, self.c[M],
                                  self.workspace, stream, flags=self.flags)
@@ -790,7 +826,7 @@ def main(argv=None):
         # ------------------------------ every workload of the metric, per M
         workloads = {}
         if not args.no_workloads and world == 1:
-            for name in ALL_WORKLOADS + BF16_WORKLOADS:
+            for name in ALL_WORKLOADS + BF16_WORKLOADS + BS_WORKLOADS:
                 w = synth.WORKLOADS[name]
                 wh = HotPath(w, list(w.m_values), device)
                 for _ in range(3):

@@ -541,13 +541,18 @@ QLIN_API qlin_status qlin_quantize_block_scaled(int fmt, const void* x, int64_t 
  *   NVFP4:  C[m,n] = bf16( ((acc[m,n] * g_a) * g_w) + bias[n] )
  *           acc[m,n] = sum over blocks of (block scales) * sum_k a_q w_q, fp32
  *
- * Plain and Split-K tiles of 128 x 128 (no Swap-AB or pair tiles); K is cut
- * into k_segments segments added in order from +0, as in qlin_scaled_mm, so
- * rows of C do not depend on M.  The dispatch table's entries are keyed
- * "mxfp8" / "nvfp4".
+ * Plain tiles of 128 x 128 and, for M <= tile_n, Swap-AB tiles of 32 or 64
+ * activation rows (one activation tile: its scales are the first rows of the
+ * first 128-row atom; no tile 16, no pair tiles), each with Split-K.  K is cut into
+ * k_segments segments added in order from +0, as in qlin_scaled_mm, so rows of
+ * C do not depend on M or on the variant.  The dispatch table's entries are
+ * keyed "mxfp8" / "nvfp4"; without one, M <= 64 runs Swap-AB and larger M
+ * plain tiles, with one K segment.
  *
  *   fmt                 QLIN_FMT_MXFP8 or QLIN_FMT_NVFP4
- *   variant             AUTO, PLAIN or SPLITK;  tile_n 0 or 128;  k_segments as qlin_scaled_mm
+ *   variant             AUTO, PLAIN, SPLITK, SWAPAB or SWAPAB_SPLITK
+ *   tile_n              0, or 128 (plain) / 32, 64 (Swap-AB, M <= tile_n);  k_segments as
+ *                       qlin_scaled_mm
  *   M, N, K             M >= 0 (0 is a no-op), N >= 16, N % 16 == 0;
  *                       K % 128 == 0 (MXFP8) or K % 256 == 0 (NVFP4)
  *   a_q, a_sf           A codes [M, K] (NVFP4: [M, K/2] packed) and tiled scales (device)

@@ -99,7 +99,7 @@ bool runs_as_cluster(int variant, int tile_n, int S) {
 }
 
 bool tile_supported(int fmt, bool swap, int tile_n, bool pair = false) {
-    if (is_block_scaled(fmt)) return !swap && !pair && tile_n == 128;
+    if (is_block_scaled(fmt)) return !pair && (swap ? (tile_n == 32 || tile_n == 64) : tile_n == 128);
     if (pair) return fmt != QLIN_FMT_FP8_BLOCK && tile_n == 256;
     if (swap) return tile_n == 16 || tile_n == 32 || tile_n == 64;
     if (fmt == QLIN_FMT_FP8_BLOCK) return tile_n == 128;
@@ -125,6 +125,20 @@ int64_t row_bytes(int fmt, int64_t K) { return fmt == QLIN_FMT_BF16 ? 2 * K : (f
 
 qlin_config default_config(int fmt, int64_t M, int64_t N, int64_t K, int num_sms) {
     qlin_config c{};
+    if (is_block_scaled(fmt)) {
+        // block-scaled: one K segment (measured fastest at every M for the
+        // attention and down-projection shapes: the running total and the
+        // Split-K partials cost more than they gain); Swap-AB 32 / 64 tiles
+        // for small M, plain 128 x 128 tiles above
+        c.k_segments = 1;
+        c.from_table = 0;
+        c.m_max = 0;
+        c.variant = M <= 64 ? QLIN_VAR_SWAPAB : QLIN_VAR_PLAIN;
+        c.tile_n = M <= 32 ? 32 : (M <= 64 ? 64 : 128);
+        size_t smem = 0;
+        gemm_kernel_info(fmt, is_swap(c.variant), c.tile_n, kModeStd, &c.stages, &smem);
+        return c;
+    }
     c.k_segments = default_segments(fmt, N, row_bytes(fmt, K), num_sms);
     c.from_table = 0;
     c.m_max = 0;
@@ -178,7 +192,7 @@ qlin_status resolve_config(int fmt, int variant, int tile_n, int k_segments, int
         const bool same_orientation = is_swap(variant) == is_swap(base.variant);
         base.tile_n = same_orientation ? base.tile_n : d.tile_n;
         if (is_swap(variant) && !same_orientation)
-            base.tile_n = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+            base.tile_n = M <= 16 && !is_block_scaled(fmt) ? 16 : (M <= 32 ? 32 : 64);
         if (variant == QLIN_VAR_PAIR) base.tile_n = 256;
         base.variant = variant;
     }
@@ -238,6 +252,9 @@ qlin_status make_gemm_plan(int fmt, int variant, int tile_n, int k_segments, int
     p.kblocks = (int)(p.k_bytes / 128);
     const bool pair = cfg.variant == QLIN_VAR_PAIR;
     if (!tile_supported(fmt, p.swap, p.tile_n, pair)) return QLIN_ERR_UNSUPPORTED;
+    // block-scaled Swap-AB: one activation tile (its scale rows are rows
+    // 0 .. tile_n - 1 of the first 128-row atom; see the kernel's Cfg)
+    if (is_block_scaled(fmt) && p.swap && M > p.tile_n) return QLIN_ERR_UNSUPPORTED;
     if (p.k_segments < 1 || p.kblocks % p.k_segments != 0) return QLIN_ERR_UNSUPPORTED;
     if (p.k_segments == 1) p.spread = false;
     p.kb_per_seg = p.kblocks / p.k_segments;
@@ -548,8 +565,8 @@ qlin_status qlin_block_scaled_mm(int fmt, int variant, int tile_n, int k_segment
     qlin_status st = check_fmt_shape(fmt, M, N, K);
     if (st != QLIN_OK) return st;
     if (flags & ~QLIN_PDL) return QLIN_ERR_INVALID_ARG;
-    if (variant != QLIN_VAR_AUTO && variant != QLIN_VAR_PLAIN && variant != QLIN_VAR_SPLITK)
-        return variant < QLIN_VAR_AUTO || variant > QLIN_VAR_PAIR ? QLIN_ERR_INVALID_ARG : QLIN_ERR_UNSUPPORTED;
+    if (variant < QLIN_VAR_AUTO || variant > QLIN_VAR_PAIR) return QLIN_ERR_INVALID_ARG;
+    if (variant == QLIN_VAR_PAIR) return QLIN_ERR_UNSUPPORTED;
     if (tile_n < 0 || k_segments < 0) return QLIN_ERR_INVALID_ARG;
     const bool nv = fmt == QLIN_FMT_NVFP4;
     if (nv != (g_a != nullptr) || nv != (g_w != nullptr)) return QLIN_ERR_INVALID_ARG;
@@ -572,7 +589,9 @@ qlin_status qlin_block_scaled_mm(int fmt, int variant, int tile_n, int k_segment
     if (g_log)
         std::fprintf(stderr, "[qlin] block_scaled_mm %s M=%lld N=%lld K=%lld -> %s tile_n=%d S=%d grid=%d\n",
                      fmt_name(fmt), (long long)M, (long long)N, (long long)K,
-                     variant_name(p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN), p.tile_n, p.k_segments, p.grid);
+                     variant_name(p.swap ? (p.spread ? QLIN_VAR_SWAPAB_SPLITK : QLIN_VAR_SWAPAB)
+                                         : (p.spread ? QLIN_VAR_SPLITK : QLIN_VAR_PLAIN)),
+                     p.tile_n, p.k_segments, p.grid);
     GemmOperands ops{a_q, g_a, w_q, g_w, bias, c_out, false, workspace, (flags & QLIN_PDL) != 0};
     ops.sf_a = a_sf;
     ops.sf_w = w_sf;

@@ -147,14 +147,24 @@ struct Cfg {
     // block-scaled (MXFP8, NVFP4): the tensor core applies per-block scale
     // factors that the MMA thread copies from shared memory into TMEM
     static constexpr bool BS = is_block_scaled(FMT);
-    static_assert(!BS || (!SWAP && !CSK && !FUSE && !PAIR && BN == 128), "block-scaled formats: plain 128 x 128 tiles");
+    // plain 128 x 128 tiles, or Swap-AB tiles of 32 / 64 activation rows.  The
+    // MMA reads the scale of its column n from TMEM column base + n / 32 of a
+    // copied 128-row atom, and its scale address must not be offset inside
+    // the atom's four columns, so a Swap-AB tile uses rows 0 .. tile_n - 1 of
+    // atom 0: the host plans Swap-AB only for M <= tile_n (one activation tile)
+    static_assert(!BS || (!CSK && !FUSE && !PAIR && (SWAP ? (BN == 32 || BN == 64) : BN == 128)),
+                  "block-scaled formats: plain 128 x 128 or Swap-AB 32 / 64 tiles");
     static constexpr int KIND =
         BS ? (FMT == QLIN_FMT_MXFP8 ? kKindMXF8 : kKindNVF4) : (INT8 ? kKindI8 : (BF16 ? kKindF16 : kKindF8));
     // scale-factor atoms (512 B: 128 rows x 4 scales) per 128-byte K block of
-    // one 128-row group: MXFP8 1 (128 elements), NVFP4 4 (256 elements)
+    // one 128-row group: MXFP8 1 (128 elements), NVFP4 4 (256 elements).  The
+    // "A" slot holds the P operand's atoms (the MMA's A: activations, or W in
+    // Swap-AB), the "B" slot the Q operand's (SF_RGQ row groups: whole atoms,
+    // also for a Swap-AB tile that uses 32 or 64 of their rows)
     static constexpr int SF_APK = FMT == QLIN_FMT_NVFP4 ? 4 : 1;
+    static constexpr int SF_RGQ = (BN + 127) / 128;
     static constexpr int SFA_BYTES = BS ? 512 * SF_APK : 0;
-    static constexpr int SFB_BYTES = BS ? 512 * SF_APK * (BN / 128) : 0;
+    static constexpr int SFB_BYTES = BS ? 512 * SF_APK * SF_RGQ : 0;
     static constexpr int SF_BYTES = SFA_BYTES + SFB_BYTES;
     static constexpr int BM = 128;                 // P rows per tile (MMA M)
     static constexpr int BK = 128;                 // K bytes per stage: one swizzle atom
@@ -187,7 +197,7 @@ struct Cfg {
     // block-scaled: two copies (alternate K blocks) of one K block's scale
     // factors, 4 columns per atom, after the accumulators and running total
     static constexpr int SF_COL = NACC * ACC_COLS + (MULTI ? ACC_COLS : 0) + ((BLOCK && SWAP) ? ACC_COLS : 0);
-    static constexpr int SF_COLS = BS ? 4 * SF_APK * (1 + BN / 128) : 0;
+    static constexpr int SF_COLS = BS ? 4 * SF_APK * (1 + SF_RGQ) : 0;
     static constexpr int TMEM_COLS = pow2_at_least(SF_COL + 2 * SF_COLS);
     static_assert(NACC * ACC_COLS <= TOTAL_COL, "accumulators overlap the running total");
     static constexpr uint32_t IDESC = BS ? make_idesc_bs(KIND, 128, BN) : make_idesc(KIND, PAIR ? 256 : 128, BN);
@@ -1048,6 +1058,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if constexpr (SWAP) {
                     load(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_w, kb * 128, un.wrow0 + un.pt * 128, fb,
                          pol_w);
+                    if constexpr (C::BS)  // W is the MMA's A: its scale atoms go to the A slot
+                        bulk_load(smem_u32(sF + (size_t)stage * C::SF_BYTES),
+                                  args.sf_w + ((size_t)un.pt * args.sf_atoms + (size_t)kb * C::SF_APK) * 512u,
+                                  (uint32_t)C::SFA_BYTES, fb, pol_w);
                 } else {
                     load(smem_u32(sQ + (size_t)stage * C::Q_BYTES), tm_w, kb * 128,
                          un.wrow0 + un.qt * BN + w_row_off, fb, pol_w);
@@ -1093,7 +1107,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     else
                         load(smem_u32(sP + (size_t)stage * C::P_BYTES), tm_a, kb * 128, un.row0 + un.pt * 128, fb,
                              pol_a);
-                    if constexpr (C::BS)  // the A tile's scale atoms of this K block
+                    if constexpr (C::BS && SWAP)  // the activation rows' 128-row atom group, B slot
+                        bulk_load(smem_u32(sF + (size_t)stage * C::SF_BYTES + C::SFA_BYTES),
+                                  args.sf_a + ((size_t)((un.qt * BN) >> 7) * args.sf_atoms +
+                                               (size_t)kb * C::SF_APK) * 512u,
+                                  (uint32_t)C::SFB_BYTES, fb, pol_a);
+                    else if constexpr (C::BS)  // the A tile's scale atoms of this K block
                         bulk_load(smem_u32(sF + (size_t)stage * C::SF_BYTES),
                                   args.sf_a + ((size_t)un.pt * args.sf_atoms + (size_t)kb * C::SF_APK) * 512u,
                                   (uint32_t)C::SFA_BYTES, fb, pol_a);
@@ -1136,7 +1155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             // this K block's scale factors into TMEM (the tensor pipe runs the
                             // copies and the MMAs in issue order); A's atoms, then W's, 4
                             // columns each: [atom][row group]
-                            constexpr int RG = BN / 128;
+                            constexpr int RG = C::SF_RGQ;
                             const uint32_t sfa_t = tmem_base + C::SF_COL + (sfi & 1u) * C::SF_COLS;
                             const uint32_t sfb_t = sfa_t + 4 * C::SF_APK;
                             const uint32_t sfs = smem_u32(sF + (size_t)stage * C::SF_BYTES);
@@ -1279,6 +1298,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         b_col[c] = (e.has_bias && q < args.N) ? bf16_to_f32(__ldg(args.bias + q)) : 0.f;
                     } else if constexpr (FUSE) {
                         s_col[c] = sa_cur[c];
+                    } else if constexpr (C::BS) {  // NVFP4: the activations' decode scale
+                        s_col[c] = FMT == QLIN_FMT_NVFP4 ? __ldg(args.s_a) : 1.f;
                     } else if constexpr (!C::BF16) {
                         s_col[c] = q < un.rows ? __ldg(args.s_a + un.row0 + q) : 0.f;
                     }
@@ -1291,7 +1312,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         e.row_scale = m < un.rows ? __ldg(args.s_a + un.row0 + m) : 0.f;
                 } else {
                     const int n = un.pt * 128 + e.row_lane;
-                    if constexpr (!C::BF16) e.row_scale = n < args.N ? __ldg(args.s_w + un.wrow0 + n) : 0.f;
+                    if constexpr (C::BS)
+                        e.row_scale = FMT == QLIN_FMT_NVFP4 ? __ldg(args.s_w) : 1.f;
+                    else if constexpr (!C::BF16)
+                        e.row_scale = n < args.N ? __ldg(args.s_w + un.wrow0 + n) : 0.f;
                     e.row_bias = (e.has_bias && n < args.N) ? bf16_to_f32(__ldg(args.bias + n)) : 0.f;
                 }
                 named_bar_sync(1, kEpiThreads);
@@ -1677,10 +1701,14 @@ void cfg_info(int* stages, size_t* smem) {
 // is applied to the one matching (swap, tile_n, mode); false if none exists.
 template <int FMT, template <int, bool, int, bool, bool, bool> class OP, typename... A>
 bool dispatch_instance(bool swap, int tile_n, int mode, A&&... args) {
-    if constexpr (is_block_scaled(FMT)) {  // plain / Split-K 128 x 128 tiles only
-        if (swap || mode != kModeStd || tile_n != 128) return false;
-        OP<FMT, false, 128, false, false, false>::run(args...);
-        return true;
+    if constexpr (is_block_scaled(FMT)) {  // plain 128 x 128 and Swap-AB 32 / 64 tiles (with Split-K)
+        if (mode != kModeStd) return false;
+        switch ((swap ? 1000 : 0) + tile_n) {
+            case 128: OP<FMT, false, 128, false, false, false>::run(args...); return true;
+            case 1032: OP<FMT, true, 32, false, false, false>::run(args...); return true;
+            case 1064: OP<FMT, true, 64, false, false, false>::run(args...); return true;
+        }
+        return false;
     } else {
     if (swap) {
         switch (mode * 1000 + tile_n) {

@@ -21,7 +21,7 @@
 // 2x L2), launched with QLIN_PDL as the hot path runs, CUDA events around the
 // graph, median of `reps` replays.
 //
-// Usage: qlin_sweep [--quick] <out.qlt> [shape ...]   shape = fmt:N:K (fmt int8|fp8|fp8_block|bf16)
+// Usage: qlin_sweep [--quick] <out.qlt> [shape ...]   shape = fmt:N:K (fmt int8|fp8|fp8_block|bf16|mxfp8|nvfp4)
 // Without shapes it sweeps the five workload shapes.  --quick (for tests):
 // buckets {1, 16, 256} only, two weight copies, short timing loops.
 #include <cuda_runtime.h>
@@ -61,10 +61,18 @@ const char* fmt_name(int f) {
         case QLIN_FMT_INT8: return "int8";
         case QLIN_FMT_FP8: return "fp8";
         case QLIN_FMT_FP8_BLOCK: return "fp8_block";
+        case QLIN_FMT_MXFP8: return "mxfp8";
+        case QLIN_FMT_NVFP4: return "nvfp4";
     }
     return "bf16";
 }
-int elem_bytes(int f) { return f == QLIN_FMT_BF16 ? 2 : 1; }
+bool block_scaled(int f) { return f == QLIN_FMT_MXFP8 || f == QLIN_FMT_NVFP4; }
+// bytes of one operand row of K elements
+int64_t row_bytes(int f, int64_t K) { return f == QLIN_FMT_BF16 ? 2 * K : (f == QLIN_FMT_NVFP4 ? K / 2 : K); }
+// bytes of the tiled scale factors of a [rows, K] block-scaled operand
+size_t sf_bytes(int f, int64_t rows, int64_t K) {
+    return (size_t)((rows + 127) / 128) * (size_t)(K / (f == QLIN_FMT_MXFP8 ? 128 : 64)) * 512u;
+}
 const char* var_name(int v) {
     switch (v) {
         case QLIN_VAR_PLAIN: return "plain";
@@ -100,6 +108,15 @@ __global__ void fill_bf16(uint16_t* p, size_t n, uint32_t seed) {
     }
 }
 
+// Block scale codes: E8M0 2^-7 .. 2^7 (MXFP8) or E4M3 0.5 .. 1.875 (NVFP4), never NaN.
+__global__ void fill_sf(uint8_t* p, size_t n, uint32_t seed, int e8m0) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        uint32_t h = (uint32_t)i * 2246822519u ^ seed;
+        h ^= h >> 15;
+        p[i] = e8m0 ? (uint8_t)(120u + h % 15u) : (uint8_t)(0x30u + h % 16u);
+    }
+}
+
 __global__ void fill_scales(float* p, size_t n, uint32_t seed) {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
         uint32_t h = (uint32_t)i * 747796405u + seed;
@@ -112,7 +129,8 @@ struct Problem {
     Shape s;
     int64_t M;
     void* a_q = nullptr;
-    float* s_a = nullptr;
+    float* s_a = nullptr;    // block-scaled formats: the tiled scale bytes
+    float* g = nullptr;      // NVFP4: the two per-tensor decode scales
     std::vector<void*> w_q;
     std::vector<float*> s_w;
     uint16_t* c = nullptr;
@@ -123,7 +141,7 @@ struct Problem {
 
 std::vector<int> segment_choices(int fmt, int64_t K) {
     std::vector<int> out;
-    const int kb = (int)(K * elem_bytes(fmt) / 128);
+    const int kb = (int)(row_bytes(fmt, K) / 128);
     for (int s : {1, 2, 3, 4, 6, 8})
         if (kb % s == 0 && kb / s >= 1) out.push_back(s);
     return out;
@@ -131,6 +149,16 @@ std::vector<int> segment_choices(int fmt, int64_t K) {
 
 std::vector<Cand> candidates(int fmt, int64_t M) {
     std::vector<Cand> c;
+    if (block_scaled(fmt)) {  // Swap-AB 32 / 64 for one activation tile; plain 128
+        for (int t : {32, 64}) {
+            if (M > t || (t == 64 && M <= 32)) continue;
+            c.push_back({QLIN_VAR_SWAPAB, t});
+            c.push_back({QLIN_VAR_SWAPAB_SPLITK, t});
+        }
+        c.push_back({QLIN_VAR_PLAIN, 128});
+        c.push_back({QLIN_VAR_SPLITK, 128});
+        return c;
+    }
     for (int t : {16, 32, 64}) {
         if (t >= 2 * M && t > 16) continue;  // a tile more than twice M only wastes the narrow side
         if (M > 64 && t < 64) continue;
@@ -155,6 +183,12 @@ qlin_status run_gemm(Problem& P, int variant, int tile, int S, size_t w, uint16_
     if (P.s.fmt == QLIN_FMT_BF16)
         return qlin_matmul_bf16(variant, tile, S, P.M, P.s.N, P.s.K, P.a_q, P.w_q[w], nullptr, c, flags, P.ws,
                                 P.ws_bytes, st);
+    if (block_scaled(P.s.fmt)) {
+        const bool nv = P.s.fmt == QLIN_FMT_NVFP4;
+        return qlin_block_scaled_mm(P.s.fmt, variant, tile, S, P.M, P.s.N, P.s.K, P.a_q, P.s_a, P.w_q[w], P.s_w[w],
+                                    nv ? P.g : nullptr, nv ? P.g + 1 : nullptr, nullptr, c, flags, P.ws, P.ws_bytes,
+                                    st);
+    }
     return qlin_scaled_mm(P.s.fmt, variant, tile, S, P.M, P.s.N, P.s.K, P.a_q, P.s_a, P.w_q[w], P.s_w[w], nullptr, c,
                           flags, P.ws, P.ws_bytes, st);
 }
@@ -233,10 +267,12 @@ int main(int argc, char** argv) {
         long long n, k;
         if (std::sscanf(argv[i], "%31[^:]:%lld:%lld", f, &n, &k) != 3) return 1;
         const std::string fs(f);
-        shapes.push_back({fs == "int8"   ? QLIN_FMT_INT8
-                          : fs == "fp8"  ? QLIN_FMT_FP8
-                          : fs == "bf16" ? QLIN_FMT_BF16
-                                         : QLIN_FMT_FP8_BLOCK,
+        shapes.push_back({fs == "int8"    ? QLIN_FMT_INT8
+                          : fs == "fp8"   ? QLIN_FMT_FP8
+                          : fs == "bf16"  ? QLIN_FMT_BF16
+                          : fs == "mxfp8" ? QLIN_FMT_MXFP8
+                          : fs == "nvfp4" ? QLIN_FMT_NVFP4
+                                          : QLIN_FMT_FP8_BLOCK,
                           n, k});
     }
     if (shapes.empty())
@@ -266,29 +302,45 @@ int main(int argc, char** argv) {
         const int64_t M_max = buckets.back();
         Problem P;
         P.s = s;
-        const size_t wbytes = (size_t)s.N * s.K * elem_bytes(s.fmt);
+        const bool bsf = block_scaled(s.fmt);
+        const size_t wbytes = (size_t)s.N * (size_t)row_bytes(s.fmt, s.K);
+        const size_t abytes = (size_t)M_max * (size_t)row_bytes(s.fmt, s.K);
         const size_t ncopy = quick ? 2 : std::max<size_t>(2, (2 * l2 + wbytes - 1) / wbytes + 1);
         const size_t sw_elems = s.fmt == QLIN_FMT_FP8_BLOCK ? (size_t)((s.N + 127) / 128) * (s.K / 128) : (size_t)s.N;
         const size_t sa_elems = s.fmt == QLIN_FMT_FP8_BLOCK ? (size_t)M_max * (s.K / 128) : (size_t)M_max;
-        CK(cudaMalloc(&P.a_q, (size_t)M_max * s.K * elem_bytes(s.fmt)));
-        CK(cudaMalloc(&P.s_a, sa_elems * 4));
+        // scale storage in bytes: fp32 scales, or the tiled block-scale bytes
+        const size_t sa_bytes = bsf ? sf_bytes(s.fmt, M_max, s.K) : sa_elems * 4;
+        const size_t sw_bytes = bsf ? sf_bytes(s.fmt, s.N, s.K) : sw_elems * 4;
+        CK(cudaMalloc(&P.a_q, abytes));
+        CK(cudaMalloc(&P.s_a, sa_bytes));
         if (s.fmt == QLIN_FMT_BF16)
-            fill_bf16<<<1024, 256, 0, st>>>(static_cast<uint16_t*>(P.a_q), (size_t)M_max * s.K, 17u);
+            fill_bf16<<<1024, 256, 0, st>>>(static_cast<uint16_t*>(P.a_q), abytes / 2, 17u);
         else
-            fill_codes<<<1024, 256, 0, st>>>(static_cast<uint8_t*>(P.a_q), (size_t)M_max * s.K, 17u,
-                                             s.fmt != QLIN_FMT_INT8);
-        fill_scales<<<256, 256, 0, st>>>(P.s_a, sa_elems, 5u);
+            fill_codes<<<1024, 256, 0, st>>>(static_cast<uint8_t*>(P.a_q), abytes, 17u,
+                                             s.fmt != QLIN_FMT_INT8 && s.fmt != QLIN_FMT_NVFP4);
+        if (bsf) {
+            fill_sf<<<256, 256, 0, st>>>(reinterpret_cast<uint8_t*>(P.s_a), sa_bytes, 5u, s.fmt == QLIN_FMT_MXFP8);
+            const float g[2] = {1e-2f, 2e-3f};
+            CK(cudaMalloc(&P.g, sizeof g));
+            CK(cudaMemcpy(P.g, g, sizeof g, cudaMemcpyHostToDevice));
+        } else {
+            fill_scales<<<256, 256, 0, st>>>(P.s_a, sa_elems, 5u);
+        }
         for (size_t i = 0; i < ncopy; ++i) {
             void* w;
             float* sw;
             CK(cudaMalloc(&w, wbytes));
-            CK(cudaMalloc(&sw, sw_elems * 4));
+            CK(cudaMalloc(&sw, sw_bytes));
             if (s.fmt == QLIN_FMT_BF16)
                 fill_bf16<<<2048, 256, 0, st>>>(static_cast<uint16_t*>(w), wbytes / 2, 1000u + (uint32_t)i);
             else
                 fill_codes<<<2048, 256, 0, st>>>(static_cast<uint8_t*>(w), wbytes, 1000u + (uint32_t)i,
-                                                 s.fmt != QLIN_FMT_INT8);
-            fill_scales<<<256, 256, 0, st>>>(sw, sw_elems, 77u);
+                                                 s.fmt != QLIN_FMT_INT8 && s.fmt != QLIN_FMT_NVFP4);
+            if (bsf)
+                fill_sf<<<256, 256, 0, st>>>(reinterpret_cast<uint8_t*>(sw), sw_bytes, 77u + (uint32_t)i,
+                                             s.fmt == QLIN_FMT_MXFP8);
+            else
+                fill_scales<<<256, 256, 0, st>>>(sw, sw_elems, 77u);
             P.w_q.push_back(w);
             P.s_w.push_back(sw);
         }
@@ -355,6 +407,7 @@ int main(int argc, char** argv) {
         std::fflush(out);
         cudaFree(P.a_q);
         cudaFree(P.s_a);
+        if (P.g) cudaFree(P.g);
         for (auto p : P.w_q) cudaFree(p);
         for (auto p : P.s_w) cudaFree(p);
         cudaFree(P.c);

@@ -40,6 +40,8 @@ FMT_INT8 = 0
 FMT_FP8 = 1
 FMT_FP8_BLOCK = 2
 FMT_BF16 = 3
+FMT_MXFP8 = 4
+FMT_NVFP4 = 5
 
 M_SWEEP = (1, 4, 8, 16, 32, 64, 256, 512, 1024, 2048)
 LM_HEAD_M = (1, 8, 64, 256, 1024, 2048)
@@ -69,6 +71,13 @@ WORKLOADS = {
     "bf16_attn": Workload("bf16_attn", FMT_BF16, 4096, 2048, M_SWEEP, False, False, False),
     "bf16_lm_head": Workload("bf16_lm_head", FMT_BF16, 151936, 2048, M_SWEEP, False, False, False),
     "bf16_square": Workload("bf16_square", FMT_BF16, 2048, 2048, M_SWEEP, False, False, False),
+    # the block-scaled formats (NVFP4 is listed among vLLM's linear-layer formats)
+    # on the attention-projection, MLP down-projection and lm_head shapes, with
+    # the same activation recipes as the FP8 / Block-FP8 workloads of those shapes
+    "mxfp8_attn": Workload("mxfp8_attn", FMT_MXFP8, 4096, 2048, M_SWEEP, True, True, False),
+    "nvfp4_attn": Workload("nvfp4_attn", FMT_NVFP4, 4096, 2048, M_SWEEP, True, True, False),
+    "mxfp8_down": Workload("mxfp8_down", FMT_MXFP8, 2048, 6144, M_SWEEP, False, False, True),
+    "nvfp4_lm_head": Workload("nvfp4_lm_head", FMT_NVFP4, 151936, 2048, LM_HEAD_M, False, False, False),
 }
 
 

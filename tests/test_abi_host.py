@@ -260,8 +260,22 @@ def test_block_scaled_entry_points_reject_bad_arguments_before_launch(q):
     assert _bsmm(q, fmt=5, K=384, ga=16, gw=16) == q.QLIN_ERR_UNSUPPORTED   # NVFP4: K % 256
     assert _bsmm(q, fmt=5) == q.QLIN_ERR_INVALID_ARG                 # NVFP4 needs both decode scales
     assert _bsmm(q, ga=16, gw=16) == q.QLIN_ERR_INVALID_ARG          # MXFP8 takes none
-    assert _bsmm(q, variant=q.QLIN_VAR_SWAPAB) == q.QLIN_ERR_UNSUPPORTED
     assert _bsmm(q, variant=q.QLIN_VAR_PAIR) == q.QLIN_ERR_UNSUPPORTED
+    # tile support is planned without a device: through the workspace query
+    import ctypes
+
+    def ws(fmt, variant, tile_n):
+        out = ctypes.c_size_t(0)
+        return q.lib.qlin_scaled_mm_workspace_size(fmt, variant, tile_n, 0, 16, 256, 256, ctypes.byref(out))
+
+    assert ws(4, q.QLIN_VAR_SWAPAB, 16) == q.QLIN_ERR_UNSUPPORTED     # whole 32-row quadrants only
+    assert ws(4, q.QLIN_VAR_SWAPAB, 32) == q.QLIN_OK
+    assert ws(4, q.QLIN_VAR_SWAPAB_SPLITK, 64) == q.QLIN_OK
+    out = ctypes.c_size_t(0)
+    assert q.lib.qlin_scaled_mm_workspace_size(4, q.QLIN_VAR_SWAPAB, 32, 0, 33, 256, 256,
+                                               ctypes.byref(out)) == q.QLIN_ERR_UNSUPPORTED  # one activation tile
+    assert ws(4, q.QLIN_VAR_PLAIN, 256) == q.QLIN_ERR_UNSUPPORTED
+    assert ws(4, q.QLIN_VAR_PLAIN, 128) == q.QLIN_OK
     assert _bsmm(q, variant=9) == q.QLIN_ERR_INVALID_ARG
     assert _bsmm(q, flags=q.QLIN_SPLITK_CLUSTER) == q.QLIN_ERR_INVALID_ARG
     assert _bsmm(q, asf=None) == q.QLIN_ERR_INVALID_ARG
@@ -279,11 +293,12 @@ def test_block_scaled_entry_points_reject_bad_arguments_before_launch(q):
     assert L.qlin_quantize_block_scaled(4, 16, 0, 256, 256, None, 16, 16, 0, None) == q.QLIN_OK
 
 
-def test_block_scaled_dispatch_uses_plain_128_tiles(q):
+def test_block_scaled_dispatch_rule(q):
     for fmt in (q.QLIN_FMT_MXFP8, q.QLIN_FMT_NVFP4):
         for M in (1, 16, 64, 256, 2048):
             c = q.qlin_dispatch_query(fmt, M, 4096, 2048)
-            assert c["variant"] in (q.QLIN_VAR_PLAIN, q.QLIN_VAR_SPLITK) and c["tile_n"] == 128, (fmt, M, c)
+            want = (q.QLIN_VAR_SWAPAB, 32 if M <= 32 else 64) if M <= 64 else (q.QLIN_VAR_PLAIN, 128)
+            assert (c["variant"], c["tile_n"], c["k_segments"]) == (*want, 1), (fmt, M, c)
         assert q.qlin_scaled_mm_workspace_size(fmt, 64, 4096, 2048, q.QLIN_VAR_PLAIN) == 0
         ws = q.qlin_scaled_mm_workspace_size(fmt, 64, 4096, 2048, q.QLIN_VAR_SPLITK, 0, 4)
         assert ws == 65536 + 4 * 32 * 128 * 128 * 4

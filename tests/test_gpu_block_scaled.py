@@ -9,9 +9,10 @@ their public definitions (readings in ``oracle/qlin_oracle.c``).
     saturating blocks and a wide spread of block magnitudes;
   - GEMM (tcgen05 block-scaled MMA, scale factors in TMEM): on the oracle's
     codes and scales, within |d| <= 1e-2 |ref| + 1e-3 of the oracle's GEMM,
-    for plain and Split-K tiles, ragged M and N, with and without bias;
-    every variant with the same K segmentation bitwise equal; AUTO dispatch
-    batch-invariant (the first rows of C do not change with M);
+    for plain, Split-K and Swap-AB (32 / 64) tiles, ragged M and N, with and
+    without bias; every variant with the same K segmentation bitwise equal;
+    AUTO dispatch (Swap-AB at small M, plain above) batch-invariant: the first
+    rows of C do not change with M;
   - the chain (GPU quantiser -> GPU GEMM) at the attention-projection shape
     N = 4096, K = 2048, sampled rows against the oracle.
 """
@@ -142,7 +143,8 @@ def _ref(fmt, aq, asf, wq, wsf, ga, gw, b, m_idx=None):
 
 
 @pytest.mark.parametrize("fmt", [MX, NV], ids=["mxfp8", "nvfp4"])
-@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (77, 384, 1024), (300, 272, 768), (129, 128, 2048)])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 512), (29, 384, 1024), (64, 272, 768), (77, 384, 1024),
+                                   (300, 272, 768), (129, 128, 2048)])
 def test_gemm_matches_oracle(fmt, M, N, K):
     if fmt == NV and K % 256:
         K = 1024
@@ -156,16 +158,19 @@ def test_gemm_matches_oracle(fmt, M, N, K):
     check_status()
     assert_fp_parity(bits_u16(c_plain), ref, f"fmt {fmt} plain S=1")
     kblocks = (K // 2 if fmt == NV else K) // 128
+    run = lambda v, t, S: bits_u16(gpu_block_scaled_mm(fmt, d[0], d[1], d[2], d[3], d[6], d[4], d[5], variant=v,
+                                                       tile_n=t, k_segments=S))
+    swap_tiles = [t for t in (32, 64) if M <= t]  # Swap-AB: one activation tile
+    for t in swap_tiles:  # bitwise the plain tile's result
+        assert np.array_equal(run(qlin.QLIN_VAR_SWAPAB, t, 1), bits_u16(c_plain)), f"Swap-AB {t} S=1"
     for S in (2, 4):
         if kblocks % S:
             continue
-        cp = gpu_block_scaled_mm(fmt, d[0], d[1], d[2], d[3], d[6], d[4], d[5], variant=qlin.QLIN_VAR_PLAIN,
-                                 k_segments=S)
-        cs = gpu_block_scaled_mm(fmt, d[0], d[1], d[2], d[3], d[6], d[4], d[5], variant=qlin.QLIN_VAR_SPLITK,
-                                 k_segments=S)
-        torch.cuda.synchronize()
-        assert np.array_equal(bits_u16(cp), bits_u16(cs)), f"S={S}: Split-K differs from plain"
-        assert_fp_parity(bits_u16(cs), ref, f"fmt {fmt} S={S}")
+        cp = run(qlin.QLIN_VAR_PLAIN, 128, S)
+        assert_fp_parity(cp, ref, f"fmt {fmt} S={S}")
+        for v, t in [(qlin.QLIN_VAR_SPLITK, 128)] + [(qlin.QLIN_VAR_SWAPAB, t) for t in swap_tiles] + \
+                [(qlin.QLIN_VAR_SWAPAB_SPLITK, t) for t in swap_tiles]:
+            assert np.array_equal(run(v, t, S), cp), f"S={S}: variant {v} tile {t} differs from plain"
     check_status()
 
 
@@ -215,3 +220,34 @@ def test_quantise_then_gemm_attention_projection(fmt, M):
     assert np.array_equal(bits_u8(aq)[rows], raq)
     ref = _ref(fmt, raq, rasf, rwq, rwsf, ga, gw, b)
     assert_fp_parity(bits_u16(c)[rows], ref, f"fmt {fmt} M={M}")
+
+
+@pytest.mark.parametrize("fmt", [MX, NV], ids=["mxfp8", "nvfp4"])
+def test_shipped_table_dispatch_is_batch_invariant(fmt):
+    """The shipped dispatch table's entries for the attention projection
+    (Swap-AB Split-K at small M, plain tiles above, one K segmentation):
+    the first 16 rows of C are bitwise the same at every M, and match the
+    oracle."""
+    import os
+
+    qlin = _q()
+    table = os.path.join(os.path.dirname(qlin.__file__), "tables", "b200.qlt")
+    qlin.qlin_dispatch_table_load(table)
+    try:
+        N, K = 4096, 2048
+        a, w, b, aq, asf, wq, wsf, ga, gw = _operands(fmt, 600, N, K, seed=21)
+        segs = {qlin.qlin_dispatch_query(fmt, M, N, K)["k_segments"] for M in (1, 64, 128, 600)}
+        assert len(segs) == 1 and all(qlin.qlin_dispatch_query(fmt, M, N, K)["from_table"] for M in (1, 600))
+        first = None
+        for M in (16, 1, 5, 33, 64, 100, 600):
+            d = _dev_ops(fmt, aq[:M], asf[:M], wq, wsf, ga, gw, b)
+            c = bits_u16(gpu_block_scaled_mm(fmt, d[0], d[1], d[2], d[3], d[6], d[4], d[5], flags=qlin.QLIN_PDL))
+            torch.cuda.synchronize()
+            r = min(M, 16)
+            if first is None:
+                first = c[:16].copy()
+                assert_fp_parity(first, _ref(fmt, aq[:16], asf[:16], wq, wsf, ga, gw, b), f"fmt {fmt}")
+            assert np.array_equal(c[:r], first[:r]), f"M={M}"
+        check_status()
+    finally:
+        qlin.qlin_dispatch_table_clear()
