@@ -201,10 +201,11 @@ struct Cfg {
     static constexpr int TMEM_COLS = pow2_at_least(SF_COL + 2 * SF_COLS);
     static_assert(NACC * ACC_COLS <= TOTAL_COL, "accumulators overlap the running total");
     static constexpr uint32_t IDESC = BS ? make_idesc_bs(KIND, 128, BN) : make_idesc(KIND, PAIR ? 256 : 128, BN);
-    // K blocks the MMA thread takes per pass: 4 for the dense Swap-AB tiles
-    // (measured: 3-8 % less time at small M, bitwise the same C); 1 elsewhere,
+    // K blocks the MMA thread takes per pass: 4 for the Swap-AB tiles with rings
+    // of 8 stages or more (measured: 3-8 % less time at small M, bitwise the
+    // same C); 1 elsewhere,
     // where the 4-6 stage rings of the wide tiles need each stage released at once
-    static constexpr int MMA_GROUP = (SWAP && !BS && !FUSE && !BLOCK && STAGES >= 8) ? 4 : 1;
+    static constexpr int MMA_GROUP = (SWAP && !FUSE && !BLOCK && STAGES >= 8) ? 4 : 1;
     static constexpr size_t STAGING_OFF = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t SCALE_OFF = STAGING_OFF + kStagingBytes;
     static constexpr size_t BSCALE_OFF = SCALE_OFF + kScaleBytes;
@@ -1146,53 +1147,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!acc_free) goto done;
                     tc_fence_after();
                     const uint32_t d = tmem_base + abuf * C::ACC_COLS;
-                    for (int kb = c0; kb < c0 + un.chunk_kb; ++kb) {
-                        if constexpr (C::MMA_GROUP > 1) {
-                            // Swap-AB: G K blocks per pass (G waits, 4G MMAs, G commits).
-                            // The narrow MMAs are cheap for the tensor pipe and the
-                            // issuing thread's per-K-block work sets the pace; one pass
-                            // over G stages spends it once.  Same MMAs in the same order.
-                            constexpr int G = C::MMA_GROUP;
-                            if (((kb - c0) % G) == 0 && kb + G <= c0 + un.chunk_kb) {
-                                uint32_t sg[G], pg[G];
-                                sg[0] = stage;
-                                pg[0] = phase;
-#pragma unroll
-                                for (int g = 1; g < G; ++g) {
-                                    const bool wrap = sg[g - 1] + 1 == STAGES;
-                                    sg[g] = wrap ? 0u : sg[g - 1] + 1;
-                                    pg[g] = wrap ? (pg[g - 1] ^ 1u) : pg[g - 1];
-                                }
-#pragma unroll
-                                for (int g = 0; g < G; ++g)
-                                    if (!mbar_wait(full0 + 8 * sg[g], pg[g])) goto done;
-                                tc_fence_after();
-#pragma unroll
-                                for (int g = 0; g < G; ++g) {
-                                    const uint64_t ad = smem_desc_k_sw128(smem_u32(sP + (size_t)sg[g] * C::P_BYTES));
-                                    const uint64_t bd = smem_desc_k_sw128(smem_u32(sQ + (size_t)sg[g] * C::Q_BYTES));
-#pragma unroll
-                                    for (int k = 0; k < 4; ++k)
-                                        tc_mma<C::KIND>(d, ad + 2 * k, bd + 2 * k, C::IDESC,
-                                                        (kb + g > c0 || k > 0) ? 1u : 0u);
-                                }
-#pragma unroll
-                                for (int g = 0; g < G; ++g) tc_commit(empty0 + 8 * sg[g]);
-                                const bool wrap = sg[G - 1] + 1 == STAGES;
-                                stage = wrap ? 0u : sg[G - 1] + 1;
-                                phase = wrap ? (pg[G - 1] ^ 1u) : pg[G - 1];
-                                kb += G - 1;
-                                continue;
-                            }
-                        }
-                        const bool landed = PAIR ? mbar_wait_cluster(full0 + 8 * stage, phase)
-                                                 : mbar_wait(full0 + 8 * stage, phase);
-                        if (!landed) goto done;
-                        tc_fence_after();
-                        const uint64_t adesc = smem_desc_k_sw128(smem_u32(sP + (size_t)stage * C::P_BYTES));
+                    // the four MMAs (32 bytes of K each) of K block kb from stage st
+                    auto issue_stage = [&](uint32_t st, int kb) {
+                        const uint64_t adesc = smem_desc_k_sw128(smem_u32(sP + (size_t)st * C::P_BYTES));
                         const uint64_t bdesc =
                             FUSE ? smem_desc_k_sw128(sA + (uint32_t)((kb - un.kb0) * BN * 128))
-                                 : smem_desc_k_sw128(smem_u32(sQ + (size_t)stage * C::Q_BYTES));
+                                 : smem_desc_k_sw128(smem_u32(sQ + (size_t)st * C::Q_BYTES));
                         if constexpr (C::BS) {
                             // this K block's scale factors into TMEM (the tensor pipe runs the
                             // copies and the MMAs in issue order); A's atoms, then W's, 4
@@ -1200,7 +1160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             constexpr int RG = C::SF_RGQ;
                             const uint32_t sfa_t = tmem_base + C::SF_COL + (sfi & 1u) * C::SF_COLS;
                             const uint32_t sfb_t = sfa_t + 4 * C::SF_APK;
-                            const uint32_t sfs = smem_u32(sF + (size_t)stage * C::SF_BYTES);
+                            const uint32_t sfs = smem_u32(sF + (size_t)st * C::SF_BYTES);
 #pragma unroll
                             for (int at = 0; at < C::SF_APK; ++at) {
                                 tc_cp_sf(sfa_t + 4 * at, smem_desc_sf(sfs + 512 * at));
@@ -1223,7 +1183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ++sfi;
                         } else {
 #pragma unroll
-                            for (int k = 0; k < 4; ++k) {  // 4 x K=32 bytes per 128-byte stage
+                            for (int k = 0; k < 4; ++k) {
                                 const uint32_t accum = (kb > c0 || k > 0) ? 1u : 0u;
                                 if constexpr (PAIR)
                                     tc_mma_pair<C::KIND>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
@@ -1231,6 +1191,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     tc_mma<C::KIND>(d, adesc + 2 * k, bdesc + 2 * k, C::IDESC, accum);
                             }
                         }
+                    };
+                    for (int kb = c0; kb < c0 + un.chunk_kb; ++kb) {
+                        if constexpr (C::MMA_GROUP > 1) {
+                            // Swap-AB: G K blocks per pass (G waits, 4G MMAs, G commits).
+                            // The narrow MMAs are cheap for the tensor pipe and the
+                            // issuing thread's per-K-block work sets the pace; one pass
+                            // over G stages spends it once.  Same MMAs in the same order.
+                            constexpr int G = C::MMA_GROUP;
+                            if (((kb - c0) % G) == 0 && kb + G <= c0 + un.chunk_kb) {
+                                uint32_t sg[G], pg[G];
+                                sg[0] = stage;
+                                pg[0] = phase;
+#pragma unroll
+                                for (int g = 1; g < G; ++g) {
+                                    const bool wrap = sg[g - 1] + 1 == STAGES;
+                                    sg[g] = wrap ? 0u : sg[g - 1] + 1;
+                                    pg[g] = wrap ? (pg[g - 1] ^ 1u) : pg[g - 1];
+                                }
+#pragma unroll
+                                for (int g = 0; g < G; ++g)
+                                    if (!mbar_wait(full0 + 8 * sg[g], pg[g])) goto done;
+                                tc_fence_after();
+#pragma unroll
+                                for (int g = 0; g < G; ++g) issue_stage(sg[g], kb + g);
+#pragma unroll
+                                for (int g = 0; g < G; ++g) tc_commit(empty0 + 8 * sg[g]);
+                                const bool wrap = sg[G - 1] + 1 == STAGES;
+                                stage = wrap ? 0u : sg[G - 1] + 1;
+                                phase = wrap ? (pg[G - 1] ^ 1u) : pg[G - 1];
+                                kb += G - 1;
+                                continue;
+                            }
+                        }
+                        const bool landed = PAIR ? mbar_wait_cluster(full0 + 8 * stage, phase)
+                                                 : mbar_wait(full0 + 8 * stage, phase);
+                        if (!landed) goto done;
+                        tc_fence_after();
+                        issue_stage(stage, kb);
                         if constexpr (PAIR)
                             tc_commit_pair(empty0 + 8 * stage, 0x3);  // both CTAs may refill the stage
                         else
