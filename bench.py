@@ -15,13 +15,17 @@ Prints one JSON line (rank 0):
               resident, one CUDA graph per step
   e2e         the same steps through the same C ABI calls with the bf16
               activations copied in from pinned host memory and C copied back
+              (eager launches; the copies run on two copy streams ordered by
+              events, so they overlap each other and the kernels)
   roofline    the dominant kernel of the headline workload (largest share of
               device time) against the measured HBM / tensor peak
   per_m       per (M, N, K, format) of the headline workload: GEMM and
               quantiser time, TFLOP/s, HBM GB/s, roofline fraction
   workloads   the same per-M table, step time and dominant-kernel roofline for
               every workload of the metric (INT8 smoke, FP8 attention,
-              Block-FP8 down projection, lm_head, FP8 12288 x 2048, INT8 2048^2)
+              Block-FP8 down projection, lm_head, FP8 12288 x 2048, INT8 2048^2),
+              the bf16 matmul on its five shapes, the MXFP8 / NVFP4 workloads
+              and the FP8 MoE layer
   tensor_peaks  dense FP8 (torch._scaled_mm) and INT8 (torch._int_mm) library
               GEMM throughput at 8192^3 measured on this GPU (burst, best of 10)
   cpu_baseline  the CPU oracle on a bounded sample (rank 0, N = 1 only), on one
@@ -408,21 +412,65 @@ class HotPath:
         return graphs
 
     def step_e2e(self, stream):
-        """Same step with the activations copied in from pinned host memory and
-        C copied back; returns (h2d bytes, d2h bytes)."""
+        """The same step through the C ABI, with each M's activations copied in
+        from pinned host memory and its C copied back.  The copies run on two
+        copy streams, ordered against the kernels by events (copy-in ->
+        quantise + GEMM -> copy-out), so transfers in both directions overlap
+        each other and the kernels of other M.  Two activation sets alternate
+        between steps.  Returns (h2d bytes, d2h bytes) of the step."""
         hb = db = 0
-        self.act = 0
         if self.a_host is None:
             self.a_host = {M: self.a_cpu[M].pin_memory() for M in self.ms}
             self.c_host = {M: torch.empty(M, self.w.N, dtype=torch.bfloat16).pin_memory() for M in self.ms}
+            self.s_in = torch.cuda.Stream(self.device)
+            self.s_out = torch.cuda.Stream(self.device)
+            self.e2e_step = 0
+            self.ev_act_free = {}  # (set, M): the kernels that read that activation buffer are done
+            self.ev_c_free = {}    # M: C[M] has been copied out
+        slot = self.e2e_step % min(2, self.n_act_sets)
+        if self.e2e_step == 0:  # the copy streams start after everything issued before
+            start = torch.cuda.Event()
+            start.record(stream)
+            self.s_in.wait_event(start)
+            self.s_out.wait_event(start)
+        self.e2e_step += 1
         for M in self.ms:
-            self.a_sets[0][M].copy_(self.a_host[M], non_blocking=True)
+            ev = self.ev_act_free.get((slot, M))
+            if ev is not None:
+                self.s_in.wait_event(ev)
+            with torch.cuda.stream(self.s_in):
+                self.a_sets[slot][M].copy_(self.a_host[M], non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(self.s_in)
             hb += self.a_host[M].numel() * 2
+            stream.wait_event(ev_in)
+            if M in self.ev_c_free:
+                stream.wait_event(self.ev_c_free[M])
+            self.act = slot
             self.launch_quant(M, stream)
             self.launch_gemm(M, stream)
-            self.c_host[M].copy_(self.c[M], non_blocking=True)
+            ev_k = torch.cuda.Event()
+            ev_k.record(stream)
+            self.ev_act_free[(slot, M)] = ev_k
+            self.s_out.wait_event(ev_k)
+            with torch.cuda.stream(self.s_out):
+                self.c_host[M].copy_(self.c[M], non_blocking=True)
+            ev_out = torch.cuda.Event()
+            ev_out.record(self.s_out)
+            self.ev_c_free[M] = ev_out
             db += self.c[M].numel() * 2
         return hb, db
+
+    def e2e_after(self, event):
+        """Order the copy streams after `event` (the start of the timed region)."""
+        self.s_in.wait_event(event)
+        self.s_out.wait_event(event)
+
+    def e2e_join(self, stream):
+        """Make `stream` wait for the last copy-out issued (steps overlap: the next
+        step's copy-in and kernels may start before this one's copies end)."""
+        if self.ev_c_free:
+            stream.wait_event(self.ev_c_free[self.ms[-1]])
 
 
 class MoEPath:
@@ -805,9 +853,11 @@ def main(argv=None):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        hp.e2e_after(e0)
         hb = db = 0
         for _ in range(args.steps):
             hb, db = hp.step_e2e(stream)
+        hp.e2e_join(stream)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -871,6 +921,8 @@ def main(argv=None):
                        "l2": ("inputs larger than L2: weights rotate per GEMM and activations per step, "
                               "> 2x L2 between two uses of one copy"),
                        "parallelism": "replicas" if world > 1 else "single GPU", "cuda_graph": args.graph,
+                       "e2e": ("each M's activations copied in from pinned host memory and C copied back, on "
+                               "two copy streams ordered by events, overlapping the kernels; eager launches"),
                        "pdl": True,
                        "table": (not args.no_table and os.path.exists(args.table))},
             "roofline": roof,
