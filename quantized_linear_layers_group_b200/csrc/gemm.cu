@@ -201,11 +201,14 @@ struct Cfg {
     static constexpr int TMEM_COLS = pow2_at_least(SF_COL + 2 * SF_COLS);
     static_assert(NACC * ACC_COLS <= TOTAL_COL, "accumulators overlap the running total");
     static constexpr uint32_t IDESC = BS ? make_idesc_bs(KIND, 128, BN) : make_idesc(KIND, PAIR ? 256 : 128, BN);
-    // K blocks the MMA thread takes per pass: 4 for the Swap-AB tiles with rings
-    // of 8 stages or more (measured: 3-8 % less time at small M, bitwise the
-    // same C); 1 elsewhere,
-    // where the 4-6 stage rings of the wide tiles need each stage released at once
-    static constexpr int MMA_GROUP = (SWAP && !FUSE && !BLOCK && STAGES >= 8) ? 4 : 1;
+    // K blocks the MMA thread takes per pass (measured; the MMAs and their order
+    // are the same, so C is bitwise the same): 4 for Swap-AB tiles with rings of
+    // 8+ stages (3-8 % less time at small M), 2 for plain 128-column tiles
+    // (6-stage rings, 3-5 %), 1 for the 256-column tiles, whose 4-stage rings
+    // need each stage released at once (grouping them cost 10-50 %)
+    static constexpr int MMA_GROUP = (FUSE || BLOCK || PAIR) ? 1
+                                     : (SWAP && STAGES >= 8) ? 4
+                                     : (!SWAP && BN == 128 && STAGES >= 6) ? 2 : 1;
     static constexpr size_t STAGING_OFF = (size_t)STAGES * STAGE_BYTES;
     static constexpr size_t SCALE_OFF = STAGING_OFF + kStagingBytes;
     static constexpr size_t BSCALE_OFF = SCALE_OFF + kScaleBytes;
@@ -1194,10 +1197,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     };
                     for (int kb = c0; kb < c0 + un.chunk_kb; ++kb) {
                         if constexpr (C::MMA_GROUP > 1) {
-                            // Swap-AB: G K blocks per pass (G waits, 4G MMAs, G commits).
-                            // The narrow MMAs are cheap for the tensor pipe and the
-                            // issuing thread's per-K-block work sets the pace; one pass
-                            // over G stages spends it once.  Same MMAs in the same order.
+                            // G K blocks per pass (G waits, 4G MMAs, G commits): the
+                            // issuing thread's per-K-block work (barrier test, fence,
+                            // loop) sets the pace of narrow tiles; one pass over G
+                            // stages spends it once.  Same MMAs in the same order.
                             constexpr int G = C::MMA_GROUP;
                             if (((kb - c0) % G) == 0 && kb + G <= c0 + un.chunk_kb) {
                                 uint32_t sg[G], pg[G];
