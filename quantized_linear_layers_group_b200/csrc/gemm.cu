@@ -1414,26 +1414,71 @@ __global__ void __launch_bounds__(kThreads, 1)
                         asm volatile("ld.shared.f32 %0, [%1];"
                                      : "=f"(row_scale)
                                      : "r"(bsc + (uint32_t)((c0 - win0) * C::BS_PITCH + e.row_lane) * 4u));
-                        if (!acc_wait(tfull0 + 8 * abuf, aphase)) goto done;
-                        tc_fence_after();
-                        uint32_t v[2 * SW];
-                        tmem_ld64(t_lane + abuf * C::ACC_COLS + e.half * 2 * SW, v);
-                        tc_wait_ld();
-                        tc_fence_before();
-                        acc_release(tempty0 + 8 * abuf);
-                        next_acc<NACC>(abuf, aphase);
-                        if (seg_start) {
+                        if (kin + 1 < kbps && c0 + 1 < un.kb1 && c0 + 1 - win0 < C::BS_KB) {
+                            // two K blocks of the segment in one pass: one accumulator
+                            // wait covers both (the second buffer's commit arrives only
+                            // after every earlier MMA has completed), the same fmas in
+                            // the same order
+                            float row_scale1;
+                            asm volatile("ld.shared.f32 %0, [%1];"
+                                         : "=f"(row_scale1)
+                                         : "r"(bsc + (uint32_t)((c0 + 1 - win0) * C::BS_PITCH + e.row_lane) * 4u));
+                            uint32_t abuf1 = abuf, aphase1 = aphase;
+                            next_acc<NACC>(abuf1, aphase1);
+                            if (!acc_wait(tfull0 + 8 * abuf1, aphase1)) goto done;
+                            tc_fence_after();
+                            uint32_t v[2 * SW];
+                            tmem_ld64(t_lane + abuf * C::ACC_COLS + e.half * 2 * SW, v);
+                            tc_wait_ld();
+                            tc_fence_before();
+                            acc_release(tempty0 + 8 * abuf);
+                            if (seg_start) {
+#pragma unroll
+                                for (int c = 0; c < 2 * SW; c += 2)
+                                    fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                            row_scale, 0.f, 0.f);
+                            } else {
+#pragma unroll
+                                for (int c = 0; c < 2 * SW; c += 2)
+                                    fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                            row_scale, sg[c], sg[c + 1]);
+                            }
+                            tmem_ld64(t_lane + abuf1 * C::ACC_COLS + e.half * 2 * SW, v);
+                            tc_wait_ld();
+                            tc_fence_before();
+                            acc_release(tempty0 + 8 * abuf1);
+                            abuf = abuf1;
+                            aphase = aphase1;
+                            next_acc<NACC>(abuf, aphase);
 #pragma unroll
                             for (int c = 0; c < 2 * SW; c += 2)
-                                fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]), row_scale,
-                                        0.f, 0.f);
+                                fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                        row_scale1, sg[c], sg[c + 1]);
+                            ++c0;
+                            kin += 2;
+                            if (kin < kbps) continue;
                         } else {
+                            if (!acc_wait(tfull0 + 8 * abuf, aphase)) goto done;
+                            tc_fence_after();
+                            uint32_t v[2 * SW];
+                            tmem_ld64(t_lane + abuf * C::ACC_COLS + e.half * 2 * SW, v);
+                            tc_wait_ld();
+                            tc_fence_before();
+                            acc_release(tempty0 + 8 * abuf);
+                            next_acc<NACC>(abuf, aphase);
+                            if (seg_start) {
 #pragma unroll
-                            for (int c = 0; c < 2 * SW; c += 2)
-                                fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]), row_scale,
-                                        sg[c], sg[c + 1]);
+                                for (int c = 0; c < 2 * SW; c += 2)
+                                    fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]), row_scale,
+                                            0.f, 0.f);
+                            } else {
+#pragma unroll
+                                for (int c = 0; c < 2 * SW; c += 2)
+                                    fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]), row_scale,
+                                            sg[c], sg[c + 1]);
+                            }
+                            if (++kin < kbps) continue;
                         }
-                        if (++kin < kbps) continue;
                         kin = 0;
                         // segment end: Split-K writes the segment out; otherwise
                         // total = total + seg in segment order from +0 (the total
