@@ -206,6 +206,9 @@ struct Cfg {
     // 8+ stages (3-8 % less time at small M), 2 for plain 128-column tiles
     // (6-stage rings, 3-5 %), 1 for the 256-column tiles, whose 4-stage rings
     // need each stage released at once (grouping them cost 10-50 %)
+    // Block-FP8 plain tiles: K blocks the epilogue folds in per accumulator wait
+    // (at most NACC - 1, so the MMA always has a free buffer)
+    static constexpr int BLOCK_PASS = 2;
     static constexpr int MMA_GROUP = (FUSE || BLOCK || PAIR) ? 1
                                      : (SWAP && STAGES >= 8) ? 4
                                      : (!SWAP && BN == 128 && STAGES >= 6) ? 2 : 1;
@@ -1414,48 +1417,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                         asm volatile("ld.shared.f32 %0, [%1];"
                                      : "=f"(row_scale)
                                      : "r"(bsc + (uint32_t)((c0 - win0) * C::BS_PITCH + e.row_lane) * 4u));
-                        if (kin + 1 < kbps && c0 + 1 < un.kb1 && c0 + 1 - win0 < C::BS_KB) {
-                            // two K blocks of the segment in one pass: one accumulator
-                            // wait covers both (the second buffer's commit arrives only
-                            // after every earlier MMA has completed), the same fmas in
+                        constexpr int P = C::BLOCK_PASS;
+                        if (kin + P - 1 < kbps && c0 + P - 1 < un.kb1 && c0 + P - 1 - win0 < C::BS_KB) {
+                            // P K blocks of the segment in one pass: one accumulator
+                            // wait covers them all (the last buffer's commit arrives
+                            // only after every earlier MMA has completed); each block
+                            // is then loaded, released and folded in, the same fmas in
                             // the same order
-                            float row_scale1;
-                            asm volatile("ld.shared.f32 %0, [%1];"
-                                         : "=f"(row_scale1)
-                                         : "r"(bsc + (uint32_t)((c0 + 1 - win0) * C::BS_PITCH + e.row_lane) * 4u));
-                            uint32_t abuf1 = abuf, aphase1 = aphase;
-                            next_acc<NACC>(abuf1, aphase1);
-                            if (!acc_wait(tfull0 + 8 * abuf1, aphase1)) goto done;
+                            float rs[P];
+                            rs[0] = row_scale;
+#pragma unroll
+                            for (int q = 1; q < P; ++q)
+                                asm volatile("ld.shared.f32 %0, [%1];"
+                                             : "=f"(rs[q])
+                                             : "r"(bsc + (uint32_t)((c0 + q - win0) * C::BS_PITCH + e.row_lane) * 4u));
+                            uint32_t bl = abuf, pl = aphase;
+#pragma unroll
+                            for (int q = 1; q < P; ++q) next_acc<NACC>(bl, pl);
+                            if (!acc_wait(tfull0 + 8 * bl, pl)) goto done;
                             tc_fence_after();
-                            uint32_t v[2 * SW];
-                            tmem_ld64(t_lane + abuf * C::ACC_COLS + e.half * 2 * SW, v);
-                            tc_wait_ld();
-                            tc_fence_before();
-                            acc_release(tempty0 + 8 * abuf);
-                            if (seg_start) {
 #pragma unroll
-                                for (int c = 0; c < 2 * SW; c += 2)
-                                    fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                                            row_scale, 0.f, 0.f);
-                            } else {
+                            for (int q = 0; q < P; ++q) {
+                                uint32_t v[2 * SW];
+                                tmem_ld64(t_lane + abuf * C::ACC_COLS + e.half * 2 * SW, v);
+                                tc_wait_ld();
+                                tc_fence_before();
+                                acc_release(tempty0 + 8 * abuf);
+                                next_acc<NACC>(abuf, aphase);
+                                if (q == 0 && seg_start) {
 #pragma unroll
-                                for (int c = 0; c < 2 * SW; c += 2)
-                                    fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                                            row_scale, sg[c], sg[c + 1]);
+                                    for (int c = 0; c < 2 * SW; c += 2)
+                                        fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                                rs[q], 0.f, 0.f);
+                                } else {
+#pragma unroll
+                                    for (int c = 0; c < 2 * SW; c += 2)
+                                        fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                                rs[q], sg[c], sg[c + 1]);
+                                }
                             }
-                            tmem_ld64(t_lane + abuf1 * C::ACC_COLS + e.half * 2 * SW, v);
-                            tc_wait_ld();
-                            tc_fence_before();
-                            acc_release(tempty0 + 8 * abuf1);
-                            abuf = abuf1;
-                            aphase = aphase1;
-                            next_acc<NACC>(abuf, aphase);
-#pragma unroll
-                            for (int c = 0; c < 2 * SW; c += 2)
-                                fma2_rn(sg[c], sg[c + 1], __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                                        row_scale1, sg[c], sg[c + 1]);
-                            ++c0;
-                            kin += 2;
+                            c0 += P - 1;
+                            kin += P;
                             if (kin < kbps) continue;
                         } else {
                             if (!acc_wait(tfull0 + 8 * abuf, aphase)) goto done;
