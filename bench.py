@@ -32,6 +32,10 @@ Prints one JSON line (rank 0):
               thread and on every host core
 
   --impl reference  times the CPU oracle as the reference arm instead.
+  --fused           runs each layer through qlin_linear with QLIN_FUSED: one
+                    kernel where the configuration is Swap-AB (the GEMM
+                    quantises its own activation rows), else the same two
+                    kernels; gpu_launches counts what is launched.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs the same
 independent step on its own GPU (no data-path collective; weak scaling); the
@@ -302,12 +306,15 @@ class HotPath:
     (one CUDA graph) reads its own set of activation copies, so that the bytes
     read between two uses of one copy exceed 2x L2 for both."""
 
-    def __init__(self, workload: synth.Workload, m_values, device, seed=0):
+    def __init__(self, workload: synth.Workload, m_values, device, seed=0, fused=False):
         from quantized_linear_layers_group_b200 import linear, qlin
 
         self.qlin, self.linear = qlin, linear
         self.w = workload
         self.fmt = workload.fmt
+        # fused: each M goes through qlin_linear with QLIN_FUSED (one kernel
+        # where the configuration is Swap-AB, else the quantiser + the GEMM)
+        self.fused = fused and self.fmt in (0, 1, 2)
         self.ms = list(m_values)
         self.device = device
         N, K = workload.N, workload.K
@@ -392,12 +399,38 @@ class HotPath:
         self.qlin.qlin_scaled_mm(self.fmt, self.a_q[M], self.s_a[M], w_q, s_w, self.bias, self.c[M],
                                  self.workspace, stream, flags=self.flags)
 
+    def layer_is_fused(self, M):
+        """Whether qlin_linear runs M as one kernel: Swap-AB configurations
+        whose unit of K blocks fits the resident activation operand (64 KiB)."""
+        if not self.fused:
+            return False
+        cfg = self.configs[M]
+        if cfg["variant"] not in (self.qlin.QLIN_VAR_SWAPAB, self.qlin.QLIN_VAR_SWAPAB_SPLITK):
+            return False
+        kblocks = self.w.K // 128
+        per_unit = kblocks // cfg["k_segments"] if cfg["k_segments"] > 1 else kblocks
+        return per_unit <= 65536 // (cfg["tile_n"] * 128)
+
+    def kernels_per_step(self):
+        return sum(1 if (self.fmt == 3 or self.layer_is_fused(M)) else 2 for M in self.ms)
+
+    def launch_layer(self, M, stream):
+        """Quantise + GEMM for one M: two PDL-chained kernels, or one call of
+        qlin_linear with QLIN_FUSED."""
+        if not self.fused:
+            self.launch_quant(M, stream)
+            self.launch_gemm(M, stream)
+            return
+        w_q, s_w = self.w_copies[self.calls % self.n_copies]
+        self.calls += 1
+        self.qlin.qlin_linear(self.fmt, self.a_sets[self.act][M], self.a_q[M], self.s_a[M], w_q, s_w, self.bias,
+                              self.c[M], self.workspace, stream, flags=self.flags | self.qlin.QLIN_FUSED)
+
     def step(self, stream, act_set=None):
         """Issue one step: for each M, the quantiser then the GEMM (PDL)."""
         self.act = (self.act + 1) % self.n_act_sets if act_set is None else act_set
         for M in self.ms:
-            self.launch_quant(M, stream)
-            self.launch_gemm(M, stream)
+            self.launch_layer(M, stream)
 
     def capture_graphs(self, stream):
         """One CUDA graph per step of a rotation: graph g reads activation set
@@ -447,8 +480,7 @@ class HotPath:
             if M in self.ev_c_free:
                 stream.wait_event(self.ev_c_free[M])
             self.act = slot
-            self.launch_quant(M, stream)
-            self.launch_gemm(M, stream)
+            self.launch_layer(M, stream)
             ev_k = torch.cuda.Event()
             ev_k.record(stream)
             self.ev_act_free[(slot, M)] = ev_k
@@ -806,6 +838,8 @@ def main(argv=None):
     ap.add_argument("--table", default=os.path.join(ROOT, "quantized_linear_layers_group_b200", "tables",
                                                     "b200.qlt"))
     ap.add_argument("--no-table", action="store_true")
+    ap.add_argument("--fused", action="store_true",
+                    help="quantise inside the GEMM where the configuration is Swap-AB (qlin_linear, QLIN_FUSED)")
     ap.add_argument("--graph", dest="graph", action="store_true", default=True,
                     help="replay each device-timed step as a CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false")
@@ -834,7 +868,7 @@ def main(argv=None):
     peaks = load_peaks()
 
     with torch.cuda.stream(stream):
-        hp = HotPath(workload, ms, device)
+        hp = HotPath(workload, ms, device, fused=args.fused)
         for _ in range(args.warmup):
             hp.step(stream)
         torch.cuda.synchronize()
@@ -867,6 +901,7 @@ def main(argv=None):
         tpk = None if args.no_peaks else measure_tensor_peaks(device)
         qt, gt = per_kernel_times(hp, stream)
         per_m, roof, tc_peak, tc_src = workload_report(hp, qt, gt, peaks, tpk)
+        kernels_per_step = hp.kernels_per_step()
         st = qlin.qlin_sync_status(stream)
         if st != 0:
             raise RuntimeError(f"device status: {qlin.qlin_status_string(st)}")
@@ -921,6 +956,7 @@ def main(argv=None):
                        "l2": ("inputs larger than L2: weights rotate per GEMM and activations per step, "
                               "> 2x L2 between two uses of one copy"),
                        "parallelism": "replicas" if world > 1 else "single GPU", "cuda_graph": args.graph,
+                       "fused": bool(args.fused),
                        "e2e": ("each M's activations copied in from pinned host memory and C copied back, on "
                                "two copy streams ordered by events, overlapping the kernels; eager launches"),
                        "pdl": True,
@@ -930,7 +966,7 @@ def main(argv=None):
             "tensor_peak_used": {"value": tc_peak, "source": tc_src},
             "tensor_peaks": tpk,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db},
-            "gpu_launches": 2 * len(ms) * args.steps,
+            "gpu_launches": kernels_per_step * args.steps,
             "clocks": clk,
             "per_m": per_m}
     if workloads:

@@ -208,13 +208,14 @@ struct Cfg {
     static constexpr uint32_t IDESC = BS ? make_idesc_bs(KIND, 128, BN) : make_idesc(KIND, PAIR ? 256 : 128, BN);
     // K blocks the MMA thread takes per pass (measured; the MMAs and their order
     // are the same, so C is bitwise the same): 4 for Swap-AB tiles with rings of
-    // 8+ stages (3-8 % less time at small M), 2 for plain 128-column tiles
+    // 8+ stages, fused ones included (3-8 % less time at small M; a fused
+    // tile-16 layer at M = 1 1.2 us less), 2 for plain 128-column tiles
     // (6-stage rings, 3-5 %), 1 for the 256-column tiles, whose 4-stage rings
     // need each stage released at once (grouping them cost 10-50 %)
     // Block-FP8 plain tiles: K blocks the epilogue folds in per accumulator wait
     // (at most NACC - 1, so the MMA always has a free buffer)
     static constexpr int BLOCK_PASS = 2;
-    static constexpr int MMA_GROUP = (FUSE || BLOCK || PAIR) ? 1
+    static constexpr int MMA_GROUP = (BLOCK || PAIR) ? 1
                                      : (SWAP && STAGES >= 8) ? 4
                                      : (!SWAP && BN == 128 && STAGES >= 6) ? 2 : 1;
     static constexpr size_t STAGING_OFF = (size_t)STAGES * STAGE_BYTES;
@@ -317,6 +318,9 @@ __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
 __device__ __forceinline__ void sts_u4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
+}
+__device__ __forceinline__ void sts_u2(uint32_t addr, uint2 v) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y) : "memory");
 }
 __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
     uint4 v;
@@ -712,6 +716,21 @@ __device__ __forceinline__ bool consume_segment_slice(const GemmArgs& a, const U
     return true;
 }
 
+// End of a fused unit: rows past M get zero codes (what the TMA's
+// out-of-bounds fill gives), then the generic-proxy stores are made visible
+// to the tensor core.  sA as in fused_quantize_unit; cpr: 16-byte chunks per
+// row of the unit.
+template <int BN>
+__device__ __forceinline__ void finish_fused_rows(uint32_t sA, int rows, int cpr) {
+    for (int i = threadIdx.x; i < (BN - rows) * cpr; i += kEpiThreads) {
+        const int r = rows + i / cpr, ch = i % cpr;
+        const int kbl = ch >> 3, c = ch & 7;
+        sts_u4(sA + (uint32_t)(kbl * BN * 128 + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)),
+               make_uint4(0u, 0u, 0u, 0u));
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Fused activation quantisation of one Swap-AB unit (the 256 epilogue
 // threads, which all call it): rows m0..m0+BN-1 of x, K blocks kb0..kb1-1,
 // into the resident operand sA ([K block][BN rows x 128 B], 16-byte chunk c of
@@ -720,13 +739,15 @@ __device__ __forceinline__ bool consume_segment_slice(const GemmArgs& a, const U
 // [BN][MAXKB]).  The arithmetic is the stand-alone quantisers'
 // (quant_math.cuh), so codes and scales are theirs bit for bit.  Only rows
 // below M are read; the work is spread over all threads by element, not by
-// row, and every thread issues its loads before it uses them, so a batch of
-// one row costs about two L2 round trips.  Rows past M get zero codes.
+// row.  Per token: when a thread's share of its row fits in registers (rows
+// of up to 16 x 256 x 8 elements per unit), all its loads go out at once and
+// the codes are made from the registers, so a unit costs one L2 round trip;
+// longer rows take two passes.  Rows past M get zero codes.
 // rmax: BN words of scratch shared memory (per-token formats).  xs: a
 // shared-memory buffer of xs_bytes; when the unit's slice of x (rows x its K
 // range in bf16) fits, pass 1 keeps that slice there and pass 2 reads it back
 // instead of going to memory a second time.
-template <int FMT, int BN, int MAXKB>
+template <int FMT, int BN, int MAXKB, bool IN_REGS = false>
 __device__ __forceinline__ void fused_quantize_unit(const GemmArgs& a, const Unit& un, uint32_t sA, float* sa,
                                                     uint32_t* rmax, uint32_t xs, int xs_bytes) {
     constexpr int T = kEpiThreads;
@@ -746,6 +767,7 @@ __device__ __forceinline__ void fused_quantize_unit(const GemmArgs& a, const Uni
     auto xrow = [&](int r) { return reinterpret_cast<const uint4*>(a.x + (size_t)(m0 + r) * a.ld_x); };
     if constexpr (FMT != QLIN_FMT_FP8_BLOCK) {
         constexpr float QMAX = (FMT == QLIN_FMT_INT8) ? 127.f : 448.f;
+        constexpr int RV = 16;  // 16-byte vectors of a row one thread may hold
         // TPR consecutive threads per row: the largest power of two with
         // TPR * rows <= T (so a batch of one row has all 256 threads on it)
         int tpr = T;
@@ -753,10 +775,69 @@ __device__ __forceinline__ void fused_quantize_unit(const GemmArgs& a, const Uni
         const int r = tid / tpr, sub = tid % tpr;
         const bool live = r < rows;
         const uint4* xr = xrow(live ? r : 0);
-        // pass 1: the row maximum over all of K, 16-byte vectors, loads first;
-        // the vectors of this unit's K range are kept in xs when they fit
         const int nvec = (int)(K >> 3);
         const int uv0 = un.kb0 * 16, uvn = nkb * 16;  // the unit's vectors of a row
+        uint8_t* qrow = write_out ? a.a_q_out + (size_t)(m0 + r) * K : nullptr;
+        // The row maximum from the threads' partial maxima: within the warp
+        // (a row's lanes are consecutive), then across warps for rows wider
+        // than a warp (|x| >= 0, so float order = bit order).  Writes the
+        // unit's scales (and, once per row, s_a) and returns row r's scale.
+        auto row_scale_from = [&](float amax) -> float {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float other = __shfl_xor_sync(0xffffffffu, amax, o);
+                if (o < tpr) amax = fmaxf(amax, other);
+            }
+            for (int i = tid; i < BN; i += T) rmax[i] = 0u;
+            named_bar_sync(1, T);
+            if (live && ((tid % tpr) & 31) == 0) atomicMax(&rmax[r], __float_as_uint(amax));
+            named_bar_sync(1, T);
+            for (int i = tid; i < BN; i += T) {
+                const float s = i < rows ? __fdiv_rn(__uint_as_float(rmax[i]), QMAX) : 0.f;
+                sa[i] = s;
+                if (i < rows && un.pt == 0 && un.seg == 0 && a.s_a_out) a.s_a_out[m0 + i] = s;
+            }
+            return live ? __fdiv_rn(__uint_as_float(rmax[r]), QMAX) : 0.f;
+        };
+        if (IN_REGS && (nvec + tpr - 1) / tpr <= RV) {
+            // A thread's share of its row fits in registers (RV vectors): one
+            // batch of loads, the row maximum, then the codes straight from
+            // the registers (8 codes = half a swizzled 16-byte chunk each).
+            uint4 v[RV];
+            float amax = 0.f;
+            if (live) {
+#pragma unroll
+                for (int j = 0; j < RV; ++j)
+                    if (sub + j * tpr < nvec) v[j] = __ldg(xr + sub + j * tpr);
+#pragma unroll
+                for (int j = 0; j < RV; ++j)
+                    if (sub + j * tpr < nvec) amax = fmaxf(amax, qm::absmax8(v[j]));
+            }
+            const float sc = row_scale_from(amax);
+            const qm::Divisor dv = qm::make_divisor(sc);
+            auto put = [&](int vu, uint2 q) {  // vu: vector within the unit's K range
+                sts_u2(sa_addr(r, vu >> 1) + (uint32_t)((vu & 1) * 8), q);
+                if (qrow) *reinterpret_cast<uint2*>(qrow + (size_t)(uv0 + vu) * 8) = q;
+            };
+            if (live && dv.fast) {
+#pragma unroll
+                for (int j = 0; j < RV; ++j) {
+                    const int vu = sub + j * tpr - uv0;
+                    if (vu >= 0 && vu < uvn) put(vu, qm::quant8<FMT, true>(v[j], dv));
+                }
+            } else if (live) {
+                // a scale outside the reciprocal's range: the IEEE division,
+                // one vector at a time, read again from memory
+#pragma unroll 1
+                for (int vu = sub - uv0 + ((uv0 - sub + tpr - 1) / tpr) * tpr; vu < uvn; vu += tpr)
+                    put(vu, qm::quant8<FMT>(__ldg(xr + uv0 + vu), dv));
+            }
+            finish_fused_rows<BN>(sA, rows, cpr);
+            return;
+        }
+        // Longer rows. pass 1: the row maximum over all of K, 16-byte vectors,
+        // loads first; the vectors of this unit's K range are kept in xs when
+        // they fit
         const bool staged = rows * uvn * 16 <= xs_bytes;
         float amax = 0.f;
         if (live) {
@@ -776,25 +857,10 @@ __device__ __forceinline__ void fused_quantize_unit(const GemmArgs& a, const Uni
                 }
             }
         }
-        // within the warp (a row's lanes are consecutive), then across warps
-        // for rows wider than a warp; |x| >= 0, so float order = bit order
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float other = __shfl_xor_sync(0xffffffffu, amax, o);
-            if (o < tpr) amax = fmaxf(amax, other);
-        }
-        for (int i = tid; i < BN; i += T) rmax[i] = 0u;
-        named_bar_sync(1, T);
-        if (live && (sub & 31) == 0) atomicMax(&rmax[r], __float_as_uint(amax));
-        named_bar_sync(1, T);
-        for (int i = tid; i < BN; i += T) {
-            const float sc = i < rows ? __fdiv_rn(__uint_as_float(rmax[i]), QMAX) : 0.f;
-            sa[i] = sc;
-            if (i < rows && un.pt == 0 && un.seg == 0 && a.s_a_out) a.s_a_out[m0 + i] = sc;
-        }
+        const float sc = row_scale_from(amax);
         // pass 2: the unit's K range, 16 elements -> one 16-byte chunk of codes
         if (live) {
-            const qm::Divisor dv = qm::make_divisor(__fdiv_rn(__uint_as_float(rmax[r]), QMAX));
+            const qm::Divisor dv = qm::make_divisor(sc);
             const uint4* xsrc = xr + (((int64_t)un.kb0 * 128) >> 3);
             uint8_t* qout = write_out ? a.a_q_out + (size_t)(m0 + r) * K + (int64_t)un.kb0 * 128 : nullptr;
             for (int c0 = sub; c0 < cpr; c0 += tpr * UNROLL2) {
@@ -869,10 +935,7 @@ __device__ __forceinline__ void fused_quantize_unit(const GemmArgs& a, const Uni
             }
         }
     }
-    // rows past M: zero codes (what the TMA's out-of-bounds fill gives)
-    for (int i = tid; i < (BN - rows) * cpr; i += T) sts_u4(sa_addr(rows + i / cpr, i % cpr), make_uint4(0u, 0u, 0u, 0u));
-    // make the generic-proxy stores visible to the tensor core, then hand over
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    finish_fused_rows<BN>(sA, rows, cpr);
 }
 
 // Block-FP8: stage the scale products s_a[m,kb] * s_w[n/128,kb] of a window of
@@ -1311,7 +1374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         if constexpr (FUSE) {
             if (u_first < units) {
-                fused_quantize_unit<FMT, BN, C::A_MAXKB>(args, decode_unit<FMT>(args, u_first), sA, sa_tile,
+                fused_quantize_unit<FMT, BN, C::A_MAXKB, true>(args, decode_unit<FMT>(args, u_first), sA, sa_tile,
                                                          rmax, xstage, kStagingBytes);
                 warp_arrive(a_full);
             }

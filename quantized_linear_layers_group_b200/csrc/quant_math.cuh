@@ -64,8 +64,11 @@ __device__ __forceinline__ Divisor make_divisor(float s) {
     return d;
 }
 
+// FAST_ONLY: the caller has checked d.fast, so no IEEE division is compiled
+// in (and no registers need to survive a call to it).
+template <bool FAST_ONLY = false>
 __device__ __forceinline__ float quotient(float x, const Divisor& d) {
-    if (d.fast) {
+    if (FAST_ONLY || d.fast) {
         const float q0 = __fmul_rn(x, d.r);
         const float rem = __fmaf_rn(-q0, d.s, x);
         return copysignf(__fmaf_rn(rem, d.r, q0), x);
@@ -73,13 +76,14 @@ __device__ __forceinline__ float quotient(float x, const Divisor& d) {
     return __fdiv_rn(x, d.s);
 }
 
+template <bool FAST_ONLY = false>
 __device__ __forceinline__ uint32_t quant_int8_x4(const float* f, const Divisor& d) {
     uint32_t out = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         int r = 0;
         if (d.s != 0.f) {
-            r = __float2int_rn(quotient(f[i], d));
+            r = __float2int_rn(quotient<FAST_ONLY>(f[i], d));
             r = max(-127, min(127, r));
         }
         out |= (uint32_t)(r & 0xFF) << (8 * i);
@@ -87,27 +91,28 @@ __device__ __forceinline__ uint32_t quant_int8_x4(const float* f, const Divisor&
     return out;
 }
 
+template <bool FAST_ONLY = false>
 __device__ __forceinline__ uint32_t quant_e4m3_x4(const float* f, const Divisor& d) {
     if (d.s == 0.f) return 0u;
     float v[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = fminf(fmaxf(quotient(f[i], d), -448.f), 448.f);
+    for (int i = 0; i < 4; ++i) v[i] = fminf(fmaxf(quotient<FAST_ONLY>(f[i], d), -448.f), 448.f);
     const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v[0], v[1]), __NV_SATFINITE, __NV_E4M3);
     const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(v[2], v[3]), __NV_SATFINITE, __NV_E4M3);
     return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
-template <int FMT>
+template <int FMT, bool FAST_ONLY = false>
 __device__ __forceinline__ uint2 quant8(const uint4& v, const Divisor& d) {
     float f[8];
     unpack8(v, f);
     uint2 r;
     if constexpr (FMT == QLIN_FMT_INT8) {
-        r.x = quant_int8_x4(f, d);
-        r.y = quant_int8_x4(f + 4, d);
+        r.x = quant_int8_x4<FAST_ONLY>(f, d);
+        r.y = quant_int8_x4<FAST_ONLY>(f + 4, d);
     } else {
-        r.x = quant_e4m3_x4(f, d);
-        r.y = quant_e4m3_x4(f + 4, d);
+        r.x = quant_e4m3_x4<FAST_ONLY>(f, d);
+        r.y = quant_e4m3_x4<FAST_ONLY>(f + 4, d);
     }
     return r;
 }

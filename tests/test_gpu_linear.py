@@ -126,6 +126,27 @@ def test_fused_layer_strided_activations(fmt):
                                           what=f"strided fmt={fmt} tile={tile} S={S}")
 
 
+@pytest.mark.parametrize("fmt", [oracle.FMT_INT8, oracle.FMT_FP8])
+def test_fused_layer_rows_with_scales_outside_the_reciprocal_range(fmt):
+    # Row scales amax / Qmax below 2^-68 or above 2^92 take the IEEE division
+    # instead of the reciprocal and its correction step, in the fused kernel's
+    # register-resident path (first unit of a CTA) as in the quantiser.
+    M, N, K = 8, 256, 1024
+    x, w, b = _inputs(fmt, M, N, K, seed=41 + fmt)
+    row_exp = [-80, -70, -58, 0, 96, 103, 110, None]  # None: an all-zero row
+    xf = x.float()
+    for r, e in enumerate(row_exp):
+        xf[r] = 0.0 if e is None else torch.ldexp(xf[r] / xf[r].abs().max(), torch.tensor(float(e)))
+    x = xf.to(torch.bfloat16)
+    assert torch.isfinite(x.float()).all()
+    layer = Layer(fmt, w, b)
+    x_dev = x.cuda()
+    for tile, S in ((16, 1), (32, 2), (64, 1)):
+        _check_against_unfused_and_oracle(layer, x, x_dev, K, SWAPAB if S == 1 else SWAPAB_SPLITK, tile, S,
+                                          what=f"extreme scales fmt={fmt} tile={tile} S={S}")
+    check_status()
+
+
 def test_fused_int8_accumulators_bit_exact():
     from quantized_linear_layers_group_b200 import qlin
 
