@@ -78,3 +78,31 @@ def test_dominant_kernel_groups_launches_like_the_launch_list():
     assert bench.kernel_of(1, cfg[1024]) == "qlin_gemm_kernel<1, 0, 256, 0, 0, 0>"
     assert bench.kernel_of(1, {"variant": qlin.QLIN_VAR_SWAPAB_SPLITK, "tile_n": 16}) == \
         bench.kernel_of(1, cfg[16])
+
+
+def test_fused_layers_and_kernel_count_follow_the_configurations():
+    # With --fused, a layer is one kernel when its configuration is Swap-AB
+    # and a unit's K blocks fit the resident 64 KiB activation operand
+    # (K/128/S <= 65536 / (tile_n * 128)); every other layer is the quantiser
+    # plus the GEMM.  gpu_launches is built from this count.
+    import bench
+    import synth
+    from quantized_linear_layers_group_b200 import qlin
+
+    hp = bench.HotPath.__new__(bench.HotPath)
+    hp.qlin = qlin
+    hp.w = synth.WORKLOADS["fp8_attn"]          # K = 2048: 16 K blocks
+    hp.fmt = hp.w.fmt
+    hp.ms = [1, 64, 256, 2048]
+    hp.configs = {
+        1: {"variant": qlin.QLIN_VAR_SWAPAB, "tile_n": 16, "k_segments": 1},          # 16 <= 32: fused
+        64: {"variant": qlin.QLIN_VAR_SWAPAB, "tile_n": 64, "k_segments": 1},         # 16 > 8: two kernels
+        256: {"variant": qlin.QLIN_VAR_SWAPAB_SPLITK, "tile_n": 64, "k_segments": 2},  # 8 <= 8: fused
+        2048: {"variant": qlin.QLIN_VAR_PLAIN, "tile_n": 256, "k_segments": 1},       # plain: two kernels
+    }
+    hp.fused = True
+    assert [hp.layer_is_fused(M) for M in hp.ms] == [True, False, True, False]
+    assert hp.kernels_per_step() == 1 + 2 + 1 + 2
+    hp.fused = False
+    assert not any(hp.layer_is_fused(M) for M in hp.ms)
+    assert hp.kernels_per_step() == 2 * len(hp.ms)
