@@ -253,7 +253,7 @@ QLIN_API qlin_status qlin_matmul_bf16(int variant, int tile_n, int k_segments, i
 
 /*
  * qlin_scaled_mm_noalloc -- qlin_scaled_mm for callers that cannot allocate
- * device memory and so cannot pass a workspace (the paper has no counterpart;
+ * device memory and so cannot pass a workspace (no source page describes one;
  * this is a library convenience).  Typical caller: a plugin inside a serving
  * engine that owns the whole device-memory pool and forbids allocations it
  * does not make itself, so that every byte the engine hands out is accounted
