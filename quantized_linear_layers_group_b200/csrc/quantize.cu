@@ -119,13 +119,14 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
 }
 
 // ----------------------------------------------------------------------------
-// Block-FP8 activations, 1x128 groups: WPR warps per row.  Thread t of the
-// row's group owns vectors t, t + 32*WPR, ...; in each step lanes 0-15 and
-// 16-31 of a warp hold one whole group each (16 vectors x 8 = 128), so the
-// group maximum is a 16-lane shuffle reduction.
+// Block-FP8 activations, 1x128 groups, few rows (latency first): 8 warps per
+// row.  Thread t of the row owns vectors t, t + 256, ...; in each step lanes
+// 0-15 and 16-31 of a warp hold one whole group each (16 vectors x 8 = 128),
+// so the group maximum is a 16-lane shuffle reduction.  A row is spread over
+// all 256 threads, so each lane's chain of work is short.
 template <int VPL, int WPR>
 __global__ void __launch_bounds__(kQuantWarps * 32)
-    quantize_group128_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+    quantize_group128_wide_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
                              uint8_t* __restrict__ q, float* __restrict__ s) {
     pdl_wait();
     pdl_launch_dependents();
@@ -164,6 +165,63 @@ __global__ void __launch_bounds__(kQuantWarps * 32)
                 if ((lane & 15) == 0) sr[idx >> 4] = sc;
                 const Divisor dv = make_divisor(sc);
                 qr[idx] = quant8<QLIN_FMT_FP8>(v[i], dv);
+            }
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------
+// Block-FP8 activations, 1x128 groups, many rows (instructions first): WPR warps per row.  A group's 16
+// vectors (8 elements each) belong to 4 consecutive lanes: lane l takes group
+// slot l / 4 and vectors l % 4, l % 4 + 4, l % 4 + 8 and l % 4 + 12 of it, so
+// one warp instruction of the scale computation serves 8 groups and the group
+// maximum is a 4-lane shuffle.  The row's WPR warps cover 8 * WPR groups per
+// slot; a lane takes PASSES slots per round and issues all their loads before
+// the first reduction, so a row of up to 8 * WPR * PASSES groups costs one
+// memory round trip.
+template <int PASSES, int WPR>
+__global__ void __launch_bounds__(kQuantWarps * 32)
+    quantize_group128_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                             uint8_t* __restrict__ q, float* __restrict__ s) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * (kQuantWarps / WPR) + warp / WPR;
+    if (row >= rows) return;  // warp-uniform: the shuffles below stay converged
+    const int gw = (warp % WPR) * 8 + (lane >> 2);  // this lane's group within a slot of the row
+    const int sub = lane & 3;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + row * ld);
+    const int ngroups = (int)(cols >> 7);
+    uint2* qr = reinterpret_cast<uint2*>(q + row * cols);
+    float* sr = s + row * ngroups;
+    constexpr int GPS = 8 * WPR;  // groups of the row per slot
+    for (int g0 = 0; g0 < ngroups; g0 += GPS * PASSES) {
+        uint4 v[PASSES][4];
+#pragma unroll
+        for (int p = 0; p < PASSES; ++p) {
+            const int g = g0 + p * GPS + gw;
+            if (g < ngroups) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) v[p][j] = ld_stream(xr + g * 16 + sub + 4 * j);
+            }
+        }
+#pragma unroll
+        for (int p = 0; p < PASSES; ++p) {
+            const int g = g0 + p * GPS + gw;
+            float gmax = 0.f;
+            if (g < ngroups) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) gmax = fmaxf(gmax, absmax8(v[p][j]));
+            }
+            gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 1));
+            gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 2));
+            if (g < ngroups) {
+                const float sc = __fdiv_rn(gmax, 448.f);
+                if (sub == 0) sr[g] = sc;
+                const Divisor dv = make_divisor(sc);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) qr[g * 16 + sub + 4 * j] = quant8<QLIN_FMT_FP8>(v[p][j], dv);
             }
         }
     }
@@ -251,14 +309,27 @@ cudaError_t launch_per_token_fmt(const uint16_t* x, int64_t rows, int64_t cols, 
     }
 }
 
+// Few rows: the row spread over the 256 threads of a CTA (16 lanes per group).
+cudaError_t launch_group_wide(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* q, float* s,
+                              bool pdl, cudaStream_t st) {
+    constexpr int WPR = 8;
+    const int64_t per_thread = ((cols >> 3) + 32 * WPR - 1) / (32 * WPR);
+    const dim3 grid((unsigned)rows), block(kQuantWarps * 32);
+    if (per_thread <= 1) return launch_k(quantize_group128_wide_kernel<1, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (per_thread <= 4) return launch_k(quantize_group128_wide_kernel<4, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    return launch_k(quantize_group128_wide_kernel<8, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+}
+
+// Many rows: 4 lanes per group.
 template <int WPR>
 cudaError_t launch_group_wpr(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* q, float* s,
                              bool pdl, cudaStream_t st) {
-    const int64_t per_thread = ((cols >> 3) + 32 * WPR - 1) / (32 * WPR);
+    const int64_t slots = ((cols >> 7) + 8 * WPR - 1) / (8 * WPR);  // group slots per lane
     const dim3 grid((unsigned)((rows + (kQuantWarps / WPR) - 1) / (kQuantWarps / WPR))), block(kQuantWarps * 32);
-    if (per_thread <= 1) return launch_k(quantize_group128_kernel<1, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
-    if (per_thread <= 4) return launch_k(quantize_group128_kernel<4, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
-    return launch_k(quantize_group128_kernel<8, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (slots <= 1) return launch_k(quantize_group128_kernel<1, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (slots <= 2) return launch_k(quantize_group128_kernel<2, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    if (slots <= 3) return launch_k(quantize_group128_kernel<3, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);
+    return launch_k(quantize_group128_kernel<4, WPR>, grid, block, pdl, st, x, rows, cols, ld, q, s);  // rounds of 4
 }
 
 }  // namespace
@@ -276,11 +347,16 @@ cudaError_t launch_quantize_block(const void* x, int64_t rows, int64_t cols, int
     const auto* xb = static_cast<const uint16_t*>(x);
     auto* qb = static_cast<uint8_t*>(q);
     if (block_rows == 1) {
-        switch (warps_per_row(rows)) {
-            case 8: return launch_group_wpr<8>(xb, rows, cols, ld, qb, s, pdl, st);
-            case 2: return launch_group_wpr<2>(xb, rows, cols, ld, qb, s, pdl, st);
-            default: return launch_group_wpr<1>(xb, rows, cols, ld, qb, s, pdl, st);
-        }
+        // Few rows are latency-bound: the short per-lane chains of the wide
+        // kernel win (Block-FP8 K = 6144: 2.8 against 4.1 us at M <= 64).
+        // Many rows are issue-bound: 4 lanes per group cut the instructions
+        // per element (M = 2048: 14.4 against 16.4 us).
+        if (warps_per_row(rows) == 8) return launch_group_wide(xb, rows, cols, ld, qb, s, pdl, st);
+        // no more warps on a row than it has slots of 8 groups for
+        int wpr = warps_per_row(rows);
+        while (wpr > 1 && 8 * wpr > (cols >> 7)) wpr >>= 1;
+        return wpr == 2 ? launch_group_wpr<2>(xb, rows, cols, ld, qb, s, pdl, st)
+                        : launch_group_wpr<1>(xb, rows, cols, ld, qb, s, pdl, st);
     }
     const dim3 grid((unsigned)(cols >> 7), (unsigned)((rows + 127) / 128));
     return launch_k(quantize_block128_kernel, grid, dim3(256), pdl, st, xb, rows, cols, ld, qb, s);

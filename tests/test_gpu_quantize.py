@@ -182,6 +182,17 @@ def test_group128_every_row_split(lib, rows):
     _assert_same(qg, sg, qr, sr, f"group rows={rows}")
 
 
+@pytest.mark.parametrize("rows", [3, 700, 2500])
+@pytest.mark.parametrize("cols", [640, 1152, 4224, 6272])
+def test_group128_odd_group_counts(lib, rows, cols):
+    # 5, 9, 33 and 49 groups per row: a row's last slot of 8 groups per warp is
+    # partly empty, for each warps-per-row choice the row count leads to
+    x = synth.normal((rows, cols), 1.5, rows * 7 + cols)
+    qg, sg = _gpu_block(lib, x, 1)
+    qr, sr = oracle.quantize_block(x, 1, 128)
+    _assert_same(qg, sg, qr, sr, f"group rows={rows} cols={cols}")
+
+
 def _markstein_rows(fmt, binades):
     """Rows [amax, x...] for every amax significand in the given binades: the
     row's x values are every bf16 significand at every exponent from amax's
